@@ -1,0 +1,405 @@
+"""CPU oracle of Prism's dynamic sparse video self-attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+benchmark's CPU-baseline leg may import this module; the library never does.
+It shares no code with the CUDA path.
+
+Source: "Prism: Dynamic Sparse Attention for Native 2K Joint Video-Audio
+Generation Model Training" (arXiv 2610.05416), as printed on the pages
+xyznot.com/id/paper/2610.05416 (section "Metode" 1-3, the clean equations) and
+paper.rainbus.top/paper/2610.05416 (section "方法步骤详情": Algorithm 1's
+five stages and the hyperparameters).  Each function names the step it follows.
+
+Precision.  Statistics, pooled means, logits and attention are accumulated in
+float64.  Every quantity that decides an integer (the block volume B, the
+snapped shape, the selected block set) is taken in float32, the precision of
+the CUDA path: r, v_hat, a_bar and rho are rounded to float32 after their
+float64 normalisation, and g, log2 g, l*, the snap distances, the softmax
+probabilities and the Top-p prefix sums are float32 arithmetic.
+
+Readings where the pages are silent (listed with their reasons in the design
+notes of the repository):
+  * "mean-pooled along axis d" = average over the plane orthogonal to d, giving
+    the Z_d-long profile that the variance formula indexes by i;
+  * r = (1/3, 1/3, 1/3) when the three directional variances sum to zero;
+  * audio coupling a_bar(m) = zone mean of a, divided by its maximum over the
+    zones (0 when that maximum is 0); v_hat_{a,d} = directional variance of
+    the zone's slice means of a, divided by the sum over the three axes (0 when
+    that sum is 0); a missing map (first layer) means a_bar = 0;
+  * information density rho(m) = channel mean of [mean over frames of the
+    spatial variance within the frame + variance of the frame differences],
+    divided by its maximum over the zones of the head (0 when that max is 0);
+    B = 256 if rho < tau256, else 128 if rho < tau128, else 64;
+  * the candidate set C_B lists (b_T, b_H, b_W) in ascending lexicographic
+    order; snapping takes the least squared log2 distance, ties to the lower
+    index;
+  * blocks tile the zone in raster order of block coordinates, tokens inside a
+    block in raster (t, h, w) order; permuted position = 512 m + block * B +
+    token;
+  * selection: logits Qbar_i . Kbar_j / sqrt(D), softmax over all key blocks,
+    order (P descending, j ascending); Top-p keeps the shortest prefix whose
+    float32 running sum reaches p (p >= 1 keeps all, p <= 0 none); the union
+    with Top-k of the same order is the first max(k, L) blocks.
+
+Parity status: the candidate set, the closed form l*, the snapping, the
+directional statistics, the selection rule and the attention (forward and
+backward) are pinned by the tests in tests/test_oracle_pins.py.  The rho
+formula and the a_bar / v_hat normalisations are readings; their code is
+pinned to hand-built fields and to a per-token brute force, the readings
+themselves are not pinned by the pages ("parity unpinned" for the reading).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+Z = 8  # macro-zone edge Z_T = Z_H = Z_W (section "Ide utama")
+F32 = np.float32
+
+
+# ---------------------------------------------------------------------------
+# Candidate shapes (section "Metode" 2: edges from {2, 4, 8}, product B,
+# 16 shapes over B in {64, 128, 256}).
+# ---------------------------------------------------------------------------
+def candidate_shapes():
+    """All (b_T, b_H, b_W) with edges in {2,4,8} and volume 64, 128 or 256.
+
+    Listed by volume, then lexicographically; the list index is the shape id.
+    """
+    out = []
+    for vol in (64, 128, 256):
+        for bt in (2, 4, 8):
+            for bh in (2, 4, 8):
+                for bw in (2, 4, 8):
+                    if bt * bh * bw == vol:
+                        out.append((bt, bh, bw))
+    return out
+
+
+SHAPES = candidate_shapes()
+
+
+def shapes_of_volume(vol):
+    return [(i, s) for i, s in enumerate(SHAPES) if s[0] * s[1] * s[2] == vol]
+
+
+# ---------------------------------------------------------------------------
+# Stage 1: zone statistics ("Metode" 1; Algorithm 1 stage one)
+# ---------------------------------------------------------------------------
+def zones_of(X, T, H, W):
+    """Raster [N, C] -> [Nz, 8(t), 8(h), 8(w), C], zones in raster (zt, zh, zw) order."""
+    C = X.shape[-1]
+    Y = X.reshape(T // Z, Z, H // Z, Z, W // Z, Z, C).transpose(0, 2, 4, 1, 3, 5, 6)
+    return Y.reshape(-1, Z, Z, Z, C)
+
+
+def directional_variance(Vz):
+    """sigma^2_{v,d}(m) for d = T, H, W: [Nz, 3] float64.
+
+    Profile along d: the mean of V over the plane orthogonal to d (one value
+    per slice i = 1..Z_d and channel c); variance of the profile over i around
+    its mean mu^{(d)}_{m,c}; average over the D channels.
+    """
+    Vz = np.asarray(Vz, dtype=np.float64)
+    sig = np.empty((Vz.shape[0], 3))
+    for d, plane in enumerate(((2, 3), (1, 3), (1, 2))):
+        prof = Vz.mean(axis=plane)                      # [Nz, 8, D]
+        mu = prof.mean(axis=1, keepdims=True)           # [Nz, 1, D]
+        sig[:, d] = ((prof - mu) ** 2).mean(axis=1).mean(axis=-1)
+    return sig
+
+
+def ratio(sig):
+    """r_{v,d} = sigma^2_d / sum_d' sigma^2_d'; (1/3,1/3,1/3) where the sum is 0."""
+    tot = sig.sum(axis=1, keepdims=True)
+    r = np.full_like(sig, 1.0 / 3.0)
+    nz = tot[:, 0] > 0
+    r[nz] = sig[nz] / tot[nz]
+    return r
+
+
+def audio_terms(a, T, H, W):
+    """(a_bar [Nz], v_hat [Nz, 3]) from the cached A->V norm map a [T, H, W].
+
+    The map is a float32 tensor; its values are taken as float32 and then
+    summed in float64, so a constant map gives exactly zero variance.
+    """
+    a = np.asarray(a, dtype=np.float32).astype(np.float64)
+    az = zones_of(a.reshape(-1, 1), T, H, W)[..., 0]
+    mean = az.mean(axis=(1, 2, 3))                      # zone mean of a
+    sig = np.empty((az.shape[0], 3))
+    for d, plane in enumerate(((2, 3), (1, 3), (1, 2))):
+        prof = az.mean(axis=plane)                      # [Nz, 8]
+        sig[:, d] = ((prof - mean[:, None]) ** 2).mean(axis=1)
+    tot = sig.sum(axis=1, keepdims=True)
+    vhat = np.zeros_like(sig)
+    nz = tot[:, 0] > 0
+    vhat[nz] = sig[nz] / tot[nz]
+    mx = mean.max()
+    abar = mean / mx if mx > 0 else np.zeros_like(mean)
+    return abar, vhat
+
+
+def density_raw(Vz):
+    """Unnormalised information density per zone: [Nz] float64.
+
+    Channel mean of (mean over the 8 frames of the variance over the frame's
+    8x8 tokens) + (variance over all 7x8x8 frame differences V[t+1]-V[t]).
+    """
+    Vz = np.asarray(Vz, dtype=np.float64)
+    spatial = Vz.var(axis=(2, 3)).mean(axis=1)          # [Nz, D]
+    diff = Vz[:, 1:] - Vz[:, :-1]                       # [Nz, 7, 8, 8, D]
+    temporal = diff.var(axis=(1, 2, 3))                 # [Nz, D]
+    return (spatial + temporal).mean(axis=-1)
+
+
+def normalise_by_max(x):
+    mx = x.max()
+    return x / mx if mx > 0 else np.zeros_like(x)
+
+
+# ---------------------------------------------------------------------------
+# Stage 1 (cont.): volume quantisation and shape snapping ("Metode" 2)
+# ---------------------------------------------------------------------------
+def volume(rho32, tau128, tau256):
+    """B(m) from the float32 density: 256 below tau256, 128 below tau128, else 64."""
+    t128, t256 = F32(tau128), F32(tau256)
+    return np.where(rho32 < t256, 256, np.where(rho32 < t128, 128, 64)).astype(np.int64)
+
+
+def ideal_log_edges(g32, vol):
+    """l*_d = -1/2 log2 g_d + 1/3 (S + 1/2 sum_d' log2 g_d'), S = log2 B (float32)."""
+    lg = np.log2(g32.astype(F32))
+    S = np.log2(np.asarray(vol, dtype=F32))
+    half = F32(0.5)
+    inner = S + half * lg[..., 0] + half * lg[..., 1] + half * lg[..., 2]
+    return (-half * lg + (inner / F32(3.0))[..., None]).astype(F32)
+
+
+def snap(ell32, vol):
+    """Shape id of the candidate of volume vol nearest (squared log2 distance) to l*."""
+    best, best_d = -1, None
+    for sid, s in shapes_of_volume(int(vol)):
+        e = np.log2(np.asarray(s, dtype=F32))
+        d = (e - ell32).astype(F32)
+        dist = F32(d[0] * d[0]) + F32(d[1] * d[1])
+        dist = F32(dist + F32(d[2] * d[2]))
+        if best_d is None or dist < best_d:
+            best, best_d = sid, dist
+    return best
+
+
+def snap_margin(ell64, vol):
+    """Float64 gap between the two smallest snap distances (tie margin)."""
+    ds = sorted(float(np.sum((np.log2(np.asarray(s, float)) - ell64) ** 2))
+                for _, s in shapes_of_volume(int(vol)))
+    return ds[1] - ds[0] if len(ds) > 1 else np.inf
+
+
+def zone_shapes(V, a, T, H, W, eps, tau128=0.5, tau256=0.25):
+    """Stage one for one head: V [N, D] raster, a [T,H,W] or None.
+
+    Returns dict with shape_id [Nz], B [Nz], g [Nz,3] (float32), rho [Nz]
+    (float32) and the float64 decision margins rho_margin, snap_margin.
+    """
+    Vz = zones_of(np.asarray(V, dtype=np.float64), T, H, W)
+    r = ratio(directional_variance(Vz))
+    if a is None:
+        abar = np.zeros(Vz.shape[0])
+        vhat = np.zeros((Vz.shape[0], 3))
+    else:
+        abar, vhat = audio_terms(a, T, H, W)
+    g32 = (r.astype(F32) + abar.astype(F32)[:, None] * vhat.astype(F32) + F32(eps)).astype(F32)
+    rho64 = normalise_by_max(density_raw(Vz))
+    rho32 = rho64.astype(F32)
+    B = volume(rho32, tau128, tau256)
+    ell = ideal_log_edges(g32, B.astype(F32))
+    sid = np.array([snap(ell[m], B[m]) for m in range(len(B))], dtype=np.int64)
+    g64 = r + abar[:, None] * vhat + eps
+    lg = np.log2(g64)
+    ell64 = -0.5 * lg + (np.log2(B) + 0.5 * lg.sum(axis=1))[:, None] / 3.0
+    rho_margin = np.minimum(np.abs(rho64 - tau128), np.abs(rho64 - tau256))
+    smargin = np.array([snap_margin(ell64[m], B[m]) for m in range(len(B))])
+    return dict(shape_id=sid, B=B, g=g32, rho=rho32, r=r, abar=abar, vhat=vhat,
+                ell=ell, rho_margin=rho_margin, snap_margin=smargin)
+
+
+# ---------------------------------------------------------------------------
+# Stage 2: token reorder (Algorithm 1 stage two)
+# ---------------------------------------------------------------------------
+def _local_order(shape):
+    """Zone-local raster indices (lt*64 + lh*8 + lw) in block-contiguous order."""
+    bt, bh, bw = shape
+    out = []
+    for kt in range(Z // bt):
+        for kh in range(Z // bh):
+            for kw in range(Z // bw):
+                for lt in range(bt):
+                    for lh in range(bh):
+                        for lw in range(bw):
+                            out.append(((kt * bt + lt) * Z + kh * bh + lh) * Z + kw * bw + lw)
+    return np.array(out, dtype=np.int64)
+
+
+_LOCAL = [_local_order(s) for s in SHAPES]
+
+
+def partition(shape_id, T, H, W):
+    """src [N] (raster token of each permuted position) and block starts [N_b + 1]."""
+    zh_n, zw_n = H // Z, W // Z
+    src = np.empty(T * H * W, dtype=np.int64)
+    starts = [0]
+    for m, sid in enumerate(shape_id):
+        zt, rem = divmod(m, zh_n * zw_n)
+        zh, zw = divmod(rem, zw_n)
+        loc = _LOCAL[int(sid)]
+        lt, lh, lw = loc // 64, (loc // 8) % 8, loc % 8
+        src[512 * m: 512 * (m + 1)] = ((zt * Z + lt) * H + zh * Z + lh) * W + zw * Z + lw
+        vol = int(np.prod(SHAPES[int(sid)]))
+        starts.extend(512 * m + vol * (k + 1) for k in range(512 // vol))
+    return src, np.array(starts, dtype=np.int64)
+
+
+def pool(X, src, starts):
+    """Block means (float64) of X [N, D] raster over the permuted blocks."""
+    Xp = np.asarray(X, dtype=np.float64)[src]
+    sums = np.add.reduceat(Xp, starts[:-1], axis=0)
+    return sums / np.diff(starts)[:, None]
+
+
+# ---------------------------------------------------------------------------
+# Stage 3: block scoring and hybrid Top-k U Top-p ("Metode" 3)
+# ---------------------------------------------------------------------------
+def block_probs(Qbar, Kbar):
+    """P_i = softmax_j(Qbar_i . Kbar_j / sqrt(D)) with float32 logits: (s32, P32)."""
+    D = Qbar.shape[1]
+    s = (np.asarray(Qbar, np.float64) @ np.asarray(Kbar, np.float64).T / np.sqrt(D)).astype(F32)
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    P = (e / e.sum(axis=1, keepdims=True)).astype(F32)
+    return s, P
+
+
+def select_row(P_row, k, p):
+    """Selected key blocks (ascending) of one query block: first max(k, L) of the order."""
+    nb = P_row.shape[0]
+    order = np.argsort(-P_row, kind="stable")           # P descending, j ascending
+    if p >= 1.0:
+        L = nb
+    elif p <= 0.0:
+        L = 0
+    else:
+        cum = np.cumsum(P_row[order], dtype=F32)        # sequential float32 sum
+        hit = np.nonzero(cum >= F32(p))[0]
+        L = int(hit[0]) + 1 if hit.size else nb
+    cnt = max(min(int(k), nb), L)
+    return np.sort(order[:cnt]), order, cnt
+
+
+def select(Qbar, Kbar, k, p):
+    """List of selected key-block arrays for every query block, plus (s32, P32)."""
+    s, P = block_probs(Qbar, Kbar)
+    sel = [select_row(P[i], k, p)[0] for i in range(P.shape[0])]
+    return sel, s, P
+
+
+# ---------------------------------------------------------------------------
+# Whole plan for one head
+# ---------------------------------------------------------------------------
+def plan_head(Q, K, V, a, T, H, W, k, p, eps, tau128=0.5, tau256=0.25, shape_id=None):
+    """Stages one to three for one head.  Q, K, V: [N, D] raster."""
+    st = zone_shapes(V, a, T, H, W, eps, tau128, tau256)
+    sid = st["shape_id"] if shape_id is None else np.asarray(shape_id)
+    src, starts = partition(sid, T, H, W)
+    Qbar, Kbar = pool(Q, src, starts), pool(K, src, starts)
+    sel, s, P = select(Qbar, Kbar, k, p)
+    return dict(stats=st, shape_id=sid, src=src, starts=starts, Qbar=Qbar, Kbar=Kbar,
+                sel=sel, logits=s, P=P)
+
+
+def block_of_token(src, starts):
+    """Block id of every raster token."""
+    nb = len(starts) - 1
+    bid_perm = np.repeat(np.arange(nb), np.diff(starts))
+    out = np.empty_like(bid_perm)
+    out[src] = bid_perm
+    return out
+
+
+def token_mask(src, starts, sel):
+    """Dense [N, N] bool mask M[q, n] = block(n) in S_{block(q)} (raster order)."""
+    nb = len(starts) - 1
+    bsel = np.zeros((nb, nb), dtype=bool)
+    for i, js in enumerate(sel):
+        bsel[i, js] = True
+    bt = block_of_token(src, starts)
+    return bsel[bt][:, bt]
+
+
+# ---------------------------------------------------------------------------
+# Stage 4-5: sparse attention over the selected blocks, output in raster order
+# ---------------------------------------------------------------------------
+def attention_fwd(Q, K, V, src, starts, sel):
+    """O [N, D] and LSE [N] (float64, raster order) of attention restricted to S_i."""
+    Q, K, V = (np.asarray(x, np.float64) for x in (Q, K, V))
+    D = Q.shape[1]
+    O = np.empty_like(Q)
+    lse = np.empty(Q.shape[0])
+    for i, js in enumerate(sel):
+        qi = src[starts[i]:starts[i + 1]]
+        keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in js])
+        s = Q[qi] @ K[keys].T / np.sqrt(D)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        z = e.sum(axis=1, keepdims=True)
+        O[qi] = (e / z) @ V[keys]
+        lse[qi] = (m + np.log(z))[:, 0]
+    return O, lse
+
+
+def attention_bwd(Q, K, V, dO, src, starts, sel):
+    """dQ, dK, dV (float64, raster order): exact gradients with the selection fixed."""
+    Q, K, V, dO = (np.asarray(x, np.float64) for x in (Q, K, V, dO))
+    D = Q.shape[1]
+    sc = 1.0 / np.sqrt(D)
+    O, lse = attention_fwd(Q, K, V, src, starts, sel)
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for i, js in enumerate(sel):
+        qi = src[starts[i]:starts[i + 1]]
+        keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in js])
+        P = np.exp(Q[qi] @ K[keys].T * sc - lse[qi][:, None])
+        dV[keys] += P.T @ dO[qi]
+        dP = dO[qi] @ V[keys].T
+        Di = (dO[qi] * O[qi]).sum(axis=1, keepdims=True)
+        dS = P * (dP - Di)
+        dQ[qi] = dS @ K[keys] * sc
+        dK[keys] += dS.T @ Q[qi] * sc
+    return dQ, dK, dV
+
+
+def attention_rows(Q, K, V, src, starts, sel, rows, dO=None):
+    """Forward (and dQ when dO is given) for selected raster query rows only.
+
+    Returns O [len(rows), D], LSE [len(rows)] and optionally dQ [len(rows), D].
+    """
+    Q, K, V = (np.asarray(x, np.float64) for x in (Q, K, V))
+    D = Q.shape[1]
+    sc = 1.0 / np.sqrt(D)
+    bt = block_of_token(src, starts)
+    O = np.empty((len(rows), D))
+    lse = np.empty(len(rows))
+    dQ = np.empty((len(rows), D)) if dO is not None else None
+    for r, q in enumerate(rows):
+        js = sel[bt[q]]
+        keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in js])
+        s = K[keys] @ Q[q] * sc
+        m = s.max()
+        e = np.exp(s - m)
+        z = e.sum()
+        P = e / z
+        O[r] = P @ V[keys]
+        lse[r] = m + np.log(z)
+        if dO is not None:
+            g = np.asarray(dO[q], np.float64)
+            dP = V[keys] @ g
+            Di = g @ O[r]
+            dQ[r] = (P * (dP - Di)) @ K[keys] * sc
+    return O, lse, dQ
