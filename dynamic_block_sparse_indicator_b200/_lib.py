@@ -1,0 +1,222 @@
+"""ctypes binding of libprism (include/prism.h): argument marshalling only.
+
+Every step of the plan and of the attention runs in the library's CUDA
+kernels; this module passes device pointers, sizes and the current CUDA stream
+through, allocates outputs with torch, and raises on a non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libprism.so")
+
+PRISM_OK = 0
+PRISM_ERR_INVALID_ARG = 1
+PRISM_ERR_WORKSPACE = 2
+PRISM_ERR_CUDA = 3
+PRISM_ERR_TIMEOUT = 4
+PRISM_ERR_DEVICE_CHECK = 5
+PRISM_ERR_UNSUPPORTED = 6
+
+PRISM_BF16 = 0
+PRISM_F32 = 1
+
+ITEMS = {
+    "shape_id": (0, np.uint8), "nblocks": (1, np.int32), "blk_start": (2, np.int32),
+    "sel_bits": (3, np.uint32), "row_ptr": (4, np.int32), "col_idx": (5, np.int32),
+    "col_ptr": (6, np.int32), "row_idx": (7, np.int32), "qbar": (8, np.float32),
+    "kbar": (9, np.float32), "src": (10, np.int32), "zone_stats": (11, np.float32),
+}
+
+
+class PrismParams(C.Structure):
+    _fields_ = [("T", C.c_int32), ("H", C.c_int32), ("W", C.c_int32), ("heads", C.c_int32),
+                ("head_dim", C.c_int32), ("dtype", C.c_int32), ("top_k", C.c_int32),
+                ("top_p", C.c_float), ("eps", C.c_float), ("tau128", C.c_float),
+                ("tau256", C.c_float)]
+
+
+class PrismError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> C.CDLL:
+    """Load libprism.so; raises if it is missing (there is no fallback path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"libprism.so not built at {p}: run "
+                          "`python -m dynamic_block_sparse_indicator_b200.build`")
+    lib = C.CDLL(p)
+    vp, i32, sz = C.c_void_p, C.c_int, C.c_size_t
+    pp = C.POINTER(PrismParams)
+    sig = {
+        "prism_plan_workspace_bytes": (sz, [pp]),
+        "prism_plan": (i32, [pp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
+        "prism_plan_import": (i32, [pp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
+        "prism_attn_fwd": (i32, [vp, vp, vp, vp]),
+        "prism_attn_bwd": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
+        "prism_plan_item_bytes": (sz, [vp, i32]),
+        "prism_plan_export": (i32, [vp, i32, vp, sz, vp]),
+        "prism_get_status": (i32, [vp, vp]),
+        "prism_plan_destroy": (None, [vp]),
+        "prism_status_string": (C.c_char_p, [i32]),
+        "prism_version": (C.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(st: int) -> str:
+    return load().prism_status_string(st).decode()
+
+
+def make_params(T, H, W, heads, head_dim, dtype, top_k, top_p, eps, tau128=0.5, tau256=0.25):
+    return PrismParams(T, H, W, heads, head_dim, dtype, top_k, float(top_p), float(eps),
+                       float(tau128), float(tau256))
+
+
+def workspace_bytes(params: PrismParams) -> int:
+    return int(load().prism_plan_workspace_bytes(C.byref(params)))
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+class Plan:
+    """A plan handle plus the device buffers it points into (kept alive here)."""
+
+    def __init__(self, params, handle, workspace, inputs):
+        self.params = params
+        self._h = handle
+        self._ws = workspace
+        self._inputs = inputs          # Q, K, V must outlive the plan
+
+    @property
+    def handle(self):
+        return self._h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h and _lib is not None:
+            _lib.prism_plan_destroy(h)
+            self._h = None
+
+    @property
+    def N(self):
+        p = self.params
+        return p.T * p.H * p.W
+
+    def _out_dtype(self):
+        import torch
+        return torch.float32 if self.params.dtype == PRISM_F32 else torch.bfloat16
+
+    def attn_fwd(self, O=None, lse=None, stream=None):
+        import torch
+        p = self.params
+        dev = self._ws.device
+        if O is None:
+            O = torch.empty(p.heads, self.N, p.head_dim, dtype=self._out_dtype(), device=dev)
+        if lse is None:
+            lse = torch.empty(p.heads, self.N, dtype=torch.float32, device=dev)
+        st = load().prism_attn_fwd(self._h, _ptr(O), _ptr(lse), _stream(stream))
+        if st:
+            raise PrismError(st, "prism_attn_fwd")
+        return O, lse
+
+    def attn_bwd(self, dO, O, lse, dQ=None, dK=None, dV=None, stream=None):
+        import torch
+        p = self.params
+        dev = self._ws.device
+        mk = lambda: torch.empty(p.heads, self.N, p.head_dim, dtype=self._out_dtype(), device=dev)
+        dQ = mk() if dQ is None else dQ
+        dK = mk() if dK is None else dK
+        dV = mk() if dV is None else dV
+        st = load().prism_attn_bwd(self._h, _ptr(dO), _ptr(O), _ptr(lse), _ptr(dQ), _ptr(dK),
+                                   _ptr(dV), _stream(stream))
+        if st:
+            raise PrismError(st, "prism_attn_bwd")
+        return dQ, dK, dV
+
+    def export(self, item: str, stream=None) -> np.ndarray:
+        code, dt = ITEMS[item]
+        lib = load()
+        nbytes = int(lib.prism_plan_item_bytes(self._h, code))
+        out = np.empty(nbytes // np.dtype(dt).itemsize, dtype=dt)
+        st = lib.prism_plan_export(self._h, code, out.ctypes.data_as(C.c_void_p), nbytes,
+                                   _stream(stream))
+        if st:
+            raise PrismError(st, f"prism_plan_export({item})")
+        return out
+
+    def status(self, stream=None) -> int:
+        return int(load().prism_get_status(self._h, _stream(stream)))
+
+
+def _check_inputs(Q, K, V, params):
+    import torch
+    want = torch.float32 if params.dtype == PRISM_F32 else torch.bfloat16
+    N = params.T * params.H * params.W
+    for t in (Q, K, V):
+        if t.dtype != want or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("Q, K, V must be contiguous CUDA tensors of the plan's dtype")
+        if tuple(t.shape) != (params.heads, N, params.head_dim):
+            raise ValueError(f"expected [heads, N, D] = {(params.heads, N, params.head_dim)}, "
+                             f"got {tuple(t.shape)}")
+
+
+def plan(Q, K, V, a_map, params: PrismParams, workspace=None, stream=None) -> Plan:
+    """Stages 1-3 on the GPU.  Q, K, V: [heads, N, D] CUDA tensors (raster order)."""
+    import torch
+    lib = load()
+    _check_inputs(Q, K, V, params)
+    need = workspace_bytes(params)
+    if need == 0:
+        raise PrismError(PRISM_ERR_INVALID_ARG, "prism_plan_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    h = C.c_void_p()
+    st = lib.prism_plan(C.byref(params), _ptr(Q), _ptr(K), _ptr(V), _ptr(a_map), _ptr(workspace),
+                        workspace.numel(), _stream(stream), C.byref(h))
+    if st:
+        raise PrismError(st, "prism_plan")
+    return Plan(params, h, workspace, (Q, K, V, a_map))
+
+
+def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None, stream=None) -> Plan:
+    """A plan from given shape ids [heads, Nz] (uint8) and selection bitmap (int32/uint32 words)."""
+    import torch
+    lib = load()
+    _check_inputs(Q, K, V, params)
+    need = workspace_bytes(params)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    h = C.c_void_p()
+    st = lib.prism_plan_import(C.byref(params), _ptr(Q), _ptr(K), _ptr(V), _ptr(shape_id),
+                               _ptr(sel_bits), _ptr(workspace), workspace.numel(), _stream(stream),
+                               C.byref(h))
+    if st:
+        raise PrismError(st, "prism_plan_import")
+    return Plan(params, h, workspace, (Q, K, V, shape_id, sel_bits))

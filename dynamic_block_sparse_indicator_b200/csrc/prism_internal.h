@@ -1,0 +1,66 @@
+// prism_internal.h -- host-side plan handle and the workspace layout shared by
+// the plan, forward and backward translation units of libprism.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/prism.h"
+
+#include <cuda.h>
+
+namespace prism {
+
+// Geometry derived from prism_params.
+struct Geom {
+    int T, H, W, heads, D, dtype;
+    int Zt, Zh, Zw, Nz;   // macro-zones per axis / total
+    int64_t N;            // tokens per head
+    int NB;               // max blocks per head = N / 64
+    int NT;               // 128-token tiles per head = N / 128
+    int WORDS;            // 32-bit words per selection-bitmap row = ceil(NB / 32)
+};
+
+// Byte offsets of the workspace regions (each 256-byte aligned).
+struct Layout {
+    size_t err;                         // int32[4]: error word + detail
+    size_t araw;                        // double[Nz]  zone mean of the audio map
+    size_t abar, vhat;                  // float[Nz], float[Nz][3]
+    size_t zstat;                       // float[heads][Nz][4]
+    size_t shape_id;                    // uint8[heads][Nz]
+    size_t zone_off;                    // int32[heads][Nz + 1]  first block of each zone
+    size_t nblocks;                     // int32[heads]
+    size_t blk_start;                   // int32[heads][NB + 1]
+    size_t t64_blk;                     // int32[heads][NB]      block of each 64-token tile
+    size_t src;                         // int32[heads][N]        raster token of each slot
+    size_t qbar, kbar;                  // float[heads][NB][D]
+    size_t sel, selT;                   // uint32[heads][NB][WORDS]
+    size_t row_ptr, col_idx;            // int32[heads][NB + 1], int32[heads][NB * NB]
+    size_t col_ptr, row_idx;            // CSC
+    size_t qt_ptr, qt_ent;              // int32[heads][NT + 1], int32[heads][NT * NT]
+    size_t kt_ptr, kt_ent;              // (forward / backward tile lists)
+    size_t qp, kp, vp, dop;             // bf16[heads][N][D] block-ordered copies
+    size_t lse_p, di_p;                 // float[heads][N] (backward, block order)
+    size_t total;
+};
+
+Geom make_geom(const prism_params* p);
+Layout make_layout(const Geom& g);
+int validate_params(const prism_params* p);
+
+}  // namespace prism
+
+struct prism_plan_s {
+    prism_params p;
+    prism::Geom g;
+    prism::Layout L;
+    char* ws;                 // device workspace base
+    size_t ws_bytes;
+    int device;
+    int has_audio;
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 2D [heads*N, D] bf16 maps, 128B swizzle
+};
+
+// Internal entry points of the attention translation units.
+int prism_launch_attn_fwd(prism_plan_s* P, void* O, float* lse, void* stream);
+int prism_launch_attn_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse,
+                          void* dQ, void* dK, void* dV, void* stream);

@@ -1,0 +1,1185 @@
+// prism_plan.cu -- Prism's plan (Algorithm 1, stages 1-3) on sm_100a, and the
+// host side of the C ABI (validation, workspace layout, plan handle, export).
+//
+// Method: "Prism: Dynamic Sparse Attention for Native 2K Joint Video-Audio
+// Generation Model Training" (arXiv 2610.05416).  Stage 1 follows the
+// equations of section "Metode" 1-2 (page xyznot.com/id/paper/2610.05416) and
+// the stage list of section "方法步骤详情" (page paper.rainbus.top); stage 3
+// follows section "Metode" 3.  Where the pages leave a step open, the kernels
+// take the same plain readings as the CPU oracle:
+//   - directional profiles are means over the plane orthogonal to the axis;
+//   - r = 1/3 each when the three variances sum to zero;
+//   - a_bar = zone mean of the audio norm map / its max over zones,
+//     v_hat_d = directional variance of the map's slice means / their sum;
+//   - rho = channel mean of (mean per-frame spatial variance + variance of the
+//     frame differences), divided by its max over the head's zones;
+//   - the 16 candidates are ordered by volume then lexicographically, snapping
+//     ties go to the lower index; blocks tile a zone in raster order;
+//   - Top-p keeps the shortest prefix of (P desc, j asc) whose mass reaches p,
+//     the union with Top-k is the first max(k, L) blocks of that order.
+// Every decision (B, shape, selection) is taken in fp32; the audio statistics
+// are accumulated in fp64 (the map is tiny and its constant regions must give
+// exactly zero variance).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "prism_internal.h"
+
+namespace prism {
+
+// ------------------------------------------------------------------ geometry
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Geom make_geom(const prism_params* p) {
+    Geom g{};
+    g.T = p->T; g.H = p->H; g.W = p->W; g.heads = p->heads; g.D = p->head_dim; g.dtype = p->dtype;
+    g.Zt = p->T / 8; g.Zh = p->H / 8; g.Zw = p->W / 8;
+    g.Nz = g.Zt * g.Zh * g.Zw;
+    g.N = (int64_t)p->T * p->H * p->W;
+    g.NB = (int)(g.N / 64);
+    g.NT = (int)(g.N / 128);
+    g.WORDS = (g.NB + 31) / 32;
+    return g;
+}
+
+Layout make_layout(const Geom& g) {
+    Layout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+    const size_t H = (size_t)g.heads, NB = (size_t)g.NB, NT = (size_t)g.NT, N = (size_t)g.N;
+    L.err = take(16);
+    L.araw = take(sizeof(double) * g.Nz);
+    L.abar = take(sizeof(float) * g.Nz);
+    L.vhat = take(sizeof(float) * g.Nz * 3);
+    L.zstat = take(sizeof(float) * H * g.Nz * 4);
+    L.shape_id = take(H * g.Nz);
+    L.zone_off = take(sizeof(int) * H * (g.Nz + 1));
+    L.nblocks = take(sizeof(int) * H);
+    L.blk_start = take(sizeof(int) * H * (NB + 1));
+    L.t64_blk = take(sizeof(int) * H * NB);
+    L.src = take(sizeof(int) * H * N);
+    L.qbar = take(sizeof(float) * H * NB * g.D);
+    L.kbar = take(sizeof(float) * H * NB * g.D);
+    L.sel = take(sizeof(uint32_t) * H * NB * g.WORDS);
+    L.selT = take(sizeof(uint32_t) * H * NB * g.WORDS);
+    L.row_ptr = take(sizeof(int) * H * (NB + 1));
+    L.col_idx = take(sizeof(int) * H * NB * NB);
+    L.col_ptr = take(sizeof(int) * H * (NB + 1));
+    L.row_idx = take(sizeof(int) * H * NB * NB);
+    L.qt_ptr = take(sizeof(int) * H * (NT + 1));
+    L.qt_ent = take(sizeof(int) * H * NT * NT);
+    L.kt_ptr = take(sizeof(int) * H * (NT + 1));
+    L.kt_ent = take(sizeof(int) * H * NT * NT);
+    L.qp = take(2 * H * N * g.D);
+    L.kp = take(2 * H * N * g.D);
+    L.vp = take(2 * H * N * g.D);
+    L.dop = take(2 * H * N * g.D);
+    L.lse_p = take(sizeof(float) * H * N);
+    L.di_p = take(sizeof(float) * H * N);
+    L.total = off;
+    return L;
+}
+
+int validate_params(const prism_params* p) {
+    if (!p) return PRISM_ERR_INVALID_ARG;
+    if (p->T <= 0 || p->H <= 0 || p->W <= 0) return PRISM_ERR_INVALID_ARG;
+    if (p->T % 8 || p->H % 8 || p->W % 8) return PRISM_ERR_INVALID_ARG;
+    if (p->heads < 1) return PRISM_ERR_INVALID_ARG;
+    if (p->head_dim != 64 && p->head_dim != 128) return PRISM_ERR_INVALID_ARG;
+    if (p->dtype != PRISM_BF16 && p->dtype != PRISM_F32) return PRISM_ERR_INVALID_ARG;
+    if (p->top_k < 0) return PRISM_ERR_INVALID_ARG;
+    if (!(p->top_p >= 0.f && p->top_p <= 1.f)) return PRISM_ERR_INVALID_ARG;
+    if (p->top_k < 1 && p->top_p <= 0.f) return PRISM_ERR_INVALID_ARG;
+    if (!(p->eps > 0.f) || !std::isfinite(p->eps)) return PRISM_ERR_INVALID_ARG;
+    if (!(p->tau256 >= 0.f && p->tau128 >= p->tau256 && p->tau128 <= 1e30f))
+        return PRISM_ERR_INVALID_ARG;
+    const int64_t N = (int64_t)p->T * p->H * p->W;
+    // one query-block row of block probabilities is staged in shared memory
+    if (N / 64 > 48 * 1024) return PRISM_ERR_INVALID_ARG;
+    if ((int64_t)p->heads * N >= (int64_t)1 << 31) return PRISM_ERR_INVALID_ARG;
+    return PRISM_OK;
+}
+
+// ---------------------------------------------------------- shape table
+// The 16 candidates (b_T, b_H, b_W): volume 64, 128, 256; lexicographic.
+__constant__ int8_t c_shape[16][3] = {
+    {2, 4, 8}, {2, 8, 4}, {4, 2, 8}, {4, 4, 4}, {4, 8, 2}, {8, 2, 4}, {8, 4, 2},
+    {2, 8, 8}, {4, 4, 8}, {4, 8, 4}, {8, 2, 8}, {8, 4, 4}, {8, 8, 2},
+    {4, 8, 8}, {8, 4, 8}, {8, 8, 4}};
+__constant__ int8_t c_log2shape[16][3] = {
+    {1, 2, 3}, {1, 3, 2}, {2, 1, 3}, {2, 2, 2}, {2, 3, 1}, {3, 1, 2}, {3, 2, 1},
+    {1, 3, 3}, {2, 2, 3}, {2, 3, 2}, {3, 1, 3}, {3, 2, 2}, {3, 3, 1},
+    {2, 3, 3}, {3, 2, 3}, {3, 3, 2}};
+
+struct DevPlan {
+    int T, H, W, heads, D, Zh, Zw, Nz, NB, NT, WORDS;
+    int64_t N;
+    int* err;
+    double* araw;
+    float* abar;
+    float* vhat;
+    float* zstat;
+    uint8_t* shape_id;
+    int* zone_off;
+    int* nblocks;
+    int* blk_start;
+    int* t64_blk;
+    int* src;
+    float* qbar;
+    float* kbar;
+    uint32_t* sel;
+    uint32_t* selT;
+    int* row_ptr;
+    int* col_idx;
+    int* col_ptr;
+    int* row_idx;
+    int* qt_ptr;
+    int* qt_ent;
+    int* kt_ptr;
+    int* kt_ent;
+    __nv_bfloat16* qp;
+    __nv_bfloat16* kp;
+    __nv_bfloat16* vp;
+};
+
+static DevPlan dev_plan(const prism_plan_s* P) {
+    DevPlan d{};
+    const Geom& g = P->g;
+    const Layout& L = P->L;
+    d.T = g.T; d.H = g.H; d.W = g.W; d.heads = g.heads; d.D = g.D; d.Zh = g.Zh; d.Zw = g.Zw;
+    d.Nz = g.Nz; d.NB = g.NB; d.NT = g.NT; d.WORDS = g.WORDS; d.N = g.N;
+    char* b = P->ws;
+    d.err = (int*)(b + L.err);
+    d.araw = (double*)(b + L.araw);
+    d.abar = (float*)(b + L.abar);
+    d.vhat = (float*)(b + L.vhat);
+    d.zstat = (float*)(b + L.zstat);
+    d.shape_id = (uint8_t*)(b + L.shape_id);
+    d.zone_off = (int*)(b + L.zone_off);
+    d.nblocks = (int*)(b + L.nblocks);
+    d.blk_start = (int*)(b + L.blk_start);
+    d.t64_blk = (int*)(b + L.t64_blk);
+    d.src = (int*)(b + L.src);
+    d.qbar = (float*)(b + L.qbar);
+    d.kbar = (float*)(b + L.kbar);
+    d.sel = (uint32_t*)(b + L.sel);
+    d.selT = (uint32_t*)(b + L.selT);
+    d.row_ptr = (int*)(b + L.row_ptr);
+    d.col_idx = (int*)(b + L.col_idx);
+    d.col_ptr = (int*)(b + L.col_ptr);
+    d.row_idx = (int*)(b + L.row_idx);
+    d.qt_ptr = (int*)(b + L.qt_ptr);
+    d.qt_ent = (int*)(b + L.qt_ent);
+    d.kt_ptr = (int*)(b + L.kt_ptr);
+    d.kt_ent = (int*)(b + L.kt_ent);
+    d.qp = (__nv_bfloat16*)(b + L.qp);
+    d.kp = (__nv_bfloat16*)(b + L.kp);
+    d.vp = (__nv_bfloat16*)(b + L.vp);
+    return d;
+}
+
+__device__ __forceinline__ void dev_fail(int* err, int code) { atomicCAS(err, 0, code); }
+
+// ---------------------------------------------------- block-wide reductions
+template <int NT_>
+__device__ __forceinline__ float block_sum(float v, float* red) {
+    // deterministic: warp xor tree, then warp partials summed in warp order
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float s = 0.f;
+    #pragma unroll
+    for (int i = 0; i < NT_ / 32; ++i) s += red[i];
+    return s;
+}
+template <int NT_>
+__device__ __forceinline__ int block_sum_int(int v, int* red) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    int s = 0;
+    #pragma unroll
+    for (int i = 0; i < NT_ / 32; ++i) s += red[i];
+    return s;
+}
+template <int NT_>
+__device__ __forceinline__ float block_max(float v, float* red) {
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float s = red[0];
+    #pragma unroll
+    for (int i = 1; i < NT_ / 32; ++i) s = fmaxf(s, red[i]);
+    return s;
+}
+
+// Block-wide exclusive scan of `n` ints in place (single CTA of 1024 threads);
+// a[n] receives the total.  Deterministic (integer).
+__device__ void block_exclusive_scan_inplace(int* a, int n, int* red) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int per = (n + nt - 1) / nt;
+    const int b0 = min(n, tid * per), b1 = min(n, b0 + per);
+    int s = 0;
+    for (int i = b0; i < b1; ++i) s += a[i];
+    // scan of per-thread sums over the block
+    __syncthreads();
+    red[tid] = s;
+    __syncthreads();
+    for (int o = 1; o < nt; o <<= 1) {
+        int v = tid >= o ? red[tid - o] : 0;
+        __syncthreads();
+        red[tid] += v;
+        __syncthreads();
+    }
+    int run = red[tid] - s;
+    for (int i = b0; i < b1; ++i) { int c = a[i]; a[i] = run; run += c; }
+    if (tid == nt - 1) a[n] = red[nt - 1];
+    __syncthreads();
+}
+
+// ================================================================ stage 1
+// Audio terms, head independent.  One CTA per zone; fp64 accumulation.
+__global__ void __launch_bounds__(256) k_audio_zone(DevPlan d, const float* __restrict__ amap) {
+    const int m = blockIdx.x;
+    const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
+    __shared__ double v[512];
+    __shared__ double sl[3][8];
+    for (int i = threadIdx.x; i < 512; i += 256) {
+        const int lt = i >> 6, lh = (i >> 3) & 7, lw = i & 7;
+        const int64_t n = ((int64_t)(8 * zt + lt) * d.H + 8 * zh + lh) * d.W + 8 * zw + lw;
+        v[i] = (double)amap[n];
+    }
+    __syncthreads();
+    if (threadIdx.x < 24) {
+        const int ax = threadIdx.x / 8, s = threadIdx.x % 8;
+        double acc = 0.0;
+        for (int a = 0; a < 8; ++a)
+            for (int b = 0; b < 8; ++b) {
+                int lt, lh, lw;
+                if (ax == 0) { lt = s; lh = a; lw = b; }
+                else if (ax == 1) { lt = a; lh = s; lw = b; }
+                else { lt = a; lh = b; lw = s; }
+                acc += v[(lt << 6) | (lh << 3) | lw];
+            }
+        sl[ax][s] = acc / 64.0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double mean = 0.0;
+        for (int s = 0; s < 8; ++s) mean += sl[0][s];
+        mean /= 8.0;
+        double sig[3], tot = 0.0;
+        for (int ax = 0; ax < 3; ++ax) {
+            double a = 0.0;
+            for (int s = 0; s < 8; ++s) { double e = sl[ax][s] - mean; a += e * e; }
+            sig[ax] = a / 8.0;
+            tot += sig[ax];
+        }
+        d.araw[m] = mean;
+        for (int ax = 0; ax < 3; ++ax) d.vhat[m * 3 + ax] = tot > 0.0 ? (float)(sig[ax] / tot) : 0.f;
+    }
+}
+
+__global__ void __launch_bounds__(1024) k_audio_norm(DevPlan d) {
+    __shared__ double red[32];
+    double mx = 0.0;
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) mx = fmax(mx, d.araw[m]);
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = red[0];
+    for (int i = 1; i < 32; ++i) mx = fmax(mx, red[i]);
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x)
+        d.abar[m] = mx > 0.0 ? (float)(d.araw[m] / mx) : 0.f;
+}
+
+__global__ void k_audio_none(DevPlan d) {
+    for (int m = blockIdx.x * blockDim.x + threadIdx.x; m < d.Nz; m += gridDim.x * blockDim.x) {
+        d.abar[m] = 0.f;
+        d.vhat[3 * m] = d.vhat[3 * m + 1] = d.vhat[3 * m + 2] = 0.f;
+    }
+}
+
+// Value statistics per (zone, head): sigma^2_{v,T/H/W} and the raw density.
+// Thread = (channel pair, group of h-rows of the zone); one pass over the zone
+// with the values shifted by the zone's first token (per channel).
+template <typename T>
+struct Pair { };
+template <>
+struct Pair<__nv_bfloat16> {
+    static __device__ __forceinline__ float2 load(const __nv_bfloat16* p) {
+        __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(p);
+        return __bfloat1622float2(v);
+    }
+};
+template <>
+struct Pair<float> {
+    static __device__ __forceinline__ float2 load(const float* p) {
+        return *reinterpret_cast<const float2*>(p);
+    }
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restrict__ V) {
+    constexpr int CP = D / 2;            // channel pairs
+    constexpr int G = 256 / CP;          // groups
+    constexpr int RPG = 8 / G;           // h-rows per group
+    constexpr int NV = 26;               // ST[8] SQ[8] SW[8] Dsum Dsq
+    extern __shared__ float zs_dyn[];    // [G][D][NV]
+    float (*red)[D][NV] = reinterpret_cast<float (*)[D][NV]>(zs_dyn);
+    __shared__ float shs[D][8];
+    __shared__ float cst[D][4];
+    const int m = blockIdx.x, h = blockIdx.y;
+    const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
+    const int cp = threadIdx.x % CP, grp = threadIdx.x / CP;
+    const T* Vh = V + (size_t)h * d.N * D;
+    auto tok = [&](int lt, int lh, int lw) -> int64_t {
+        return ((int64_t)(8 * zt + lt) * d.H + 8 * zh + lh) * d.W + 8 * zw + lw;
+    };
+    const float2 ref = Pair<T>::load(Vh + tok(0, 0, 0) * D + 2 * cp);
+    float ST[2][8], SQ[2][8], SW[2][8], SH[2][RPG], Ds[2], Dq[2];
+    #pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) ST[c][i] = SQ[c][i] = SW[c][i] = 0.f;
+        #pragma unroll
+        for (int i = 0; i < RPG; ++i) SH[c][i] = 0.f;
+        Ds[c] = Dq[c] = 0.f;
+    }
+    #pragma unroll
+    for (int rr = 0; rr < RPG; ++rr) {
+        const int lh = grp * RPG + rr;
+        float prev[2][8];
+        #pragma unroll
+        for (int lt = 0; lt < 8; ++lt) {
+            float2 x[8];
+            #pragma unroll
+            for (int lw = 0; lw < 8; ++lw) x[lw] = Pair<T>::load(Vh + tok(lt, lh, lw) * D + 2 * cp);
+            #pragma unroll
+            for (int lw = 0; lw < 8; ++lw) {
+                const float v0 = x[lw].x - ref.x, v1 = x[lw].y - ref.y;
+                ST[0][lt] += v0; ST[1][lt] += v1;
+                SQ[0][lt] += v0 * v0; SQ[1][lt] += v1 * v1;
+                SW[0][lw] += v0; SW[1][lw] += v1;
+                SH[0][rr] += v0; SH[1][rr] += v1;
+                if (lt > 0) {
+                    const float d0 = v0 - prev[0][lw], d1 = v1 - prev[1][lw];
+                    Ds[0] += d0; Ds[1] += d1;
+                    Dq[0] += d0 * d0; Dq[1] += d1 * d1;
+                }
+                prev[0][lw] = v0; prev[1][lw] = v1;
+            }
+        }
+    }
+    #pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        float* r = red[grp][2 * cp + c];
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) { r[i] = ST[c][i]; r[8 + i] = SQ[c][i]; r[16 + i] = SW[c][i]; }
+        r[24] = Ds[c]; r[25] = Dq[c];
+        #pragma unroll
+        for (int rr = 0; rr < RPG; ++rr) shs[2 * cp + c][grp * RPG + rr] = SH[c][rr];
+    }
+    __syncthreads();
+    if (threadIdx.x < D) {
+        const int c = threadIdx.x;
+        float st[8], sq[8], sw[8], ds = 0.f, dq = 0.f;
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) st[i] = sq[i] = sw[i] = 0.f;
+        for (int g = 0; g < G; ++g) {
+            const float* r = red[g][c];
+            #pragma unroll
+            for (int i = 0; i < 8; ++i) { st[i] += r[i]; sq[i] += r[8 + i]; sw[i] += r[16 + i]; }
+            ds += r[24]; dq += r[25];
+        }
+        float zsum = 0.f;
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) zsum += st[i];
+        const float mu = zsum / 512.f;
+        float vt = 0.f, vh = 0.f, vw = 0.f, sp = 0.f;
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float et = st[i] / 64.f - mu, eh = shs[c][i] / 64.f - mu, ew = sw[i] / 64.f - mu;
+            vt += et * et; vh += eh * eh; vw += ew * ew;
+            const float fm = st[i] / 64.f;
+            sp += sq[i] / 64.f - fm * fm;
+        }
+        const float dm = ds / 448.f;
+        const float temporal = dq / 448.f - dm * dm;
+        cst[c][0] = vt / 8.f; cst[c][1] = vh / 8.f; cst[c][2] = vw / 8.f;
+        cst[c][3] = sp / 8.f + temporal;
+    }
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        float s = 0.f;
+        for (int c = 0; c < D; ++c) s += cst[c][threadIdx.x];
+        d.zstat[((size_t)h * d.Nz + m) * 4 + threadIdx.x] = s / (float)D;
+    }
+}
+
+// Per head: rho normalisation, volume, closed form, snapping, block offsets.
+__device__ int snap_shape(const float g[3], int vol) {
+    const float lg0 = log2f(g[0]), lg1 = log2f(g[1]), lg2 = log2f(g[2]);
+    const float S = vol == 64 ? 6.f : (vol == 128 ? 7.f : 8.f);
+    float inner = __fadd_rn(S, __fmul_rn(0.5f, lg0));
+    inner = __fadd_rn(inner, __fmul_rn(0.5f, lg1));
+    inner = __fadd_rn(inner, __fmul_rn(0.5f, lg2));
+    const float third = __fdiv_rn(inner, 3.f);
+    const float e0 = __fadd_rn(__fmul_rn(-0.5f, lg0), third);
+    const float e1 = __fadd_rn(__fmul_rn(-0.5f, lg1), third);
+    const float e2 = __fadd_rn(__fmul_rn(-0.5f, lg2), third);
+    const int lo = vol == 64 ? 0 : (vol == 128 ? 7 : 13);
+    const int hi = vol == 64 ? 7 : (vol == 128 ? 13 : 16);
+    int best = lo;
+    float bd = 0.f;
+    for (int s = lo; s < hi; ++s) {
+        const float d0 = __fsub_rn((float)c_log2shape[s][0], e0);
+        const float d1 = __fsub_rn((float)c_log2shape[s][1], e1);
+        const float d2 = __fsub_rn((float)c_log2shape[s][2], e2);
+        float dist = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
+        dist = __fadd_rn(dist, __fmul_rn(d2, d2));
+        if (s == lo || dist < bd) { best = s; bd = dist; }
+    }
+    return best;
+}
+
+__global__ void __launch_bounds__(1024) k_zone_finalize(DevPlan d, float eps, float tau128,
+                                                        float tau256, int use_given_shapes) {
+    __shared__ float redf[32];
+    __shared__ int red[1024];
+    extern __shared__ int nbz[];   // [Nz + 1]
+    const int h = blockIdx.x;
+    const float* zs = d.zstat + (size_t)h * d.Nz * 4;
+    uint8_t* sid = d.shape_id + (size_t)h * d.Nz;
+    if (!use_given_shapes) {
+        float mx = 0.f;
+        for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) mx = fmaxf(mx, zs[m * 4 + 3]);
+        mx = block_max<1024>(mx, redf);
+        for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+            const float rho = mx > 0.f ? __fdiv_rn(zs[m * 4 + 3], mx) : 0.f;
+            const int vol = rho < tau256 ? 256 : (rho < tau128 ? 128 : 64);
+            const float s0 = zs[m * 4], s1 = zs[m * 4 + 1], s2 = zs[m * 4 + 2];
+            const float tot = __fadd_rn(__fadd_rn(s0, s1), s2);
+            float r[3];
+            if (tot > 0.f) { r[0] = __fdiv_rn(s0, tot); r[1] = __fdiv_rn(s1, tot); r[2] = __fdiv_rn(s2, tot); }
+            else { r[0] = r[1] = r[2] = 1.f / 3.f; }
+            const float ab = d.abar[m];
+            float g[3];
+            #pragma unroll
+            for (int ax = 0; ax < 3; ++ax)
+                g[ax] = __fadd_rn(__fadd_rn(r[ax], __fmul_rn(ab, d.vhat[3 * m + ax])), eps);
+            sid[m] = (uint8_t)snap_shape(g, vol);
+        }
+        __syncthreads();
+    }
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+        const int s = sid[m] < 16 ? sid[m] : 0;
+        if (sid[m] >= 16) dev_fail(d.err, PRISM_ERR_DEVICE_CHECK);
+        nbz[m] = 512 / (c_shape[s][0] * c_shape[s][1] * c_shape[s][2]);
+    }
+    __syncthreads();
+    block_exclusive_scan_inplace(nbz, d.Nz, red);
+    int* zoff = d.zone_off + (size_t)h * (d.Nz + 1);
+    int* bs = d.blk_start + (size_t)h * (d.NB + 1);
+    int* t64 = d.t64_blk + (size_t)h * d.NB;
+    for (int m = threadIdx.x; m <= d.Nz; m += blockDim.x) zoff[m] = nbz[m];
+    const int nb = nbz[d.Nz];
+    if (threadIdx.x == 0) d.nblocks[h] = nb;
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+        const int s = sid[m] < 16 ? sid[m] : 0;
+        const int vol = c_shape[s][0] * c_shape[s][1] * c_shape[s][2];
+        const int j0 = nbz[m], cnt = nbz[m + 1] - nbz[m];
+        for (int k = 0; k < cnt; ++k) {
+            const int st = 512 * m + k * vol;
+            bs[j0 + k] = st;
+            for (int u = 0; u < vol / 64; ++u) t64[st / 64 + u] = j0 + k;
+        }
+    }
+    for (int j = nb + threadIdx.x; j <= d.NB; j += blockDim.x) bs[j] = (int)d.N;
+}
+
+// ================================================================ stage 2
+__device__ __forceinline__ uint32_t pk2(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Gather one block: rows in block order into the bf16 copies, raster index of
+// each slot into src, and fp32 block means of Q and K (from the input values).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restrict__ Q,
+                                                     const T* __restrict__ K,
+                                                     const T* __restrict__ V) {
+    constexpr int EPC = 16 / sizeof(T);      // input elements per 16-byte chunk
+    constexpr int CPR = D / EPC;             // chunks per row
+    constexpr int RP = 256 / CPR;            // rows in flight
+    __shared__ float pq[RP][D], pk[RP][D];
+    const int j = blockIdx.x, h = blockIdx.y;
+    if (j >= d.nblocks[h]) return;
+    const int* bs = d.blk_start + (size_t)h * (d.NB + 1);
+    const int start = bs[j], vol = bs[j + 1] - start;
+    const int m = start >> 9;
+    const int s = d.shape_id[(size_t)h * d.Nz + m];
+    const int bt = c_shape[s][0], bh = c_shape[s][1], bw = c_shape[s][2];
+    const int kin = (start - 512 * m) / vol;
+    const int nkw = 8 / bw, nkh = 8 / bh;
+    const int kw = kin % nkw, kh = (kin / nkw) % nkh, kt = kin / (nkw * nkh);
+    const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
+    const int c = threadIdx.x % CPR, rl = threadIdx.x / CPR;
+    float aq[EPC], ak[EPC];
+    #pragma unroll
+    for (int e = 0; e < EPC; ++e) aq[e] = ak[e] = 0.f;
+    const size_t hoff = (size_t)h * d.N * D;
+    for (int r = rl; r < vol; r += RP) {
+        const int lw = r % bw, lh = (r / bw) % bh, lt = r / (bw * bh);
+        const int64_t n = ((int64_t)(8 * zt + kt * bt + lt) * d.H + 8 * zh + kh * bh + lh) * d.W +
+                          8 * zw + kw * bw + lw;
+        const size_t so = hoff + (size_t)n * D + (size_t)c * EPC;
+        const size_t dst = hoff + (size_t)(start + r) * D + (size_t)c * EPC;
+        if (c == 0) d.src[(size_t)h * d.N + start + r] = (int)n;
+        const uint4 q4 = *reinterpret_cast<const uint4*>(Q + so);
+        const uint4 k4 = *reinterpret_cast<const uint4*>(K + so);
+        const uint4 v4 = *reinterpret_cast<const uint4*>(V + so);
+        if constexpr (sizeof(T) == 2) {
+            *reinterpret_cast<uint4*>(d.qp + dst) = q4;
+            *reinterpret_cast<uint4*>(d.kp + dst) = k4;
+            *reinterpret_cast<uint4*>(d.vp + dst) = v4;
+            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&q4);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&k4);
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fq = __bfloat1622float2(q2[e]), fk = __bfloat1622float2(k2[e]);
+                aq[2 * e] += fq.x; aq[2 * e + 1] += fq.y;
+                ak[2 * e] += fk.x; ak[2 * e + 1] += fk.y;
+            }
+        } else {
+            const float* fq = reinterpret_cast<const float*>(&q4);
+            const float* fk = reinterpret_cast<const float*>(&k4);
+            const float* fv = reinterpret_cast<const float*>(&v4);
+            uint2 oq, ok, ov;
+            oq.x = pk2(fq[0], fq[1]); oq.y = pk2(fq[2], fq[3]);
+            ok.x = pk2(fk[0], fk[1]); ok.y = pk2(fk[2], fk[3]);
+            ov.x = pk2(fv[0], fv[1]); ov.y = pk2(fv[2], fv[3]);
+            *reinterpret_cast<uint2*>(d.qp + dst) = oq;
+            *reinterpret_cast<uint2*>(d.kp + dst) = ok;
+            *reinterpret_cast<uint2*>(d.vp + dst) = ov;
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) { aq[e] += fq[e]; ak[e] += fk[e]; }
+        }
+    }
+    #pragma unroll
+    for (int e = 0; e < EPC; ++e) { pq[rl][c * EPC + e] = aq[e]; pk[rl][c * EPC + e] = ak[e]; }
+    __syncthreads();
+    for (int ch = threadIdx.x; ch < 2 * D; ch += 256) {
+        const int cc = ch % D;
+        float s2 = 0.f;
+        if (ch < D) { for (int r = 0; r < RP; ++r) s2 += pq[r][cc]; }
+        else { for (int r = 0; r < RP; ++r) s2 += pk[r][cc]; }
+        float* out = (ch < D ? d.qbar : d.kbar) + ((size_t)h * d.NB + j) * D + cc;
+        *out = s2 / (float)vol;
+    }
+}
+
+// ================================================================ stage 3
+// One CTA per (query block, head): fp32 logits against every key block,
+// softmax, Top-k U Top-p count, and the selected set as a bitmap row.
+constexpr int SEL_THREADS = 512;
+
+__device__ __forceinline__ uint32_t fkey(float x) { return __float_as_uint(x); }
+
+template <int D>
+__global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, float top_p) {
+    extern __shared__ float prow[];                 // [NB] logits, then probabilities
+    __shared__ float redf[SEL_THREADS / 32];
+    __shared__ int redi[SEL_THREADS / 32];
+    __shared__ int tiecnt[48 * 1024 / 32 + 1];
+    const int i = blockIdx.x, h = blockIdx.y;
+    const int nb = d.nblocks[h];
+    int* rowcnt = d.row_ptr + (size_t)h * (d.NB + 1);
+    if (i >= nb) {
+        if (threadIdx.x == 0) rowcnt[i] = 0;
+        return;
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int PL = D / 32;
+    float q[PL];
+    const float* qb = d.qbar + ((size_t)h * d.NB + i) * D;
+    #pragma unroll
+    for (int e = 0; e < PL; ++e) q[e] = qb[lane + 32 * e];
+    const float* kb = d.kbar + (size_t)h * d.NB * D;
+    const float sq = sqrtf((float)D);
+    for (int j = warp; j < nb; j += SEL_THREADS / 32) {
+        const float* kr = kb + (size_t)j * D;
+        float a = 0.f;
+        #pragma unroll
+        for (int e = 0; e < PL; ++e) a = fmaf(q[e], kr[lane + 32 * e], a);
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) prow[j] = __fdiv_rn(a, sq);
+    }
+    __syncthreads();
+    float mx = -INFINITY;
+    for (int j = threadIdx.x; j < nb; j += SEL_THREADS) mx = fmaxf(mx, prow[j]);
+    mx = block_max<SEL_THREADS>(mx, redf);
+    float z = 0.f;
+    for (int j = threadIdx.x; j < nb; j += SEL_THREADS) {
+        const float e = expf(prow[j] - mx);
+        prow[j] = e;
+        z += e;
+    }
+    z = block_sum<SEL_THREADS>(z, redf);
+    for (int j = threadIdx.x; j < nb; j += SEL_THREADS) prow[j] = __fdiv_rn(prow[j], z);
+    __syncthreads();
+
+    // L = shortest prefix of (P desc, j asc) with mass >= p
+    const int K = min(top_k, nb);
+    int L;
+    if (top_p >= 1.f) L = nb;
+    else if (top_p <= 0.f) L = 0;
+    else {
+        float tot = 0.f;
+        for (int j = threadIdx.x; j < nb; j += SEL_THREADS) tot += prow[j];
+        tot = block_sum<SEL_THREADS>(tot, redf);
+        if (tot < top_p) L = nb;
+        else {
+            uint32_t lo = 0u, hi = 0x3F800001u;      // mass(P >= lo) >= p > mass(P >= hi)
+            while (hi - lo > 1u) {
+                const uint32_t mid = lo + ((hi - lo) >> 1);
+                float ms = 0.f;
+                for (int j = threadIdx.x; j < nb; j += SEL_THREADS)
+                    if (fkey(prow[j]) >= mid) ms += prow[j];
+                ms = block_sum<SEL_THREADS>(ms, redf);
+                if (ms >= top_p) lo = mid; else hi = mid;
+            }
+            float mg = 0.f;
+            int cg = 0, ct = 0;
+            for (int j = threadIdx.x; j < nb; j += SEL_THREADS) {
+                const uint32_t k = fkey(prow[j]);
+                if (k > lo) { mg += prow[j]; ++cg; }
+                else if (k == lo) ++ct;
+            }
+            mg = block_sum<SEL_THREADS>(mg, redf);
+            cg = block_sum_int<SEL_THREADS>(cg, redi);
+            ct = block_sum_int<SEL_THREADS>(ct, redi);
+            const float v = __uint_as_float(lo);
+            int c = 0;
+            float acc = mg;
+            while (c < ct && acc < top_p) { acc += v; ++c; }
+            if (c == 0) c = ct > 0 ? 1 : 0;    // the threshold element itself reached p
+            L = cg + c;
+        }
+    }
+    const int cnt = max(K, L);
+    // threshold of the first cnt elements of the order
+    uint32_t lo = 0u;
+    int cgt = 0;
+    if (cnt < nb) {
+        uint32_t hi = 0x3F800001u;                  // count(P >= lo) >= cnt > count(P >= hi)
+        while (hi - lo > 1u) {
+            const uint32_t mid = lo + ((hi - lo) >> 1);
+            int cc = 0;
+            for (int j = threadIdx.x; j < nb; j += SEL_THREADS) cc += fkey(prow[j]) >= mid;
+            cc = block_sum_int<SEL_THREADS>(cc, redi);
+            if (cc >= cnt) lo = mid; else hi = mid;
+        }
+        int cc = 0;
+        for (int j = threadIdx.x; j < nb; j += SEL_THREADS) cc += fkey(prow[j]) > lo;
+        cgt = block_sum_int<SEL_THREADS>(cc, redi);
+    }
+    const int need = cnt - cgt;                     // ties at the threshold, lowest j first
+    uint32_t* row = d.sel + ((size_t)h * d.NB + i) * d.WORDS;
+    const int nw = (nb + 31) / 32;
+    for (int w = threadIdx.x; w < nw; w += SEL_THREADS) {
+        uint32_t tb = 0u;
+        if (cnt < nb)
+            for (int b = 0; b < 32; ++b) {
+                const int j = 32 * w + b;
+                if (j < nb && fkey(prow[j]) == lo) tb |= 1u << b;
+            }
+        tiecnt[w] = __popc(tb);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int w = 0; w < nw; ++w) { const int t = tiecnt[w]; tiecnt[w] = run; run += t; }
+    }
+    __syncthreads();
+    for (int w = threadIdx.x; w < d.WORDS; w += SEL_THREADS) {
+        uint32_t bits = 0u;
+        if (w < nw) {
+            if (cnt >= nb) {
+                const int left = nb - 32 * w;
+                bits = left >= 32 ? 0xffffffffu : ((1u << left) - 1u);
+            } else {
+                int rank = tiecnt[w];
+                for (int b = 0; b < 32; ++b) {
+                    const int j = 32 * w + b;
+                    if (j >= nb) break;
+                    const uint32_t k = fkey(prow[j]);
+                    if (k > lo) bits |= 1u << b;
+                    else if (k == lo) { if (rank < need) bits |= 1u << b; ++rank; }
+                }
+            }
+        }
+        row[w] = bits;
+    }
+    if (threadIdx.x == 0) rowcnt[i] = cnt;
+}
+
+// Bitmap popcount per row (used for imported selections and for the transpose).
+__global__ void k_row_popc(const uint32_t* __restrict__ bits, int* __restrict__ cnt, const int* nblocks,
+                           int NB, int WORDS) {
+    const int h = blockIdx.y;
+    const int nb = nblocks[h];
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= NB) return;
+    int c = 0;
+    if (i < nb) {
+        const uint32_t* r = bits + ((size_t)h * NB + i) * WORDS;
+        const int nw = (nb + 31) / 32;
+        for (int w = 0; w < nw; ++w) {
+            uint32_t x = r[w];
+            if (w == nw - 1 && (nb & 31)) x &= (1u << (nb & 31)) - 1u;
+            c += __popc(x);
+        }
+    }
+    cnt[(size_t)h * (NB + 1) + i] = c;
+}
+
+// Clear bits beyond nblocks in an imported bitmap (rows and columns).
+__global__ void k_mask_bits(uint32_t* bits, const int* nblocks, int NB, int WORDS) {
+    const int h = blockIdx.y;
+    const int nb = nblocks[h];
+    const size_t n = (size_t)NB * WORDS;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+        const int i = (int)(e / WORDS), w = (int)(e % WORDS);
+        uint32_t x = bits[(size_t)h * n + e];
+        if (i >= nb || 32 * w >= nb) x = 0u;
+        else if (32 * w + 32 > nb) x &= (1u << (nb - 32 * w)) - 1u;
+        bits[(size_t)h * n + e] = x;
+    }
+}
+
+// 32x32 bit-tile transpose: selT[j][i] = sel[i][j].
+__global__ void k_transpose_bits(DevPlan d) {
+    const int tr = blockIdx.x, w = blockIdx.y, h = blockIdx.z;
+    const int lane = threadIdx.x;
+    const int i = 32 * tr + lane;
+    uint32_t x = 0u;
+    if (i < d.nblocks[h]) x = d.sel[((size_t)h * d.NB + i) * d.WORDS + w];
+    uint32_t mine = 0u;
+    #pragma unroll
+    for (int b = 0; b < 32; ++b) {
+        const uint32_t col = __ballot_sync(0xffffffffu, (x >> b) & 1u);
+        if (lane == b) mine = col;
+    }
+    const int j = 32 * w + lane;
+    if (j < d.NB && tr < d.WORDS) d.selT[((size_t)h * d.NB + j) * d.WORDS + tr] = mine;
+}
+
+// Exclusive scan of per-head count arrays [heads][n + 1] in place.
+__global__ void __launch_bounds__(1024) k_scan_heads(int* a, int n) {
+    __shared__ int red[1024];
+    block_exclusive_scan_inplace(a + (size_t)blockIdx.x * (n + 1), n, red);
+}
+
+// Bitmap rows -> ascending index lists (CSR from sel, CSC from selT).
+__global__ void k_fill_lists(const uint32_t* __restrict__ bits, const int* __restrict__ ptr,
+                             int* __restrict__ idx, const int* nblocks, int NB, int WORDS,
+                             int* err) {
+    const int i = blockIdx.x, h = blockIdx.y;
+    const int nb = nblocks[h];
+    if (i >= nb) return;
+    const int lane = threadIdx.x;
+    const uint32_t* r = bits + ((size_t)h * NB + i) * WORDS;
+    const int* p = ptr + (size_t)h * (NB + 1);
+    int* out = idx + (size_t)h * NB * NB;
+    int base = p[i];
+    const int end = p[i + 1];
+    const int nw = (nb + 31) / 32;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t x = w < nw ? r[w] : 0u;
+        if (w == nw - 1 && (nb & 31)) x &= (1u << (nb & 31)) - 1u;
+        const int pc = __popc(x);
+        int incl = pc;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int pos = base + incl - pc;
+        while (x) {
+            const int b = __ffs(x) - 1;
+            x &= x - 1u;
+            if (pos < end) out[pos] = 32 * w + b;
+            else dev_fail(err, PRISM_ERR_DEVICE_CHECK);
+            ++pos;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
+// Tile lists for the attention kernels.  A 128-token tile holds one block
+// part (volume 128/256) or two 64-token blocks; entry = (other tile << 4) | mask
+// with mask bit (qhalf * 2 + khalf) set when query half qhalf of the pair
+// attends to key half khalf.  Forward: per query tile, over key tiles (from
+// sel); backward: per key tile, over query tiles (from selT, same bit order).
+__device__ __forceinline__ int bit_of(const uint32_t* rowbits, int j) {
+    return (rowbits[j >> 5] >> (j & 31)) & 1u;
+}
+
+template <bool FILL>
+__global__ void __launch_bounds__(256) k_tile_lists(const uint32_t* __restrict__ bits,
+                                                    const int* __restrict__ t64, int* ptr,
+                                                    int* ent, int NB, int NT, int WORDS,
+                                                    int transposed, int* err) {
+    __shared__ int red[256];
+    const int t = blockIdx.x, h = blockIdx.y;
+    const int* tb = t64 + (size_t)h * NB;
+    const uint32_t* b = bits + (size_t)h * NB * WORDS;
+    // own halves: blocks of the two 64-token halves of tile t
+    const int a0 = tb[2 * t], a1 = tb[2 * t + 1];
+    const uint32_t* r0 = b + (size_t)a0 * WORDS;
+    const uint32_t* r1 = b + (size_t)a1 * WORDS;
+    const int per = (NT + 255) / 256;
+    const int c0 = min(NT, (int)threadIdx.x * per), c1 = min(NT, c0 + per);
+    auto mask_of = [&](int o) -> int {
+        const int o0 = tb[2 * o], o1 = tb[2 * o + 1];
+        // own half x (row bits rx) against other half y (block oy)
+        const int m00 = bit_of(r0, o0), m01 = bit_of(r0, o1);
+        const int m10 = bit_of(r1, o0), m11 = bit_of(r1, o1);
+        // forward: own = query halves, other = key halves: bit (q*2 + k)
+        // backward: own = key halves, other = query halves: bit (q*2 + k) = (other*2 + own)
+        if (!transposed) return m00 | (m01 << 1) | (m10 << 2) | (m11 << 3);
+        return m00 | (m10 << 1) | (m01 << 2) | (m11 << 3);
+    };
+    int cnt = 0;
+    for (int o = c0; o < c1; ++o) cnt += mask_of(o) != 0;
+    int* p = ptr + (size_t)h * (NT + 1);
+    if (!FILL) {
+        const int tot = block_sum_int<256>(cnt, red);
+        if (threadIdx.x == 0) p[t] = tot;
+        return;
+    }
+    __syncthreads();
+    red[threadIdx.x] = cnt;
+    __syncthreads();
+    for (int o = 1; o < 256; o <<= 1) {
+        const int v = threadIdx.x >= o ? red[threadIdx.x - o] : 0;
+        __syncthreads();
+        red[threadIdx.x] += v;
+        __syncthreads();
+    }
+    int pos = p[t] + red[threadIdx.x] - cnt;
+    const int end = p[t + 1];
+    int* e = ent + (size_t)h * NT * NT;
+    for (int o = c0; o < c1; ++o) {
+        const int mk = mask_of(o);
+        if (mk) {
+            if (pos < end) e[pos] = (o << 4) | mk;
+            else dev_fail(err, PRISM_ERR_DEVICE_CHECK);
+            ++pos;
+        }
+    }
+}
+
+// ------------------------------------------------------------- host helpers
+static int cuda_status(cudaError_t e) { return e == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA; }
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+static int make_tmap(CUtensorMap* m, void* base, int64_t rows, int D) {
+    auto enc = get_encode();
+    if (!enc) return PRISM_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+static int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_UNSUPPORTED;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return PRISM_ERR_UNSUPPORTED;
+    return PRISM_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int plan_common(const prism_params* p, const void* Q, const void* K, const void* V,
+                       void* workspace, size_t ws_bytes, prism_plan_s** outP) {
+    int st = validate_params(p);
+    if (st) return st;
+    if (!Q || !K || !V || !workspace) return PRISM_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V)) return PRISM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PRISM_ERR_INVALID_ARG;
+    st = check_device();
+    if (st) return st;
+    Geom g = make_geom(p);
+    Layout L = make_layout(g);
+    if (ws_bytes < L.total) return PRISM_ERR_WORKSPACE;
+    prism_plan_s* P = new (std::nothrow) prism_plan_s();
+    if (!P) return PRISM_ERR_CUDA;
+    P->p = *p;
+    P->g = g;
+    P->L = L;
+    P->ws = static_cast<char*>(workspace);
+    P->ws_bytes = ws_bytes;
+    cudaGetDevice(&P->device);
+    const int64_t rows = (int64_t)g.heads * g.N;
+    st = make_tmap(&P->tm_q, P->ws + L.qp, rows, g.D);
+    if (!st) st = make_tmap(&P->tm_k, P->ws + L.kp, rows, g.D);
+    if (!st) st = make_tmap(&P->tm_v, P->ws + L.vp, rows, g.D);
+    if (!st) st = make_tmap(&P->tm_do, P->ws + L.dop, rows, g.D);
+    if (st) { delete P; return st; }
+    *outP = P;
+    return PRISM_OK;
+}
+
+template <typename T, int D>
+static void launch_stats(prism_plan_s* P, const DevPlan& d, const void* V, cudaStream_t s) {
+    const Geom& g = P->g;
+    const int sm = (256 / (D / 2)) * D * 26 * (int)sizeof(float);
+    cudaFuncSetAttribute(k_zone_stats<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    k_zone_stats<T, D><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V);
+}
+
+template <typename T, int D>
+static void launch_gather(prism_plan_s* P, const DevPlan& d, const void* Q, const void* K,
+                          const void* V, cudaStream_t s) {
+    const Geom& g = P->g;
+    k_gather_pool<T, D><<<dim3(g.NB, g.heads), 256, 0, s>>>(d, (const T*)Q, (const T*)K, (const T*)V);
+}
+
+static void launch_lists(prism_plan_s* P, const DevPlan& d, cudaStream_t s) {
+    const Geom& g = P->g;
+    // CSR from sel (row counts already in row_ptr[0..NB))
+    k_scan_heads<<<g.heads, 1024, 0, s>>>(d.row_ptr, g.NB);
+    k_fill_lists<<<dim3(g.NB, g.heads), 32, 0, s>>>(d.sel, d.row_ptr, d.col_idx, d.nblocks, g.NB, g.WORDS, d.err);
+    // transpose and CSC
+    k_transpose_bits<<<dim3(g.WORDS, g.WORDS, g.heads), 32, 0, s>>>(d);
+    k_row_popc<<<dim3((g.NB + 255) / 256, g.heads), 256, 0, s>>>(d.selT, d.col_ptr, d.nblocks, g.NB, g.WORDS);
+    k_scan_heads<<<g.heads, 1024, 0, s>>>(d.col_ptr, g.NB);
+    k_fill_lists<<<dim3(g.NB, g.heads), 32, 0, s>>>(d.selT, d.col_ptr, d.row_idx, d.nblocks, g.NB, g.WORDS, d.err);
+    // tile lists (forward from sel, backward from selT)
+    k_tile_lists<false><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.sel, d.t64_blk, d.qt_ptr, d.qt_ent, g.NB, g.NT, g.WORDS, 0, d.err);
+    k_scan_heads<<<g.heads, 1024, 0, s>>>(d.qt_ptr, g.NT);
+    k_tile_lists<true><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.sel, d.t64_blk, d.qt_ptr, d.qt_ent, g.NB, g.NT, g.WORDS, 0, d.err);
+    k_tile_lists<false><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.selT, d.t64_blk, d.kt_ptr, d.kt_ent, g.NB, g.NT, g.WORDS, 1, d.err);
+    k_scan_heads<<<g.heads, 1024, 0, s>>>(d.kt_ptr, g.NT);
+    k_tile_lists<true><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.selT, d.t64_blk, d.kt_ptr, d.kt_ent, g.NB, g.NT, g.WORDS, 1, d.err);
+}
+
+static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V, const float* amap,
+                    const uint8_t* given_shapes, const uint32_t* given_sel, cudaStream_t s) {
+    const Geom& g = P->g;
+    const prism_params& p = P->p;
+    DevPlan d = dev_plan(P);
+    cudaMemsetAsync(P->ws + P->L.err, 0, 16, s);
+    const bool bf = p.dtype == PRISM_BF16;
+    if (!given_shapes) {
+        if (amap) {
+            k_audio_zone<<<g.Nz, 256, 0, s>>>(d, amap);
+            k_audio_norm<<<1, 1024, 0, s>>>(d);
+        } else {
+            k_audio_none<<<(g.Nz + 255) / 256, 256, 0, s>>>(d);
+        }
+        if (bf && g.D == 128) launch_stats<__nv_bfloat16, 128>(P, d, V, s);
+        else if (bf) launch_stats<__nv_bfloat16, 64>(P, d, V, s);
+        else if (g.D == 128) launch_stats<float, 128>(P, d, V, s);
+        else launch_stats<float, 64>(P, d, V, s);
+    } else {
+        cudaMemcpyAsync(d.shape_id, given_shapes, (size_t)g.heads * g.Nz, cudaMemcpyDeviceToDevice, s);
+    }
+    const size_t fin_smem = sizeof(int) * (g.Nz + 1);
+    if (fin_smem > 48 * 1024)
+        cudaFuncSetAttribute(k_zone_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
+    k_zone_finalize<<<g.heads, 1024, fin_smem, s>>>(d, p.eps, p.tau128, p.tau256, given_shapes ? 1 : 0);
+    if (bf && g.D == 128) launch_gather<__nv_bfloat16, 128>(P, d, Q, K, V, s);
+    else if (bf) launch_gather<__nv_bfloat16, 64>(P, d, Q, K, V, s);
+    else if (g.D == 128) launch_gather<float, 128>(P, d, Q, K, V, s);
+    else launch_gather<float, 64>(P, d, Q, K, V, s);
+    if (!given_sel) {
+        const size_t sm = sizeof(float) * g.NB;
+        if (g.D == 128) {
+            cudaFuncSetAttribute(k_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            k_select<128><<<dim3(g.NB, g.heads), SEL_THREADS, sm, s>>>(d, p.top_k, p.top_p);
+        } else {
+            cudaFuncSetAttribute(k_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            k_select<64><<<dim3(g.NB, g.heads), SEL_THREADS, sm, s>>>(d, p.top_k, p.top_p);
+        }
+    } else {
+        cudaMemcpyAsync(d.sel, given_sel, sizeof(uint32_t) * (size_t)g.heads * g.NB * g.WORDS,
+                        cudaMemcpyDeviceToDevice, s);
+        k_mask_bits<<<dim3(256, g.heads), 256, 0, s>>>(d.sel, d.nblocks, g.NB, g.WORDS);
+        k_row_popc<<<dim3((g.NB + 255) / 256, g.heads), 256, 0, s>>>(d.sel, d.row_ptr, d.nblocks, g.NB, g.WORDS);
+    }
+    launch_lists(P, d, s);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace prism
+
+using namespace prism;
+
+// ================================================================== C ABI
+extern "C" size_t prism_plan_workspace_bytes(const prism_params* p) {
+    if (validate_params(p) != PRISM_OK) return 0;
+    return make_layout(make_geom(p)).total;
+}
+
+extern "C" int prism_plan(const prism_params* p, const void* Q, const void* K, const void* V,
+                          const float* a_map, void* workspace, size_t ws_bytes, void* stream,
+                          prism_plan_t* out) {
+    if (!out) return PRISM_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (a_map && !aligned16(a_map)) return PRISM_ERR_INVALID_ARG;
+    prism_plan_s* P = nullptr;
+    int st = plan_common(p, Q, K, V, workspace, ws_bytes, &P);
+    if (st) return st;
+    P->has_audio = a_map != nullptr;
+    st = run_plan(P, Q, K, V, a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+    if (st) { delete P; return st; }
+    *out = P;
+    return PRISM_OK;
+}
+
+extern "C" int prism_plan_import(const prism_params* p, const void* Q, const void* K, const void* V,
+                                 const uint8_t* shape_id, const uint32_t* sel, void* workspace,
+                                 size_t ws_bytes, void* stream, prism_plan_t* out) {
+    if (!out) return PRISM_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!shape_id || !sel || !aligned16(sel)) return PRISM_ERR_INVALID_ARG;
+    prism_plan_s* P = nullptr;
+    int st = plan_common(p, Q, K, V, workspace, ws_bytes, &P);
+    if (st) return st;
+    P->has_audio = 0;
+    st = run_plan(P, Q, K, V, nullptr, shape_id, sel, static_cast<cudaStream_t>(stream));
+    if (st) { delete P; return st; }
+    *out = P;
+    return PRISM_OK;
+}
+
+extern "C" size_t prism_plan_item_bytes(prism_plan_t P, int item) {
+    if (!P) return 0;
+    const Geom& g = P->g;
+    const size_t H = g.heads, NB = g.NB;
+    switch (item) {
+        case PRISM_ITEM_SHAPE_ID: return H * g.Nz;
+        case PRISM_ITEM_NBLOCKS: return 4 * H;
+        case PRISM_ITEM_BLK_START: return 4 * H * (NB + 1);
+        case PRISM_ITEM_SEL_BITS: return 4 * H * NB * g.WORDS;
+        case PRISM_ITEM_ROW_PTR: return 4 * H * (NB + 1);
+        case PRISM_ITEM_COL_IDX: return 4 * H * NB * NB;
+        case PRISM_ITEM_COL_PTR: return 4 * H * (NB + 1);
+        case PRISM_ITEM_ROW_IDX: return 4 * H * NB * NB;
+        case PRISM_ITEM_QBAR: return 4 * H * NB * g.D;
+        case PRISM_ITEM_KBAR: return 4 * H * NB * g.D;
+        case PRISM_ITEM_SRC: return 4 * H * (size_t)g.N;
+        case PRISM_ITEM_ZONE_STATS: return 4 * H * g.Nz * 4;
+        default: return 0;
+    }
+}
+
+extern "C" int prism_plan_export(prism_plan_t P, int item, void* host_dst, size_t bytes, void* stream) {
+    if (!P || !host_dst) return PRISM_ERR_INVALID_ARG;
+    const size_t need = prism_plan_item_bytes(P, item);
+    if (need == 0 || bytes != need) return PRISM_ERR_INVALID_ARG;
+    const Layout& L = P->L;
+    size_t off;
+    switch (item) {
+        case PRISM_ITEM_SHAPE_ID: off = L.shape_id; break;
+        case PRISM_ITEM_NBLOCKS: off = L.nblocks; break;
+        case PRISM_ITEM_BLK_START: off = L.blk_start; break;
+        case PRISM_ITEM_SEL_BITS: off = L.sel; break;
+        case PRISM_ITEM_ROW_PTR: off = L.row_ptr; break;
+        case PRISM_ITEM_COL_IDX: off = L.col_idx; break;
+        case PRISM_ITEM_COL_PTR: off = L.col_ptr; break;
+        case PRISM_ITEM_ROW_IDX: off = L.row_idx; break;
+        case PRISM_ITEM_QBAR: off = L.qbar; break;
+        case PRISM_ITEM_KBAR: off = L.kbar; break;
+        case PRISM_ITEM_SRC: off = L.src; break;
+        case PRISM_ITEM_ZONE_STATS: off = L.zstat; break;
+        default: return PRISM_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
+    if (cudaMemcpy(host_dst, P->ws + off, bytes, cudaMemcpyDeviceToHost) != cudaSuccess) return PRISM_ERR_CUDA;
+    return PRISM_OK;
+}
+
+extern "C" int prism_get_status(prism_plan_t P, void* stream) {
+    if (!P) return PRISM_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
+    int e = 0;
+    if (cudaMemcpy(&e, P->ws + P->L.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PRISM_ERR_CUDA;
+    if (e) {
+        const int zero = 0;
+        cudaMemcpy(P->ws + P->L.err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    }
+    return e;
+}
+
+extern "C" void prism_plan_destroy(prism_plan_t P) { delete P; }
+
+extern "C" const char* prism_status_string(int st) {
+    switch (st) {
+        case PRISM_OK: return "ok";
+        case PRISM_ERR_INVALID_ARG: return "invalid argument";
+        case PRISM_ERR_WORKSPACE: return "workspace too small";
+        case PRISM_ERR_CUDA: return "CUDA error";
+        case PRISM_ERR_TIMEOUT: return "device wait timed out";
+        case PRISM_ERR_DEVICE_CHECK: return "device-side check failed";
+        case PRISM_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
+        default: return "unknown status";
+    }
+}
+
+extern "C" const char* prism_version(void) { return "prism-b200 0.1 sm_100a"; }
+
+extern "C" int prism_attn_fwd(prism_plan_t P, void* O, float* lse, void* stream) {
+    if (!P || !O || !lse) return PRISM_ERR_INVALID_ARG;
+    if (!aligned16(O) || !aligned16(lse)) return PRISM_ERR_INVALID_ARG;
+    return prism_launch_attn_fwd(P, O, lse, stream);
+}
+
+extern "C" int prism_attn_bwd(prism_plan_t P, const void* dO, const void* O, const float* lse,
+                              void* dQ, void* dK, void* dV, void* stream) {
+    if (!P || !dO || !O || !lse || !dQ || !dK || !dV) return PRISM_ERR_INVALID_ARG;
+    if (!aligned16(dO) || !aligned16(O) || !aligned16(lse) || !aligned16(dQ) || !aligned16(dK) ||
+        !aligned16(dV))
+        return PRISM_ERR_INVALID_ARG;
+    return prism_launch_attn_bwd(P, dO, O, lse, dQ, dK, dV, stream);
+}

@@ -1,0 +1,200 @@
+/*
+ * prism.h -- C ABI of libprism, a B200 (sm_100a) implementation of Prism's
+ * dynamic block-sparse video self-attention.
+ *
+ * Method: "Prism: Dynamic Sparse Attention for Native 2K Joint Video-Audio
+ * Generation Model Training" (arXiv 2610.05416).  The equations are those of
+ * the page xyznot.com/id/paper/2610.05416, section "Metode" 1-3; the five
+ * stages and the hyperparameters are those of the page
+ * paper.rainbus.top/paper/2610.05416, section "方法步骤详情" (Algorithm 1).
+ *
+ * Call sequence for one layer:
+ *   prism_plan()      stage 1 (zone statistics, volume, shape), stage 2 (token
+ *                     reorder), stage 3 (block pooling, scores, Top-k U Top-p)
+ *   prism_attn_fwd()  stages 4-5 (sparse attention, inverse permutation)
+ *   prism_attn_bwd()  gradients through stage 4 only (the plan is detached)
+ *
+ * Conventions
+ *   - Every call is asynchronous on the caller's CUDA stream (passed as
+ *     `void*`, i.e. a cudaStream_t; NULL = legacy default stream) and returns
+ *     an int status (PRISM_OK or a PRISM_ERR_* code).  No call aborts the
+ *     process.  Only prism_get_status() and prism_plan_export() synchronise,
+ *     and only the given stream.
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory.  The caller allocates the plan
+ *     workspace (size from prism_plan_workspace_bytes) and keeps it, and the
+ *     Q, K, V tensors, alive until prism_plan_destroy().
+ *   - Token order: raster n = (t*H + h)*W + w over the latent T x H x W grid.
+ *     Q, K, V, O, dO, dQ, dK, dV are [heads][N][head_dim] row-major in that
+ *     order, of the element type `dtype` (bf16, or fp32 for the small fp32
+ *     workload).  LSE is [heads][N] fp32 (natural log), same order.
+ *   - Pointers must be 16-byte aligned.
+ */
+#ifndef PRISM_H
+#define PRISM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PRISM_API __attribute__((visibility("default")))
+#else
+#define PRISM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define PRISM_OK               0
+#define PRISM_ERR_INVALID_ARG  1  /* bad grid / head_dim / k,p / null pointer / misaligned */
+#define PRISM_ERR_WORKSPACE    2  /* workspace smaller than prism_plan_workspace_bytes() */
+#define PRISM_ERR_CUDA         3  /* a CUDA runtime or driver call failed */
+#define PRISM_ERR_TIMEOUT      4  /* a bounded device-side wait gave up; kernel returned */
+#define PRISM_ERR_DEVICE_CHECK 5  /* a device-side bounds/consistency check failed */
+#define PRISM_ERR_UNSUPPORTED  6  /* no sm_100 device, or the build lacks the kernels */
+
+/* Element type of Q, K, V, dO and of the outputs O, dQ, dK, dV. */
+#define PRISM_BF16 0
+#define PRISM_F32  1
+
+/*
+ * Problem description.
+ *   T, H, W   latent grid, each a positive multiple of the macro-zone edge 8
+ *             (zones are 8 x 8 x 8: page xyznot.com/id, section "Ide utama").
+ *   heads     number of heads in this call (>= 1).
+ *   head_dim  D, 64 or 128.
+ *   dtype     PRISM_BF16 or PRISM_F32.  fp32 inputs feed the statistics and
+ *             the pooled means in fp32; attention runs on their bf16 rounding
+ *             (round to nearest even).
+ *   top_k     k of Top-k (>= 0); k >= number of blocks keeps every block.
+ *   top_p     p of Top-p in [0, 1]; p >= 1 keeps every block, p <= 0 none.
+ *             top_k < 1 together with top_p <= 0 is rejected (empty sets).
+ *   eps       epsilon of g_d = r_{v,d} + a_bar * v_hat_{a,d} + eps.
+ *   tau128, tau256   density thresholds (the pages use 0.5 and 0.25).
+ */
+typedef struct prism_params {
+    int32_t T, H, W;
+    int32_t heads;
+    int32_t head_dim;
+    int32_t dtype;
+    int32_t top_k;
+    float   top_p;
+    float   eps;
+    float   tau128;
+    float   tau256;
+} prism_params;
+
+/* Opaque host-side handle: a small host struct pointing into the workspace. */
+typedef struct prism_plan_s* prism_plan_t;
+
+/*
+ * Bytes of device workspace prism_plan() needs for `p` (an upper bound: the
+ * block count and the number of selected pairs are data dependent; the bound
+ * assumes N/64 blocks per head and every pair selected).  Returns 0 when `p`
+ * is invalid.
+ */
+PRISM_API size_t prism_plan_workspace_bytes(const prism_params* p);
+
+/*
+ * prism_plan -- stages 1-3 of Algorithm 1 for every head.
+ *   Stage 1 (page paper.rainbus.top, section "方法步骤详情"; equations of page
+ *   xyznot.com/id, section "Metode" 1-2): per 8x8x8 zone and head, the
+ *   directional value variances sigma^2_{v,d} of the mean-pooled V profiles,
+ *   r_{v,d}, the audio coupling a_bar and v_hat_{a,d} from a_map, g_d, the
+ *   density rho -> volume B in {64,128,256} (thresholds tau256, tau128), the
+ *   closed form l*_d = -1/2 log2 g_d + 1/3 (log2 B + 1/2 sum log2 g) snapped to
+ *   the nearest of the 16 candidate shapes.
+ *   Stage 2: reorder tokens so every block is contiguous (bf16 copies of Q,
+ *   K, V in block order, kept in the workspace).
+ *   Stage 3 ("Metode" 3): block means Qbar, Kbar; P_i = softmax(Qbar_i Kbar^T
+ *   / sqrt(D)); S_i = Top-k(P_i, k) U Top-p(P_i, p) as per-query-block CSR
+ *   key-block lists and their transpose.
+ * Arguments
+ *   Q, K, V    device, [heads][N][head_dim] of `dtype`, raster order.
+ *   a_map      device fp32 [T][H][W], the cached audio-to-video cross-attention
+ *              output norm of the previous layer, shared by all heads; NULL for
+ *              the first layer (then g_d = r_{v,d} + eps).
+ *   workspace  device, >= prism_plan_workspace_bytes(p) bytes, 256-B aligned.
+ *   stream     cudaStream_t.
+ *   out        receives the plan handle (host memory, freed by
+ *              prism_plan_destroy).  Left NULL on error.
+ */
+PRISM_API int prism_plan(const prism_params* p, const void* Q, const void* K, const void* V,
+               const float* a_map, void* workspace, size_t ws_bytes, void* stream,
+               prism_plan_t* out);
+
+/*
+ * prism_plan_import -- the same plan, but with stage 1's shapes and stage 3's
+ * selection supplied by the caller instead of computed (a fixed-shape
+ * comparator, a cached plan, or a plan computed elsewhere).  Runs stage 2
+ * (reorder) and the pooling of stage 3, then builds the CSR lists from `sel`.
+ *   shape_id  device uint8 [heads][Nz], values 0..15 (the candidate order: by
+ *             volume 64, 128, 256, then lexicographic (b_T, b_H, b_W)).
+ *   sel       device uint32 bitmap [heads][N/64][ceil((N/64)/32)]: bit j of
+ *             row i set <=> key block j is in S_i; rows and bits beyond the
+ *             head's block count are ignored.
+ */
+PRISM_API int prism_plan_import(const prism_params* p, const void* Q, const void* K, const void* V,
+                      const uint8_t* shape_id, const uint32_t* sel,
+                      void* workspace, size_t ws_bytes, void* stream, prism_plan_t* out);
+
+/*
+ * prism_attn_fwd -- stages 4-5: for every query token q of block i,
+ *   O_q = softmax_n(q . k_n / sqrt(D)) v_n over the tokens n of the key
+ *   blocks in S_i (fp32 online softmax, bf16 tensor-core products), written
+ *   back in raster order (inverse permutation).
+ *   O    device [heads][N][head_dim] of `dtype`.
+ *   lse  device fp32 [heads][N], log-sum-exp of the scaled logits, raster order.
+ */
+PRISM_API int prism_attn_fwd(prism_plan_t plan, void* O, float* lse, void* stream);
+
+/*
+ * prism_attn_bwd -- exact gradients of prism_attn_fwd with the plan fixed (the
+ *   statistics, shapes and selection are detached: page xyznot.com/th, section
+ *   on training).  dO, O, lse as produced/consumed by prism_attn_fwd.
+ *   dQ, dK, dV device [heads][N][head_dim] of `dtype`, raster order.
+ */
+PRISM_API int prism_attn_bwd(prism_plan_t plan, const void* dO, const void* O, const float* lse,
+                   void* dQ, void* dK, void* dV, void* stream);
+
+/* ---- inspection -------------------------------------------------------- */
+#define PRISM_ITEM_SHAPE_ID   0  /* uint8  [heads][Nz]                         */
+#define PRISM_ITEM_NBLOCKS    1  /* int32  [heads]                             */
+#define PRISM_ITEM_BLK_START  2  /* int32  [heads][N/64 + 1] (first nblocks+1)  */
+#define PRISM_ITEM_SEL_BITS   3  /* uint32 [heads][N/64][ceil(N/64 / 32)]       */
+#define PRISM_ITEM_ROW_PTR    4  /* int32  [heads][N/64 + 1]  CSR              */
+#define PRISM_ITEM_COL_IDX    5  /* int32  [heads][(N/64)^2]  CSR (row_ptr'd)  */
+#define PRISM_ITEM_COL_PTR    6  /* int32  [heads][N/64 + 1]  CSC              */
+#define PRISM_ITEM_ROW_IDX    7  /* int32  [heads][(N/64)^2]  CSC              */
+#define PRISM_ITEM_QBAR       8  /* fp32   [heads][N/64][head_dim]             */
+#define PRISM_ITEM_KBAR       9  /* fp32   [heads][N/64][head_dim]             */
+#define PRISM_ITEM_SRC       10  /* int32  [heads][N] raster token of each permuted slot */
+#define PRISM_ITEM_ZONE_STATS 11 /* fp32   [heads][Nz][4] sigma2_T, sigma2_H, sigma2_W, rho_raw */
+#define PRISM_ITEM_COUNT     12
+
+/* Bytes of an item (0 for an unknown item). */
+PRISM_API size_t prism_plan_item_bytes(prism_plan_t plan, int item);
+
+/* Synchronises `stream` and copies an item into host memory (bytes must equal
+ * prism_plan_item_bytes). */
+PRISM_API int prism_plan_export(prism_plan_t plan, int item, void* host_dst, size_t bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the plan's device error word:
+ * PRISM_OK, PRISM_ERR_TIMEOUT or PRISM_ERR_DEVICE_CHECK (or PRISM_ERR_CUDA). */
+PRISM_API int prism_get_status(prism_plan_t plan, void* stream);
+
+/* Frees the host handle (the workspace stays the caller's). */
+PRISM_API void prism_plan_destroy(prism_plan_t plan);
+
+/* Static description of a status code. */
+PRISM_API const char* prism_status_string(int status);
+
+/* Library version, e.g. "prism-b200 0.1 sm_100a". */
+PRISM_API const char* prism_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PRISM_H */

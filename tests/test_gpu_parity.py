@@ -1,0 +1,167 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Small grids that the oracle finishes in seconds but that still span several
+zones, 128-token tiles and block volumes; plus the degenerate cases (every
+block selected, a single block selected, one zone, no audio map).
+"""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from dynamic_block_sparse_indicator_b200 import _lib
+from dynamic_block_sparse_indicator_b200 import synthetic as syn
+from oracle import prism_oracle as po
+
+pytestmark = pytest.mark.gpu
+
+
+def _dtype_code(w):
+    return _lib.PRISM_F32 if w.dtype == "f32" else _lib.PRISM_BF16
+
+
+def _inputs(w, heads, with_audio=True):
+    Q, K, V = syn.make_qkv(w, heads=heads)
+    a = syn.make_amap(w) if with_audio else None
+    return Q, K, V, a
+
+
+def _to_dev(*xs):
+    return [None if x is None else x.cuda() for x in xs]
+
+
+def _params(w, heads):
+    return _lib.make_params(w.T, w.H, w.W, heads, w.head_dim, _dtype_code(w), w.top_k, w.top_p,
+                            w.eps)
+
+
+def _oracle_plans(w, Q, K, V, a, heads):
+    an = None if a is None else a.numpy()
+    return [po.plan_head(Q[h].double().numpy(), K[h].double().numpy(), V[h].double().numpy(), an,
+                         w.T, w.H, w.W, w.top_k, w.top_p, w.eps) for h in range(heads)]
+
+
+def _check_plan(pl, orc, w, heads):
+    """Stage-wise comparison; returns per head the set of query blocks whose
+    selection equals the oracle's exactly (None when the shapes differ)."""
+    NB, WORDS, Nz, N = w.N // 64, (w.N // 64 + 31) // 32, w.zones, w.N
+    sid = pl.export("shape_id").reshape(heads, Nz)
+    nblocks = pl.export("nblocks")
+    bstart = pl.export("blk_start").reshape(heads, NB + 1)
+    src = pl.export("src").reshape(heads, N)
+    qbar = pl.export("qbar").reshape(heads, NB, w.head_dim)
+    kbar = pl.export("kbar").reshape(heads, NB, w.head_dim)
+    bits = pl.export("sel_bits").reshape(heads, NB, WORDS)
+    row_ptr = pl.export("row_ptr").reshape(heads, NB + 1)
+    col_idx = pl.export("col_idx").reshape(heads, NB * NB)
+    col_ptr = pl.export("col_ptr").reshape(heads, NB + 1)
+    row_idx = pl.export("row_idx").reshape(heads, NB * NB)
+    exact_rows = []
+    for h in range(heads):
+        o = orc[h]
+        ok, tie, bad = parity.shapes_agree(sid[h], o["stats"])
+        assert not bad, f"head {h}: shape mismatch outside the tie margin in zones {bad}"
+        if tie:
+            exact_rows.append(None)
+            continue
+        nb = len(o["starts"]) - 1
+        assert nblocks[h] == nb
+        np.testing.assert_array_equal(bstart[h, :nb + 1], o["starts"])
+        np.testing.assert_array_equal(src[h], o["src"])
+        np.testing.assert_allclose(qbar[h, :nb], o["Qbar"], rtol=1e-5, atol=1e-6)
+        np.testing.assert_allclose(kbar[h, :nb], o["Kbar"], rtol=1e-5, atol=1e-6)
+        gsets = parity.bits_to_sets(bits[h], nb, WORDS)
+        exact = set()
+        for i in range(nb):
+            assert parity.selection_agrees(gsets[i], o["logits"][i], o["P"][i], w.top_k, w.top_p), \
+                f"head {h} row {i}: selection differs beyond the tie margin"
+            if np.array_equal(gsets[i], o["sel"][i]):
+                exact.add(i)
+        # CSR rows = the bitmap rows; CSC = the transpose
+        for i in range(nb):
+            np.testing.assert_array_equal(col_idx[h, row_ptr[h, i]:row_ptr[h, i + 1]], gsets[i])
+        cols = [[] for _ in range(nb)]
+        for i in range(nb):
+            for j in gsets[i]:
+                cols[j].append(i)
+        for j in range(nb):
+            np.testing.assert_array_equal(row_idx[h, col_ptr[h, j]:col_ptr[h, j + 1]], cols[j])
+        exact_rows.append(exact)
+    return exact_rows
+
+
+def _rows_of_blocks(o, blocks):
+    return np.concatenate([o["src"][o["starts"][i]:o["starts"][i + 1]] for i in sorted(blocks)])
+
+
+CASES = {
+    "tiny_fp32_d64": (syn.workload(0), 2, True),
+    "grid16x32x32_bf16_d128": (syn.workload(2, T=16, H=32, W=32), 2, True),
+    "grid8x8x8_single_zone_no_audio": (syn.workload(1, T=8, H=8, W=8), 1, False),
+    "grid8x16x24_k1_p0": (syn.workload(1, T=8, H=16, W=24, top_k=1, top_p=0.0), 2, True),
+    "grid16x16x16_all_blocks": (syn.workload(2, T=16, H=16, W=16, top_k=10 ** 6, top_p=0.0), 1, True),
+    "grid8x16x16_p1": (syn.workload(0, top_p=1.0, top_k=1), 1, True),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_plan_and_forward_match_oracle(name, cuda_device):
+    w, heads, audio = CASES[name]
+    Q, K, V, a = _inputs(w, heads, audio)
+    Qd, Kd, Vd, ad = _to_dev(Q, K, V, a)
+    pl = _lib.plan(Qd, Kd, Vd, ad, _params(w, heads))
+    O, lse = pl.attn_fwd()
+    torch.cuda.synchronize()
+    assert pl.status() == 0
+    orc = _oracle_plans(w, Q, K, V, a, heads)
+    exact = _check_plan(pl, orc, w, heads)
+    O, lse = O.double().cpu().numpy(), lse.double().cpu().numpy()
+    for h in range(heads):
+        if exact[h] is None:
+            continue
+        o = orc[h]
+        Oo, lo = po.attention_fwd(Q[h].double().numpy(), K[h].double().numpy(), V[h].double().numpy(),
+                                  o["src"], o["starts"], o["sel"])
+        rows = _rows_of_blocks(o, exact[h])
+        assert len(rows) >= 0.95 * w.N
+        good, rl2, ma = parity.close(O[h][rows], Oo[rows])
+        assert good, f"{name} head {h}: O relL2 {rl2:.2e} maxabs {ma:.2e}"
+        np.testing.assert_allclose(lse[h][rows], lo[rows], atol=2e-2, rtol=1e-3)
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32_d64", "grid16x32x32_bf16_d128"])
+def test_imported_oracle_plan_forward(name, cuda_device):
+    """The oracle's own shapes and selection fed through prism_plan_import:
+    every output row is compared."""
+    w, heads, audio = CASES[name]
+    Q, K, V, a = _inputs(w, heads, audio)
+    orc = _oracle_plans(w, Q, K, V, a, heads)
+    NB, WORDS = w.N // 64, (w.N // 64 + 31) // 32
+    sid = np.stack([o["shape_id"] for o in orc]).astype(np.uint8)
+    bits = np.stack([parity.sets_to_bits(o["sel"], NB, WORDS) for o in orc])
+    Qd, Kd, Vd = _to_dev(Q, K, V)
+    sid_d = torch.from_numpy(sid).cuda()
+    bits_d = torch.from_numpy(bits.view(np.int32)).cuda()
+    pl = _lib.plan_import(Qd, Kd, Vd, sid_d, bits_d, _params(w, heads))
+    O, lse = pl.attn_fwd()
+    torch.cuda.synchronize()
+    assert pl.status() == 0
+    O, lse = O.double().cpu().numpy(), lse.double().cpu().numpy()
+    for h in range(heads):
+        o = orc[h]
+        Oo, lo = po.attention_fwd(Q[h].double().numpy(), K[h].double().numpy(), V[h].double().numpy(),
+                                  o["src"], o["starts"], o["sel"])
+        good, rl2, ma = parity.close(O[h], Oo)
+        assert good, f"{name} head {h}: O relL2 {rl2:.2e} maxabs {ma:.2e}"
+        np.testing.assert_allclose(lse[h], lo, atol=2e-2, rtol=1e-3)
+
+
+def test_invalid_workspace_is_rejected(cuda_device):
+    w = syn.workload(0)
+    Q, K, V, a = _inputs(w, 1)
+    Qd, Kd, Vd, ad = _to_dev(Q, K, V, a)
+    p = _params(w, 1)
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(_lib.PrismError) as e:
+        _lib.plan(Qd, Kd, Vd, ad, p, workspace=small)
+    assert e.value.status == _lib.PRISM_ERR_WORKSPACE
