@@ -35,7 +35,8 @@ ITEMS = {
 
 class PrismParams(C.Structure):
     _fields_ = [("T", C.c_int32), ("H", C.c_int32), ("W", C.c_int32), ("heads", C.c_int32),
-                ("head_dim", C.c_int32), ("dtype", C.c_int32), ("top_k", C.c_int32),
+                ("head_dim", C.c_int32), ("dtype", C.c_int32), ("out_dtype", C.c_int32),
+                ("top_k", C.c_int32),
                 ("top_p", C.c_float), ("eps", C.c_float), ("tau128", C.c_float),
                 ("tau256", C.c_float)]
 
@@ -86,9 +87,10 @@ def status_string(st: int) -> str:
     return load().prism_status_string(st).decode()
 
 
-def make_params(T, H, W, heads, head_dim, dtype, top_k, top_p, eps, tau128=0.5, tau256=0.25):
-    return PrismParams(T, H, W, heads, head_dim, dtype, top_k, float(top_p), float(eps),
-                       float(tau128), float(tau256))
+def make_params(T, H, W, heads, head_dim, dtype, top_k, top_p, eps, tau128=0.5, tau256=0.25,
+                out_dtype=PRISM_F32):
+    return PrismParams(T, H, W, heads, head_dim, dtype, out_dtype, top_k, float(top_p),
+                       float(eps), float(tau128), float(tau256))
 
 
 def workspace_bytes(params: PrismParams) -> int:
@@ -131,7 +133,7 @@ class Plan:
 
     def _out_dtype(self):
         import torch
-        return torch.float32 if self.params.dtype == PRISM_F32 else torch.bfloat16
+        return torch.float32 if self.params.out_dtype == PRISM_F32 else torch.bfloat16
 
     def attn_fwd(self, O=None, lse=None, stream=None):
         import torch

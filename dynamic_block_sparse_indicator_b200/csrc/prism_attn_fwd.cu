@@ -27,6 +27,13 @@
 namespace prism {
 
 constexpr int FWD_STAGES = 2;
+#ifndef PRISM_RESCALE_LOG2
+#define PRISM_RESCALE_LOG2 0.0f
+#endif
+// O is rescaled whenever a row max grows by more than this (log2 units).
+// A lazy threshold (P up to 2^8 between rescales) measured ~3x the output
+// error of exact rescaling on these kernels, so the default is exact.
+constexpr float kRescaleLog2 = PRISM_RESCALE_LOG2;
 constexpr int SLAB = 128 * 64 * 2;   // bytes of a 128-row x 64-column bf16 slab
 
 template <int HD>
@@ -82,7 +89,10 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         sm.abort = 0;
         mbar_fence_init();
     }
-    if (warp == 4) tmem_alloc(&sm.tmem_base, 512);
+    if (warp == 4) {
+        __syncwarp();
+        tmem_alloc(&sm.tmem_base, 512);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -98,7 +108,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             for (int j = 0; j < n; ++j) {
                 const int s = j % FWD_STAGES;
                 if (j >= FWD_STAGES &&
-                    !mbar_wait(&sm.kv_empty[s], ((j / FWD_STAGES) - 1) & 1, a.err)) break;
+                    !mbar_wait(&sm.kv_empty[s], ((j / FWD_STAGES) - 1) & 1, a.err, 401)) break;
                 const int kt = ents[j] >> 4;
                 const int krow = (int)((int64_t)h * a.N + (int64_t)kt * 128);
                 mbar_expect_tx(&sm.kv_full[s], 2 * NSL * SLAB);
@@ -114,11 +124,11 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(128, HD, 0, 1);
             const uint32_t q_s = smem_u32(sm.q[0]);
-            bool ok = mbar_wait(&sm.bar_q, 0, a.err);
+            bool ok = mbar_wait(&sm.bar_q, 0, a.err, 501);
             for (int j = 0; ok && j <= n; ++j) {
                 if (j < n) {
                     const int s = j % FWD_STAGES, b = j & 1;
-                    if (!mbar_wait(&sm.kv_full[s], (j / FWD_STAGES) & 1, a.err)) { ok = false; break; }
+                    if (!mbar_wait(&sm.kv_full[s], (j / FWD_STAGES) & 1, a.err, 502)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t k_s = smem_u32(sm.k[s][0]);
                     #pragma unroll
@@ -129,7 +139,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
                 if (j >= 1) {
                     const int jj = j - 1, b = jj & 1, s = jj % FWD_STAGES;
-                    if (!mbar_wait(&sm.p_full[b], (jj >> 1) & 1, a.err)) { ok = false; break; }
+                    if (!mbar_wait(&sm.p_full[b], (jj >> 1) & 1, a.err, 503)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t p_s = smem_u32(sm.p[b][0]);
                     const uint32_t v_s = smem_u32(sm.v[s][0]);
@@ -145,16 +155,18 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
     } else {
         // ------------------------------------------------ softmax + epilogue
+        // tcgen05.ld/st are warp-collective (.sync.aligned): every decision that
+        // guards one is made warp-uniform (__all_sync / __any_sync).
         const int r = threadIdx.x;                 // query row of the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const int qh = r >> 6;
+        const int qh = r >> 6;                     // uniform per warp (32 | 64)
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n; ++j) {
             const int b = j & 1;
             const int msk = ents[j] & 15;
             const bool v0 = (msk >> (qh * 2)) & 1, v1 = (msk >> (qh * 2 + 1)) & 1;
-            if (!mbar_wait(&sm.s_full[b], (j >> 1) & 1, a.err)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (j >> 1) & 1, a.err, 1))) { ok = false; break; }
             tc_fence_after();
             uint32_t sr[128];
             PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 0, (sr + 0));
@@ -173,13 +185,17 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }
             mx *= a.scale_log2;
             const float m_new = fmaxf(m_ref, mx);
-            bool rescaled = false;
-            if (m_ref == -INFINITY || j == 0) {
-                m_ref = m_new;
-            } else if (m_new > m_ref + 8.f) {
-                const float f = ex2(m_ref - m_new);
-                if (!mbar_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err)) { ok = false; break; }
+            const bool first = (j == 0) || (m_ref == -INFINITY);
+            const bool need = !first && (m_new > m_ref + kRescaleLog2);
+            if (first) m_ref = m_new;
+            const bool rescale = __any_sync(0xffffffffu, need);
+            if (rescale) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err, 2))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
+                const float f = need ? ex2(m_ref - m_new) : 1.f;
                 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
                     uint32_t o[32];
@@ -189,11 +205,12 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
                     PRISM_TMEM_ST32(tmem + lane_off + 256 + 32 * c, o);
                 }
-                l *= f;
-                m_ref = m_new;
-                rescaled = true;
+                if (need) { l *= f; m_ref = m_new; }
             }
-            if (j >= 2 && !mbar_wait(&sm.pv_done[b], ((j - 2) >> 1) & 1, a.err)) { ok = false; break; }
+            if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[b], ((j - 2) >> 1) & 1, a.err, 3))) {
+                ok = false;
+                break;
+            }
             const float neg = -m_ref;
             const uint32_t p_s = smem_u32(sm.p[b][0]);
             #pragma unroll
@@ -217,7 +234,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
             }
             fence_proxy_async_smem();
-            if (rescaled) tmem_wait_st();
+            if (rescale) tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
         }
@@ -225,7 +242,10 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const int row_perm = t * 128 + r;
         const int dst = a.src[(size_t)h * a.N + row_perm];
         const size_t orow = (size_t)h * a.N + (size_t)dst;
-        if (ok && n > 0 && mbar_wait(&sm.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err)) {
+        bool fin = false;
+        if (ok && n > 0)
+            fin = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err, 4));
+        if (fin) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             #pragma unroll
@@ -261,7 +281,10 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) tmem_dealloc(tmem, 512);
+    if (warp == 4) {
+        __syncwarp();
+        tmem_dealloc(tmem, 512);
+    }
 }
 
 template <int HD>
@@ -276,7 +299,7 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
     a.lse = lse;
     a.N = g.N;
     a.NT = g.NT;
-    a.out_f32 = g.dtype == PRISM_F32;
+    a.out_f32 = P->p.out_dtype == PRISM_F32;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
     a.err = (int*)(b + P->L.err);
     const int smem = (int)sizeof(FwdSmem<HD>) + 1024;

@@ -12,7 +12,13 @@
 
 namespace prism {
 
-constexpr uint32_t kWaitLimit = 1u << 26;   // polls (with back-off) before giving up
+constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s of wall-clock per wait before giving up
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -41,15 +47,23 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait for the phase of parity `parity`; false (and the error word
-// set) if it did not complete within the limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// set, with `where` in err[1]) if it did not complete within kWaitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int where = 0) {
     if (mbar_try(bar, parity)) return true;
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0;; ++i) {
         if (mbar_try(bar, parity)) return true;
-        if (i > 32) __nanosleep(64);
-        if ((i & 1023) == 0 && *(volatile int*)err != 0) return false;   // another CTA gave up
+        if (i > 16) __nanosleep(128);
+        if ((i & 255) == 0) {
+            if (*(volatile int*)err != 0) return false;          // someone else gave up
+            if (globaltimer_ns() - t0 > kWaitNs) break;
+        }
     }
-    atomicCAS(err, 0, PRISM_ERR_TIMEOUT);
+    if (atomicCAS(err, 0, PRISM_ERR_TIMEOUT) == 0) {
+        err[1] = where;
+        err[2] = (int)blockIdx.x;
+        err[3] = (int)threadIdx.x;
+    }
     return false;
 }
 

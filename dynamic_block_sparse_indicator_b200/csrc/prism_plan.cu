@@ -95,6 +95,7 @@ int validate_params(const prism_params* p) {
     if (p->heads < 1) return PRISM_ERR_INVALID_ARG;
     if (p->head_dim != 64 && p->head_dim != 128) return PRISM_ERR_INVALID_ARG;
     if (p->dtype != PRISM_BF16 && p->dtype != PRISM_F32) return PRISM_ERR_INVALID_ARG;
+    if (p->out_dtype != PRISM_BF16 && p->out_dtype != PRISM_F32) return PRISM_ERR_INVALID_ARG;
     if (p->top_k < 0) return PRISM_ERR_INVALID_ARG;
     if (!(p->top_p >= 0.f && p->top_p <= 1.f)) return PRISM_ERR_INVALID_ARG;
     if (p->top_k < 1 && p->top_p <= 0.f) return PRISM_ERR_INVALID_ARG;

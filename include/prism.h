@@ -26,8 +26,8 @@
  *     Q, K, V tensors, alive until prism_plan_destroy().
  *   - Token order: raster n = (t*H + h)*W + w over the latent T x H x W grid.
  *     Q, K, V, O, dO, dQ, dK, dV are [heads][N][head_dim] row-major in that
- *     order, of the element type `dtype` (bf16, or fp32 for the small fp32
- *     workload).  LSE is [heads][N] fp32 (natural log), same order.
+ *     order; Q, K, V of element type `dtype`, the others of `out_dtype`.
+ *     LSE is [heads][N] fp32 (natural log), same order.
  *   - Pointers must be 16-byte aligned.
  */
 #ifndef PRISM_H
@@ -55,7 +55,7 @@ extern "C" {
 #define PRISM_ERR_DEVICE_CHECK 5  /* a device-side bounds/consistency check failed */
 #define PRISM_ERR_UNSUPPORTED  6  /* no sm_100 device, or the build lacks the kernels */
 
-/* Element type of Q, K, V, dO and of the outputs O, dQ, dK, dV. */
+/* Element types (prism_params.dtype / out_dtype). */
 #define PRISM_BF16 0
 #define PRISM_F32  1
 
@@ -65,9 +65,12 @@ extern "C" {
  *             (zones are 8 x 8 x 8: page xyznot.com/id, section "Ide utama").
  *   heads     number of heads in this call (>= 1).
  *   head_dim  D, 64 or 128.
- *   dtype     PRISM_BF16 or PRISM_F32.  fp32 inputs feed the statistics and
- *             the pooled means in fp32; attention runs on their bf16 rounding
- *             (round to nearest even).
+ *   dtype     element type of Q, K, V: PRISM_BF16 or PRISM_F32.  fp32 inputs
+ *             feed the statistics and the pooled means in fp32; attention runs
+ *             on their bf16 rounding (round to nearest even).
+ *   out_dtype element type of O, dO, dQ, dK, dV: PRISM_BF16 or PRISM_F32.
+ *             The tensor-core products are bf16 with fp32 accumulation either
+ *             way; fp32 outputs keep the fp32 accumulators unrounded.
  *   top_k     k of Top-k (>= 0); k >= number of blocks keeps every block.
  *   top_p     p of Top-p in [0, 1]; p >= 1 keeps every block, p <= 0 none.
  *             top_k < 1 together with top_p <= 0 is rejected (empty sets).
@@ -79,6 +82,7 @@ typedef struct prism_params {
     int32_t heads;
     int32_t head_dim;
     int32_t dtype;
+    int32_t out_dtype;
     int32_t top_k;
     float   top_p;
     float   eps;
@@ -145,7 +149,7 @@ PRISM_API int prism_plan_import(const prism_params* p, const void* Q, const void
  *   O_q = softmax_n(q . k_n / sqrt(D)) v_n over the tokens n of the key
  *   blocks in S_i (fp32 online softmax, bf16 tensor-core products), written
  *   back in raster order (inverse permutation).
- *   O    device [heads][N][head_dim] of `dtype`.
+ *   O    device [heads][N][head_dim] of `out_dtype`.
  *   lse  device fp32 [heads][N], log-sum-exp of the scaled logits, raster order.
  */
 PRISM_API int prism_attn_fwd(prism_plan_t plan, void* O, float* lse, void* stream);
@@ -154,7 +158,7 @@ PRISM_API int prism_attn_fwd(prism_plan_t plan, void* O, float* lse, void* strea
  * prism_attn_bwd -- exact gradients of prism_attn_fwd with the plan fixed (the
  *   statistics, shapes and selection are detached: page xyznot.com/th, section
  *   on training).  dO, O, lse as produced/consumed by prism_attn_fwd.
- *   dQ, dK, dV device [heads][N][head_dim] of `dtype`, raster order.
+ *   dO, dQ, dK, dV device [heads][N][head_dim] of `out_dtype`, raster order.
  */
 PRISM_API int prism_attn_bwd(prism_plan_t plan, const void* dO, const void* O, const float* lse,
                    void* dQ, void* dK, void* dV, void* stream);

@@ -55,7 +55,7 @@ def test_workspace_bytes_and_validation(lib):
     # grows with heads; invalid problems give 0
     assert _lib.workspace_bytes(_params(heads=4)) > n
     for bad in (dict(T=12), dict(H=0), dict(head_dim=96), dict(top_k=0, top_p=0.0),
-                dict(top_p=1.5), dict(top_p=float("nan")), dict(eps=0.0), dict(dtype=7),
+                dict(top_p=1.5), dict(top_p=float("nan")), dict(eps=0.0), dict(dtype=7), dict(out_dtype=3),
                 dict(heads=0), dict(tau128=0.1, tau256=0.2)):
         assert _lib.workspace_bytes(_params(**bad)) == 0, bad
 
