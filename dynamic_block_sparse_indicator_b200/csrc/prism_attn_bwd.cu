@@ -1,9 +1,618 @@
-// prism_attn_bwd.cu -- gradients of the block-sparse attention (placeholder
-// until the tensor-core backward lands).
+// prism_attn_bwd.cu -- gradients of the block-sparse attention on sm_100a.
+//
+// "Prism: Dynamic Sparse Attention for Native 2K Joint Video-Audio Generation
+// Model Training" detaches the plan (statistics, shapes, selection): gradients
+// flow only through the attention over the selected key blocks (page
+// xyznot.com/th, section on training).  The pages give no backward kernel; the
+// kernels below compute the exact gradients of the forward with the selection
+// fixed, FlashAttention-style, restricted to the selected (query, key) pairs:
+//   D_i = rowsum(dO o O);  P = exp(S/sqrt(d) - LSE);  dV = P^T dO;
+//   dP = dO V^T;  dS = P o (dP - D);  dK = dS^T Q / sqrt(d);  dQ = dS K / sqrt(d).
+//
+// Three kernels, no atomics (deterministic):
+//   k_bwd_absmax / k_bwd_pre   per row: D_i, dO in fp16 block order (scaled
+//               by an exact per-head power of two so that max |dO| lies in
+//               [0.5, 1): gradients of any magnitude keep fp16's precision and
+//               dS cannot overflow), LSE in block order.
+//   k_bwd_dkdv  one CTA per 128-key tile; iterates the 64-row query halves of
+//               the key tile's transposed list; S^T = K Q^T and dP^T = V dO^T
+//               into TMEM (double-buffered), softmax warps form P^T and dS^T in
+//               fp16 shared memory, dV += P^T dO and dK += dS^T Q accumulate in
+//               TMEM.
+//   k_bwd_dq    one CTA per 128-row query tile; iterates the 64-key halves of
+//               the forward list; S = Q K^T, dP = dO V^T, dS -> shared memory,
+//               dQ += dS K in TMEM.
+// Warp roles as in the forward: 0-3 softmax/epilogue (thread = TMEM lane),
+// 4 TMA producer + TMEM allocator, 5 MMA issuer.  All waits are bounded and
+// every TMEM access is warp-uniform.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "prism_dev.cuh"
 #include "prism_internal.h"
 
-int prism_launch_attn_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse,
-                          void* dQ, void* dK, void* dV, void* stream) {
-    (void)P; (void)dO; (void)O; (void)lse; (void)dQ; (void)dK; (void)dV; (void)stream;
-    return PRISM_ERR_UNSUPPORTED;
+namespace prism {
+
+constexpr int BWD_STAGES = 2;
+constexpr int SLAB128 = 128 * 128;   // bytes: 128 rows x 64 fp16
+constexpr int SLAB64 = 64 * 128;     // bytes:  64 rows x 64 fp16
+constexpr float kLog2e = 1.4426950408889634f;
+
+// --------------------------------------------------------------- preprocess
+template <typename OT>
+__global__ void __launch_bounds__(256) k_bwd_absmax(const OT* __restrict__ dO, uint32_t* dmax, int64_t n_per_head) {
+    const int h = blockIdx.y;
+    const OT* x = dO + (size_t)h * n_per_head;
+    float m = 0.f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_per_head;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = fabsf((float)x[i]);
+        m = (v > m || v != v) ? v : m;                    // keeps a NaN
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        const float y = __shfl_xor_sync(0xffffffffu, m, o);
+        m = (y > m || y != y) ? y : m;
+    }
+    if ((threadIdx.x & 31) == 0) atomicMax(dmax + h, __float_as_uint(m));  // |x| bits order like values
+}
+
+// Exponent E with max |dO| in [2^(E-1), 2^E); dO is multiplied by 2^-E.
+__device__ __forceinline__ int dscale_exp(uint32_t bits, int* err) {
+    const float mx = __uint_as_float(bits);
+    if (!(mx <= 3.0e38f)) { atomicCAS(err, 0, PRISM_ERR_DEVICE_CHECK); return 0; }
+    if (mx == 0.f) return 0;
+    int e;
+    frexpf(mx, &e);
+    return e;
+}
+
+template <typename OT>
+__global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, const OT* __restrict__ O,
+                                                 const float* __restrict__ lse,
+                                                 const int* __restrict__ src, const uint32_t* dmax,
+                                                 __half* __restrict__ dOp, float* __restrict__ lse_p,
+                                                 float* __restrict__ di_p, int64_t N, int HD, int* err) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t p = (int64_t)blockIdx.x * 8 + warp;
+    const int h = blockIdx.y;
+    if (p >= N) return;
+    const float sc = ldexpf(1.f, -dscale_exp(dmax[h], err));
+    const int64_t n = src[(size_t)h * N + p];
+    const OT* dr = dO + ((size_t)h * N + n) * HD;
+    const OT* orow = O + ((size_t)h * N + n) * HD;
+    __half* out = dOp + ((size_t)h * N + p) * HD;
+    float acc = 0.f;
+    for (int c = lane; c < HD; c += 32) {
+        const float g = (float)dr[c];
+        acc = fmaf(g, (float)orow[c], acc);
+        out[c] = __float2half_rn(g * sc);
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+        di_p[(size_t)h * N + p] = acc * sc;
+        lse_p[(size_t)h * N + p] = lse[(size_t)h * N + n] * kLog2e;
+    }
+}
+
+// Iterator over the 64-token halves of a tile list.  Each entry is
+// (other tile << 4) | mask, mask bit (qhalf * 2 + khalf).  `own_is_key`
+// selects which side of the bit pair belongs to the CTA's own tile: the
+// iterated half is the other side, and the returned 2-bit mask says which of
+// the own tile's halves take part.
+struct HalfIter {
+    const int* ents;
+    int n, e, half;
+    int own_is_key;
+    __device__ bool next(int& row64, int& mask2) {
+        while (e < n) {
+            const int ent = ents[e];
+            const int other = ent >> 4, mk = ent & 15;
+            const int hf = half;
+            if (++half == 2) { half = 0; ++e; }
+            int m2;
+            if (own_is_key)   // iterated = query half hf; own halves = key halves
+                m2 = (mk >> (hf * 2)) & 3;
+            else              // iterated = key half hf; own halves = query halves
+                m2 = ((mk >> hf) & 1) | (((mk >> (2 + hf)) & 1) << 1);
+            if (m2) { row64 = other * 2 + hf; mask2 = m2; return true; }
+        }
+        return false;
+    }
+};
+
+__device__ __forceinline__ int count_units(const int* ents, int n, int own_is_key) {
+    HalfIter it{ents, n, 0, 0, own_is_key};
+    int r, m, c = 0;
+    while (it.next(r, m)) ++c;
+    return c;
+}
+
+struct BwdArgs {
+    const int* ptr;        // [heads][NT + 1]
+    const int* ent;        // [heads][NT * NT]
+    const int* src;        // [heads][N]
+    const float* lse_p;    // [heads][N] log2-scaled, block order
+    const float* di_p;     // [heads][N]  (scaled like dO)
+    const uint32_t* dmax;  // [heads] max |dO| bits: outputs are divided by the dO scale
+    void* out0;            // dK (dkdv) or dQ (dq), raster order
+    void* out1;            // dV (dkdv)
+    int64_t N;
+    int NT;
+    int out_f32;
+    float scale_log2;      // log2(e) / sqrt(d)
+    float inv_sqrt_d;
+    int* err;
+};
+
+__device__ __forceinline__ void store_row(void* base, size_t row, int HD, int c0, const uint32_t* v,
+                                          float mul, int out_f32) {
+    if (out_f32) {
+        float4* op = reinterpret_cast<float4*>(static_cast<float*>(base) + row * HD + c0);
+        #pragma unroll
+        for (int e = 0; e < 8; ++e)
+            op[e] = make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
+                                __uint_as_float(v[4 * e + 2]) * mul, __uint_as_float(v[4 * e + 3]) * mul);
+    } else {
+        uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + row * HD + c0);
+        #pragma unroll
+        for (int e = 0; e < 4; ++e)
+            op[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]) * mul, __uint_as_float(v[8 * e + 1]) * mul),
+                               pack_bf16(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul),
+                               pack_bf16(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul),
+                               pack_bf16(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul));
+    }
+}
+
+__device__ __forceinline__ void zero_row(void* base, size_t row, int HD, int out_f32) {
+    for (int c = 0; c < HD; ++c) {
+        if (out_f32) static_cast<float*>(base)[row * HD + c] = 0.f;
+        else static_cast<__nv_bfloat16*>(base)[row * HD + c] = __float2bfloat16(0.f);
+    }
+}
+
+// ------------------------------------------------------------------- dK, dV
+template <int HD>
+struct DkdvSmem {
+    static constexpr int NSL = HD / 64;
+    alignas(1024) uint8_t k[NSL][SLAB128];
+    alignas(1024) uint8_t v[NSL][SLAB128];
+    alignas(1024) uint8_t q[BWD_STAGES][NSL][SLAB64];
+    alignas(1024) uint8_t dO[BWD_STAGES][NSL][SLAB64];
+    alignas(1024) uint8_t p[2][SLAB128];      // P^T  [128 keys][64 queries]
+    alignas(1024) uint8_t ds[2][SLAB128];     // dS^T [128 keys][64 queries]
+    alignas(16) float lse[BWD_STAGES][64];
+    alignas(16) float di[BWD_STAGES][64];
+    uint64_t bar_kv;
+    uint64_t st_full[BWD_STAGES], st_empty[BWD_STAGES];
+    uint64_t s_full[2], s_free[2], p_full[2], pd_done[2];
+    uint32_t tmem_base;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+           const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
+           BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    DkdvSmem<HD>& sm = *reinterpret_cast<DkdvSmem<HD>*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int NSL = HD / 64;
+    const int t = blockIdx.x, h = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e0 = a.ptr[(size_t)h * (a.NT + 1) + t];
+    const int ne = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - e0;
+    const int* ents = a.ent + (size_t)h * a.NT * a.NT + e0;
+    const int U = count_units(ents, ne, 1);
+    // TMEM columns: S^T[b] at 64b, dP^T[b] at 128 + 64b, dV at 256, dK at 256 + HD
+    constexpr uint32_t TS = 0, TDP = 128, TDV = 256, TDK = 256 + HD;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_kv, 1);
+        for (int s = 0; s < BWD_STAGES; ++s) { mbar_init(&sm.st_full[s], 1); mbar_init(&sm.st_empty[s], 1); }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.s_free[b], 128);
+            mbar_init(&sm.p_full[b], 128);
+            mbar_init(&sm.pd_done[b], 1);
+        }
+        mbar_fence_init();
+    }
+    if (warp == 4) { __syncwarp(); tmem_alloc(&sm.tmem_base, 512); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int64_t hrow = (int64_t)h * a.N;
+
+    if (warp == 4) {
+        if (lane == 0 && U > 0) {
+            const int krow = (int)(hrow + (int64_t)t * 128);
+            mbar_expect_tx(&sm.bar_kv, 2 * NSL * SLAB128);
+            for (int c = 0; c < NSL; ++c) {
+                tma_load_2d(sm.k[c], &tm_k, &sm.bar_kv, 64 * c, krow);
+                tma_load_2d(sm.v[c], &tm_v, &sm.bar_kv, 64 * c, krow);
+            }
+            HalfIter it{ents, ne, 0, 0, 1};
+            int r64, m2;
+            for (int u = 0; it.next(r64, m2); ++u) {
+                const int s = u % BWD_STAGES;
+                if (u >= BWD_STAGES &&
+                    !mbar_wait(&sm.st_empty[s], ((u / BWD_STAGES) - 1) & 1, a.err, 1401)) break;
+                const int64_t qrow = hrow + (int64_t)r64 * 64;
+                mbar_expect_tx(&sm.st_full[s], 2 * NSL * SLAB64 + 2 * 256);
+                for (int c = 0; c < NSL; ++c) {
+                    tma_load_2d(sm.q[s][c], &tm_q64, &sm.st_full[s], 64 * c, (int)qrow);
+                    tma_load_2d(sm.dO[s][c], &tm_do64, &sm.st_full[s], 64 * c, (int)qrow);
+                }
+                bulk_load(sm.lse[s], a.lse_p + qrow, 256, &sm.st_full[s]);
+                bulk_load(sm.di[s], a.di_p + qrow, 256, &sm.st_full[s]);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0 && U > 0) {
+            constexpr uint32_t id_s = idesc_f16(128, 64, 0, 0);
+            constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
+            const uint32_t k_s = smem_u32(sm.k[0]), v_s = smem_u32(sm.v[0]);
+            bool ok = mbar_wait(&sm.bar_kv, 0, a.err, 1501);
+            for (int u = 0; ok && u <= U; ++u) {
+                if (u < U) {
+                    const int s = u % BWD_STAGES, b = u & 1;
+                    if (!mbar_wait(&sm.st_full[s], (u / BWD_STAGES) & 1, a.err, 1502)) break;
+                    if (u >= 2 && !mbar_wait(&sm.s_free[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
+                    tc_fence_after();
+                    const uint32_t q_s = smem_u32(sm.q[s][0]), do_s = smem_u32(sm.dO[s][0]);
+                    #pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_f16(tmem + TS + 64 * b, desc_kmajor(k_s, kk, SLAB128),
+                                  desc_kmajor(q_s, kk, SLAB64), id_s, kk > 0);
+                    #pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_f16(tmem + TDP + 64 * b, desc_kmajor(v_s, kk, SLAB128),
+                                  desc_kmajor(do_s, kk, SLAB64), id_s, kk > 0);
+                    umma_commit(&sm.s_full[b]);
+                }
+                if (u >= 1) {
+                    const int uu = u - 1, b = uu & 1, s = uu % BWD_STAGES;
+                    if (!mbar_wait(&sm.p_full[b], (uu >> 1) & 1, a.err, 1504)) break;
+                    tc_fence_after();
+                    const uint32_t p_s = smem_u32(sm.p[b]), ds_s = smem_u32(sm.ds[b]);
+                    const uint32_t q_s = smem_u32(sm.q[s][0]), do_s = smem_u32(sm.dO[s][0]);
+                    #pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + TDV, desc_kmajor(p_s, kk, SLAB128), desc_mnmajor(do_s, kk, SLAB64),
+                                  id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
+                    #pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + TDK, desc_kmajor(ds_s, kk, SLAB128), desc_mnmajor(q_s, kk, SLAB64),
+                                  id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&sm.pd_done[b]);
+                    umma_commit(&sm.st_empty[s]);
+                }
+            }
+        }
+    } else {
+        const int r = threadIdx.x;                  // key row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int kh = r >> 6;                      // warp-uniform
+        bool ok = true;
+        HalfIter it{ents, ne, 0, 0, 1};
+        int r64, m2;
+        for (int u = 0; it.next(r64, m2); ++u) {
+            const int b = u & 1, s = u % BWD_STAGES;
+            const bool valid = (m2 >> kh) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (u >> 1) & 1, a.err, 1001))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full[s], (u / BWD_STAGES) & 1, a.err, 1002))) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sv[64], dp[64];
+            PRISM_TMEM_LD32(tmem + lane_off + TS + 64 * b, sv);
+            PRISM_TMEM_LD32(tmem + lane_off + TS + 64 * b + 32, (sv + 32));
+            PRISM_TMEM_LD32(tmem + lane_off + TDP + 64 * b, dp);
+            PRISM_TMEM_LD32(tmem + lane_off + TDP + 64 * b + 32, (dp + 32));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.s_free[b]);
+            if (u >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1003))) {
+                ok = false;
+                break;
+            }
+            const float* lq = sm.lse[s];
+            const float* dq = sm.di[s];
+            const uint32_t p_s = smem_u32(sm.p[b]), ds_s = smem_u32(sm.ds[b]);
+            #pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t wp[4], wd[4];
+                #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = ch * 8 + 2 * e;
+                    float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+                    if (valid) {
+                        p0 = ex2(fmaf(__uint_as_float(sv[c]), a.scale_log2, -lq[c]));
+                        p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), a.scale_log2, -lq[c + 1]));
+                        d0 = p0 * (__uint_as_float(dp[c]) - dq[c]);
+                        d1 = p1 * (__uint_as_float(dp[c + 1]) - dq[c + 1]);
+                    }
+                    wp[e] = pack_f16(p0, p1);
+                    wd[e] = pack_f16(d0, d1);
+                }
+                st_shared_v4(p_s + swz128(r, ch), wp[0], wp[1], wp[2], wp[3]);
+                st_shared_v4(ds_s + swz128(r, ch), wd[0], wd[1], wd[2], wd[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&sm.p_full[b]);
+        }
+        const size_t orow = (size_t)hrow + (size_t)a.src[(size_t)hrow + (size_t)t * 128 + r];
+        bool fin = false;
+        if (ok && U > 0)
+            fin = __all_sync(0xffffffffu, mbar_wait(&sm.pd_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, 1004));
+        if (fin) {
+            tc_fence_after();
+            const float unscale = ldexpf(1.f, dscale_exp(a.dmax[h], a.err));
+            #pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                uint32_t o[32];
+                PRISM_TMEM_LD32(tmem + lane_off + TDV + 32 * c, o);
+                tmem_wait_ld();
+                store_row(a.out1, orow, HD, 32 * c, o, unscale, a.out_f32);
+                PRISM_TMEM_LD32(tmem + lane_off + TDK + 32 * c, o);
+                tmem_wait_ld();
+                store_row(a.out0, orow, HD, 32 * c, o, a.inv_sqrt_d * unscale, a.out_f32);
+            }
+        } else if (U == 0) {
+            zero_row(a.out0, orow, HD, a.out_f32);
+            zero_row(a.out1, orow, HD, a.out_f32);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 4) { __syncwarp(); tmem_dealloc(tmem, 512); }
+}
+
+// ------------------------------------------------------------------------ dQ
+template <int HD>
+struct DqSmem {
+    static constexpr int NSL = HD / 64;
+    alignas(1024) uint8_t q[NSL][SLAB128];
+    alignas(1024) uint8_t dO[NSL][SLAB128];
+    alignas(1024) uint8_t k[BWD_STAGES][NSL][SLAB64];
+    alignas(1024) uint8_t v[BWD_STAGES][NSL][SLAB64];
+    alignas(1024) uint8_t ds[2][SLAB128];     // dS [128 queries][64 keys]
+    uint64_t bar_q;
+    uint64_t st_full[BWD_STAGES], st_empty[BWD_STAGES];
+    uint64_t s_full[2], s_free[2], ds_full[2], dq_done[2];
+    uint32_t tmem_base;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+         const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
+         BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    DqSmem<HD>& sm = *reinterpret_cast<DqSmem<HD>*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int NSL = HD / 64;
+    const int t = blockIdx.x, h = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e0 = a.ptr[(size_t)h * (a.NT + 1) + t];
+    const int ne = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - e0;
+    const int* ents = a.ent + (size_t)h * a.NT * a.NT + e0;
+    const int U = count_units(ents, ne, 0);
+    constexpr uint32_t TS = 0, TDP = 128, TDQ = 256;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_q, 1);
+        for (int s = 0; s < BWD_STAGES; ++s) { mbar_init(&sm.st_full[s], 1); mbar_init(&sm.st_empty[s], 1); }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.s_free[b], 128);
+            mbar_init(&sm.ds_full[b], 128);
+            mbar_init(&sm.dq_done[b], 1);
+        }
+        mbar_fence_init();
+    }
+    if (warp == 4) { __syncwarp(); tmem_alloc(&sm.tmem_base, 512); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int64_t hrow = (int64_t)h * a.N;
+
+    if (warp == 4) {
+        if (lane == 0 && U > 0) {
+            const int qrow = (int)(hrow + (int64_t)t * 128);
+            mbar_expect_tx(&sm.bar_q, 2 * NSL * SLAB128);
+            for (int c = 0; c < NSL; ++c) {
+                tma_load_2d(sm.q[c], &tm_q, &sm.bar_q, 64 * c, qrow);
+                tma_load_2d(sm.dO[c], &tm_do, &sm.bar_q, 64 * c, qrow);
+            }
+            HalfIter it{ents, ne, 0, 0, 0};
+            int r64, m2;
+            for (int u = 0; it.next(r64, m2); ++u) {
+                const int s = u % BWD_STAGES;
+                if (u >= BWD_STAGES &&
+                    !mbar_wait(&sm.st_empty[s], ((u / BWD_STAGES) - 1) & 1, a.err, 2401)) break;
+                const int krow = (int)(hrow + (int64_t)r64 * 64);
+                mbar_expect_tx(&sm.st_full[s], 2 * NSL * SLAB64);
+                for (int c = 0; c < NSL; ++c) {
+                    tma_load_2d(sm.k[s][c], &tm_k64, &sm.st_full[s], 64 * c, krow);
+                    tma_load_2d(sm.v[s][c], &tm_v64, &sm.st_full[s], 64 * c, krow);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0 && U > 0) {
+            constexpr uint32_t id_s = idesc_f16(128, 64, 0, 0);
+            constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
+            const uint32_t q_s = smem_u32(sm.q[0]), do_s = smem_u32(sm.dO[0]);
+            bool ok = mbar_wait(&sm.bar_q, 0, a.err, 2501);
+            for (int u = 0; ok && u <= U; ++u) {
+                if (u < U) {
+                    const int s = u % BWD_STAGES, b = u & 1;
+                    if (!mbar_wait(&sm.st_full[s], (u / BWD_STAGES) & 1, a.err, 2502)) break;
+                    if (u >= 2 && !mbar_wait(&sm.s_free[b], ((u - 2) >> 1) & 1, a.err, 2503)) break;
+                    tc_fence_after();
+                    const uint32_t k_s = smem_u32(sm.k[s][0]), v_s = smem_u32(sm.v[s][0]);
+                    #pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_f16(tmem + TS + 64 * b, desc_kmajor(q_s, kk, SLAB128),
+                                  desc_kmajor(k_s, kk, SLAB64), id_s, kk > 0);
+                    #pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_f16(tmem + TDP + 64 * b, desc_kmajor(do_s, kk, SLAB128),
+                                  desc_kmajor(v_s, kk, SLAB64), id_s, kk > 0);
+                    umma_commit(&sm.s_full[b]);
+                }
+                if (u >= 1) {
+                    const int uu = u - 1, b = uu & 1, s = uu % BWD_STAGES;
+                    if (!mbar_wait(&sm.ds_full[b], (uu >> 1) & 1, a.err, 2504)) break;
+                    tc_fence_after();
+                    const uint32_t ds_s = smem_u32(sm.ds[b]), k_s = smem_u32(sm.k[s][0]);
+                    #pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + TDQ, desc_kmajor(ds_s, kk, SLAB128), desc_mnmajor(k_s, kk, SLAB64),
+                                  id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&sm.dq_done[b]);
+                    umma_commit(&sm.st_empty[s]);
+                }
+            }
+        }
+    } else {
+        const int r = threadIdx.x;                  // query row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int qh = r >> 6;
+        const size_t prow = (size_t)hrow + (size_t)t * 128 + r;
+        const float lse2 = a.lse_p[prow];
+        const float di = a.di_p[prow];
+        bool ok = true;
+        HalfIter it{ents, ne, 0, 0, 0};
+        int r64, m2;
+        for (int u = 0; it.next(r64, m2); ++u) {
+            const int b = u & 1;
+            const bool valid = (m2 >> qh) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (u >> 1) & 1, a.err, 2001))) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sv[64], dp[64];
+            PRISM_TMEM_LD32(tmem + lane_off + TS + 64 * b, sv);
+            PRISM_TMEM_LD32(tmem + lane_off + TS + 64 * b + 32, (sv + 32));
+            PRISM_TMEM_LD32(tmem + lane_off + TDP + 64 * b, dp);
+            PRISM_TMEM_LD32(tmem + lane_off + TDP + 64 * b + 32, (dp + 32));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.s_free[b]);
+            if (u >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.dq_done[b], ((u - 2) >> 1) & 1, a.err, 2003))) {
+                ok = false;
+                break;
+            }
+            const uint32_t ds_s = smem_u32(sm.ds[b]);
+            #pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t wd[4];
+                #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = ch * 8 + 2 * e;
+                    float d0 = 0.f, d1 = 0.f;
+                    if (valid) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sv[c]), a.scale_log2, -lse2));
+                        const float p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), a.scale_log2, -lse2));
+                        d0 = p0 * (__uint_as_float(dp[c]) - di);
+                        d1 = p1 * (__uint_as_float(dp[c + 1]) - di);
+                    }
+                    wd[e] = pack_f16(d0, d1);
+                }
+                st_shared_v4(ds_s + swz128(r, ch), wd[0], wd[1], wd[2], wd[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&sm.ds_full[b]);
+        }
+        const size_t orow = (size_t)hrow + (size_t)a.src[prow];
+        bool fin = false;
+        if (ok && U > 0)
+            fin = __all_sync(0xffffffffu, mbar_wait(&sm.dq_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, 2004));
+        if (fin) {
+            tc_fence_after();
+            const float unscale = ldexpf(1.f, dscale_exp(a.dmax[h], a.err));
+            #pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                uint32_t o[32];
+                PRISM_TMEM_LD32(tmem + lane_off + TDQ + 32 * c, o);
+                tmem_wait_ld();
+                store_row(a.out0, orow, HD, 32 * c, o, a.inv_sqrt_d * unscale, a.out_f32);
+            }
+        } else if (U == 0) {
+            zero_row(a.out0, orow, HD, a.out_f32);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 4) { __syncwarp(); tmem_dealloc(tmem, 512); }
+}
+
+template <int HD>
+static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse, void* dQ,
+                      void* dK, void* dV, cudaStream_t s) {
+    const Geom& g = P->g;
+    char* b = P->ws;
+    const int* src = (const int*)(b + P->L.src);
+    __half* dOp = (__half*)(b + P->L.dop);
+    float* lse_p = (float*)(b + P->L.lse_p);
+    float* di_p = (float*)(b + P->L.di_p);
+    uint32_t* dmax = (uint32_t*)(b + P->L.dmax);
+    int* err = (int*)(b + P->L.err);
+    cudaMemsetAsync(dmax, 0, sizeof(uint32_t) * g.heads, s);
+    const dim3 gmax(296, g.heads);
+    const dim3 gpre((unsigned)((g.N + 7) / 8), g.heads);
+    if (P->p.out_dtype == PRISM_F32) {
+        k_bwd_absmax<float><<<gmax, 256, 0, s>>>((const float*)dO, dmax, g.N * HD);
+        k_bwd_pre<float><<<gpre, 256, 0, s>>>((const float*)dO, (const float*)O, lse, src, dmax, dOp, lse_p,
+                                              di_p, g.N, HD, err);
+    } else {
+        k_bwd_absmax<__nv_bfloat16><<<gmax, 256, 0, s>>>((const __nv_bfloat16*)dO, dmax, g.N * HD);
+        k_bwd_pre<__nv_bfloat16><<<gpre, 256, 0, s>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)O, lse,
+                                                      src, dmax, dOp, lse_p, di_p, g.N, HD, err);
+    }
+    BwdArgs a{};
+    a.src = src;
+    a.lse_p = lse_p;
+    a.di_p = di_p;
+    a.dmax = dmax;
+    a.N = g.N;
+    a.NT = g.NT;
+    a.out_f32 = P->p.out_dtype == PRISM_F32;
+    a.scale_log2 = kLog2e / sqrtf((float)HD);
+    a.inv_sqrt_d = 1.f / sqrtf((float)HD);
+    a.err = err;
+    // dK, dV per key tile over the transposed lists
+    a.ptr = (const int*)(b + P->L.kt_ptr);
+    a.ent = (const int*)(b + P->L.kt_ent);
+    a.out0 = dK;
+    a.out1 = dV;
+    const int sm1 = (int)sizeof(DkdvSmem<HD>) + 1024;
+    if (cudaFuncSetAttribute(k_bwd_dkdv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1) != cudaSuccess)
+        return PRISM_ERR_CUDA;
+    k_bwd_dkdv<HD><<<dim3(g.NT, g.heads), 192, sm1, s>>>(P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, a);
+    // dQ per query tile over the forward lists
+    a.ptr = (const int*)(b + P->L.qt_ptr);
+    a.ent = (const int*)(b + P->L.qt_ent);
+    a.out0 = dQ;
+    a.out1 = nullptr;
+    const int sm2 = (int)sizeof(DqSmem<HD>) + 1024;
+    if (cudaFuncSetAttribute(k_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2) != cudaSuccess)
+        return PRISM_ERR_CUDA;
+    k_bwd_dq<HD><<<dim3(g.NT, g.heads), 192, sm2, s>>>(P->tm_q, P->tm_do, P->tm_k64, P->tm_v64, a);
+    return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+}  // namespace prism
+
+int prism_launch_attn_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse, void* dQ,
+                          void* dK, void* dV, void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return P->g.D == 128 ? prism::launch_bwd<128>(P, dO, O, lse, dQ, dK, dV, s)
+                         : prism::launch_bwd<64>(P, dO, O, lse, dQ, dK, dV, s);
 }

@@ -9,11 +9,11 @@
 // Design (B200): one CTA per 128-token query tile.  The plan's tile list gives,
 // for the tile, the 128-token key tiles to visit with a 4-bit mask (which
 // 64-token query half attends to which 64-token key half).  Per key tile:
-//   TMA (128B swizzle) K, V -> shared memory (2-stage ring)
+//   TMA (128B swizzle) K, V (fp16 block-ordered copies) -> shared memory (2-stage ring)
 //   tcgen05.mma S = Q K^T into TMEM (double-buffered, 2 x 128 columns)
 //   4 softmax warps (thread = query row = TMEM lane) read S, mask, update the
 //     running max (rescaling O in TMEM only when it grows by more than 2^8),
-//     write P = 2^(s - m) as bf16 to shared memory
+//     write P = 2^(s - m) as fp16 to shared memory
 //   tcgen05.mma O += P V into TMEM (128 + head_dim columns)
 // Warp roles: 0-3 softmax/epilogue, 4 TMA producer (and TMEM allocator),
 // 5 MMA issuer.  Every barrier wait is bounded (PRISM_ERR_TIMEOUT).
@@ -34,7 +34,7 @@ constexpr int FWD_STAGES = 2;
 // A lazy threshold (P up to 2^8 between rescales) measured ~3x the output
 // error of exact rescaling on these kernels, so the default is exact.
 constexpr float kRescaleLog2 = PRISM_RESCALE_LOG2;
-constexpr int SLAB = 128 * 64 * 2;   // bytes of a 128-row x 64-column bf16 slab
+constexpr int SLAB = 128 * 64 * 2;   // bytes of a 128-row x 64-column fp16 slab
 
 template <int HD>
 struct FwdSmem {
@@ -121,8 +121,8 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     } else if (warp == 5) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16(128, HD, 0, 1);
+            constexpr uint32_t idesc_qk = idesc_f16(128, 128, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_f16(128, HD, 0, 1);
             const uint32_t q_s = smem_u32(sm.q[0]);
             bool ok = mbar_wait(&sm.bar_q, 0, a.err, 501);
             for (int j = 0; ok && j <= n; ++j) {
@@ -133,7 +133,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     const uint32_t k_s = smem_u32(sm.k[s][0]);
                     #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_bf16(tmem + 128 * b, desc_kmajor(q_s, kk, SLAB), desc_kmajor(k_s, kk, SLAB),
+                        umma_f16(tmem + 128 * b, desc_kmajor(q_s, kk, SLAB), desc_kmajor(k_s, kk, SLAB),
                                   idesc_qk, kk > 0);
                     umma_commit(&sm.s_full[b]);
                 }
@@ -145,7 +145,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     const uint32_t v_s = smem_u32(sm.v[s][0]);
                     #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(tmem + 256, desc_kmajor(p_s, kk, SLAB), desc_mnmajor(v_s, kk, SLAB),
+                        umma_f16(tmem + 256, desc_kmajor(p_s, kk, SLAB), desc_mnmajor(v_s, kk, SLAB),
                                   idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sm.pv_done[b]);
                     umma_commit(&sm.kv_empty[s]);
@@ -228,7 +228,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, neg));
                         }
                         l += p0 + p1;
-                        w[e] = pack_bf16(p0, p1);
+                        w[e] = pack_f16(p0, p1);
                     }
                     st_shared_v4(p_s + half * SLAB + swz128(r, ch), w[0], w[1], w[2], w[3]);
                 }

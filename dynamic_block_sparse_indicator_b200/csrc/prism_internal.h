@@ -38,8 +38,9 @@ struct Layout {
     size_t col_ptr, row_idx;            // CSC
     size_t qt_ptr, qt_ent;              // int32[heads][NT + 1], int32[heads][NT * NT]
     size_t kt_ptr, kt_ent;              // (forward / backward tile lists)
-    size_t qp, kp, vp, dop;             // bf16[heads][N][D] block-ordered copies
+    size_t qp, kp, vp, dop;             // fp16[heads][N][D] block-ordered copies
     size_t lse_p, di_p;                 // float[heads][N] (backward, block order)
+    size_t dmax;                        // uint32[heads]: max |dO| bits (backward scaling)
     size_t total;
 };
 
@@ -57,7 +58,8 @@ struct prism_plan_s {
     size_t ws_bytes;
     int device;
     int has_audio;
-    CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 2D [heads*N, D] bf16 maps, 128B swizzle
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;       // 2D [heads*N, D] fp16, 128-row boxes, 128B swizzle
+    CUtensorMap tm_q64, tm_k64, tm_v64, tm_do64;  // the same with 64-row boxes
 };
 
 // Internal entry points of the attention translation units.

@@ -22,6 +22,7 @@
 // exactly zero variance).
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -84,6 +85,7 @@ Layout make_layout(const Geom& g) {
     L.dop = take(2 * H * N * g.D);
     L.lse_p = take(sizeof(float) * H * N);
     L.di_p = take(sizeof(float) * H * N);
+    L.dmax = take(sizeof(uint32_t) * H);
     L.total = off;
     return L;
 }
@@ -146,9 +148,9 @@ struct DevPlan {
     int* qt_ent;
     int* kt_ptr;
     int* kt_ent;
-    __nv_bfloat16* qp;
-    __nv_bfloat16* kp;
-    __nv_bfloat16* vp;
+    __half* qp;
+    __half* kp;
+    __half* vp;
 };
 
 static DevPlan dev_plan(const prism_plan_s* P) {
@@ -181,9 +183,9 @@ static DevPlan dev_plan(const prism_plan_s* P) {
     d.qt_ent = (int*)(b + L.qt_ent);
     d.kt_ptr = (int*)(b + L.kt_ptr);
     d.kt_ent = (int*)(b + L.kt_ent);
-    d.qp = (__nv_bfloat16*)(b + L.qp);
-    d.kp = (__nv_bfloat16*)(b + L.kp);
-    d.vp = (__nv_bfloat16*)(b + L.vp);
+    d.qp = (__half*)(b + L.qp);
+    d.kp = (__half*)(b + L.kp);
+    d.vp = (__half*)(b + L.vp);
     return d;
 }
 
@@ -514,12 +516,17 @@ __global__ void __launch_bounds__(1024) k_zone_finalize(DevPlan d, float eps, fl
 }
 
 // ================================================================ stage 2
-__device__ __forceinline__ uint32_t pk2(float a, float b) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+// The block-ordered copies are fp16: bf16 values inside +-65504 convert
+// exactly, and fp16 operands keep the tensor-core products' rounding error 8x
+// below bf16's.  A value outside the fp16 range is a device-check error.
+constexpr float kHalfMax = 65504.f;
+
+__device__ __forceinline__ uint32_t ph2(float a, float b) {
+    __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Gather one block: rows in block order into the bf16 copies, raster index of
+// Gather one block: rows in block order into the fp16 copies, raster index of
 // each slot into src, and fp32 block means of Q and K (from the input values).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restrict__ Q,
@@ -544,6 +551,7 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
     float aq[EPC], ak[EPC];
     #pragma unroll
     for (int e = 0; e < EPC; ++e) aq[e] = ak[e] = 0.f;
+    float amax = 0.f;
     const size_t hoff = (size_t)h * d.N * D;
     for (int r = rl; r < vol; r += RP) {
         const int lw = r % bw, lh = (r / bw) % bh, lt = r / (bw * bh);
@@ -555,33 +563,51 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
         const uint4 q4 = *reinterpret_cast<const uint4*>(Q + so);
         const uint4 k4 = *reinterpret_cast<const uint4*>(K + so);
         const uint4 v4 = *reinterpret_cast<const uint4*>(V + so);
+        float fq[EPC], fk[EPC], fv[EPC];
         if constexpr (sizeof(T) == 2) {
-            *reinterpret_cast<uint4*>(d.qp + dst) = q4;
-            *reinterpret_cast<uint4*>(d.kp + dst) = k4;
-            *reinterpret_cast<uint4*>(d.vp + dst) = v4;
             const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&q4);
             const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&k4);
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
             #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 fq = __bfloat1622float2(q2[e]), fk = __bfloat1622float2(k2[e]);
-                aq[2 * e] += fq.x; aq[2 * e + 1] += fq.y;
-                ak[2 * e] += fk.x; ak[2 * e + 1] += fk.y;
+                const float2 a0 = __bfloat1622float2(q2[e]), a1 = __bfloat1622float2(k2[e]),
+                             a2 = __bfloat1622float2(v2[e]);
+                fq[2 * e] = a0.x; fq[2 * e + 1] = a0.y;
+                fk[2 * e] = a1.x; fk[2 * e + 1] = a1.y;
+                fv[2 * e] = a2.x; fv[2 * e + 1] = a2.y;
             }
         } else {
-            const float* fq = reinterpret_cast<const float*>(&q4);
-            const float* fk = reinterpret_cast<const float*>(&k4);
-            const float* fv = reinterpret_cast<const float*>(&v4);
-            uint2 oq, ok, ov;
-            oq.x = pk2(fq[0], fq[1]); oq.y = pk2(fq[2], fq[3]);
-            ok.x = pk2(fk[0], fk[1]); ok.y = pk2(fk[2], fk[3]);
-            ov.x = pk2(fv[0], fv[1]); ov.y = pk2(fv[2], fv[3]);
-            *reinterpret_cast<uint2*>(d.qp + dst) = oq;
-            *reinterpret_cast<uint2*>(d.kp + dst) = ok;
-            *reinterpret_cast<uint2*>(d.vp + dst) = ov;
             #pragma unroll
-            for (int e = 0; e < 4; ++e) { aq[e] += fq[e]; ak[e] += fk[e]; }
+            for (int e = 0; e < 4; ++e) {
+                fq[e] = reinterpret_cast<const float*>(&q4)[e];
+                fk[e] = reinterpret_cast<const float*>(&k4)[e];
+                fv[e] = reinterpret_cast<const float*>(&v4)[e];
+            }
+        }
+        uint32_t oq[EPC / 2], ok[EPC / 2], ov[EPC / 2];
+        #pragma unroll
+        for (int e = 0; e < EPC / 2; ++e) {
+            oq[e] = ph2(fq[2 * e], fq[2 * e + 1]);
+            ok[e] = ph2(fk[2 * e], fk[2 * e + 1]);
+            ov[e] = ph2(fv[2 * e], fv[2 * e + 1]);
+        }
+        #pragma unroll
+        for (int e = 0; e < EPC; ++e) {
+            aq[e] += fq[e];
+            ak[e] += fk[e];
+            amax = fmaxf(amax, fmaxf(fabsf(fq[e]), fmaxf(fabsf(fk[e]), fabsf(fv[e]))));
+        }
+        if constexpr (EPC == 8) {
+            *reinterpret_cast<uint4*>(d.qp + dst) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+            *reinterpret_cast<uint4*>(d.kp + dst) = make_uint4(ok[0], ok[1], ok[2], ok[3]);
+            *reinterpret_cast<uint4*>(d.vp + dst) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+        } else {
+            *reinterpret_cast<uint2*>(d.qp + dst) = make_uint2(oq[0], oq[1]);
+            *reinterpret_cast<uint2*>(d.kp + dst) = make_uint2(ok[0], ok[1]);
+            *reinterpret_cast<uint2*>(d.vp + dst) = make_uint2(ov[0], ov[1]);
         }
     }
+    if (!(amax <= kHalfMax)) dev_fail(d.err, PRISM_ERR_DEVICE_CHECK);   // also catches NaN
     #pragma unroll
     for (int e = 0; e < EPC; ++e) { pq[rl][c * EPC + e] = aq[e]; pk[rl][c * EPC + e] = ak[e]; }
     __syncthreads();
@@ -913,14 +939,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-static int make_tmap(CUtensorMap* m, void* base, int64_t rows, int D) {
+static int make_tmap(CUtensorMap* m, void* base, int64_t rows, int D, int box_rows) {
     auto enc = get_encode();
     if (!enc) return PRISM_ERR_CUDA;
     cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
@@ -959,10 +985,14 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
     P->ws_bytes = ws_bytes;
     cudaGetDevice(&P->device);
     const int64_t rows = (int64_t)g.heads * g.N;
-    st = make_tmap(&P->tm_q, P->ws + L.qp, rows, g.D);
-    if (!st) st = make_tmap(&P->tm_k, P->ws + L.kp, rows, g.D);
-    if (!st) st = make_tmap(&P->tm_v, P->ws + L.vp, rows, g.D);
-    if (!st) st = make_tmap(&P->tm_do, P->ws + L.dop, rows, g.D);
+    st = make_tmap(&P->tm_q, P->ws + L.qp, rows, g.D, 128);
+    if (!st) st = make_tmap(&P->tm_k, P->ws + L.kp, rows, g.D, 128);
+    if (!st) st = make_tmap(&P->tm_v, P->ws + L.vp, rows, g.D, 128);
+    if (!st) st = make_tmap(&P->tm_do, P->ws + L.dop, rows, g.D, 128);
+    if (!st) st = make_tmap(&P->tm_q64, P->ws + L.qp, rows, g.D, 64);
+    if (!st) st = make_tmap(&P->tm_k64, P->ws + L.kp, rows, g.D, 64);
+    if (!st) st = make_tmap(&P->tm_v64, P->ws + L.vp, rows, g.D, 64);
+    if (!st) st = make_tmap(&P->tm_do64, P->ws + L.dop, rows, g.D, 64);
     if (st) { delete P; return st; }
     *outP = P;
     return PRISM_OK;

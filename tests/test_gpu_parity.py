@@ -91,10 +91,10 @@ def _check_plan(pl, orc, w, heads):
 
 
 def _attn_inputs(w, Q, K, V, h):
-    """Values the attention kernels compute on: the inputs, rounded to bf16 for
-    the fp32 workload (the path's documented precision)."""
+    """Values the attention kernels compute on: the tensor-core operands are
+    fp16, so fp32 inputs are rounded to fp16 (bf16 inputs convert exactly)."""
     if w.dtype == "f32":
-        return [x[h].to(torch.bfloat16).double().numpy() for x in (Q, K, V)]
+        return [x[h].to(torch.float16).double().numpy() for x in (Q, K, V)]
     return [x[h].double().numpy() for x in (Q, K, V)]
 
 
@@ -175,3 +175,57 @@ def test_invalid_workspace_is_rejected(cuda_device):
     with pytest.raises(_lib.PrismError) as e:
         _lib.plan(Qd, Kd, Vd, ad, p, workspace=small)
     assert e.value.status == _lib.PRISM_ERR_WORKSPACE
+
+
+def _dout(w, heads):
+    """dO ~ N(0,1), cast to bf16 (as every synthetic tensor), held in fp32."""
+    return syn.make_dout(w, heads=heads, out_dtype=torch.bfloat16).float()
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32_d64", "grid16x32x32_bf16_d128", "grid8x16x24_k1_p0"])
+def test_imported_oracle_plan_backward(name, cuda_device):
+    """dQ, dK, dV with the oracle's own plan imported: every element compared."""
+    w, heads, audio = CASES[name]
+    Q, K, V, a = _inputs(w, heads, audio)
+    dO = _dout(w, heads)
+    orc = _oracle_plans(w, Q, K, V, a, heads)
+    NB, WORDS = w.N // 64, (w.N // 64 + 31) // 32
+    sid = np.stack([o["shape_id"] for o in orc]).astype(np.uint8)
+    bits = np.stack([parity.sets_to_bits(o["sel"], NB, WORDS) for o in orc])
+    Qd, Kd, Vd, dOd = _to_dev(Q, K, V, dO)
+    pl = _lib.plan_import(Qd, Kd, Vd, torch.from_numpy(sid).cuda(),
+                          torch.from_numpy(bits.view(np.int32)).cuda(), _params(w, heads))
+    O, lse = pl.attn_fwd()
+    dQ, dK, dV = pl.attn_bwd(dOd, O, lse)
+    torch.cuda.synchronize()
+    assert pl.status() == 0
+    for h in range(heads):
+        o = orc[h]
+        qa, ka, va = _attn_inputs(w, Q, K, V, h)
+        ref = po.attention_bwd(qa, ka, va, dO[h].double().numpy(), o["src"], o["starts"], o["sel"])
+        for got, want, nm in zip((dQ, dK, dV), ref, ("dQ", "dK", "dV")):
+            good, rl2, ma = parity.close(got[h].double().cpu().numpy(), want)
+            assert good, f"{name} head {h} {nm}: relL2 {rl2:.2e} maxabs {ma:.2e}"
+
+
+def test_full_pipeline_backward_tiny(cuda_device):
+    """GPU plan + forward + backward on the tiny fp32 workload against the oracle."""
+    w, heads, audio = CASES["tiny_fp32_d64"]
+    Q, K, V, a = _inputs(w, heads, audio)
+    dO = _dout(w, heads)
+    Qd, Kd, Vd, ad, dOd = _to_dev(Q, K, V, a, dO)
+    pl = _lib.plan(Qd, Kd, Vd, ad, _params(w, heads))
+    O, lse = pl.attn_fwd()
+    dQ, dK, dV = pl.attn_bwd(dOd, O, lse)
+    torch.cuda.synchronize()
+    assert pl.status() == 0
+    orc = _oracle_plans(w, Q, K, V, a, heads)
+    exact = _check_plan(pl, orc, w, heads)
+    for h in range(heads):
+        o = orc[h]
+        assert exact[h] is not None and len(exact[h]) == len(o["starts"]) - 1
+        ref = po.attention_bwd(*_attn_inputs(w, Q, K, V, h), dO[h].double().numpy(), o["src"],
+                               o["starts"], o["sel"])
+        for got, want, nm in zip((dQ, dK, dV), ref, ("dQ", "dK", "dV")):
+            good, rl2, ma = parity.close(got[h].double().cpu().numpy(), want)
+            assert good, f"head {h} {nm}: relL2 {rl2:.2e} maxabs {ma:.2e}"
