@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Prism sparse video self-attention benchmark on B200.
+
+One step = one head-layer of the 2K training workload (grid 72x88x160,
+1,013,760 tokens, head_dim 128, bf16 inputs, Top-k 16, Top-p 0.9): the plan
+(zone statistics, shapes, reorder, pooling, selection), the sparse attention
+forward and its backward, heads processed in sequence.  With N GPUs (one
+process each, launched by torchrun) every rank runs its own heads: weak
+scaling, no collective on the data path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl prism|reference]
+
+Prints one JSON line (rank 0).  `value` is milliseconds per head-layer for the
+whole job (lower is better); the dominant kernel's roofline, the end-to-end
+number through the C ABI with host buffers, and the CPU oracle baseline ride
+along.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Prism sparse-attn fwd+bwd ms/head-layer @1M tokens; achieved tensor TFLOP/s"
+UNIT = "ms/head-layer"
+
+
+def args_():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["prism", "reference"], default="prism")
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="attention sample budget of the CPU oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+def selected_pairs(pl, head=0):
+    """Pi = sum_i |B_i| * sum_{j in S_i} |B_j| of a plan (exported, host)."""
+    import numpy as np
+    p = pl.params
+    N = p.T * p.H * p.W
+    NB = N // 64
+    words = (NB + 31) // 32
+    nb = int(pl.export("nblocks")[head])
+    st = pl.export("blk_start").reshape(-1, NB + 1)[head, :nb + 1].astype(np.int64)
+    size = np.diff(st)
+    bits = pl.export("sel_bits").reshape(-1, NB, words)[head, :nb]
+    sel = np.unpackbits(bits.view(np.uint8), axis=1, bitorder="little")[:, :nb].astype(np.int64)
+    keys = sel @ size
+    return int((size * keys).sum()), nb, float(sel.sum(1).mean())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self):
+        import statistics
+        rows = []
+        self.f.flush()
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        mx = max(r[1] for r in rows)
+        load = [r[0] for r in rows if r[0] > 0.5 * mx] or [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        return {}
+
+
+# --------------------------------------------------------- CPU oracle leg
+def oracle_head_ms(Qh, Kh, Vh, dOh, a, w, budget_s, seed=0):
+    """The oracle on one head: full plan, then forward + backward on a seeded
+    sample of query blocks until `budget_s` elapses; the attention time is
+    extrapolated to the head by the share of selected pairs.  Returns
+    (ms per head-layer, description, threads)."""
+    import numpy as np
+    from oracle import prism_oracle as po
+    t0 = time.perf_counter()
+    pl = po.plan_head(Qh, Kh, Vh, a, w.T, w.H, w.W, w.top_k, w.top_p, w.eps)
+    t_plan = time.perf_counter() - t0
+    src, st, sel = pl["src"], pl["starts"], pl["sel"]
+    size = np.diff(st)
+    pairs = np.array([size[i] * size[js].sum() for i, js in enumerate(sel)], dtype=np.float64)
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(len(sel))
+    # O and LSE of the sampled blocks come from the oracle forward on those rows
+    O = np.zeros_like(Qh)
+    lse = np.zeros(Qh.shape[0])
+    dQ, dK, dV = np.zeros_like(Qh), np.zeros_like(Kh), np.zeros_like(Vh)
+    t1 = time.perf_counter()
+    done, pi_s = 0, 0.0
+    for i in order:
+        qi = src[st[i]:st[i + 1]]
+        keys = np.concatenate([src[st[j]:st[j + 1]] for j in sel[i]])
+        s = Qh[qi] @ Kh[keys].T / np.sqrt(Qh.shape[1])
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        z = e.sum(axis=1, keepdims=True)
+        O[qi] = (e / z) @ Vh[keys]
+        lse[qi] = (m + np.log(z))[:, 0]
+        po.block_grads(Qh, Kh, Vh, dOh, O, lse, src, st, sel, i, dQ, dK, dV)
+        done += 1
+        pi_s += pairs[i]
+        if time.perf_counter() - t1 > budget_s:
+            break
+    t_attn = (time.perf_counter() - t1) * pairs.sum() / pi_s
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count() or 1
+    desc = (f"full oracle plan of one head ({t_plan:.1f} s) + forward and backward of {done} of "
+            f"{len(sel)} query blocks ({100 * pi_s / pairs.sum():.2f}% of the selected pairs), "
+            f"attention time extrapolated by pair share")
+    return 1e3 * (t_plan + t_attn), desc, threads
+
+
+# ------------------------------------------------------------- main paths
+def emit(d):
+    print(json.dumps(d), flush=True)
+
+
+def run_reference(a, rank, world):
+    """The oracle on the host cores, on the same workload and metric."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    from dynamic_block_sparse_indicator_b200 import synthetic as syn
+    w = syn.workload(a.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    heads = min(w.heads, a.steps + 1)
+    Q, K, V = syn.make_qkv(w, device=dev, heads=heads)
+    dO = syn.make_dout(w, device=dev, heads=heads, out_dtype=torch.bfloat16)
+    amap = syn.make_amap(w, device=dev).cpu().numpy()
+    host = lambda t, h: t[h].to("cpu", torch.float64).numpy()
+    # warm-up steps: a one-second sample on head 0
+    for _ in range(a.warmup):
+        oracle_head_ms(host(Q, 0), host(K, 0), host(V, 0), host(dO, 0), amap, w, 1.0)
+    vals, desc, threads = [], "", 1
+    t0 = time.perf_counter()
+    for s in range(a.steps):
+        h = s % heads
+        ms, desc, threads = oracle_head_ms(host(Q, h), host(K, h), host(V, h), host(dO, h), amap, w,
+                                           a.cpu_seconds / 4, seed=s)
+        vals.append(ms)
+    wall = time.perf_counter() - t0
+    v = float(np.mean(vals))
+    emit({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+          "steps": a.steps, "warmup": a.warmup, "ms_per_step": v, "higher_is_better": False,
+          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+          "config": {"workload": w.name(), "grid": [w.T, w.H, w.W], "tokens": w.N,
+                     "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p},
+          "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                           "sample": desc, "wall_s": wall},
+          "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+
+
+def run_prism(a, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from dynamic_block_sparse_indicator_b200 import _lib
+    from dynamic_block_sparse_indicator_b200 import synthetic as syn
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = syn.workload(a.workload)
+    lib = _lib.load()
+    need = a.warmup + a.steps
+    heads = min(w.heads, need)
+    # this rank's heads: offsets by rank, so ranks work on different heads
+    order = [(rank * need + i) % w.heads for i in range(need)]
+    gen_heads = max(order) + 1
+    Q, K, V = syn.make_qkv(w, device=dev, heads=gen_heads)
+    dO = syn.make_dout(w, device=dev, heads=gen_heads, out_dtype=torch.bfloat16).float()
+    amap = syn.make_amap(w, device=dev)
+    params = _lib.make_params(w.T, w.H, w.W, 1, w.head_dim, _lib.PRISM_BF16, w.top_k, w.top_p,
+                              w.eps, out_dtype=_lib.PRISM_F32)
+    ws = torch.empty(_lib.workspace_bytes(params), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    O = torch.empty(1, w.N, w.head_dim, **f32)
+    lse = torch.empty(1, w.N, **f32)
+    dQ, dK, dV = (torch.empty(1, w.N, w.head_dim, **f32) for _ in range(3))
+
+    def step(h, prof=False, pev=None):
+        if pev is not None:
+            pev[0].record()
+        pl = _lib.plan(Q[h:h + 1], K[h:h + 1], V[h:h + 1], amap, params, workspace=ws)
+        if pev is not None:
+            pev[1].record()
+        if prof:
+            pl.profile(True)
+        pl.attn_fwd(O, lse)
+        pl.attn_bwd(dO[h:h + 1], O, lse, dQ, dK, dV)
+        return pl
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    for i in range(a.warmup):
+        pl = step(order[i])
+    barrier()
+    st = pl.status()
+    if st:
+        raise RuntimeError(f"device status after warm-up: {_lib.status_string(st)}")
+    del pl
+    # ---------------------------------------------------------- timed region
+    stage_ms = {k: 0.0 for k in _lib.Plan.STAGES}
+    stage_n = {k: 0 for k in _lib.Plan.STAGES}
+    plan_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(a.steps)]
+    launches = 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    plans = []
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        e0.record()
+        for i in range(a.steps):
+            pl = step(order[a.warmup + i], prof=True, pev=plan_ev[i])
+            plans.append(pl)
+        e1.record()
+        barrier()
+    clocks = clk.summary()
+    elapsed = e0.elapsed_time(e1)
+    for pl in plans:
+        for k, (ms, n) in pl.profile_read().items():
+            stage_ms[k] += ms
+            stage_n[k] += n
+        launches += pl.launches()
+        st = pl.status()
+        if st:
+            raise RuntimeError(f"device status: {_lib.status_string(st)}")
+    plan_ms = sum(a_.elapsed_time(b_) for a_, b_ in plan_ev)
+    del plans, pl
+    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_max = float(t.item())
+    # selected pairs of the timed heads (plans are deterministic: re-plan, untimed)
+    pis = []
+    for i in range(a.steps):
+        h = order[a.warmup + i]
+        pl = _lib.plan(Q[h:h + 1], K[h:h + 1], V[h:h + 1], amap, params, workspace=ws)
+        pis.append(selected_pairs(pl))
+        del pl
+    Pi = float(np.mean([p[0] for p in pis]))
+    nb_mean = float(np.mean([p[1] for p in pis]))
+    sel_mean = float(np.mean([p[2] for p in pis]))
+    D = w.head_dim
+    flops = {"fwd": 4 * D * Pi, "bwd_dkdv": 8 * D * Pi, "bwd_dq": 2 * D * Pi}
+    pk = peaks()
+    peak = pk.get("bf16_tflops_sustained") or 1400.0
+    peak_src = "measured sustained bf16 (fp16 operands, same kind::f16 rate)" if pk else "fallback"
+    per_launch = {k: stage_ms[k] / max(stage_n[k], 1) for k in stage_ms}
+    dom = max(("fwd", "bwd_dkdv", "bwd_dq"), key=lambda k: stage_ms[k])
+    ach = flops[dom] / (per_launch[dom] * 1e-3) / 1e12
+    attn_ms = (stage_ms["fwd"] + stage_ms["bwd_pre"] + stage_ms["bwd_dkdv"] + stage_ms["bwd_dq"]) / a.steps
+    attn_tflops = 14 * D * Pi / (attn_ms * 1e-3) / 1e12
+    value = elapsed_max / (a.steps * world)
+    # --------------------------------------------------- end to end (host)
+    e2e = None
+    if a.e2e_steps > 0:
+        pin = lambda t: t.cpu().pin_memory()
+        hq, hk, hv = pin(Q[:1]), pin(K[:1]), pin(V[:1])
+        hdo, ha = pin(dO[:1]), pin(amap)
+        outs = [torch.empty(1, w.N, D, dtype=torch.float32).pin_memory() for _ in range(4)]
+        hlse = torch.empty(1, w.N, dtype=torch.float32).pin_memory()
+        dq_, dk_, dv_ = (torch.empty_like(Q[:1]) for _ in range(3))
+        bufs = dict(q=dq_, k=dk_, v=dv_, do=torch.empty_like(dO[:1]), a=torch.empty_like(amap))
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo, ha))
+        d2h = sum(x.numel() * x.element_size() for x in outs) + hlse.numel() * 4
+        barrier()
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record()
+        for _ in range(a.e2e_steps):
+            bufs["q"].copy_(hq, non_blocking=True)
+            bufs["k"].copy_(hk, non_blocking=True)
+            bufs["v"].copy_(hv, non_blocking=True)
+            bufs["do"].copy_(hdo, non_blocking=True)
+            bufs["a"].copy_(ha, non_blocking=True)
+            pl = _lib.plan(bufs["q"], bufs["k"], bufs["v"], bufs["a"], params, workspace=ws)
+            pl.attn_fwd(O, lse)
+            pl.attn_bwd(bufs["do"], O, lse, dQ, dK, dV)
+            for hbuf, dbuf in zip(outs, (O, dQ, dK, dV)):
+                hbuf.copy_(dbuf, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+        x1.record()
+        barrier()
+        te = torch.tensor([x0.elapsed_time(x1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": float(te.item()) / (a.e2e_steps * world), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    # --------------------------------------------------- CPU oracle baseline
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        h = order[a.warmup]
+        host = lambda t: t[h].to("cpu", torch.float64).numpy()
+        ms, desc, threads = oracle_head_ms(host(Q), host(K), host(V), host(dO),
+                                           amap.cpu().numpy(), w, a.cpu_seconds)
+        cpu = {"value": ms, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        emit({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+              "warmup": a.warmup, "ms_per_step": elapsed_max / a.steps, "higher_is_better": False,
+              "scaling": "weak", "vs_baseline": None, "dtype": "fp16-operand tensor cores, fp32 accumulate",
+              "data": "synthetic",
+              "config": {"workload": w.name(), "grid": [w.T, w.H, w.W], "tokens": w.N,
+                         "heads_in_sequence": True, "head_dim": D, "input_dtype": "bf16",
+                         "output_dtype": "fp32", "top_k": w.top_k, "top_p": w.top_p,
+                         "l2": "inputs larger than L2 (259 MB per tensor per head)"},
+              "tflops": {"fwd_bwd_selected": attn_tflops,
+                         "fraction_of_peak": attn_tflops / peak},
+              "stages_ms_per_head": {"plan": plan_ms / a.steps,
+                                     **{k: stage_ms[k] / a.steps for k in stage_ms}},
+              "plan_stats": {"blocks_per_head": nb_mean, "mean_selected_blocks": sel_mean,
+                             "selected_pairs": Pi, "pair_density": Pi / float(w.N) ** 2},
+              "roofline": {"kernel": {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv",
+                                      "bwd_dq": "k_bwd_dq"}[dom],
+                           "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                           "frac": ach / peak, "peak_source": peak_src, "traffic": None},
+              "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks})
+
+
+def main():
+    a = args_()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        run_reference(a, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600))
+    try:
+        run_prism(a, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

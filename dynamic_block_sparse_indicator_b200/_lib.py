@@ -74,6 +74,9 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_plan_destroy": (None, [vp]),
         "prism_status_string": (C.c_char_p, [i32]),
         "prism_version": (C.c_char_p, []),
+        "prism_profile_enable": (i32, [vp, i32]),
+        "prism_profile_read": (i32, [vp, C.POINTER(C.c_float), C.POINTER(C.c_int), vp]),
+        "prism_launch_count": (C.c_int64, [vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -172,6 +175,23 @@ class Plan:
         if st:
             raise PrismError(st, f"prism_plan_export({item})")
         return out
+
+    STAGES = ("fwd", "bwd_pre", "bwd_dkdv", "bwd_dq")
+
+    def profile(self, on: bool = True):
+        load().prism_profile_enable(self._h, 1 if on else 0)
+
+    def profile_read(self, stream=None):
+        """{stage: (ms, launches)} accumulated since the last read (synchronises)."""
+        ms = (C.c_float * len(self.STAGES))()
+        n = (C.c_int * len(self.STAGES))()
+        st = load().prism_profile_read(self._h, ms, n, _stream(stream))
+        if st:
+            raise PrismError(st, "prism_profile_read")
+        return {k: (float(ms[i]), int(n[i])) for i, k in enumerate(self.STAGES)}
+
+    def launches(self) -> int:
+        return int(load().prism_launch_count(self._h))
 
     def status(self, stream=None) -> int:
         return int(load().prism_get_status(self._h, _stream(stream)))

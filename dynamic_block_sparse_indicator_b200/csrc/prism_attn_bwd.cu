@@ -567,6 +567,9 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     cudaMemsetAsync(dmax, 0, sizeof(uint32_t) * g.heads, s);
     const dim3 gmax(296, g.heads);
     const dim3 gpre((unsigned)((g.N + 7) / 8), g.heads);
+    P->launches += 4;
+    {
+    PrismProf prof(P, PRISM_STAGE_BWD_PRE, s);
     if (P->p.out_dtype == PRISM_F32) {
         k_bwd_absmax<float><<<gmax, 256, 0, s>>>((const float*)dO, dmax, g.N * HD);
         k_bwd_pre<float><<<gpre, 256, 0, s>>>((const float*)dO, (const float*)O, lse, src, dmax, dOp, lse_p,
@@ -575,6 +578,7 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
         k_bwd_absmax<__nv_bfloat16><<<gmax, 256, 0, s>>>((const __nv_bfloat16*)dO, dmax, g.N * HD);
         k_bwd_pre<__nv_bfloat16><<<gpre, 256, 0, s>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)O, lse,
                                                       src, dmax, dOp, lse_p, di_p, g.N, HD, err);
+    }
     }
     BwdArgs a{};
     a.src = src;
@@ -595,7 +599,10 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     const int sm1 = (int)sizeof(DkdvSmem<HD>) + 1024;
     if (cudaFuncSetAttribute(k_bwd_dkdv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    k_bwd_dkdv<HD><<<dim3(g.NT, g.heads), 192, sm1, s>>>(P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, a);
+    {
+        PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
+        k_bwd_dkdv<HD><<<dim3(g.NT, g.heads), 192, sm1, s>>>(P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, a);
+    }
     // dQ per query tile over the forward lists
     a.ptr = (const int*)(b + P->L.qt_ptr);
     a.ent = (const int*)(b + P->L.qt_ent);
@@ -604,7 +611,10 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     const int sm2 = (int)sizeof(DqSmem<HD>) + 1024;
     if (cudaFuncSetAttribute(k_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    k_bwd_dq<HD><<<dim3(g.NT, g.heads), 192, sm2, s>>>(P->tm_q, P->tm_do, P->tm_k64, P->tm_v64, a);
+    {
+        PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
+        k_bwd_dq<HD><<<dim3(g.NT, g.heads), 192, sm2, s>>>(P->tm_q, P->tm_do, P->tm_k64, P->tm_v64, a);
+    }
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 

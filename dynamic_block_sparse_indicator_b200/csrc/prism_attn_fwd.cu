@@ -305,7 +305,11 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
     const int smem = (int)sizeof(FwdSmem<HD>) + 1024;
     if (cudaFuncSetAttribute(k_attn_fwd<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
-    k_attn_fwd<HD><<<dim3(g.NT, g.heads), 192, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+    {
+        PrismProf prof(P, PRISM_STAGE_FWD, s);
+        k_attn_fwd<HD><<<dim3(g.NT, g.heads), 192, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+    }
+    P->launches += 1;
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 

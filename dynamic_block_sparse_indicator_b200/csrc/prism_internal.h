@@ -7,6 +7,9 @@
 #include "../../include/prism.h"
 
 #include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <vector>
 
 namespace prism {
 
@@ -60,6 +63,28 @@ struct prism_plan_s {
     int has_audio;
     CUtensorMap tm_q, tm_k, tm_v, tm_do;       // 2D [heads*N, D] fp16, 128-row boxes, 128B swizzle
     CUtensorMap tm_q64, tm_k64, tm_v64, tm_do64;  // the same with 64-row boxes
+    int64_t launches;                             // kernels launched so far
+    int profile;                                  // per-stage event timing on?
+    struct Timed { int stage; cudaEvent_t a, b; };
+    std::vector<Timed> timed;                     // pending event pairs
+};
+
+// Event pair around one launch when profiling is on.
+struct PrismProf {
+    prism_plan_s* P;
+    int stage;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    PrismProf(prism_plan_s* P_, int stage_, cudaStream_t s_) : P(P_), stage(stage_), s(s_) {
+        if (P->profile && cudaEventCreate(&a) == cudaSuccess && cudaEventCreate(&b) == cudaSuccess)
+            cudaEventRecord(a, s);
+    }
+    ~PrismProf() {
+        if (a && b) {
+            cudaEventRecord(b, s);
+            P->timed.push_back({stage, a, b});
+        }
+    }
 };
 
 // Internal entry points of the attention translation units.

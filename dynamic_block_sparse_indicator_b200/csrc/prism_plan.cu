@@ -1034,6 +1034,9 @@ static void launch_lists(prism_plan_s* P, const DevPlan& d, cudaStream_t s) {
 
 static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V, const float* amap,
                     const uint8_t* given_shapes, const uint32_t* given_sel, cudaStream_t s) {
+    // kernels launched below: audio 1-2, stats 1, finalize 1, gather 1, select (or
+    // mask + popcount) 1-2, lists 12
+    P->launches += (given_shapes ? 0 : (amap ? 3 : 2)) + 2 + (given_sel ? 2 : 1) + 12;
     const Geom& g = P->g;
     const prism_params& p = P->p;
     DevPlan d = dev_plan(P);
@@ -1183,7 +1186,42 @@ extern "C" int prism_get_status(prism_plan_t P, void* stream) {
     return e;
 }
 
-extern "C" void prism_plan_destroy(prism_plan_t P) { delete P; }
+static void drop_events(prism_plan_s* P) {
+    for (auto& t : P->timed) { cudaEventDestroy(t.a); cudaEventDestroy(t.b); }
+    P->timed.clear();
+}
+
+extern "C" void prism_plan_destroy(prism_plan_t P) {
+    if (!P) return;
+    drop_events(P);
+    delete P;
+}
+
+extern "C" int prism_profile_enable(prism_plan_t P, int on) {
+    if (!P) return PRISM_ERR_INVALID_ARG;
+    P->profile = on ? 1 : 0;
+    return PRISM_OK;
+}
+
+extern "C" int prism_profile_read(prism_plan_t P, float* ms, int* launches, void* stream) {
+    if (!P || !ms) return PRISM_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PRISM_ERR_CUDA;
+    for (int i = 0; i < PRISM_STAGE_COUNT; ++i) { ms[i] = 0.f; if (launches) launches[i] = 0; }
+    int st = PRISM_OK;
+    for (auto& t : P->timed) {
+        float e = 0.f;
+        if (cudaEventSynchronize(t.b) != cudaSuccess || cudaEventElapsedTime(&e, t.a, t.b) != cudaSuccess)
+            st = PRISM_ERR_CUDA;
+        if (t.stage >= 0 && t.stage < PRISM_STAGE_COUNT) {
+            ms[t.stage] += e;
+            if (launches) launches[t.stage] += 1;
+        }
+    }
+    drop_events(P);
+    return st;
+}
+
+extern "C" int64_t prism_launch_count(prism_plan_t P) { return P ? P->launches : 0; }
 
 extern "C" const char* prism_status_string(int st) {
     switch (st) {

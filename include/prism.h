@@ -195,6 +195,26 @@ PRISM_API void prism_plan_destroy(prism_plan_t plan);
 /* Static description of a status code. */
 PRISM_API const char* prism_status_string(int status);
 
+/* ---- profiling ---------------------------------------------------------- */
+/* Per-kernel CUDA-event timing of the attention launches (events recorded on
+ * the caller's stream around each launch). */
+#define PRISM_STAGE_FWD       0  /* k_attn_fwd                         */
+#define PRISM_STAGE_BWD_PRE   1  /* dO scaling, D_i, block-order dO     */
+#define PRISM_STAGE_BWD_DKDV  2  /* dK, dV per key tile                 */
+#define PRISM_STAGE_BWD_DQ    3  /* dQ per query tile                   */
+#define PRISM_STAGE_COUNT     4
+
+/* Turns per-stage timing on (1) or off (0) for later calls on this plan. */
+PRISM_API int prism_profile_enable(prism_plan_t plan, int on);
+
+/* Synchronises `stream`, writes the milliseconds spent per stage (and the
+ * number of launches per stage into `launches`, may be NULL) since the last
+ * read, and resets the accumulators.  ms has PRISM_STAGE_COUNT entries. */
+PRISM_API int prism_profile_read(prism_plan_t plan, float* ms, int* launches, void* stream);
+
+/* Number of kernels this plan has launched (plan, forward and backward). */
+PRISM_API int64_t prism_launch_count(prism_plan_t plan);
+
 /* Library version, e.g. "prism-b200 0.1 sm_100a". */
 PRISM_API const char* prism_version(void);
 

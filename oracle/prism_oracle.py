@@ -355,23 +355,29 @@ def attention_fwd(Q, K, V, src, starts, sel):
     return O, lse
 
 
+def block_grads(Q, K, V, dO, O, lse, src, starts, sel, i, dQ, dK, dV):
+    """Gradient contributions of query block i (float64, raster order):
+    dQ rows of the block, and its terms of dK, dV over the keys of S_i."""
+    D = Q.shape[1]
+    sc = 1.0 / np.sqrt(D)
+    qi = src[starts[i]:starts[i + 1]]
+    keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in sel[i]])
+    P = np.exp(Q[qi] @ K[keys].T * sc - lse[qi][:, None])
+    dV[keys] += P.T @ dO[qi]
+    dP = dO[qi] @ V[keys].T
+    Di = (dO[qi] * O[qi]).sum(axis=1, keepdims=True)
+    dS = P * (dP - Di)
+    dQ[qi] = dS @ K[keys] * sc
+    dK[keys] += dS.T @ Q[qi] * sc
+
+
 def attention_bwd(Q, K, V, dO, src, starts, sel):
     """dQ, dK, dV (float64, raster order): exact gradients with the selection fixed."""
     Q, K, V, dO = (np.asarray(x, np.float64) for x in (Q, K, V, dO))
-    D = Q.shape[1]
-    sc = 1.0 / np.sqrt(D)
     O, lse = attention_fwd(Q, K, V, src, starts, sel)
     dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
-    for i, js in enumerate(sel):
-        qi = src[starts[i]:starts[i + 1]]
-        keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in js])
-        P = np.exp(Q[qi] @ K[keys].T * sc - lse[qi][:, None])
-        dV[keys] += P.T @ dO[qi]
-        dP = dO[qi] @ V[keys].T
-        Di = (dO[qi] * O[qi]).sum(axis=1, keepdims=True)
-        dS = P * (dP - Di)
-        dQ[qi] = dS @ K[keys] * sc
-        dK[keys] += dS.T @ Q[qi] * sc
+    for i in range(len(sel)):
+        block_grads(Q, K, V, dO, O, lse, src, starts, sel, i, dQ, dK, dV)
     return dQ, dK, dV
 
 
