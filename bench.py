@@ -40,6 +40,8 @@ def args_():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["prism", "reference"], default="prism")
     ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--grid", type=int, nargs=3, default=None, metavar=("T", "H", "W"),
+                    help="override the grid (smaller cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="attention sample budget of the CPU oracle baseline")
@@ -222,6 +224,8 @@ def run_prism(a, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = syn.workload(a.workload)
+    if a.grid:
+        w = syn.workload(a.workload, T=a.grid[0], H=a.grid[1], W=a.grid[2])
     lib = _lib.load()
     need = a.warmup + a.steps
     heads = min(w.heads, need)
