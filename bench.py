@@ -50,6 +50,23 @@ def args_():
 
 
 # ----------------------------------------------------------------- helpers
+def head_order(rank, world, need, heads):
+    """The heads a rank processes, in order: `need` consecutive heads starting
+    at rank * need (mod heads), so ranks work on different heads while
+    rank * need < heads."""
+    return [(rank * need + i) % heads for i in range(need)]
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a per-rank float over all ranks (the job's time is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def selected_pairs(pl, head=0):
     """Pi = sum_i |B_i| * sum_{j in S_i} |B_j| of a plan (exported, host)."""
     import numpy as np
@@ -230,7 +247,7 @@ def run_prism(a, rank, world, local_rank):
     need = a.warmup + a.steps
     heads = min(w.heads, need)
     # this rank's heads: offsets by rank, so ranks work on different heads
-    order = [(rank * need + i) % w.heads for i in range(need)]
+    order = head_order(rank, world, need, w.heads)
     gen_heads = max(order) + 1
     Q, K, V = syn.make_qkv(w, device=dev, heads=gen_heads)
     dO = syn.make_dout(w, device=dev, heads=gen_heads, out_dtype=torch.bfloat16).float()
@@ -285,6 +302,7 @@ def run_prism(a, rank, world, local_rank):
         barrier()
     clocks = clk.summary()
     elapsed = e0.elapsed_time(e1)
+    elapsed_max = max_over_ranks(elapsed, world, dev)
     for pl in plans:
         for k, (ms, n) in pl.profile_read().items():
             stage_ms[k] += ms
@@ -295,10 +313,6 @@ def run_prism(a, rank, world, local_rank):
             raise RuntimeError(f"device status: {_lib.status_string(st)}")
     plan_ms = sum(a_.elapsed_time(b_) for a_, b_ in plan_ev)
     del plans, pl
-    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_max = float(t.item())
     # selected pairs of the timed heads (plans are deterministic: re-plan, untimed)
     pis = []
     for i in range(a.steps):
@@ -349,10 +363,8 @@ def run_prism(a, rank, world, local_rank):
             hlse.copy_(lse, non_blocking=True)
         x1.record()
         barrier()
-        te = torch.tensor([x0.elapsed_time(x1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": float(te.item()) / (a.e2e_steps * world), "unit": UNIT,
+        te = max_over_ranks(x0.elapsed_time(x1), world, dev)
+        e2e = {"value": te / (a.e2e_steps * world), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     # --------------------------------------------------- CPU oracle baseline
     cpu = None
