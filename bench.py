@@ -324,7 +324,11 @@ def run_prism(a, rank, world, local_rank):
     nb_mean = float(np.mean([p[1] for p in pis]))
     sel_mean = float(np.mean([p[2] for p in pis]))
     D = w.head_dim
-    flops = {"fwd": 4 * D * Pi, "bwd_dkdv": 8 * D * Pi, "bwd_dq": 2 * D * Pi}
+    # head_dim 128 folds dQ into the dK/dV kernel (10 D Pi there, the dQ stage is a
+    # scatter); head_dim 64 keeps a separate dQ kernel (8 D Pi + 2 D Pi)
+    fused = D == 128
+    flops = {"fwd": 4 * D * Pi, "bwd_dkdv": (10 if fused else 8) * D * Pi,
+             "bwd_dq": 0.0 if fused else 2 * D * Pi}
     pk = peaks()
     peak = pk.get("bf16_tflops_sustained") or 1400.0
     peak_src = "measured sustained bf16 (fp16 operands, same kind::f16 rate)" if pk else "fallback"
@@ -390,7 +394,7 @@ def run_prism(a, rank, world, local_rank):
               "plan_stats": {"blocks_per_head": nb_mean, "mean_selected_blocks": sel_mean,
                              "selected_pairs": Pi, "pair_density": Pi / float(w.N) ** 2},
               "roofline": {"kernel": {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv",
-                                      "bwd_dq": "k_bwd_dq"}[dom],
+                                      "bwd_dq": "k_dq_finalize" if fused else "k_bwd_dq"}[dom],
                            "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                            "frac": ach / peak, "peak_source": peak_src, "traffic": None},
               "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks})

@@ -9,7 +9,7 @@
 //   D_i = rowsum(dO o O);  P = exp(S/sqrt(d) - LSE);  dV = P^T dO;
 //   dP = dO V^T;  dS = P o (dP - D);  dK = dS^T Q / sqrt(d);  dQ = dS K / sqrt(d).
 //
-// Three kernels, no atomics (deterministic):
+// Kernels:
 //   k_bwd_absmax / k_bwd_pre   per row: D_i, dO in fp16 block order (scaled
 //               by an exact per-head power of two so that max |dO| lies in
 //               [0.5, 1): gradients of any magnitude keep fp16's precision and
@@ -19,9 +19,12 @@
 //               into TMEM (double-buffered), softmax warps form P^T and dS^T in
 //               fp16 shared memory, dV += P^T dO and dK += dS^T Q accumulate in
 //               TMEM.
-//   k_bwd_dq    one CTA per 128-row query tile; iterates the 64-key halves of
-//               the forward list; S = Q K^T, dP = dO V^T, dS -> shared memory,
-//               dQ += dS K in TMEM.
+//               For head_dim 128 the same CTA also forms dQ^T = K^T dS^T per
+//               unit and TMA reduce-adds it into an fp32 accumulator
+//               (k_dq_finalize scatters it to raster order).
+//   k_bwd_dq    (head_dim 64) one CTA per 128-row query tile; iterates the
+//               64-key halves of the forward list; S = Q K^T, dP = dO V^T,
+//               dS -> shared memory, dQ += dS K in TMEM.
 // Warp roles as in the forward: 0-3 softmax/epilogue (thread = TMEM lane),
 // 4 TMA producer + TMEM allocator, 5 MMA issuer.  All waits are bounded and
 // every TMEM access is warp-uniform.
@@ -173,7 +176,12 @@ __device__ __forceinline__ void zero_row(void* base, size_t row, int HD, int out
 }
 
 // ------------------------------------------------------------------- dK, dV
-template <int HD>
+// FUSE (head_dim 128): the same CTA also forms dQ^T = K^T dS^T for every
+// 64-query unit into the TMEM columns that S^T just vacated; a drain warpgroup
+// (warps 6-9) moves it through shared memory and TMA reduce-adds it into an
+// fp32 dQ accumulator in block order, so dQ costs one more MMA instead of a
+// second kernel that recomputes S and dP.
+template <int HD, bool FUSE>
 struct DkdvSmem {
     static constexpr int NSL = HD / 64;
     alignas(1024) uint8_t k[NSL][SLAB128];
@@ -182,21 +190,23 @@ struct DkdvSmem {
     alignas(1024) uint8_t dO[BWD_STAGES][NSL][SLAB64];
     alignas(1024) uint8_t p[2][SLAB128];      // P^T  [128 keys][64 queries]
     alignas(1024) uint8_t ds[2][SLAB128];     // dS^T [128 keys][64 queries]
+    alignas(1024) float stage_dq[FUSE ? 32 * HD : 4];   // [32 queries][HD] fp32
     alignas(16) float lse[BWD_STAGES][64];
     alignas(16) float di[BWD_STAGES][64];
     uint64_t bar_kv;
     uint64_t st_full[BWD_STAGES], st_empty[BWD_STAGES];
     uint64_t s_full[2], s_free[2], p_full[2], pd_done[2];
+    uint64_t dq_full[2], dq_free[2];
     uint32_t tmem_base;
 };
 
-template <int HD>
-__global__ void __launch_bounds__(192, 1)
+template <int HD, bool FUSE>
+__global__ void __launch_bounds__(FUSE ? 320 : 192, 1)
 k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
            const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
-           BwdArgs a) {
+           const __grid_constant__ CUtensorMap tm_dq, BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    DkdvSmem<HD>& sm = *reinterpret_cast<DkdvSmem<HD>*>(
+    DkdvSmem<HD, FUSE>& sm = *reinterpret_cast<DkdvSmem<HD, FUSE>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NSL = HD / 64;
     const int t = blockIdx.x, h = blockIdx.y;
@@ -205,8 +215,9 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     const int ne = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - e0;
     const int* ents = a.ent + (size_t)h * a.NT * a.NT + e0;
     const int U = count_units(ents, ne, 1);
-    // TMEM columns: S^T[b] at 64b, dP^T[b] at 128 + 64b, dV at 256, dK at 256 + HD
-    constexpr uint32_t TS = 0, TDP = 128, TDV = 256, TDK = 256 + HD;
+    // TMEM columns: buffer b = [128b, 128b + 128): S^T at 128b, dP^T at 128b + 64
+    // (dQ^T of the unit reuses the S^T columns); dV at 256, dK at 256 + HD.
+    constexpr uint32_t TDV = 256, TDK = 256 + HD;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_kv, 1);
@@ -216,6 +227,8 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             mbar_init(&sm.s_free[b], 128);
             mbar_init(&sm.p_full[b], 128);
             mbar_init(&sm.pd_done[b], 1);
+            mbar_init(&sm.dq_full[b], 1);
+            mbar_init(&sm.dq_free[b], 128);
         }
         mbar_fence_init();
     }
@@ -254,6 +267,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         if (lane == 0 && U > 0) {
             constexpr uint32_t id_s = idesc_f16(128, 64, 0, 0);
             constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
+            constexpr uint32_t id_dq = idesc_f16(128, 64, 1, 1);
             const uint32_t k_s = smem_u32(sm.k[0]), v_s = smem_u32(sm.v[0]);
             bool ok = mbar_wait(&sm.bar_kv, 0, a.err, 1501);
             for (int u = 0; ok && u <= U; ++u) {
@@ -261,16 +275,17 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     const int s = u % BWD_STAGES, b = u & 1;
                     if (!mbar_wait(&sm.st_full[s], (u / BWD_STAGES) & 1, a.err, 1502)) break;
                     if (u >= 2 && !mbar_wait(&sm.s_free[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
+                    if (FUSE && u >= 2 && !mbar_wait(&sm.dq_free[b], ((u - 2) >> 1) & 1, a.err, 1505)) break;
                     tc_fence_after();
                     const uint32_t q_s = smem_u32(sm.q[s][0]), do_s = smem_u32(sm.dO[s][0]);
                     #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + TS + 64 * b, desc_kmajor(k_s, kk, SLAB128),
-                                  desc_kmajor(q_s, kk, SLAB64), id_s, kk > 0);
+                        umma_f16(tmem + 128 * b, desc_kmajor(k_s, kk, SLAB128),
+                                 desc_kmajor(q_s, kk, SLAB64), id_s, kk > 0);
                     #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + TDP + 64 * b, desc_kmajor(v_s, kk, SLAB128),
-                                  desc_kmajor(do_s, kk, SLAB64), id_s, kk > 0);
+                        umma_f16(tmem + 128 * b + 64, desc_kmajor(v_s, kk, SLAB128),
+                                 desc_kmajor(do_s, kk, SLAB64), id_s, kk > 0);
                     umma_commit(&sm.s_full[b]);
                 }
                 if (u >= 1) {
@@ -282,17 +297,25 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16(tmem + TDV, desc_kmajor(p_s, kk, SLAB128), desc_mnmajor(do_s, kk, SLAB64),
-                                  id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
+                                 id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
                     #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16(tmem + TDK, desc_kmajor(ds_s, kk, SLAB128), desc_mnmajor(q_s, kk, SLAB64),
-                                  id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
+                                 id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
+                    if (FUSE) {
+                        // dQ^T [HD x 64 queries] = K^T [HD x 128 keys] . dS^T [128 keys x 64 queries]
+                        #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_f16(tmem + 128 * b, desc_mnmajor(k_s, kk, SLAB128),
+                                     desc_mnmajor(ds_s, kk, SLAB128), id_dq, kk > 0);
+                        umma_commit(&sm.dq_full[b]);
+                    }
                     umma_commit(&sm.pd_done[b]);
                     umma_commit(&sm.st_empty[s]);
                 }
             }
         }
-    } else {
+    } else if (warp < 4) {
         const int r = threadIdx.x;                  // key row of the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const int kh = r >> 6;                      // warp-uniform
@@ -306,10 +329,10 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full[s], (u / BWD_STAGES) & 1, a.err, 1002))) { ok = false; break; }
             tc_fence_after();
             uint32_t sv[64], dp[64];
-            PRISM_TMEM_LD32(tmem + lane_off + TS + 64 * b, sv);
-            PRISM_TMEM_LD32(tmem + lane_off + TS + 64 * b + 32, (sv + 32));
-            PRISM_TMEM_LD32(tmem + lane_off + TDP + 64 * b, dp);
-            PRISM_TMEM_LD32(tmem + lane_off + TDP + 64 * b + 32, (dp + 32));
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b, sv);
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 32, (sv + 32));
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64, dp);
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 96, (dp + 32));
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.s_free[b]);
@@ -364,11 +387,60 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             zero_row(a.out0, orow, HD, a.out_f32);
             zero_row(a.out1, orow, HD, a.out_f32);
         }
+    } else if (FUSE) {
+        // ---------------------------------------------- dQ drain (warps 6-9)
+        const int d = (warp & 3) * 32 + lane;       // head-dim row of dQ^T = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        HalfIter it{ents, ne, 0, 0, 1};
+        int r64, m2;
+        for (int u = 0; it.next(r64, m2); ++u) {
+            const int b = u & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.dq_full[b], (u >> 1) & 1, a.err, 3001))) break;
+            tc_fence_after();
+            uint32_t v[64];
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b, v);
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 32, (v + 32));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.dq_free[b]);
+            const int64_t qrow = hrow + (int64_t)r64 * 64;
+            #pragma unroll
+            for (int pass = 0; pass < 2; ++pass) {
+                if (leader) bulk_wait_read0();      // the previous reduce has read the stage
+                named_bar(1, 128);
+                #pragma unroll
+                for (int qq = 0; qq < 32; ++qq) sm.stage_dq[qq * HD + d] = __uint_as_float(v[pass * 32 + qq]);
+                fence_proxy_async_smem();
+                named_bar(1, 128);
+                if (leader) {
+                    tma_reduce_add_2d(&tm_dq, sm.stage_dq, 0, (int)(qrow + 32 * pass));
+                    bulk_commit();
+                }
+            }
+        }
+        if (leader) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 4) { __syncwarp(); tmem_dealloc(tmem, 512); }
+}
+
+// dQ accumulator (block order, fp32) -> dQ output (raster order, scaled).
+template <typename OT>
+__global__ void __launch_bounds__(256) k_dq_finalize(const float* __restrict__ acc, const int* __restrict__ src,
+                                                     const uint32_t* dmax, OT* __restrict__ dQ, int64_t N,
+                                                     int HD, float inv_sqrt_d, int* err) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t p = (int64_t)blockIdx.x * 8 + warp;
+    const int h = blockIdx.y;
+    if (p >= N) return;
+    const float mul = inv_sqrt_d * ldexpf(1.f, dscale_exp(dmax[h], err));
+    const int64_t n = src[(size_t)h * N + p];
+    const float* in = acc + ((size_t)h * N + p) * HD;
+    OT* out = dQ + ((size_t)h * N + n) * HD;
+    for (int c = lane; c < HD; c += 32) out[c] = (OT)(in[c] * mul);
 }
 
 // ------------------------------------------------------------------------ dQ
@@ -591,19 +663,33 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     a.scale_log2 = kLog2e / sqrtf((float)HD);
     a.inv_sqrt_d = 1.f / sqrtf((float)HD);
     a.err = err;
-    // dK, dV per key tile over the transposed lists
+    // dK, dV (and for head_dim 128 dQ) per key tile over the transposed lists
+    constexpr bool FUSE = HD == 128;
     a.ptr = (const int*)(b + P->L.kt_ptr);
     a.ent = (const int*)(b + P->L.kt_ent);
     a.out0 = dK;
     a.out1 = dV;
-    const int sm1 = (int)sizeof(DkdvSmem<HD>) + 1024;
-    if (cudaFuncSetAttribute(k_bwd_dkdv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1) != cudaSuccess)
+    float* dq_acc = (float*)(b + P->L.dq_acc);
+    if (FUSE) cudaMemsetAsync(dq_acc, 0, sizeof(float) * (size_t)g.heads * g.N * HD, s);
+    const int sm1 = (int)sizeof(DkdvSmem<HD, FUSE>) + 1024;
+    if (cudaFuncSetAttribute(k_bwd_dkdv<HD, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1) != cudaSuccess)
         return PRISM_ERR_CUDA;
     {
         PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
-        k_bwd_dkdv<HD><<<dim3(g.NT, g.heads), 192, sm1, s>>>(P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, a);
+        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, g.heads), FUSE ? 320 : 192, sm1, s>>>(
+            P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, a);
     }
-    // dQ per query tile over the forward lists
+    if (FUSE) {
+        PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
+        const dim3 gfin((unsigned)((g.N + 7) / 8), g.heads);
+        if (a.out_f32)
+            k_dq_finalize<float><<<gfin, 256, 0, s>>>(dq_acc, src, dmax, (float*)dQ, g.N, HD, a.inv_sqrt_d, err);
+        else
+            k_dq_finalize<__nv_bfloat16><<<gfin, 256, 0, s>>>(dq_acc, src, dmax, (__nv_bfloat16*)dQ, g.N, HD,
+                                                              a.inv_sqrt_d, err);
+        return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+    }
+    // dQ per query tile over the forward lists (head_dim 64)
     a.ptr = (const int*)(b + P->L.qt_ptr);
     a.ent = (const int*)(b + P->L.qt_ent);
     a.out0 = dQ;

@@ -86,6 +86,7 @@ Layout make_layout(const Geom& g) {
     L.lse_p = take(sizeof(float) * H * N);
     L.di_p = take(sizeof(float) * H * N);
     L.dmax = take(sizeof(uint32_t) * H);
+    L.dq_acc = take(sizeof(float) * H * N * g.D);
     L.total = off;
     return L;
 }
@@ -952,6 +953,19 @@ static int make_tmap(CUtensorMap* m, void* base, int64_t rows, int D, int box_ro
     return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
+static int make_tmap_f32(CUtensorMap* m, void* base, int64_t rows, int D, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return PRISM_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+    cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
 static int check_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_UNSUPPORTED;
@@ -993,6 +1007,7 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
     if (!st) st = make_tmap(&P->tm_k64, P->ws + L.kp, rows, g.D, 64);
     if (!st) st = make_tmap(&P->tm_v64, P->ws + L.vp, rows, g.D, 64);
     if (!st) st = make_tmap(&P->tm_do64, P->ws + L.dop, rows, g.D, 64);
+    if (!st) st = make_tmap_f32(&P->tm_dq, P->ws + L.dq_acc, rows, g.D, 32);
     if (st) { delete P; return st; }
     *outP = P;
     return PRISM_OK;
