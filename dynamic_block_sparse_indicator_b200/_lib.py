@@ -21,6 +21,7 @@ PRISM_ERR_CUDA = 3
 PRISM_ERR_TIMEOUT = 4
 PRISM_ERR_DEVICE_CHECK = 5
 PRISM_ERR_UNSUPPORTED = 6
+PRISM_ERR_SCRATCH_LIMIT = 7
 
 PRISM_BF16 = 0
 PRISM_F32 = 1
@@ -77,6 +78,7 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_profile_enable": (i32, [vp, i32]),
         "prism_profile_read": (i32, [vp, C.POINTER(C.c_float), C.POINTER(C.c_int), vp]),
         "prism_launch_count": (C.c_int64, [vp]),
+        "prism_zone_shapes_noalloc": (i32, [pp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

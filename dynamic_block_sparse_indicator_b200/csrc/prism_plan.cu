@@ -1247,6 +1247,7 @@ extern "C" const char* prism_status_string(int st) {
         case PRISM_ERR_TIMEOUT: return "device wait timed out";
         case PRISM_ERR_DEVICE_CHECK: return "device-side check failed";
         case PRISM_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
+        case PRISM_ERR_SCRATCH_LIMIT: return "problem larger than the no-allocation entry point's static scratch";
         default: return "unknown status";
     }
 }
@@ -1266,4 +1267,127 @@ extern "C" int prism_attn_bwd(prism_plan_t P, const void* dO, const void* O, con
         !aligned16(dV))
         return PRISM_ERR_INVALID_ARG;
     return prism_launch_attn_bwd(P, dO, O, lse, dQ, dK, dV, stream);
+}
+
+// ====================================================== no-allocation stage 1
+// Some callers cannot allocate device memory at all: a plugin that lives inside
+// another engine's fixed memory plan and may only use the buffers it is handed,
+// code on a latency-critical path where cudaMalloc's implicit device
+// synchronisation is not acceptable, or a deployment whose device memory budget
+// is fixed up front.  For them stage 1 (zone statistics -> block volume ->
+// shape) runs with its intermediates in this file-scope device array instead
+// of a caller workspace.  Every GPU that loads the library holds the array
+// until the process exits.
+namespace prism {
+
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;   // 4 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// Floats of scratch used for (Nz zones, heads): audio zone means (fp64), a_bar,
+// v_hat and the per-head zone statistics, each region 256-byte aligned.
+static size_t noalloc_floats(int Nz, int heads, size_t* off_abar, size_t* off_vhat, size_t* off_zstat) {
+    auto up = [](size_t f) { return (f + 63) & ~size_t(63); };
+    size_t o = up(2 * (size_t)Nz);
+    *off_abar = o;
+    o = up(o + Nz);
+    *off_vhat = o;
+    o = up(o + 3 * (size_t)Nz);
+    *off_zstat = o;
+    return o + 4 * (size_t)Nz * heads;
+}
+
+// Variant of k_zone_finalize that stops at the shapes: shape id per zone and
+// the head's block count, no block offsets.
+__global__ void __launch_bounds__(1024) k_zone_shapes_static(DevPlan d, float eps, float tau128, float tau256,
+                                                             uint8_t* __restrict__ sid_out,
+                                                             int* __restrict__ nblocks_out) {
+    __shared__ float redf[32];
+    __shared__ int redi[32];
+    const int h = blockIdx.x;
+    const float* zs = d.zstat + (size_t)h * d.Nz * 4;
+    float mx = 0.f;
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) mx = fmaxf(mx, zs[m * 4 + 3]);
+    mx = block_max<1024>(mx, redf);
+    int blocks = 0;
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+        const float rho = mx > 0.f ? __fdiv_rn(zs[m * 4 + 3], mx) : 0.f;
+        const int vol = rho < tau256 ? 256 : (rho < tau128 ? 128 : 64);
+        const float s0 = zs[m * 4], s1 = zs[m * 4 + 1], s2 = zs[m * 4 + 2];
+        const float tot = __fadd_rn(__fadd_rn(s0, s1), s2);
+        float r[3];
+        if (tot > 0.f) { r[0] = __fdiv_rn(s0, tot); r[1] = __fdiv_rn(s1, tot); r[2] = __fdiv_rn(s2, tot); }
+        else { r[0] = r[1] = r[2] = 1.f / 3.f; }
+        const float ab = d.abar[m];
+        float g[3];
+        #pragma unroll
+        for (int ax = 0; ax < 3; ++ax)
+            g[ax] = __fadd_rn(__fadd_rn(r[ax], __fmul_rn(ab, d.vhat[3 * m + ax])), eps);
+        sid_out[(size_t)h * d.Nz + m] = (uint8_t)snap_shape(g, vol);
+        blocks += 512 / vol;
+    }
+    blocks = block_sum_int<1024>(blocks, redi);
+    if (threadIdx.x == 0) nblocks_out[h] = blocks;
+}
+
+template <typename T, int D>
+static void noalloc_stats(const Geom& g, const DevPlan& d, const void* V, cudaStream_t s) {
+    const int sm = (256 / (D / 2)) * D * 26 * (int)sizeof(float);
+    cudaFuncSetAttribute(k_zone_stats<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    k_zone_stats<T, D><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V);
+}
+
+// Device address of the scratch array, looked up once per device (with that
+// device current) the first time the entry point runs on it.
+static float* noalloc_scratch_ptr(int dev) {
+    static float* ptrs[64] = {};
+    if (dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<float*>(p);
+    }
+    return ptrs[dev];
+}
+
+}  // namespace prism
+
+extern "C" int prism_zone_shapes_noalloc(const prism_params* p, const void* V, const float* a_map,
+                                         uint8_t* shape_id, int32_t* nblocks, void* stream) {
+    using namespace prism;
+    int st = validate_params(p);
+    if (st) return st;
+    if (!V || !shape_id || !nblocks || !aligned16(V) || (a_map && !aligned16(a_map)))
+        return PRISM_ERR_INVALID_ARG;
+    st = check_device();
+    if (st) return st;
+    const Geom g = make_geom(p);
+    size_t o_abar, o_vhat, o_zstat;
+    if (noalloc_floats(g.Nz, g.heads, &o_abar, &o_vhat, &o_zstat) > kNoAllocScratchFloats)
+        return PRISM_ERR_SCRATCH_LIMIT;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+    float* base = noalloc_scratch_ptr(dev);
+    if (!base) return PRISM_ERR_CUDA;
+    DevPlan d{};
+    d.T = g.T; d.H = g.H; d.W = g.W; d.heads = g.heads; d.D = g.D; d.Zh = g.Zh; d.Zw = g.Zw;
+    d.Nz = g.Nz; d.N = g.N;
+    d.araw = reinterpret_cast<double*>(base);
+    d.abar = base + o_abar;
+    d.vhat = base + o_vhat;
+    d.zstat = base + o_zstat;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // every scratch value below is written before it is read: nothing to clear
+    if (a_map) {
+        k_audio_zone<<<g.Nz, 256, 0, s>>>(d, a_map);
+        k_audio_norm<<<1, 1024, 0, s>>>(d);
+    } else {
+        k_audio_none<<<(g.Nz + 255) / 256, 256, 0, s>>>(d);
+    }
+    const bool bf = p->dtype == PRISM_BF16;
+    if (bf && g.D == 128) noalloc_stats<__nv_bfloat16, 128>(g, d, V, s);
+    else if (bf) noalloc_stats<__nv_bfloat16, 64>(g, d, V, s);
+    else if (g.D == 128) noalloc_stats<float, 128>(g, d, V, s);
+    else noalloc_stats<float, 64>(g, d, V, s);
+    k_zone_shapes_static<<<g.heads, 1024, 0, s>>>(d, p->eps, p->tau128, p->tau256, shape_id, nblocks);
+    return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }

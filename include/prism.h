@@ -54,6 +54,7 @@ extern "C" {
 #define PRISM_ERR_TIMEOUT      4  /* a bounded device-side wait gave up; kernel returned */
 #define PRISM_ERR_DEVICE_CHECK 5  /* a device-side bounds/consistency check failed */
 #define PRISM_ERR_UNSUPPORTED  6  /* no sm_100 device, or the build lacks the kernels */
+#define PRISM_ERR_SCRATCH_LIMIT 7 /* too large for prism_zone_shapes_noalloc's static scratch */
 
 /* Element types (prism_params.dtype / out_dtype). */
 #define PRISM_BF16 0
@@ -162,6 +163,33 @@ PRISM_API int prism_attn_fwd(prism_plan_t plan, void* O, float* lse, void* strea
  */
 PRISM_API int prism_attn_bwd(prism_plan_t plan, const void* dO, const void* O, const float* lse,
                    void* dQ, void* dK, void* dV, void* stream);
+
+/*
+ * prism_zone_shapes_noalloc -- stage 1 alone (zone statistics, block volume,
+ *   snapped shape) for callers that cannot allocate device memory: a plugin
+ *   that may only use the buffers another engine's memory plan hands it, a
+ *   latency-critical path where cudaMalloc's implicit device synchronisation
+ *   is not acceptable, or a deployment whose device memory is budgeted up
+ *   front.  The paper has no counterpart: it is a packaging of prism_plan's
+ *   first stage, computing the same shape ids and block counts.
+ *   Inputs as for prism_plan (V device [heads][N][head_dim] of `dtype`; a_map
+ *   device fp32 [T][H][W] or NULL).  Outputs (device, caller-allocated):
+ *     shape_id  uint8 [heads][Nz], the candidate index per zone and head;
+ *     nblocks   int32 [heads], blocks of the head (sum over zones of 512 / B).
+ *   Scratch: a file-scope static device array of 4 MiB (2^20 floats) that
+ *   every GPU loading the library holds until the process exits.  Its use is
+ *   2*Nz + Nz + 3*Nz + 4*heads*Nz floats (each part rounded up to 64 floats);
+ *   larger problems return PRISM_ERR_SCRATCH_LIMIT (the 2K layer, Nz = 1,980,
+ *   fits up to 130 heads).  No allocation of any kind is made.
+ *   The first call on a device looks the array's device address up (one
+ *   cudaGetSymbolAddress with that device current); make that first call
+ *   before any stream capture.  Every call shares the one array and leaves its
+ *   contents behind; each value is written before it is read, so nothing needs
+ *   clearing, but calls whose kernels overlap on the GPU (other streams, other
+ *   host threads) race on it and must be serialised by the caller.
+ */
+PRISM_API int prism_zone_shapes_noalloc(const prism_params* p, const void* V, const float* a_map,
+                                        uint8_t* shape_id, int32_t* nblocks, void* stream);
 
 /* ---- inspection -------------------------------------------------------- */
 #define PRISM_ITEM_SHAPE_ID   0  /* uint8  [heads][Nz]                         */
