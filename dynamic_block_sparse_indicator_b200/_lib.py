@@ -56,7 +56,7 @@ def load(path: str | None = None) -> C.CDLL:
     global _lib
     if _lib is not None:
         return _lib
-    p = path or LIB_PATH
+    p = path or os.environ.get("PRISM_LIB") or LIB_PATH
     if not os.path.exists(p):
         raise ImportError(f"libprism.so not built at {p}: run "
                           "`python -m dynamic_block_sparse_indicator_b200.build`")
