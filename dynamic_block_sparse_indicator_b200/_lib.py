@@ -72,6 +72,8 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_plan_item_bytes": (sz, [vp, i32]),
         "prism_plan_export": (i32, [vp, i32, vp, sz, vp]),
         "prism_get_status": (i32, [vp, vp]),
+        "prism_get_status_ex": (i32, [vp, C.POINTER(C.c_int32), vp]),
+        "prism_selftest_timeout": (i32, [vp, vp]),
         "prism_plan_destroy": (None, [vp]),
         "prism_status_string": (C.c_char_p, [i32]),
         "prism_version": (C.c_char_p, []),
@@ -197,6 +199,17 @@ class Plan:
 
     def status(self, stream=None) -> int:
         return int(load().prism_get_status(self._h, _stream(stream)))
+
+    def status_ex(self, stream=None):
+        """(status, site of a timed-out wait) -- synchronises and clears."""
+        site = C.c_int32(0)
+        st = load().prism_get_status_ex(self._h, C.byref(site), _stream(stream))
+        return int(st), int(site.value)
+
+    def selftest_timeout(self, stream=None):
+        st = load().prism_selftest_timeout(self._h, _stream(stream))
+        if st:
+            raise PrismError(st, "prism_selftest_timeout")
 
 
 def _check_inputs(Q, K, V, params):

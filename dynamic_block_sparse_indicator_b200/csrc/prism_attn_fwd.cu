@@ -287,6 +287,19 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
 }
 
+// Failure-detection self-test: one thread waits on an mbarrier that nothing
+// ever arrives at.  The bounded wait gives up after kWaitNs, records
+// PRISM_ERR_TIMEOUT (site 9001) in the error word and the kernel returns.
+__global__ void k_selftest_wait(int* err) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, err, 9001);
+}
+
 template <int HD>
 static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
     const Geom& g = P->g;
@@ -314,6 +327,12 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
 }
 
 }  // namespace prism
+
+int prism_launch_selftest_wait(prism_plan_s* P, void* stream) {
+    prism::k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((int*)(P->ws + P->L.err));
+    P->launches += 1;
+    return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
 
 int prism_launch_attn_fwd(prism_plan_s* P, void* O, float* lse, void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

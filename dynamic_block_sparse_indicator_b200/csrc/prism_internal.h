@@ -91,5 +91,6 @@ struct PrismProf {
 
 // Internal entry points of the attention translation units.
 int prism_launch_attn_fwd(prism_plan_s* P, void* O, float* lse, void* stream);
+int prism_launch_selftest_wait(prism_plan_s* P, void* stream);
 int prism_launch_attn_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse,
                           void* dQ, void* dK, void* dV, void* stream);

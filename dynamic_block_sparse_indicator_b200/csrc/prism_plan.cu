@@ -1189,16 +1189,21 @@ extern "C" int prism_plan_export(prism_plan_t P, int item, void* host_dst, size_
 }
 
 extern "C" int prism_get_status(prism_plan_t P, void* stream) {
+    return prism_get_status_ex(P, nullptr, stream);
+}
+
+extern "C" int prism_get_status_ex(prism_plan_t P, int32_t* site, void* stream) {
     if (!P) return PRISM_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
-    int e = 0;
-    if (cudaMemcpy(&e, P->ws + P->L.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PRISM_ERR_CUDA;
-    if (e) {
-        const int zero = 0;
-        cudaMemcpy(P->ws + P->L.err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    int e[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(e, P->ws + P->L.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return PRISM_ERR_CUDA;
+    if (site) *site = e[0] ? e[1] : 0;
+    if (e[0]) {
+        const int zero[4] = {0, 0, 0, 0};
+        cudaMemcpy(P->ws + P->L.err, zero, sizeof(zero), cudaMemcpyHostToDevice);
     }
-    return e;
+    return e[0];
 }
 
 static void drop_events(prism_plan_s* P) {
@@ -1234,6 +1239,11 @@ extern "C" int prism_profile_read(prism_plan_t P, float* ms, int* launches, void
     }
     drop_events(P);
     return st;
+}
+
+extern "C" int prism_selftest_timeout(prism_plan_t P, void* stream) {
+    if (!P) return PRISM_ERR_INVALID_ARG;
+    return prism_launch_selftest_wait(P, stream);
 }
 
 extern "C" int64_t prism_launch_count(prism_plan_t P) { return P ? P->launches : 0; }

@@ -217,6 +217,17 @@ PRISM_API int prism_plan_export(prism_plan_t plan, int item, void* host_dst, siz
  * PRISM_OK, PRISM_ERR_TIMEOUT or PRISM_ERR_DEVICE_CHECK (or PRISM_ERR_CUDA). */
 PRISM_API int prism_get_status(prism_plan_t plan, void* stream);
 
+/* As prism_get_status, and writes the site of a timed-out wait (an id of the
+ * kernel role and barrier, 0 if none) into *site when site is not NULL. */
+PRISM_API int prism_get_status_ex(prism_plan_t plan, int32_t* site, void* stream);
+
+/* Failure-detection self-test: launches one thread that waits on a barrier
+ * nothing ever arrives at.  The bounded device wait gives up after about a
+ * second, records PRISM_ERR_TIMEOUT (site 9001) in the plan's error word and
+ * the kernel returns; the next prism_get_status reports it.  No fault and no
+ * hang: the context stays usable. */
+PRISM_API int prism_selftest_timeout(prism_plan_t plan, void* stream);
+
 /* Frees the host handle (the workspace stays the caller's). */
 PRISM_API void prism_plan_destroy(prism_plan_t plan);
 

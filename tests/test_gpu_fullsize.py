@@ -1,0 +1,88 @@
+"""Parity at the full 1M-token size, in the launch configuration bench.py times.
+
+The 2K training layer (grid 72x88x160, 1,013,760 tokens, head_dim 128, bf16,
+Top-k 16, Top-p 0.9), one head planned at a time, fp32 outputs:
+  * the plan (shapes, block offsets, permutation, every selected set) against
+    the oracle's full plan of the head, with the near-tie rules;
+  * O, LSE and dQ on sampled query rows against the oracle row by row;
+  * dV and dK through identities that hold at any size: the rows of dV sum to
+    the rows of dO (each row's softmax weights sum to one) and the rows of dK
+    sum to zero (each query row's dS sums to zero).
+"""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from dynamic_block_sparse_indicator_b200 import _lib
+from dynamic_block_sparse_indicator_b200 import synthetic as syn
+from oracle import prism_oracle as po
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def run(cuda_device):
+    w = syn.workload(3)
+    Q, K, V = syn.make_qkv(w, device="cuda", heads=1)
+    dO = syn.make_dout(w, device="cuda", heads=1, out_dtype=torch.bfloat16).float()
+    a = syn.make_amap(w, device="cuda")
+    p = _lib.make_params(w.T, w.H, w.W, 1, w.head_dim, _lib.PRISM_BF16, w.top_k, w.top_p, w.eps)
+    pl = _lib.plan(Q, K, V, a, p)
+    O, lse = pl.attn_fwd()
+    dQ, dK, dV = pl.attn_bwd(dO, O, lse)
+    torch.cuda.synchronize()
+    assert pl.status() == _lib.PRISM_OK
+    host = lambda t: t[0].double().cpu().numpy()
+    q, k, v, g = host(Q), host(K), host(V), host(dO)
+    orc = po.plan_head(q, k, v, a.cpu().numpy(), w.T, w.H, w.W, w.top_k, w.top_p, w.eps)
+    return dict(w=w, pl=pl, q=q, k=k, v=v, g=g, orc=orc, O=host(O), lse=lse[0].double().cpu().numpy(),
+                dQ=host(dQ), dK=host(dK), dV=host(dV))
+
+
+def test_fullsize_plan(run):
+    w, pl, o = run["w"], run["pl"], run["orc"]
+    NB, WORDS = w.N // 64, (w.N // 64 + 31) // 32
+    ok, tie, bad = parity.shapes_agree(pl.export("shape_id"), o["stats"])
+    assert not bad
+    if tie:
+        pytest.skip(f"accepted near-tie shapes in zones {tie}: downstream stages differ legitimately")
+    nb = len(o["starts"]) - 1
+    assert pl.export("nblocks")[0] == nb
+    np.testing.assert_array_equal(pl.export("blk_start")[:nb + 1], o["starts"])
+    np.testing.assert_array_equal(pl.export("src"), o["src"])
+    gsets = parity.bits_to_sets(pl.export("sel_bits").reshape(NB, WORDS), nb, WORDS)
+    exact = 0
+    for i in range(nb):
+        assert parity.selection_agrees(gsets[i], o["logits"][i], o["P"][i], w.top_k, w.top_p), i
+        exact += np.array_equal(gsets[i], o["sel"][i])
+    assert exact >= 0.99 * nb
+    run["gsets"] = gsets
+
+
+def test_fullsize_sampled_rows(run):
+    o = run["orc"]
+    gsets = run.get("gsets")
+    if gsets is None:
+        pytest.skip("plan comparison did not run")
+    nb = len(o["starts"]) - 1
+    rng = np.random.default_rng(3)
+    blocks = [i for i in rng.permutation(nb) if np.array_equal(gsets[i], o["sel"][i])][:6]
+    rows = np.array([o["src"][o["starts"][i] + int(rng.integers(o["starts"][i + 1] - o["starts"][i]))]
+                     for i in blocks])
+    Oo, lo, dQo = po.attention_rows(run["q"], run["k"], run["v"], o["src"], o["starts"], o["sel"], rows,
+                                    dO=run["g"])
+    for got, want, nm in ((run["O"][rows], Oo, "O"), (run["dQ"][rows], dQo, "dQ")):
+        good, rl2, ma = parity.close(got, want)
+        assert good, f"{nm}: relL2 {rl2:.2e} maxabs {ma:.2e}"
+    np.testing.assert_allclose(run["lse"][rows], lo, atol=2e-2, rtol=1e-3)
+
+
+def test_fullsize_gradient_identities(run):
+    dV, dK, g = run["dV"], run["dK"], run["g"]
+    sv = dV.sum(axis=0)
+    sg = g.sum(axis=0)
+    scale = np.abs(dV).sum(axis=0)
+    assert np.all(np.abs(sv - sg) <= 1e-3 * scale + 1e-3)
+    sk = dK.sum(axis=0)
+    assert np.all(np.abs(sk) <= 1e-3 * np.abs(dK).sum(axis=0) + 1e-3)
