@@ -42,6 +42,7 @@ constexpr int BWD_STAGES = 2;
 constexpr int SLAB128 = 128 * 128;   // bytes: 128 rows x 64 fp16
 constexpr int SLAB64 = 64 * 128;     // bytes:  64 rows x 64 fp16
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kPScale = 32768.f;          // 2^15: scale of the P operand of dV += P^T dO
 
 // --------------------------------------------------------------- preprocess
 template <typename OT>
@@ -356,7 +357,9 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                         d0 = p0 * (__uint_as_float(dp[c]) - dq[c]);
                         d1 = p1 * (__uint_as_float(dp[c + 1]) - dq[c + 1]);
                     }
-                    wp[e] = pack_f16(p0, p1);
+                    // the dV operand is 2^15 P (normal in fp16 down to P = 2^-29);
+                    // dV is unscaled in the epilogue
+                    wp[e] = pack_f16(p0 * kPScale, p1 * kPScale);
                     wd[e] = pack_f16(d0, d1);
                 }
                 st_shared_v4(p_s + swz128(r, ch), wp[0], wp[1], wp[2], wp[3]);
@@ -378,7 +381,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 uint32_t o[32];
                 PRISM_TMEM_LD32(tmem + lane_off + TDV + 32 * c, o);
                 tmem_wait_ld();
-                store_row(a.out1, orow, HD, 32 * c, o, unscale, a.out_f32);
+                store_row(a.out1, orow, HD, 32 * c, o, unscale / kPScale, a.out_f32);
                 PRISM_TMEM_LD32(tmem + lane_off + TDK + 32 * c, o);
                 tmem_wait_ld();
                 store_row(a.out0, orow, HD, 32 * c, o, a.inv_sqrt_d * unscale, a.out_f32);
