@@ -16,9 +16,9 @@
 //               dS cannot overflow), LSE in block order.
 //   k_bwd_dkdv  one CTA per 128-key tile; iterates the 64-row query halves of
 //               the key tile's transposed list; S^T = K Q^T and dP^T = V dO^T
-//               into TMEM (double-buffered), softmax warps form P^T and dS^T in
-//               fp16 shared memory, dV += P^T dO and dK += dS^T Q accumulate in
-//               TMEM.
+//               into TMEM (double-buffered), softmax warps form P^T (into TMEM, over
+//               dP^T) and dS^T (fp16 shared memory), dV += P^T dO and
+//               dK += dS^T Q accumulate in TMEM.
 //               For head_dim 128 the same CTA also forms dQ^T = K^T dS^T per
 //               unit and TMA reduce-adds it into an fp32 accumulator
 //               (k_dq_finalize scatters it to raster order).
@@ -39,6 +39,7 @@
 namespace prism {
 
 constexpr int BWD_STAGES = 2;
+constexpr int DKDV_STAGES = 3;   // Q/dO prefetch depth of the dK/dV kernel
 constexpr int SLAB128 = 128 * 128;   // bytes: 128 rows x 64 fp16
 constexpr int SLAB64 = 64 * 128;     // bytes:  64 rows x 64 fp16
 constexpr float kLog2e = 1.4426950408889634f;
@@ -179,7 +180,7 @@ __device__ __forceinline__ void zero_row(void* base, size_t row, int HD, int out
 // ------------------------------------------------------------------- dK, dV
 // FUSE (head_dim 128): the same CTA also forms dQ^T = K^T dS^T for every
 // 64-query unit into the TMEM columns that S^T just vacated; a drain warpgroup
-// (warps 6-9) moves it through shared memory and TMA reduce-adds it into an
+// (warps 10-13) moves it through shared memory and TMA reduce-adds it into an
 // fp32 dQ accumulator in block order, so dQ costs one more MMA instead of a
 // second kernel that recomputes S and dP.
 template <int HD, bool FUSE>
@@ -187,22 +188,21 @@ struct DkdvSmem {
     static constexpr int NSL = HD / 64;
     alignas(1024) uint8_t k[NSL][SLAB128];
     alignas(1024) uint8_t v[NSL][SLAB128];
-    alignas(1024) uint8_t q[BWD_STAGES][NSL][SLAB64];
-    alignas(1024) uint8_t dO[BWD_STAGES][NSL][SLAB64];
-    alignas(1024) uint8_t p[2][SLAB128];      // P^T  [128 keys][64 queries]
-    alignas(1024) uint8_t ds[2][SLAB128];     // dS^T [128 keys][64 queries]
+    alignas(1024) uint8_t q[DKDV_STAGES][NSL][SLAB64];
+    alignas(1024) uint8_t dO[DKDV_STAGES][NSL][SLAB64];
+    alignas(1024) uint8_t ds[2][SLAB128];     // dS^T [128 keys][64 queries] (P^T lives in TMEM)
     alignas(1024) float stage_dq[FUSE ? 32 * HD : 4];   // [32 queries][HD] fp32
-    alignas(16) float lse[BWD_STAGES][64];
-    alignas(16) float di[BWD_STAGES][64];
+    alignas(16) float lse[DKDV_STAGES][64];
+    alignas(16) float di[DKDV_STAGES][64];
     uint64_t bar_kv;
-    uint64_t st_full[BWD_STAGES], st_empty[BWD_STAGES];
+    uint64_t st_full[DKDV_STAGES], st_empty[DKDV_STAGES];
     uint64_t s_full[2], s_free[2], p_full[2], pd_done[2];
     uint64_t dq_full[2], dq_free[2];
     uint32_t tmem_base;
 };
 
 template <int HD, bool FUSE>
-__global__ void __launch_bounds__(FUSE ? 320 : 192, 1)
+__global__ void __launch_bounds__(FUSE ? 448 : 320, 1)
 k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
            const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
            const __grid_constant__ CUtensorMap tm_dq, BwdArgs a) {
@@ -222,25 +222,29 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_kv, 1);
-        for (int s = 0; s < BWD_STAGES; ++s) { mbar_init(&sm.st_full[s], 1); mbar_init(&sm.st_empty[s], 1); }
+        for (int s = 0; s < DKDV_STAGES; ++s) { mbar_init(&sm.st_full[s], 1); mbar_init(&sm.st_empty[s], 1); }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.s_free[b], 128);
-            mbar_init(&sm.p_full[b], 128);
+            mbar_init(&sm.s_free[b], 256);
+            mbar_init(&sm.p_full[b], 256);
             mbar_init(&sm.pd_done[b], 1);
             mbar_init(&sm.dq_full[b], 1);
             mbar_init(&sm.dq_free[b], 128);
         }
         mbar_fence_init();
     }
-    if (warp == 4) { __syncwarp(); tmem_alloc(&sm.tmem_base, 512); }
+    // warps 0-7: two softmax warpgroups (same 128 key rows, one 32-query half of
+    // the unit each); warp 8: TMA producer + TMEM allocator; warp 9: MMA issuer;
+    // warps 10-13 (FUSE): dQ drain.
+    constexpr int W_PROD = 8, W_MMA = 9;
+    if (warp == W_PROD) { __syncwarp(); tmem_alloc(&sm.tmem_base, 512); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int64_t hrow = (int64_t)h * a.N;
 
-    if (warp == 4) {
+    if (warp == W_PROD) {
         if (lane == 0 && U > 0) {
             const int krow = (int)(hrow + (int64_t)t * 128);
             mbar_expect_tx(&sm.bar_kv, 2 * NSL * SLAB128);
@@ -251,9 +255,9 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             HalfIter it{ents, ne, 0, 0, 1};
             int r64, m2;
             for (int u = 0; it.next(r64, m2); ++u) {
-                const int s = u % BWD_STAGES;
-                if (u >= BWD_STAGES &&
-                    !mbar_wait(&sm.st_empty[s], ((u / BWD_STAGES) - 1) & 1, a.err, 1401)) break;
+                const int s = u % DKDV_STAGES;
+                if (u >= DKDV_STAGES &&
+                    !mbar_wait(&sm.st_empty[s], ((u / DKDV_STAGES) - 1) & 1, a.err, 1401)) break;
                 const int64_t qrow = hrow + (int64_t)r64 * 64;
                 mbar_expect_tx(&sm.st_full[s], 2 * NSL * SLAB64 + 2 * 256);
                 for (int c = 0; c < NSL; ++c) {
@@ -264,7 +268,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 bulk_load(sm.di[s], a.di_p + qrow, 256, &sm.st_full[s]);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == W_MMA) {
         if (lane == 0 && U > 0) {
             constexpr uint32_t id_s = idesc_f16(128, 64, 0, 0);
             constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
@@ -273,8 +277,8 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             bool ok = mbar_wait(&sm.bar_kv, 0, a.err, 1501);
             for (int u = 0; ok && u <= U; ++u) {
                 if (u < U) {
-                    const int s = u % BWD_STAGES, b = u & 1;
-                    if (!mbar_wait(&sm.st_full[s], (u / BWD_STAGES) & 1, a.err, 1502)) break;
+                    const int s = u % DKDV_STAGES, b = u & 1;
+                    if (!mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1502)) break;
                     if (u >= 2 && !mbar_wait(&sm.s_free[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
                     if (FUSE && u >= 2 && !mbar_wait(&sm.dq_free[b], ((u - 2) >> 1) & 1, a.err, 1505)) break;
                     tc_fence_after();
@@ -290,15 +294,16 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     umma_commit(&sm.s_full[b]);
                 }
                 if (u >= 1) {
-                    const int uu = u - 1, b = uu & 1, s = uu % BWD_STAGES;
+                    const int uu = u - 1, b = uu & 1, s = uu % DKDV_STAGES;
                     if (!mbar_wait(&sm.p_full[b], (uu >> 1) & 1, a.err, 1504)) break;
                     tc_fence_after();
-                    const uint32_t p_s = smem_u32(sm.p[b]), ds_s = smem_u32(sm.ds[b]);
+                    const uint32_t ds_s = smem_u32(sm.ds[b]);
                     const uint32_t q_s = smem_u32(sm.q[s][0]), do_s = smem_u32(sm.dO[s][0]);
+                    // dV += P^T dO with P^T (fp16) read from TMEM over the dP^T columns
                     #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + TDV, desc_kmajor(p_s, kk, SLAB128), desc_mnmajor(do_s, kk, SLAB64),
-                                 id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16_ts(tmem + TDV, tmem + 128 * b + 64 + 8 * kk, desc_mnmajor(do_s, kk, SLAB64),
+                                    id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
                     #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16(tmem + TDK, desc_kmajor(ds_s, kk, SLAB128), desc_mnmajor(q_s, kk, SLAB64),
@@ -316,37 +321,40 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 }
             }
         }
-    } else if (warp < 4) {
-        const int r = threadIdx.x;                  // key row of the tile = TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    } else if (warp < 8) {
+        const int wg = warp >> 2;                   // which 32 queries of the unit
+        const int r = (warp & 3) * 32 + lane;       // key row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const int kh = r >> 6;                      // warp-uniform
+        const int c0 = 32 * wg;
         bool ok = true;
         HalfIter it{ents, ne, 0, 0, 1};
         int r64, m2;
         for (int u = 0; it.next(r64, m2); ++u) {
-            const int b = u & 1, s = u % BWD_STAGES;
+            const int b = u & 1, s = u % DKDV_STAGES;
             const bool valid = (m2 >> kh) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (u >> 1) & 1, a.err, 1001))) { ok = false; break; }
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full[s], (u / BWD_STAGES) & 1, a.err, 1002))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1002))) { ok = false; break; }
             tc_fence_after();
-            uint32_t sv[64], dp[64];
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b, sv);
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 32, (sv + 32));
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64, dp);
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 96, (dp + 32));
+            uint32_t sv[32], dp[32];
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + c0, sv);
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64 + c0, dp);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.s_free[b]);
+            // both warpgroups of this lane quarter have read dP^T before P^T overwrites it
+            named_bar(2 + (warp & 3), 64);
             if (u >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1003))) {
                 ok = false;
                 break;
             }
-            const float* lq = sm.lse[s];
-            const float* dq = sm.di[s];
-            const uint32_t p_s = smem_u32(sm.p[b]), ds_s = smem_u32(sm.ds[b]);
+            const float* lq = sm.lse[s] + c0;
+            const float* dq = sm.di[s] + c0;
+            const uint32_t ds_s = smem_u32(sm.ds[b]);
+            uint32_t pt[16];
             #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t wp[4], wd[4];
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t wd[4];
                 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = ch * 8 + 2 * e;
@@ -359,39 +367,40 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     }
                     // the dV operand is 2^15 P (normal in fp16 down to P = 2^-29);
                     // dV is unscaled in the epilogue
-                    wp[e] = pack_f16(p0 * kPScale, p1 * kPScale);
+                    pt[ch * 4 + e] = pack_f16(p0 * kPScale, p1 * kPScale);
                     wd[e] = pack_f16(d0, d1);
                 }
-                st_shared_v4(p_s + swz128(r, ch), wp[0], wp[1], wp[2], wp[3]);
-                st_shared_v4(ds_s + swz128(r, ch), wd[0], wd[1], wd[2], wd[3]);
+                st_shared_v4(ds_s + swz128(r, 4 * wg + ch), wd[0], wd[1], wd[2], wd[3]);
             }
+            PRISM_TMEM_ST16(tmem + lane_off + 128 * b + 64 + 16 * wg, pt);
             fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
         }
+        // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (same rows)
         const size_t orow = (size_t)hrow + (size_t)a.src[(size_t)hrow + (size_t)t * 128 + r];
+        void* out = wg ? a.out0 : a.out1;
         bool fin = false;
         if (ok && U > 0)
             fin = __all_sync(0xffffffffu, mbar_wait(&sm.pd_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, 1004));
         if (fin) {
             tc_fence_after();
             const float unscale = ldexpf(1.f, dscale_exp(a.dmax[h], a.err));
+            const float mul = wg ? a.inv_sqrt_d * unscale : unscale / kPScale;
+            const uint32_t col = wg ? TDK : TDV;
             #pragma unroll
             for (int c = 0; c < HD / 32; ++c) {
                 uint32_t o[32];
-                PRISM_TMEM_LD32(tmem + lane_off + TDV + 32 * c, o);
+                PRISM_TMEM_LD32(tmem + lane_off + col + 32 * c, o);
                 tmem_wait_ld();
-                store_row(a.out1, orow, HD, 32 * c, o, unscale / kPScale, a.out_f32);
-                PRISM_TMEM_LD32(tmem + lane_off + TDK + 32 * c, o);
-                tmem_wait_ld();
-                store_row(a.out0, orow, HD, 32 * c, o, a.inv_sqrt_d * unscale, a.out_f32);
+                store_row(out, orow, HD, 32 * c, o, mul, a.out_f32);
             }
         } else if (U == 0) {
-            zero_row(a.out0, orow, HD, a.out_f32);
-            zero_row(a.out1, orow, HD, a.out_f32);
+            zero_row(out, orow, HD, a.out_f32);
         }
-    } else if (FUSE) {
-        // ---------------------------------------------- dQ drain (warps 6-9)
+    } else if (FUSE && warp >= 10) {
+        // ---------------------------------------------- dQ drain (warps 10-13)
         const int d = (warp & 3) * 32 + lane;       // head-dim row of dQ^T = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const bool leader = (warp & 3) == 0 && lane == 0;
@@ -427,7 +436,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) { __syncwarp(); tmem_dealloc(tmem, 512); }
+    if (warp == W_PROD) { __syncwarp(); tmem_dealloc(tmem, 512); }
 }
 
 // dQ accumulator (block order, fp32) -> dQ output (raster order, scaled).
@@ -679,7 +688,7 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
         return PRISM_ERR_CUDA;
     {
         PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
-        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, g.heads), FUSE ? 320 : 192, sm1, s>>>(
+        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, g.heads), FUSE ? 448 : 320, sm1, s>>>(
             P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, a);
     }
     if (FUSE) {

@@ -9,14 +9,14 @@
 // Design (B200): one CTA per 128-token query tile.  The plan's tile list gives,
 // for the tile, the 128-token key tiles to visit with a 4-bit mask (which
 // 64-token query half attends to which 64-token key half).  Per key tile:
-//   TMA (128B swizzle) K, V (fp16 block-ordered copies) -> shared memory (2-stage ring)
+//   TMA (128B swizzle) K (2-stage ring) and V (one buffer), fp16 block-ordered copies
 //   tcgen05.mma S = Q K^T into TMEM (double-buffered, 2 x 128 columns)
-//   4 softmax warps (thread = query row = TMEM lane) read S, mask, update the
+//   8 softmax warps (2 per TMEM lane quarter, 64 keys each) read S, mask, update the
 //     running max (rescaling O in TMEM only when it grows by more than 2^8),
-//     write P = 2^(s - m) as fp16 to shared memory
-//   tcgen05.mma O += P V into TMEM (128 + head_dim columns)
-// Warp roles: 0-3 softmax/epilogue, 4 TMA producer (and TMEM allocator),
-// 5 MMA issuer.  Every barrier wait is bounded (PRISM_ERR_TIMEOUT).
+//     write P = 2^(s - m) as fp16 into TMEM
+//   tcgen05.mma O += P V (P read from TMEM, V from shared memory) into TMEM
+// Warp roles: 0-7 softmax/epilogue (two warpgroups, one per 64-key half),
+// 8 TMA producer (and TMEM allocator), 9 MMA issuer.  Every barrier wait is bounded (PRISM_ERR_TIMEOUT).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -42,11 +42,14 @@ struct FwdSmem {
     static constexpr int NSL = HD / 64;
     alignas(1024) uint8_t q[NSL][SLAB];
     alignas(1024) uint8_t k[FWD_STAGES][NSL][SLAB];
-    alignas(1024) uint8_t v[FWD_STAGES][NSL][SLAB];
+    alignas(1024) uint8_t v[NSL][SLAB];           // one V tile: PV_j runs long after QK_j+1
     alignas(1024) uint8_t p[2][2][SLAB];          // [buffer][64-key slab]
     uint64_t bar_q;
-    uint64_t kv_full[FWD_STAGES], kv_empty[FWD_STAGES];
+    uint64_t k_full[FWD_STAGES], k_empty[FWD_STAGES];
+    uint64_t v_full, v_empty;
     uint64_t s_full[2], p_full[2], pv_done[2];
+    float pmax[2][2][128];                        // [step parity][warpgroup][row] partial max
+    float psum[2][128];                           // [warpgroup][row] partial sum (epilogue)
     uint32_t tmem_base;
     int abort;
 };
@@ -65,7 +68,7 @@ struct FwdArgs {
 };
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, FwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -81,16 +84,22 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < FWD_STAGES; ++s) { mbar_init(&sm.kv_full[s], 1); mbar_init(&sm.kv_empty[s], 1); }
+        for (int s = 0; s < FWD_STAGES; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
+        mbar_init(&sm.v_full, 1);
+        mbar_init(&sm.v_empty, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.p_full[b], 128);
+            mbar_init(&sm.p_full[b], 256);
             mbar_init(&sm.pv_done[b], 1);
         }
         sm.abort = 0;
         mbar_fence_init();
     }
-    if (warp == 4) {
+    // warps 0-7: two softmax warpgroups (same 128 query rows; warpgroup g takes
+    // the 64 keys of key half g of every tile); warp 8: TMA producer + TMEM
+    // allocator; warp 9: MMA issuer.
+    constexpr int W_PROD = 8, W_MMA = 9;
+    if (warp == W_PROD) {
         __syncwarp();
         tmem_alloc(&sm.tmem_base, 512);
     }
@@ -98,10 +107,13 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // TMEM columns: S double-buffered at 0 and 128, O at 256 (HD columns)
+    constexpr uint32_t TS = 0, TO = 256;
     const int64_t qrow0 = (int64_t)h * a.N + (int64_t)t * 128;
 
-    if (warp == 4) {
+    if (warp == W_PROD) {
         // ------------------------------------------------ TMA producer
+        // lane 0 streams Q and the K ring, lane 1 the V ring
         if (lane == 0 && n > 0) {
             tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
             mbar_expect_tx(&sm.bar_q, NSL * SLAB);
@@ -109,17 +121,20 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             for (int j = 0; j < n; ++j) {
                 const int s = j % FWD_STAGES;
                 if (j >= FWD_STAGES &&
-                    !mbar_wait(&sm.kv_empty[s], ((j / FWD_STAGES) - 1) & 1, a.err, 401)) break;
-                const int kt = ents[j] >> 4;
-                const int krow = (int)((int64_t)h * a.N + (int64_t)kt * 128);
-                mbar_expect_tx(&sm.kv_full[s], 2 * NSL * SLAB);
-                for (int c = 0; c < NSL; ++c) {
-                    tma_load_2d(sm.k[s][c], &tm_k, &sm.kv_full[s], 64 * c, krow);
-                    tma_load_2d(sm.v[s][c], &tm_v, &sm.kv_full[s], 64 * c, krow);
-                }
+                    !mbar_wait(&sm.k_empty[s], ((j / FWD_STAGES) - 1) & 1, a.err, 401)) break;
+                const int krow = (int)((int64_t)h * a.N + (int64_t)(ents[j] >> 4) * 128);
+                mbar_expect_tx(&sm.k_full[s], NSL * SLAB);
+                for (int c = 0; c < NSL; ++c) tma_load_2d(sm.k[s][c], &tm_k, &sm.k_full[s], 64 * c, krow);
+            }
+        } else if (lane == 1 && n > 0) {
+            for (int j = 0; j < n; ++j) {
+                if (j >= 1 && !mbar_wait(&sm.v_empty, (j - 1) & 1, a.err, 402)) break;
+                const int krow = (int)((int64_t)h * a.N + (int64_t)(ents[j] >> 4) * 128);
+                mbar_expect_tx(&sm.v_full, NSL * SLAB);
+                for (int c = 0; c < NSL; ++c) tma_load_2d(sm.v[c], &tm_v, &sm.v_full, 64 * c, krow);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == W_MMA) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
             constexpr uint32_t idesc_qk = idesc_f16(128, 128, 0, 0);
@@ -129,27 +144,29 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             for (int j = 0; ok && j <= n; ++j) {
                 if (j < n) {
                     const int s = j % FWD_STAGES, b = j & 1;
-                    if (!mbar_wait(&sm.kv_full[s], (j / FWD_STAGES) & 1, a.err, 502)) { ok = false; break; }
+                    if (!mbar_wait(&sm.k_full[s], (j / FWD_STAGES) & 1, a.err, 502)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t k_s = smem_u32(sm.k[s][0]);
                     #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + 128 * b, desc_kmajor(q_s, kk, SLAB), desc_kmajor(k_s, kk, SLAB),
+                        umma_f16(tmem + TS + 128 * b, desc_kmajor(q_s, kk, SLAB), desc_kmajor(k_s, kk, SLAB),
                                   idesc_qk, kk > 0);
                     umma_commit(&sm.s_full[b]);
+                    umma_commit(&sm.k_empty[s]);
                 }
                 if (j >= 1) {
-                    const int jj = j - 1, b = jj & 1, s = jj % FWD_STAGES;
+                    const int jj = j - 1, b = jj & 1;
                     if (!mbar_wait(&sm.p_full[b], (jj >> 1) & 1, a.err, 503)) { ok = false; break; }
+                    if (!mbar_wait(&sm.v_full, jj & 1, a.err, 504)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t p_s = smem_u32(sm.p[b][0]);
-                    const uint32_t v_s = smem_u32(sm.v[s][0]);
+                    const uint32_t v_s = smem_u32(sm.v[0]);
                     #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_f16(tmem + 256, desc_kmajor(p_s, kk, SLAB), desc_mnmajor(v_s, kk, SLAB),
-                                  idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16(tmem + TO, desc_kmajor(p_s, kk, SLAB), desc_mnmajor(v_s, kk, SLAB),
+                                 idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sm.pv_done[b]);
-                    umma_commit(&sm.kv_empty[s]);
+                    umma_commit(&sm.v_empty);
                 }
             }
             if (!ok) sm.abort = 1;
@@ -157,34 +174,40 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     } else {
         // ------------------------------------------------ softmax + epilogue
         // tcgen05.ld/st are warp-collective (.sync.aligned): every decision that
-        // guards one is made warp-uniform (__all_sync / __any_sync).
-        const int r = threadIdx.x;                 // query row of the tile = TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // guards one is made warp-uniform (__all_sync / __any_sync).  The two
+        // warps sharing a TMEM lane quarter (w and w + 4) combine their row maxima
+        // through shared memory and a 64-thread named barrier, so both take the
+        // same rescaling decisions.
+        const int wg = warp >> 2;                  // key half handled by this warpgroup
+        const int r = (warp & 3) * 32 + lane;      // query row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const int pair_bar = 1 + (warp & 3);
         const int qh = r >> 6;                     // uniform per warp (32 | 64)
-        float m_ref = -INFINITY, l = 0.f;
+        constexpr int OC = HD / 2;                 // O columns rescaled / written per warpgroup
+        const uint32_t ocol = TO + OC * wg;
+        float m_ref = -INFINITY, l = 0.f;          // l: this warpgroup's share of the row sum
         bool ok = true;
         for (int j = 0; j < n; ++j) {
             const int b = j & 1;
             const int msk = ents[j] & 15;
-            const bool v0 = (msk >> (qh * 2)) & 1, v1 = (msk >> (qh * 2 + 1)) & 1;
+            const bool valid = (msk >> (qh * 2 + wg)) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (j >> 1) & 1, a.err, 1))) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[128];
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 0, (sr + 0));
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 32, (sr + 32));
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64, (sr + 64));
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 96, (sr + 96));
+            uint32_t sr[64];
+            PRISM_TMEM_LD32(tmem + lane_off + TS + 128 * b + 64 * wg, (sr + 0));
+            PRISM_TMEM_LD32(tmem + lane_off + TS + 128 * b + 64 * wg + 32, (sr + 32));
             tmem_wait_ld();
             float mx = -INFINITY;
-            if (v0) {
+            if (valid) {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 #pragma unroll
-                for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-            }
-            if (v1) {
-                #pragma unroll
-                for (int c = 64; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+                for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             }
             mx *= a.scale_log2;
+            sm.pmax[j & 1][wg][r] = mx;
+            named_bar(pair_bar, 64);
+            mx = fmaxf(mx, sm.pmax[j & 1][wg ^ 1][r]);
             const float m_new = fmaxf(m_ref, mx);
             const bool first = (j == 0) || (m_ref == -INFINITY);
             const bool need = !first && (m_new > m_ref + kRescaleLog2);
@@ -198,13 +221,13 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 tc_fence_after();
                 const float f = need ? ex2(m_ref - m_new) : 1.f;
                 #pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
+                for (int c = 0; c < OC / 32; ++c) {
                     uint32_t o[32];
-                    PRISM_TMEM_LD32(tmem + lane_off + 256 + 32 * c, o);
+                    PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * c, o);
                     tmem_wait_ld();
                     #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    PRISM_TMEM_ST32(tmem + lane_off + 256 + 32 * c, o);
+                    PRISM_TMEM_ST32(tmem + lane_off + ocol + 32 * c, o);
                 }
                 if (need) { l *= f; m_ref = m_new; }
             }
@@ -217,33 +240,31 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             // of a 1M-token head sit near 1e-6, fp16's subnormal range), and the
             // 2^15 cancels in O = acc / l because l sums the same scaled values.
             const float neg = kPScaleLog2 - m_ref;
-            const uint32_t p_s = smem_u32(sm.p[b][0]);
+            const uint32_t p_s = smem_u32(sm.p[b][wg]);
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
             #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const bool valid = half ? v1 : v0;
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t w[4];
                 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t w[4];
-                    #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = half * 64 + ch * 8 + 2 * e;
-                        float p0 = 0.f, p1 = 0.f;
-                        if (valid) {
-                            p0 = ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, neg));
-                            p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, neg));
-                        }
-                        l += p0 + p1;
-                        w[e] = pack_f16(p0, p1);
+                for (int e = 0; e < 4; ++e) {
+                    const int c = ch * 8 + 2 * e;
+                    float p0 = 0.f, p1 = 0.f;
+                    if (valid) {
+                        p0 = ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, neg));
+                        p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, neg));
                     }
-                    st_shared_v4(p_s + half * SLAB + swz128(r, ch), w[0], w[1], w[2], w[3]);
+                    l4[e] += p0 + p1;
+                    w[e] = pack_f16(p0, p1);
                 }
+                st_shared_v4(p_s + swz128(r, ch), w[0], w[1], w[2], w[3]);
             }
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             fence_proxy_async_smem();
             if (rescale) tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
         }
-        // epilogue: O / l, scattered to raster order
+        // epilogue: both warpgroups add their row sums, each writes half of O
         const int row_perm = t * 128 + r;
         const int dst = a.src[(size_t)h * a.N + row_perm];
         const size_t orow = (size_t)h * a.N + (size_t)dst;
@@ -251,21 +272,25 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (ok && n > 0)
             fin = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err, 4));
         if (fin) {
+            sm.psum[wg][r] = l;
+            named_bar(pair_bar, 64);
+            const float lt = sm.psum[0][r] + sm.psum[1][r];
             tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
             #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
+            for (int c = 0; c < OC / 32; ++c) {
                 uint32_t o[32];
-                PRISM_TMEM_LD32(tmem + lane_off + 256 + 32 * c, o);
+                PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * c, o);
                 tmem_wait_ld();
+                const int c0 = OC * wg + 32 * c;
                 if (a.out_f32) {
-                    float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * HD + 32 * c);
+                    float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * HD + c0);
                     #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         op[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
                                             __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
                 } else {
-                    uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + orow * HD + 32 * c);
+                    uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + orow * HD + c0);
                     #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         op[e] = make_uint4(pack_bf16(__uint_as_float(o[8 * e]) * inv, __uint_as_float(o[8 * e + 1]) * inv),
@@ -274,19 +299,20 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                            pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv));
                 }
             }
-            a.lse[orow] = l > 0.f ? (m_ref - kPScaleLog2) * 0.69314718055994531f + logf(l) : -INFINITY;
+            if (wg == 0)
+                a.lse[orow] = lt > 0.f ? (m_ref - kPScaleLog2) * 0.69314718055994531f + logf(lt) : -INFINITY;
         } else if (n == 0) {
-            for (int c = 0; c < HD; ++c) {
+            for (int c = OC * wg; c < OC * wg + OC; ++c) {
                 if (a.out_f32) static_cast<float*>(a.O)[orow * HD + c] = 0.f;
                 else static_cast<__nv_bfloat16*>(a.O)[orow * HD + c] = __float2bfloat16(0.f);
             }
-            a.lse[orow] = -INFINITY;
+            if (wg == 0) a.lse[orow] = -INFINITY;
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) {
+    if (warp == W_PROD) {
         __syncwarp();
         tmem_dealloc(tmem, 512);
     }
@@ -325,7 +351,7 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
         return PRISM_ERR_CUDA;
     {
         PrismProf prof(P, PRISM_STAGE_FWD, s);
-        k_attn_fwd<HD><<<dim3(g.NT, g.heads), 192, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+        k_attn_fwd<HD><<<dim3(g.NT, g.heads), 320, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
     }
     P->launches += 1;
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
