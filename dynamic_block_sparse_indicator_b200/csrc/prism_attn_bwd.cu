@@ -328,6 +328,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         const int kh = r >> 6;                      // warp-uniform
         const int c0 = 32 * wg;
         bool ok = true;
+        int nbar = 0;                               // quarter barriers taken in the loop
         HalfIter it{ents, ne, 0, 0, 1};
         int r64, m2;
         for (int u = 0; it.next(r64, m2); ++u) {
@@ -344,6 +345,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             mbar_arrive(&sm.s_free[b]);
             // both warpgroups of this lane quarter have read dP^T before P^T overwrites it
             named_bar(2 + (warp & 3), 64);
+            ++nbar;
             if (u >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1003))) {
                 ok = false;
                 break;
@@ -378,6 +380,9 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
         }
+        // a warp that left the loop on a failed wait still takes the barriers
+        // the other warpgroup will take, so that one is never left at a barrier
+        for (; nbar < U; ++nbar) named_bar(2 + (warp & 3), 64);
         // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (same rows)
         const size_t orow = (size_t)hrow + (size_t)a.src[(size_t)hrow + (size_t)t * 128 + r];
         void* out = wg ? a.out0 : a.out1;
@@ -406,7 +411,8 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         const bool leader = (warp & 3) == 0 && lane == 0;
         HalfIter it{ents, ne, 0, 0, 1};
         int r64, m2;
-        for (int u = 0; it.next(r64, m2); ++u) {
+        int u = 0;                                  // units drained
+        for (; it.next(r64, m2); ++u) {
             const int b = u & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.dq_full[b], (u >> 1) & 1, a.err, 3001))) break;
             tc_fence_after();
@@ -431,6 +437,9 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 }
             }
         }
+        // after a failed wait, the four barriers of every undrained unit, which
+        // the other drain warps may still take
+        for (int k = 4 * u; k < 4 * U; ++k) named_bar(1, 128);
         if (leader) bulk_wait0();
     }
     tc_fence_before();

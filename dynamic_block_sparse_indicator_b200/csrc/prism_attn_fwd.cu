@@ -187,6 +187,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const uint32_t ocol = TO + OC * wg;
         float m_ref = -INFINITY, l = 0.f;          // l: this warpgroup's share of the row sum
         bool ok = true;
+        int nbar = 0;                              // pair barriers taken in the loop
         for (int j = 0; j < n; ++j) {
             const int b = j & 1;
             const int msk = ents[j] & 15;
@@ -207,6 +208,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             mx *= a.scale_log2;
             sm.pmax[j & 1][wg][r] = mx;
             named_bar(pair_bar, 64);
+            ++nbar;
             mx = fmaxf(mx, sm.pmax[j & 1][wg ^ 1][r]);
             const float m_new = fmaxf(m_ref, mx);
             const bool first = (j == 0) || (m_ref == -INFINITY);
@@ -268,12 +270,16 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const int row_perm = t * 128 + r;
         const int dst = a.src[(size_t)h * a.N + row_perm];
         const size_t orow = (size_t)h * a.N + (size_t)dst;
+        // A warp that left the loop on a failed wait still takes the pair barriers
+        // its partner will take (one per tile, then the epilogue's), so the
+        // partner is never left at a barrier.
+        for (; nbar < n; ++nbar) named_bar(pair_bar, 64);
         bool fin = false;
         if (ok && n > 0)
             fin = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err, 4));
+        sm.psum[wg][r] = l;
+        named_bar(pair_bar, 64);
         if (fin) {
-            sm.psum[wg][r] = l;
-            named_bar(pair_bar, 64);
             const float lt = sm.psum[0][r] + sm.psum[1][r];
             tc_fence_after();
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
