@@ -197,6 +197,7 @@ struct DkdvSmem {
     uint64_t bar_kv;
     uint64_t st_full[DKDV_STAGES], st_empty[DKDV_STAGES];
     uint64_t s_full[2], s_free[2], p_full[2], pd_done[2];
+    uint64_t acc_done;                        // every MMA of the CTA has completed
     uint64_t dq_full[2], dq_free[2];
     uint32_t tmem_base;
 };
@@ -216,12 +217,16 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     const int ne = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - e0;
     const int* ents = a.ent + (size_t)h * a.NT * a.NT + e0;
     const int U = count_units(ents, ne, 1);
-    // TMEM columns: buffer b = [128b, 128b + 128): S^T at 128b, dP^T at 128b + 64
-    // (dQ^T of the unit reuses the S^T columns); dV at 256, dK at 256 + HD.
+    // TMEM columns: buffer b = [128b, 128b + 128): S^T at 128b, dP^T at 128b + 64.
+    // The softmax writes P^T (fp16 pairs) over the first half of dP^T; dQ^T of
+    // the unit then overwrites all 64 dP^T columns after dV has read P^T (the
+    // MMAs of one issuer run in order), so the next S^T into the buffer does not
+    // wait for the dQ drain -- only the next dP^T does.  dV at 256, dK at 256 + HD.
     constexpr uint32_t TDV = 256, TDK = 256 + HD;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_kv, 1);
+        mbar_init(&sm.acc_done, 1);
         for (int s = 0; s < DKDV_STAGES; ++s) { mbar_init(&sm.st_full[s], 1); mbar_init(&sm.st_empty[s], 1); }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
@@ -273,53 +278,63 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             constexpr uint32_t id_s = idesc_f16(128, 64, 0, 0);
             constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
             constexpr uint32_t id_dq = idesc_f16(128, 64, 1, 1);
-            const uint32_t k_s = smem_u32(sm.k[0]), v_s = smem_u32(sm.v[0]);
+            // descriptor low words; every K step below adds an immediate
+            const uint32_t kA = desc_lo(smem_u32(sm.k[0]), 16), vA = desc_lo(smem_u32(sm.v[0]), 16);
+            const uint32_t kT = desc_lo(smem_u32(sm.k[0]), SLAB128);       // K^T (MN-major) for dQ^T
             bool ok = mbar_wait(&sm.bar_kv, 0, a.err, 1501);
-            for (int u = 0; ok && u <= U; ++u) {
+            int u = 0;
+            for (; ok && u <= U; ++u) {
                 if (u < U) {
                     const int s = u % DKDV_STAGES, b = u & 1;
                     if (!mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1502)) break;
+                    // both softmax warpgroups have loaded S^T(u - 2)
                     if (u >= 2 && !mbar_wait(&sm.s_free[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
+                    tc_fence_after();
+                    const uint32_t qB = desc_lo(smem_u32(sm.q[s][0]), 16), doB = desc_lo(smem_u32(sm.dO[s][0]), 16);
+                    #pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_f16(tmem + 128 * b, desc_from_lo(kA + kmajor_step(kk, SLAB128)),
+                                 desc_from_lo(qB + kmajor_step(kk, SLAB64)), id_s, kk > 0);
+                    // dP^T overwrites dQ^T(u - 2): wait until the drain has read it
                     if (FUSE && u >= 2 && !mbar_wait(&sm.dq_free[b], ((u - 2) >> 1) & 1, a.err, 1505)) break;
                     tc_fence_after();
-                    const uint32_t q_s = smem_u32(sm.q[s][0]), do_s = smem_u32(sm.dO[s][0]);
                     #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + 128 * b, desc_kmajor(k_s, kk, SLAB128),
-                                 desc_kmajor(q_s, kk, SLAB64), id_s, kk > 0);
-                    #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + 128 * b + 64, desc_kmajor(v_s, kk, SLAB128),
-                                 desc_kmajor(do_s, kk, SLAB64), id_s, kk > 0);
+                        umma_f16(tmem + 128 * b + 64, desc_from_lo(vA + kmajor_step(kk, SLAB128)),
+                                 desc_from_lo(doB + kmajor_step(kk, SLAB64)), id_s, kk > 0);
                     umma_commit(&sm.s_full[b]);
                 }
                 if (u >= 1) {
                     const int uu = u - 1, b = uu & 1, s = uu % DKDV_STAGES;
                     if (!mbar_wait(&sm.p_full[b], (uu >> 1) & 1, a.err, 1504)) break;
                     tc_fence_after();
-                    const uint32_t ds_s = smem_u32(sm.ds[b]);
-                    const uint32_t q_s = smem_u32(sm.q[s][0]), do_s = smem_u32(sm.dO[s][0]);
+                    const uint32_t dsA = desc_lo(smem_u32(sm.ds[b]), 16);          // dS^T, K-major
+                    const uint32_t dsT = desc_lo(smem_u32(sm.ds[b]), SLAB128);     // dS^T as MN-major B
+                    const uint32_t qT = desc_lo(smem_u32(sm.q[s][0]), SLAB64);
+                    const uint32_t doT = desc_lo(smem_u32(sm.dO[s][0]), SLAB64);
                     // dV += P^T dO with P^T (fp16) read from TMEM over the dP^T columns
                     #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tmem + TDV, tmem + 128 * b + 64 + 8 * kk, desc_mnmajor(do_s, kk, SLAB64),
+                        umma_f16_ts(tmem + TDV, tmem + 128 * b + 64 + 8 * kk, desc_from_lo(doT + mnmajor_step(kk)),
                                     id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
-                    #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + TDK, desc_kmajor(ds_s, kk, SLAB128), desc_mnmajor(q_s, kk, SLAB64),
-                                 id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
                     if (FUSE) {
-                        // dQ^T [HD x 64 queries] = K^T [HD x 128 keys] . dS^T [128 keys x 64 queries]
+                        // dQ^T [HD x 64 queries] = K^T [HD x 128 keys] . dS^T [128 keys x 64 queries],
+                        // over the dP^T columns (after dV above has read P^T there)
                         #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            umma_f16(tmem + 128 * b, desc_mnmajor(k_s, kk, SLAB128),
-                                     desc_mnmajor(ds_s, kk, SLAB128), id_dq, kk > 0);
+                            umma_f16(tmem + 128 * b + 64, desc_from_lo(kT + mnmajor_step(kk)),
+                                     desc_from_lo(dsT + mnmajor_step(kk)), id_dq, kk > 0);
                         umma_commit(&sm.dq_full[b]);
                     }
+                    #pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + TDK, desc_from_lo(dsA + kmajor_step(kk, SLAB128)),
+                                 desc_from_lo(qT + mnmajor_step(kk)), id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sm.pd_done[b]);
                     umma_commit(&sm.st_empty[s]);
                 }
             }
+            if (u > U) umma_commit(&sm.acc_done);   // dV and dK are final
         }
     } else if (warp < 8) {
         const int wg = warp >> 2;                   // which 32 queries of the unit
@@ -388,7 +403,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         void* out = wg ? a.out0 : a.out1;
         bool fin = false;
         if (ok && U > 0)
-            fin = __all_sync(0xffffffffu, mbar_wait(&sm.pd_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, 1004));
+            fin = __all_sync(0xffffffffu, mbar_wait(&sm.acc_done, 0, a.err, 1004));
         if (fin) {
             tc_fence_after();
             const float unscale = ldexpf(1.f, dscale_exp(a.dmax[h], a.err));
@@ -417,8 +432,8 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.dq_full[b], (u >> 1) & 1, a.err, 3001))) break;
             tc_fence_after();
             uint32_t v[64];
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b, v);
-            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 32, (v + 32));
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64, v);
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 96, (v + 32));
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.dq_free[b]);

@@ -139,18 +139,20 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (lane == 0 && n > 0) {
             constexpr uint32_t idesc_qk = idesc_f16(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = idesc_f16(128, HD, 0, 1);
-            const uint32_t q_s = smem_u32(sm.q[0]);
+            // descriptor low words; every K step below adds an immediate
+            const uint32_t qA = desc_lo(smem_u32(sm.q[0]), 16);
+            const uint32_t vT = desc_lo(smem_u32(sm.v[0]), SLAB);
             bool ok = mbar_wait(&sm.bar_q, 0, a.err, 501);
             for (int j = 0; ok && j <= n; ++j) {
                 if (j < n) {
                     const int s = j % FWD_STAGES, b = j & 1;
                     if (!mbar_wait(&sm.k_full[s], (j / FWD_STAGES) & 1, a.err, 502)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t k_s = smem_u32(sm.k[s][0]);
+                    const uint32_t kB = desc_lo(smem_u32(sm.k[s][0]), 16);
                     #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + TS + 128 * b, desc_kmajor(q_s, kk, SLAB), desc_kmajor(k_s, kk, SLAB),
-                                  idesc_qk, kk > 0);
+                        umma_f16(tmem + TS + 128 * b, desc_from_lo(qA + kmajor_step(kk, SLAB)),
+                                 desc_from_lo(kB + kmajor_step(kk, SLAB)), idesc_qk, kk > 0);
                     umma_commit(&sm.s_full[b]);
                     umma_commit(&sm.k_empty[s]);
                 }
@@ -159,12 +161,11 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     if (!mbar_wait(&sm.p_full[b], (jj >> 1) & 1, a.err, 503)) { ok = false; break; }
                     if (!mbar_wait(&sm.v_full, jj & 1, a.err, 504)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t p_s = smem_u32(sm.p[b][0]);
-                    const uint32_t v_s = smem_u32(sm.v[0]);
+                    const uint32_t pA = desc_lo(smem_u32(sm.p[b][0]), 16);
                     #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_f16(tmem + TO, desc_kmajor(p_s, kk, SLAB), desc_mnmajor(v_s, kk, SLAB),
-                                 idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16(tmem + TO, desc_from_lo(pA + kmajor_step(kk, SLAB)),
+                                 desc_from_lo(vT + mnmajor_step(kk)), idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sm.pv_done[b]);
                     umma_commit(&sm.v_empty);
                 }

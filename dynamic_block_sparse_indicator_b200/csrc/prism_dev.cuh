@@ -14,6 +14,9 @@
 namespace prism {
 
 constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s of wall-clock per wait before giving up
+#ifndef PRISM_WAIT_SUSPEND
+#define PRISM_WAIT_SUSPEND 1
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
@@ -47,11 +50,30 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
                  : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes (it is woken at once) or about `ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
 // Bounded wait for the phase of parity `parity`; false (and the error word
-// set, with `where` in err[1]) if it did not complete within kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int where = 0) {
-    if (mbar_try(bar, parity)) return true;
+// set, with `where` in err[1]) if it did not complete within kWaitNs.  The
+// first poll is inline; the polling loop is an out-of-line call, which keeps
+// the inline code of every wait short (the MMA issuer is a single warp whose
+// instructions must stay in the instruction cache next to busy softmax warps).
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int* err, int where) {
     const uint64_t t0 = globaltimer_ns();
+#if PRISM_WAIT_SUSPEND
+    for (;;) {
+        if (mbar_try_suspend(bar, parity, 20000)) return true;
+        if (*(volatile int*)err != 0) return false;              // someone else gave up
+        if (globaltimer_ns() - t0 > kWaitNs) break;
+    }
+#else
     for (uint32_t i = 0;; ++i) {
         if (mbar_try(bar, parity)) return true;
         if (i > 16) __nanosleep(128);
@@ -60,12 +82,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
             if (globaltimer_ns() - t0 > kWaitNs) break;
         }
     }
+#endif
     if (atomicCAS(err, 0, PRISM_ERR_TIMEOUT) == 0) {
         err[1] = where;
         err[2] = (int)blockIdx.x;
         err[3] = (int)threadIdx.x;
     }
     return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int where = 0) {
+    if (mbar_try(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, err, where);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -205,16 +232,58 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 // K-major operand (rows = M or N, the contraction dim contiguous): the k-th
 // 16-element step starts 32*k bytes into the row (inside a slab) or in the
 // next slab.  SBO = 1024 (next 8-row group); LBO unused for swizzled K-major.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int k16, uint32_t slab_bytes) {
-    uint32_t a = tile_saddr + (uint32_t)(k16 >> 2) * slab_bytes + (uint32_t)(k16 & 3) * 32u;
-    return sdesc(a, 16, 1024);
+// The same descriptors split into a constant high word (SBO 1024 B, version 1,
+// 128-byte swizzle) and a low word (start address, LBO).  Within one tile the
+// K steps only add an immediate to the low word (the start field is 14 bits of
+// a shared address below 256 KB, so the add never carries out of it), which
+// keeps the MMA issuer's instruction stream short.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr >> 4) & 0x3FFFu) | ((lbo >> 4) << 16);
 }
-// MN-major operand (rows of the smem tile = the contraction dim, the M or N dim
-// contiguous inside 64-wide slabs): the k-th 16-row step starts 16*128 bytes
-// further; LBO = distance between slabs along M/N; SBO = 1024 (8 rows).
+__device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) {
+    return ((uint64_t)kDescHi << 32) | lo;
+}
+// low-word offset of K step k16 of a K-major tile of 64-column slabs
+__host__ __device__ constexpr uint32_t kmajor_step(int k16, uint32_t slab_bytes) {
+    return ((uint32_t)(k16 >> 2) * slab_bytes + (uint32_t)(k16 & 3) * 32u) >> 4;
+}
+// low-word offset of K step k16 of an MN-major tile
+__host__ __device__ constexpr uint32_t mnmajor_step(int k16) { return (uint32_t)k16 * (2048u >> 4); }
+// K-major tile of 64-column slabs: K step k16 moves 32 B inside a slab, a new
+// slab every 4 steps.
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int k16, uint32_t slab_bytes) {
+    return desc_from_lo(desc_lo(tile_saddr, 16) + kmajor_step(k16, slab_bytes));
+}
+// MN-major tile (MN contiguous, 64-element slabs slab_bytes apart): K step
+// k16 moves 16 rows of 128 B.
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_saddr, int k16, uint32_t slab_bytes) {
-    uint32_t a = tile_saddr + (uint32_t)k16 * 2048u;
-    return sdesc(a, slab_bytes, 1024);
+    return desc_from_lo(desc_lo(tile_saddr, slab_bytes) + mnmajor_step(k16));
+}
+
+// One accumulation chain of n MMAs (K = 16 each) with the loop kept rolled:
+// A and B are shared-memory tiles given by descriptor low words, K-major
+// (slab bytes apart every 4 steps) or MN-major.  A short loop keeps the MMA
+// issuer's instruction stream small.
+template <bool A_KMAJOR, bool B_KMAJOR>
+__device__ __forceinline__ void umma_chain(uint32_t d_tmem, uint32_t a_lo, uint32_t a_slab, uint32_t b_lo,
+                                           uint32_t b_slab, uint32_t idesc, int n, bool acc) {
+    #pragma unroll 1
+    for (int kk = 0; kk < n; ++kk) {
+        const uint32_t ao = A_KMAJOR ? kmajor_step(kk, a_slab) : mnmajor_step(kk);
+        const uint32_t bo = B_KMAJOR ? kmajor_step(kk, b_slab) : mnmajor_step(kk);
+        umma_f16(d_tmem, desc_from_lo(a_lo + ao), desc_from_lo(b_lo + bo), idesc, (acc || kk > 0) ? 1u : 0u);
+    }
+}
+// The same with A (M x K, 16-bit) in TMEM: 8 columns per K step.
+template <bool B_KMAJOR>
+__device__ __forceinline__ void umma_chain_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_slab,
+                                              uint32_t idesc, int n, bool acc) {
+    #pragma unroll 1
+    for (int kk = 0; kk < n; ++kk) {
+        const uint32_t bo = B_KMAJOR ? kmajor_step(kk, b_slab) : mnmajor_step(kk);
+        umma_f16_ts(d_tmem, a_tmem + 8 * kk, desc_from_lo(b_lo + bo), idesc, (acc || kk > 0) ? 1u : 0u);
+    }
 }
 
 // Instruction descriptor, kind::f16 with fp16 A/B and fp32 accumulate.
