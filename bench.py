@@ -46,6 +46,8 @@ def args_():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="attention sample budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip the dense same-shape comparison (torch SDPA and all-blocks Prism)")
     return ap.parse_args()
 
 
@@ -231,6 +233,70 @@ def run_reference(a, rank, world):
           "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
 
 
+def dense_same_shape(Q, K, V, dO, amap, w, ws, O, lse, dQ, dK, dV, h, peak):
+    """Dense attention over all N tokens of one head, fwd + bwd (14 D N^2 flops):
+    torch SDPA (flash and cuDNN back ends, where available) and this library with
+    every block selected (k >= N_b, p = 1)."""
+    import torch
+    from dynamic_block_sparse_indicator_b200 import _lib
+    D, N = w.head_dim, w.N
+    flops = 14.0 * D * float(N) ** 2
+    out = {"flops": flops, "tokens": N}
+
+    def timed(fn, reps=1):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    q = Q[h:h + 1].unsqueeze(0).to(torch.bfloat16).detach().requires_grad_(True)
+    k = K[h:h + 1].unsqueeze(0).to(torch.bfloat16).detach().requires_grad_(True)
+    v = V[h:h + 1].unsqueeze(0).to(torch.bfloat16).detach().requires_grad_(True)
+    g = dO[h:h + 1].unsqueeze(0).to(torch.bfloat16)
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        backends = {"sdpa_flash": SDPBackend.FLASH_ATTENTION, "sdpa_cudnn": SDPBackend.CUDNN_ATTENTION}
+    except ImportError:
+        backends = {}
+    for name, be in backends.items():
+        try:
+            def run():
+                with sdpa_kernel([be]):
+                    o = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+                torch.autograd.backward(o, g)
+                q.grad = k.grad = v.grad = None
+            ms = timed(run)
+            out[name] = {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12}
+        except Exception as exc:  # noqa: BLE001
+            out[name] = {"unavailable": str(exc).splitlines()[0][:160]}
+    del q, k, v, g
+    params = _lib.make_params(w.T, w.H, w.W, 1, D, _lib.PRISM_BF16, 1 << 30, 1.0, w.eps,
+                              out_dtype=_lib.PRISM_F32)
+
+    last = []
+
+    def prism_all():
+        pl = _lib.plan(Q[h:h + 1], K[h:h + 1], V[h:h + 1], amap, params, workspace=ws)
+        pl.attn_fwd(O, lse)
+        pl.attn_bwd(dO[h:h + 1], O, lse, dQ, dK, dV)
+        last[:] = [pl]
+
+    ms = timed(prism_all)
+    st = last[0].status()
+    if st:
+        raise RuntimeError(f"device status (all blocks): {_lib.status_string(st)}")
+    last.clear()
+    out["prism_all_blocks"] = {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                               "fraction_of_peak": flops / (ms * 1e-3) / 1e12 / peak,
+                               "note": "plan + fwd + bwd with k >= N_b and p = 1 (every block selected)"}
+    return out
+
+
 def run_prism(a, rank, world, local_rank):
     import numpy as np
     import torch
@@ -292,6 +358,7 @@ def run_prism(a, rank, world, local_rank):
     launches = 0
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     plans = []
+    _lib.profile_plans(True)          # the timed plans also time their own kernels
     with ClockSampler(local_rank) as clk:
         barrier()
         e0.record()
@@ -300,6 +367,7 @@ def run_prism(a, rank, world, local_rank):
             plans.append(pl)
         e1.record()
         barrier()
+    _lib.profile_plans(False)
     clocks = clk.summary()
     elapsed = e0.elapsed_time(e1)
     elapsed_max = max_over_ranks(elapsed, world, dev)
@@ -338,6 +406,29 @@ def run_prism(a, rank, world, local_rank):
     attn_ms = (stage_ms["fwd"] + stage_ms["bwd_pre"] + stage_ms["bwd_dkdv"] + stage_ms["bwd_dq"]) / a.steps
     attn_tflops = 14 * D * Pi / (attn_ms * 1e-3) / 1e12
     value = elapsed_max / (a.steps * world)
+    # plan kernels against their own bounds: HBM for the statistics (one read of
+    # V) and the gather (Q, K, V read, fp16 copies written); plain ALU for the
+    # block scores (2 D N_b^2 flops + N_b^2 exp)
+    hbm = pk.get("hbm_gbs") or 6650.0
+    per_head = lambda k: stage_ms[k] / a.steps
+    stats_bytes = 2.0 * D * w.N + 4.0 * w.N
+    gather_bytes = 12.0 * D * w.N
+    plan_kernels = {
+        "stats": {"ms": per_head("plan_stats"), "bytes": stats_bytes,
+                  "GB/s": stats_bytes / (per_head("plan_stats") * 1e-3) / 1e9 if per_head("plan_stats") else None},
+        "shapes": {"ms": per_head("plan_shapes")},
+        "gather": {"ms": per_head("plan_gather"), "bytes": gather_bytes,
+                   "GB/s": gather_bytes / (per_head("plan_gather") * 1e-3) / 1e9 if per_head("plan_gather") else None},
+        "select": {"ms": per_head("plan_select"), "flops": 2.0 * D * nb_mean ** 2, "exp": nb_mean ** 2,
+                   "GFLOP/s": 2.0 * D * nb_mean ** 2 / (per_head("plan_select") * 1e-3) / 1e9
+                   if per_head("plan_select") else None},
+        "lists": {"ms": per_head("plan_lists")},
+        "hbm_peak_GB/s": hbm, "peak_source": "measured" if pk.get("hbm_gbs") else "fallback",
+    }
+    # ------------------------------------------- dense attention of the same shape
+    dense = None
+    if world == 1 and not a.no_dense:
+        dense = dense_same_shape(Q, K, V, dO, amap, w, ws, O, lse, dQ, dK, dV, order[a.warmup], peak)
     # --------------------------------------------------- end to end (host)
     e2e = None
     if a.e2e_steps > 0:
@@ -397,6 +488,7 @@ def run_prism(a, rank, world, local_rank):
                                       "bwd_dq": "k_dq_finalize" if fused else "k_bwd_dq"}[dom],
                            "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                            "frac": ach / peak, "peak_source": peak_src, "traffic": None},
+              "plan_kernels": plan_kernels, "dense_same_shape": dense,
               "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks})
 
 

@@ -78,6 +78,7 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_status_string": (C.c_char_p, [i32]),
         "prism_version": (C.c_char_p, []),
         "prism_profile_enable": (i32, [vp, i32]),
+        "prism_profile_plans": (i32, [i32]),
         "prism_profile_read": (i32, [vp, C.POINTER(C.c_float), C.POINTER(C.c_int), vp]),
         "prism_launch_count": (C.c_int64, [vp]),
         "prism_zone_shapes_noalloc": (i32, [pp, vp, vp, vp, vp, vp]),
@@ -88,6 +89,11 @@ def load(path: str | None = None) -> C.CDLL:
         f.argtypes = args
     _lib = lib
     return lib
+
+
+def profile_plans(on: bool = True) -> bool:
+    """Plans created afterwards time their own plan kernels (process-wide); returns the old setting."""
+    return bool(load().prism_profile_plans(1 if on else 0))
 
 
 def status_string(st: int) -> str:
@@ -180,7 +186,8 @@ class Plan:
             raise PrismError(st, f"prism_plan_export({item})")
         return out
 
-    STAGES = ("fwd", "bwd_pre", "bwd_dkdv", "bwd_dq")
+    STAGES = ("fwd", "bwd_pre", "bwd_dkdv", "bwd_dq", "plan_stats", "plan_shapes", "plan_gather",
+              "plan_select", "plan_lists")
 
     def profile(self, on: bool = True):
         load().prism_profile_enable(self._h, 1 if on else 0)

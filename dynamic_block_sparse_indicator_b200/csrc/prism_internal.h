@@ -81,12 +81,15 @@ struct PrismProf {
         if (P->profile && cudaEventCreate(&a) == cudaSuccess && cudaEventCreate(&b) == cudaSuccess)
             cudaEventRecord(a, s);
     }
-    ~PrismProf() {
+    // records the closing event now (idempotent; the destructor calls it)
+    void close() {
         if (a && b) {
             cudaEventRecord(b, s);
             P->timed.push_back({stage, a, b});
+            a = b = nullptr;
         }
     }
+    ~PrismProf() { close(); }
 };
 
 // Internal entry points of the attention translation units.

@@ -978,6 +978,8 @@ static int check_device() {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+static int g_profile_plans = 0;   // prism_profile_plans: timing state of new plans
+
 static int plan_common(const prism_params* p, const void* Q, const void* K, const void* V,
                        void* workspace, size_t ws_bytes, prism_plan_s** outP) {
     int st = validate_params(p);
@@ -997,6 +999,7 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
     P->L = L;
     P->ws = static_cast<char*>(workspace);
     P->ws_bytes = ws_bytes;
+    P->profile = g_profile_plans;
     cudaGetDevice(&P->device);
     const int64_t rows = (int64_t)g.heads * g.N;
     st = make_tmap(&P->tm_q, P->ws + L.qp, rows, g.D, 128);
@@ -1058,6 +1061,7 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
     cudaMemsetAsync(P->ws + P->L.err, 0, 16, s);
     const bool bf = p.dtype == PRISM_BF16;
     if (!given_shapes) {
+        PrismProf prof(P, PRISM_STAGE_PLAN_STATS, s);
         if (amap) {
             k_audio_zone<<<g.Nz, 256, 0, s>>>(d, amap);
             k_audio_norm<<<1, 1024, 0, s>>>(d);
@@ -1071,14 +1075,21 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
     } else {
         cudaMemcpyAsync(d.shape_id, given_shapes, (size_t)g.heads * g.Nz, cudaMemcpyDeviceToDevice, s);
     }
-    const size_t fin_smem = sizeof(int) * (g.Nz + 1);
-    if (fin_smem > 48 * 1024)
-        cudaFuncSetAttribute(k_zone_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
-    k_zone_finalize<<<g.heads, 1024, fin_smem, s>>>(d, p.eps, p.tau128, p.tau256, given_shapes ? 1 : 0);
-    if (bf && g.D == 128) launch_gather<__nv_bfloat16, 128>(P, d, Q, K, V, s);
-    else if (bf) launch_gather<__nv_bfloat16, 64>(P, d, Q, K, V, s);
-    else if (g.D == 128) launch_gather<float, 128>(P, d, Q, K, V, s);
-    else launch_gather<float, 64>(P, d, Q, K, V, s);
+    {
+        PrismProf prof(P, PRISM_STAGE_PLAN_SHAPES, s);
+        const size_t fin_smem = sizeof(int) * (g.Nz + 1);
+        if (fin_smem > 48 * 1024)
+            cudaFuncSetAttribute(k_zone_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
+        k_zone_finalize<<<g.heads, 1024, fin_smem, s>>>(d, p.eps, p.tau128, p.tau256, given_shapes ? 1 : 0);
+    }
+    {
+        PrismProf prof(P, PRISM_STAGE_PLAN_GATHER, s);
+        if (bf && g.D == 128) launch_gather<__nv_bfloat16, 128>(P, d, Q, K, V, s);
+        else if (bf) launch_gather<__nv_bfloat16, 64>(P, d, Q, K, V, s);
+        else if (g.D == 128) launch_gather<float, 128>(P, d, Q, K, V, s);
+        else launch_gather<float, 64>(P, d, Q, K, V, s);
+    }
+    PrismProf prof_sel(P, PRISM_STAGE_PLAN_SELECT, s);
     if (!given_sel) {
         const size_t sm = sizeof(float) * g.NB;
         if (g.D == 128) {
@@ -1094,7 +1105,11 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
         k_mask_bits<<<dim3(256, g.heads), 256, 0, s>>>(d.sel, d.nblocks, g.NB, g.WORDS);
         k_row_popc<<<dim3((g.NB + 255) / 256, g.heads), 256, 0, s>>>(d.sel, d.row_ptr, d.nblocks, g.NB, g.WORDS);
     }
-    launch_lists(P, d, s);
+    prof_sel.close();
+    {
+        PrismProf prof(P, PRISM_STAGE_PLAN_LISTS, s);
+        launch_lists(P, d, s);
+    }
     return cuda_status(cudaGetLastError());
 }
 
@@ -1215,6 +1230,12 @@ extern "C" void prism_plan_destroy(prism_plan_t P) {
     if (!P) return;
     drop_events(P);
     delete P;
+}
+
+extern "C" int prism_profile_plans(int on) {
+    const int prev = g_profile_plans;
+    g_profile_plans = on ? 1 : 0;
+    return prev;
 }
 
 extern "C" int prism_profile_enable(prism_plan_t P, int on) {

@@ -241,10 +241,23 @@ PRISM_API const char* prism_status_string(int status);
 #define PRISM_STAGE_BWD_PRE   1  /* dO scaling, D_i, block-order dO     */
 #define PRISM_STAGE_BWD_DKDV  2  /* dK, dV per key tile                 */
 #define PRISM_STAGE_BWD_DQ    3  /* dQ per query tile                   */
-#define PRISM_STAGE_COUNT     4
+/* Plan stages, timed only for plans created while prism_profile_plans(1) is
+ * in force (the plan is built inside prism_plan, before a handle exists). */
+#define PRISM_STAGE_PLAN_STATS  4  /* audio terms + zone statistics of V    */
+#define PRISM_STAGE_PLAN_SHAPES 5  /* finalize: g_d, B, l*, snapped shapes  */
+#define PRISM_STAGE_PLAN_GATHER 6  /* block-order fp16 Q, K, V + pooled means */
+#define PRISM_STAGE_PLAN_SELECT 7  /* block scores, Top-k u Top-p selection  */
+#define PRISM_STAGE_PLAN_LISTS  8  /* CSR, CSC and the per-tile lists        */
+#define PRISM_STAGE_COUNT       9
 
 /* Turns per-stage timing on (1) or off (0) for later calls on this plan. */
 PRISM_API int prism_profile_enable(prism_plan_t plan, int on);
+
+/* Process-wide switch: plans created after prism_profile_plans(1) start with
+ * timing on and record their own plan kernels under PRISM_STAGE_PLAN_*
+ * (read back with prism_profile_read).  Returns the previous setting.  Not
+ * synchronised with concurrent prism_plan calls on other host threads. */
+PRISM_API int prism_profile_plans(int on);
 
 /* Synchronises `stream`, writes the milliseconds spent per stage (and the
  * number of launches per stage into `launches`, may be NULL) since the last
