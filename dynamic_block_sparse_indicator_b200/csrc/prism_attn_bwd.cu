@@ -196,14 +196,14 @@ struct DkdvSmem {
     alignas(16) float di[DKDV_STAGES][64];
     uint64_t bar_kv;
     uint64_t st_full[DKDV_STAGES], st_empty[DKDV_STAGES];
-    uint64_t s_full[2], s_free[2], p_full[2], pd_done[2];
+    uint64_t s_full[2], p_full[2], pd_done[2];
     uint64_t acc_done;                        // every MMA of the CTA has completed
     uint64_t dq_full[2], dq_free[2];
     uint32_t tmem_base;
 };
 
 template <int HD, bool FUSE>
-__global__ void __launch_bounds__(FUSE ? 448 : 320, 1)
+__global__ void __launch_bounds__(FUSE ? 480 : 352, 1)
 k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
            const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
            const __grid_constant__ CUtensorMap tm_dq, BwdArgs a) {
@@ -230,7 +230,6 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         for (int s = 0; s < DKDV_STAGES; ++s) { mbar_init(&sm.st_full[s], 1); mbar_init(&sm.st_empty[s], 1); }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.s_free[b], 256);
             mbar_init(&sm.p_full[b], 256);
             mbar_init(&sm.pd_done[b], 1);
             mbar_init(&sm.dq_full[b], 1);
@@ -239,9 +238,13 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         mbar_fence_init();
     }
     // warps 0-7: two softmax warpgroups (same 128 key rows, one 32-query half of
-    // the unit each); warp 8: TMA producer + TMEM allocator; warp 9: MMA issuer;
-    // warps 10-13 (FUSE): dQ drain.
-    constexpr int W_PROD = 8, W_MMA = 9;
+    // the unit each); warp 8: TMA producer + TMEM allocator; warp 9: issuer of
+    // S^T and dP^T; warps 10-13 (FUSE): dQ drain; warp 14 (10 without FUSE):
+    // issuer of dV, dQ^T and dK.  Two issuers on different SM sub-partitions:
+    // an issuing thread that waits on a barrier stalls until its queued MMAs
+    // have been handed to the tensor core, so with one issuer every wait left
+    // the tensor pipe idle; each issuer now waits while the other one feeds it.
+    constexpr int W_PROD = 8, W_MMA = 9, W_MMB = FUSE ? 14 : 10;
     if (warp == W_PROD) { __syncwarp(); tmem_alloc(&sm.tmem_base, 512); }
     tc_fence_before();
     __syncthreads();
@@ -274,67 +277,76 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             }
         }
     } else if (warp == W_MMA) {
+        // ------------------------------------------------ S^T and dP^T issuer
         if (lane == 0 && U > 0) {
             constexpr uint32_t id_s = idesc_f16(128, 64, 0, 0);
-            constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
-            constexpr uint32_t id_dq = idesc_f16(128, 64, 1, 1);
             // descriptor low words; every K step below adds an immediate
             const uint32_t kA = desc_lo(smem_u32(sm.k[0]), 16), vA = desc_lo(smem_u32(sm.v[0]), 16);
-            const uint32_t kT = desc_lo(smem_u32(sm.k[0]), SLAB128);       // K^T (MN-major) for dQ^T
             bool ok = mbar_wait(&sm.bar_kv, 0, a.err, 1501);
-            int u = 0;
-            for (; ok && u <= U; ++u) {
-                if (u < U) {
-                    const int s = u % DKDV_STAGES, b = u & 1;
-                    if (!mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1502)) break;
-                    // both softmax warpgroups have loaded S^T(u - 2)
-                    if (u >= 2 && !mbar_wait(&sm.s_free[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
-                    tc_fence_after();
-                    const uint32_t qB = desc_lo(smem_u32(sm.q[s][0]), 16), doB = desc_lo(smem_u32(sm.dO[s][0]), 16);
-                    #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + 128 * b, desc_from_lo(kA + kmajor_step(kk, SLAB128)),
-                                 desc_from_lo(qB + kmajor_step(kk, SLAB64)), id_s, kk > 0);
-                    // dP^T overwrites dQ^T(u - 2): wait until the drain has read it
-                    if (FUSE && u >= 2 && !mbar_wait(&sm.dq_free[b], ((u - 2) >> 1) & 1, a.err, 1505)) break;
-                    tc_fence_after();
-                    #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + 128 * b + 64, desc_from_lo(vA + kmajor_step(kk, SLAB128)),
-                                 desc_from_lo(doB + kmajor_step(kk, SLAB64)), id_s, kk > 0);
-                    umma_commit(&sm.s_full[b]);
+            for (int u = 0; ok && u < U; ++u) {
+                const int s = u % DKDV_STAGES, b = u & 1;
+                if (!mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1502)) break;
+                // the softmax is done with unit u - 2: S^T(u - 2) has been read
+                if (u >= 2 && !mbar_wait(&sm.p_full[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
+                tc_fence_after();
+                const uint32_t qB = desc_lo(smem_u32(sm.q[s][0]), 16), doB = desc_lo(smem_u32(sm.dO[s][0]), 16);
+                #pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_f16(tmem + 128 * b, desc_from_lo(kA + kmajor_step(kk, SLAB128)),
+                             desc_from_lo(qB + kmajor_step(kk, SLAB64)), id_s, kk > 0);
+                // dP^T overwrites P^T(u - 2) and (FUSE) dQ^T(u - 2): wait until dV(u - 2)
+                // has read P^T (pd_done) and the drain has read dQ^T (dq_free)
+                if (u >= 2) {
+                    if (FUSE ? !mbar_wait(&sm.dq_free[b], ((u - 2) >> 1) & 1, a.err, 1505)
+                             : !mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1506))
+                        break;
                 }
-                if (u >= 1) {
-                    const int uu = u - 1, b = uu & 1, s = uu % DKDV_STAGES;
-                    if (!mbar_wait(&sm.p_full[b], (uu >> 1) & 1, a.err, 1504)) break;
-                    tc_fence_after();
-                    const uint32_t dsA = desc_lo(smem_u32(sm.ds[b]), 16);          // dS^T, K-major
-                    const uint32_t dsT = desc_lo(smem_u32(sm.ds[b]), SLAB128);     // dS^T as MN-major B
-                    const uint32_t qT = desc_lo(smem_u32(sm.q[s][0]), SLAB64);
-                    const uint32_t doT = desc_lo(smem_u32(sm.dO[s][0]), SLAB64);
-                    // dV += P^T dO with P^T (fp16) read from TMEM over the dP^T columns
-                    #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tmem + TDV, tmem + 128 * b + 64 + 8 * kk, desc_from_lo(doT + mnmajor_step(kk)),
-                                    id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
-                    if (FUSE) {
-                        // dQ^T [HD x 64 queries] = K^T [HD x 128 keys] . dS^T [128 keys x 64 queries],
-                        // over the dP^T columns (after dV above has read P^T there)
-                        #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_f16(tmem + 128 * b + 64, desc_from_lo(kT + mnmajor_step(kk)),
-                                     desc_from_lo(dsT + mnmajor_step(kk)), id_dq, kk > 0);
-                        umma_commit(&sm.dq_full[b]);
-                    }
-                    #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + TDK, desc_from_lo(dsA + kmajor_step(kk, SLAB128)),
-                                 desc_from_lo(qT + mnmajor_step(kk)), id_acc, (uu > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&sm.pd_done[b]);
-                    umma_commit(&sm.st_empty[s]);
-                }
+                tc_fence_after();
+                #pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    umma_f16(tmem + 128 * b + 64, desc_from_lo(vA + kmajor_step(kk, SLAB128)),
+                             desc_from_lo(doB + kmajor_step(kk, SLAB64)), id_s, kk > 0);
+                umma_commit(&sm.s_full[b]);
             }
-            if (u > U) umma_commit(&sm.acc_done);   // dV and dK are final
+        }
+    } else if (warp == W_MMB) {
+        // ------------------------------------------------ dV, dQ^T and dK issuer
+        if (lane == 0 && U > 0) {
+            constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
+            constexpr uint32_t id_dq = idesc_f16(128, 64, 1, 1);
+            const uint32_t kT = desc_lo(smem_u32(sm.k[0]), SLAB128);       // K^T (MN-major) for dQ^T
+            int u = 0;
+            for (; u < U; ++u) {
+                const int b = u & 1, s = u % DKDV_STAGES;
+                // P^T (TMEM) and dS^T (shared memory) of unit u are complete
+                if (!mbar_wait(&sm.p_full[b], (u >> 1) & 1, a.err, 1504)) break;
+                tc_fence_after();
+                const uint32_t dsA = desc_lo(smem_u32(sm.ds[b]), 16);          // dS^T, K-major
+                const uint32_t dsT = desc_lo(smem_u32(sm.ds[b]), SLAB128);     // dS^T as MN-major B
+                const uint32_t qT = desc_lo(smem_u32(sm.q[s][0]), SLAB64);
+                const uint32_t doT = desc_lo(smem_u32(sm.dO[s][0]), SLAB64);
+                // dV += P^T dO with P^T (fp16) read from TMEM over the dP^T columns
+                #pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16_ts(tmem + TDV, tmem + 128 * b + 64 + 8 * kk, desc_from_lo(doT + mnmajor_step(kk)),
+                                id_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                if (FUSE) {
+                    // dQ^T [HD x 64 queries] = K^T [HD x 128 keys] . dS^T [128 keys x 64 queries],
+                    // over the dP^T columns (after dV above has read P^T there)
+                    #pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16(tmem + 128 * b + 64, desc_from_lo(kT + mnmajor_step(kk)),
+                                 desc_from_lo(dsT + mnmajor_step(kk)), id_dq, kk > 0);
+                    umma_commit(&sm.dq_full[b]);
+                }
+                #pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + TDK, desc_from_lo(dsA + kmajor_step(kk, SLAB128)),
+                             desc_from_lo(qT + mnmajor_step(kk)), id_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&sm.pd_done[b]);
+                umma_commit(&sm.st_empty[s]);
+            }
+            if (u == U) umma_commit(&sm.acc_done);   // dV and dK are final
         }
     } else if (warp < 8) {
         const int wg = warp >> 2;                   // which 32 queries of the unit
@@ -356,8 +368,6 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             PRISM_TMEM_LD32(tmem + lane_off + 128 * b + c0, sv);
             PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64 + c0, dp);
             tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.s_free[b]);
             // both warpgroups of this lane quarter have read dP^T before P^T overwrites it
             named_bar(2 + (warp & 3), 64);
             ++nbar;
@@ -712,7 +722,7 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
         return PRISM_ERR_CUDA;
     {
         PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
-        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, g.heads), FUSE ? 448 : 320, sm1, s>>>(
+        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, g.heads), FUSE ? 480 : 352, sm1, s>>>(
             P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, a);
     }
     if (FUSE) {
