@@ -14,14 +14,17 @@
 //               by an exact per-head power of two so that max |dO| lies in
 //               [0.5, 1): gradients of any magnitude keep fp16's precision and
 //               dS cannot overflow), LSE in block order.
-//   k_bwd_dkdv  one CTA per 128-key tile; iterates the 64-row query halves of
-//               the key tile's transposed list; S^T = K Q^T and dP^T = V dO^T
-//               into TMEM (double-buffered), softmax warps form P^T (into TMEM, over
+//   k_bwd_dkdv  one CTA per (128-key tile, chunk of 512 query tiles); iterates
+//               the 64-row query halves of that range of the key tile's
+//               transposed list; S^T = K Q^T and dP^T = V dO^T into TMEM
+//               (double-buffered), softmax warps form P^T (into TMEM, over
 //               dP^T) and dS^T (fp16 shared memory), dV += P^T dO and
-//               dK += dS^T Q accumulate in TMEM.
-//               For head_dim 128 the same CTA also forms dQ^T = K^T dS^T per
-//               unit and TMA reduce-adds it into an fp32 accumulator
-//               (k_dq_finalize scatters it to raster order).
+//               dK += dS^T Q accumulate in TMEM and are TMA reduce-added into
+//               fp32 accumulators at the end of the chunk.  For head_dim 128
+//               the same CTA also forms dQ^T = K^T dS^T per unit and TMA
+//               reduce-adds it into an fp32 accumulator.  The grid runs chunk
+//               by chunk, so the dQ rows being accumulated stay in L2.
+//   k_acc_finalize  scales the accumulators and scatters them to raster order.
 //   k_bwd_dq    (head_dim 64) one CTA per 128-row query tile; iterates the
 //               64-key halves of the forward list; S = Q K^T, dP = dO V^T,
 //               dS -> shared memory, dQ += dS K in TMEM.
@@ -40,6 +43,7 @@ namespace prism {
 
 constexpr int BWD_STAGES = 2;
 constexpr int DKDV_STAGES = 3;   // Q/dO prefetch depth of the dK/dV kernel
+constexpr int kChunkTiles = 512; // query tiles per chunk of the dK/dV grid
 constexpr int SLAB128 = 128 * 128;   // bytes: 128 rows x 64 fp16
 constexpr int SLAB64 = 64 * 128;     // bytes:  64 rows x 64 fp16
 constexpr float kLog2e = 1.4426950408889634f;
@@ -148,8 +152,20 @@ struct BwdArgs {
     int out_f32;
     float scale_log2;      // log2(e) / sqrt(d)
     float inv_sqrt_d;
+    int CQ;                // query tiles per chunk of the dK/dV grid
     int* err;
 };
+
+// First index in the ascending list e[0, n) whose tile (entry >> 4) is >= key.
+__device__ __forceinline__ int tiles_lower_bound(const int* e, int n, int key) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((e[mid] >> 4) < key) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
 
 __device__ __forceinline__ void store_row(void* base, size_t row, int HD, int c0, const uint32_t* v,
                                           float mul, int out_f32) {
@@ -200,23 +216,45 @@ struct DkdvSmem {
     uint64_t acc_done;                        // every MMA of the CTA has completed
     uint64_t dq_full[2], dq_free[2];
     uint32_t tmem_base;
+    int e0, ne, U;                            // this chunk's entries and 64-query units
 };
+
+// the dK / dV epilogue stages 8 warps x 32 rows x HD fp32 values in q, dO and ds
+template <int HD, bool FUSE>
+constexpr bool epilogue_fits() {
+    using S = DkdvSmem<HD, FUSE>;
+    return offsetof(S, stage_dq) - offsetof(S, q) >= 8 * 32 * HD * sizeof(float);
+}
 
 template <int HD, bool FUSE>
 __global__ void __launch_bounds__(FUSE ? 480 : 352, 1)
 k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
            const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
-           const __grid_constant__ CUtensorMap tm_dq, BwdArgs a) {
+           const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+           const __grid_constant__ CUtensorMap tm_dv, BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     DkdvSmem<HD, FUSE>& sm = *reinterpret_cast<DkdvSmem<HD, FUSE>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NSL = HD / 64;
-    const int t = blockIdx.x, h = blockIdx.y;
+    // one CTA per (key tile t, chunk c of CQ query tiles): the grid runs chunk
+    // after chunk, so the dQ accumulator rows and the Q / dO tiles that all CTAs
+    // in flight touch are one chunk's (about 32 MB), resident in L2
+    const int t = blockIdx.x, c = blockIdx.y, h = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e0 = a.ptr[(size_t)h * (a.NT + 1) + t];
-    const int ne = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - e0;
+    if (threadIdx.x == 0) {
+        const int p0 = a.ptr[(size_t)h * (a.NT + 1) + t];
+        const int n0 = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - p0;
+        const int* all = a.ent + (size_t)h * a.NT * a.NT + p0;
+        const int lo = tiles_lower_bound(all, n0, c * a.CQ);
+        const int hi = tiles_lower_bound(all, n0, (c + 1) * a.CQ);
+        sm.e0 = p0 + lo;
+        sm.ne = hi - lo;
+        sm.U = count_units(all + lo, hi - lo, 1);
+    }
+    __syncthreads();
+    const int e0 = sm.e0, ne = sm.ne, U = sm.U;
+    if (U == 0) return;                            // nothing selected in this chunk
     const int* ents = a.ent + (size_t)h * a.NT * a.NT + e0;
-    const int U = count_units(ents, ne, 1);
     // TMEM columns: buffer b = [128b, 128b + 128): S^T at 128b, dP^T at 128b + 64.
     // The softmax writes P^T (fp16 pairs) over the first half of dP^T; dQ^T of
     // the unit then overwrites all 64 dP^T columns after dV has read P^T (the
@@ -408,26 +446,36 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         // a warp that left the loop on a failed wait still takes the barriers
         // the other warpgroup will take, so that one is never left at a barrier
         for (; nbar < U; ++nbar) named_bar(2 + (warp & 3), 64);
-        // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (same rows)
-        const size_t orow = (size_t)hrow + (size_t)a.src[(size_t)hrow + (size_t)t * 128 + r];
-        void* out = wg ? a.out0 : a.out1;
+        // epilogue: this chunk's share of dV (warpgroup 0) and dK (warpgroup 1)
+        // is TMA reduce-added into the fp32 accumulators (block order, unscaled).
+        // Each warp stages its 32 rows in the Q / dO / dS^T buffers, idle once
+        // every MMA of the CTA has completed (8 x 32 x HD floats fit there).
         bool fin = false;
-        if (ok && U > 0)
+        if (ok)
             fin = __all_sync(0xffffffffu, mbar_wait(&sm.acc_done, 0, a.err, 1004));
         if (fin) {
             tc_fence_after();
-            const float unscale = ldexpf(1.f, dscale_exp(a.dmax[h], a.err));
-            const float mul = wg ? a.inv_sqrt_d * unscale : unscale / kPScale;
+            float* stage = reinterpret_cast<float*>(&sm.q[0][0][0]) + (size_t)warp * 32 * HD;
             const uint32_t col = wg ? TDK : TDV;
             #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
+            for (int c4 = 0; c4 < HD / 32; ++c4) {
                 uint32_t o[32];
-                PRISM_TMEM_LD32(tmem + lane_off + col + 32 * c, o);
+                PRISM_TMEM_LD32(tmem + lane_off + col + 32 * c4, o);
                 tmem_wait_ld();
-                store_row(out, orow, HD, 32 * c, o, mul, a.out_f32);
+                float4* dst = reinterpret_cast<float4*>(stage + (size_t)lane * HD + 32 * c4);
+                #pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                         __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
             }
-        } else if (U == 0) {
-            zero_row(out, orow, HD, a.out_f32);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_reduce_add_2d(wg ? &tm_dk : &tm_dv, stage, 0, (int)(hrow + (int64_t)t * 128 + 32 * (warp & 3)));
+                bulk_commit();
+                bulk_wait0();
+            }
+            __syncwarp();
         }
     } else if (FUSE && warp >= 10) {
         // ---------------------------------------------- dQ drain (warps 10-13)
@@ -473,20 +521,24 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     if (warp == W_PROD) { __syncwarp(); tmem_dealloc(tmem, 512); }
 }
 
-// dQ accumulator (block order, fp32) -> dQ output (raster order, scaled).
+// fp32 accumulators (block order, unscaled) -> outputs (raster order): one
+// warp per row p, out[src[p]] = acc[p] * scale * 2^-e (the per-head dO scale).
+// Two accumulators (dK, dV) or one (dQ, acc1 == nullptr) per launch.
 template <typename OT>
-__global__ void __launch_bounds__(256) k_dq_finalize(const float* __restrict__ acc, const int* __restrict__ src,
-                                                     const uint32_t* dmax, OT* __restrict__ dQ, int64_t N,
-                                                     int HD, float inv_sqrt_d, int* err) {
+__global__ void __launch_bounds__(256) k_acc_finalize(const float* __restrict__ acc0, float scale0, OT* __restrict__ out0,
+                                                      const float* __restrict__ acc1, float scale1,
+                                                      OT* __restrict__ out1, const int* __restrict__ src,
+                                                      const uint32_t* dmax, int64_t N, int HD, int* err) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t p = (int64_t)blockIdx.x * 8 + warp;
     const int h = blockIdx.y;
     if (p >= N) return;
-    const float mul = inv_sqrt_d * ldexpf(1.f, dscale_exp(dmax[h], err));
+    const float unscale = ldexpf(1.f, dscale_exp(dmax[h], err));
     const int64_t n = src[(size_t)h * N + p];
-    const float* in = acc + ((size_t)h * N + p) * HD;
-    OT* out = dQ + ((size_t)h * N + n) * HD;
-    for (int c = lane; c < HD; c += 32) out[c] = (OT)(in[c] * mul);
+    const size_t ir = ((size_t)h * N + p) * HD, orow = ((size_t)h * N + n) * HD;
+    for (int c = lane; c < HD; c += 32) out0[orow + c] = (OT)(acc0[ir + c] * (scale0 * unscale));
+    if (acc1)
+        for (int c = lane; c < HD; c += 32) out1[orow + c] = (OT)(acc1[ir + c] * (scale1 * unscale));
 }
 
 // ------------------------------------------------------------------------ dQ
@@ -715,24 +767,43 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     a.ent = (const int*)(b + P->L.kt_ent);
     a.out0 = dK;
     a.out1 = dV;
+    static_assert(epilogue_fits<HD, FUSE>(), "dK/dV staging does not fit in the Q/dO/dS buffers");
     float* dq_acc = (float*)(b + P->L.dq_acc);
-    if (FUSE) cudaMemsetAsync(dq_acc, 0, sizeof(float) * (size_t)g.heads * g.N * HD, s);
+    float* dk_acc = (float*)(b + P->L.dk_acc);
+    float* dv_acc = (float*)(b + P->L.dv_acc);
+    const size_t acc_bytes = sizeof(float) * (size_t)g.heads * g.N * HD;
     const int sm1 = (int)sizeof(DkdvSmem<HD, FUSE>) + 1024;
     if (cudaFuncSetAttribute(k_bwd_dkdv<HD, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1) != cudaSuccess)
         return PRISM_ERR_CUDA;
+    // chunks of kChunkTiles query tiles (65536 tokens): about 32 MB of dQ
+    // accumulator per chunk, so the reduce-adds of the CTAs in flight stay in L2
+    a.CQ = kChunkTiles;
+    const unsigned chunks = (unsigned)((g.NT + kChunkTiles - 1) / kChunkTiles);
+    const dim3 gfin((unsigned)((g.N + 7) / 8), g.heads);
+    P->launches += 1;
     {
         PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
-        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, g.heads), FUSE ? 480 : 352, sm1, s>>>(
-            P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, a);
+        if (FUSE) cudaMemsetAsync(dq_acc, 0, acc_bytes, s);
+        cudaMemsetAsync(dk_acc, 0, acc_bytes, s);
+        cudaMemsetAsync(dv_acc, 0, acc_bytes, s);
+        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, chunks, g.heads), FUSE ? 480 : 352, sm1, s>>>(
+            P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, P->tm_dk, P->tm_dv, a);
+        if (a.out_f32)
+            k_acc_finalize<float><<<gfin, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (float*)dK, dv_acc, 1.f / kPScale,
+                                                       (float*)dV, src, dmax, g.N, HD, err);
+        else
+            k_acc_finalize<__nv_bfloat16><<<gfin, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (__nv_bfloat16*)dK, dv_acc,
+                                                               1.f / kPScale, (__nv_bfloat16*)dV, src, dmax, g.N,
+                                                               HD, err);
     }
     if (FUSE) {
         PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
-        const dim3 gfin((unsigned)((g.N + 7) / 8), g.heads);
         if (a.out_f32)
-            k_dq_finalize<float><<<gfin, 256, 0, s>>>(dq_acc, src, dmax, (float*)dQ, g.N, HD, a.inv_sqrt_d, err);
+            k_acc_finalize<float><<<gfin, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (float*)dQ, nullptr, 0.f, nullptr,
+                                                       src, dmax, g.N, HD, err);
         else
-            k_dq_finalize<__nv_bfloat16><<<gfin, 256, 0, s>>>(dq_acc, src, dmax, (__nv_bfloat16*)dQ, g.N, HD,
-                                                              a.inv_sqrt_d, err);
+            k_acc_finalize<__nv_bfloat16><<<gfin, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (__nv_bfloat16*)dQ, nullptr,
+                                                               0.f, nullptr, src, dmax, g.N, HD, err);
         return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
     }
     // dQ per query tile over the forward lists (head_dim 64)

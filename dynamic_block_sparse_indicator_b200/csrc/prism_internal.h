@@ -45,6 +45,7 @@ struct Layout {
     size_t lse_p, di_p;                 // float[heads][N] (backward, block order)
     size_t dmax;                        // uint32[heads]: max |dO| bits (backward scaling)
     size_t dq_acc;                      // float[heads][N][D]: dQ accumulated in block order
+    size_t dk_acc, dv_acc;              // float[heads][N][D]: dK, dV accumulated in block order
     size_t total;
 };
 
@@ -65,6 +66,7 @@ struct prism_plan_s {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;       // 2D [heads*N, D] fp16, 128-row boxes, 128B swizzle
     CUtensorMap tm_q64, tm_k64, tm_v64, tm_do64;  // the same with 64-row boxes
     CUtensorMap tm_dq;                            // fp32 dQ accumulator, 32-row boxes, no swizzle
+    CUtensorMap tm_dk, tm_dv;                     // fp32 dK, dV accumulators, the same boxes
     int64_t launches;                             // kernels launched so far
     int profile;                                  // per-stage event timing on?
     struct Timed { int stage; cudaEvent_t a, b; };

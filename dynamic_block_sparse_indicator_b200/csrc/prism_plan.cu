@@ -87,6 +87,8 @@ Layout make_layout(const Geom& g) {
     L.di_p = take(sizeof(float) * H * N);
     L.dmax = take(sizeof(uint32_t) * H);
     L.dq_acc = take(sizeof(float) * H * N * g.D);
+    L.dk_acc = take(sizeof(float) * H * N * g.D);
+    L.dv_acc = take(sizeof(float) * H * N * g.D);
     L.total = off;
     return L;
 }
@@ -1011,6 +1013,8 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
     if (!st) st = make_tmap(&P->tm_v64, P->ws + L.vp, rows, g.D, 64);
     if (!st) st = make_tmap(&P->tm_do64, P->ws + L.dop, rows, g.D, 64);
     if (!st) st = make_tmap_f32(&P->tm_dq, P->ws + L.dq_acc, rows, g.D, 32);
+    if (!st) st = make_tmap_f32(&P->tm_dk, P->ws + L.dk_acc, rows, g.D, 32);
+    if (!st) st = make_tmap_f32(&P->tm_dv, P->ws + L.dv_acc, rows, g.D, 32);
     if (st) { delete P; return st; }
     *outP = P;
     return PRISM_OK;
