@@ -48,6 +48,8 @@ constexpr int SLAB128 = 128 * 128;   // bytes: 128 rows x 64 fp16
 constexpr int SLAB64 = 64 * 128;     // bytes:  64 rows x 64 fp16
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kPScale = 32768.f;          // 2^15: scale of the P operand of dV += P^T dO
+constexpr float kPScaleLog2 = 15.f;
+constexpr float kPScaleInv = 1.f / 32768.f;
 
 // --------------------------------------------------------------- preprocess
 template <typename OT>
@@ -99,9 +101,13 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, cons
         out[c] = __float2half_rn(g * sc);
     }
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    // stored for the softmax of the backward kernels, which form P' = 2^15 P as
+    // ex2(s * log2(e)/sqrt(d) + lse_p) and dS = P' (dP 2^-15 + di_p) with one
+    // fused multiply-add each: lse_p = 15 - LSE log2(e), di_p = -D 2^-15 (D in
+    // the dO scale)
     if (lane == 0) {
-        di_p[(size_t)h * N + p] = acc * sc;
-        lse_p[(size_t)h * N + p] = lse[(size_t)h * N + n] * kLog2e;
+        di_p[(size_t)h * N + p] = -acc * sc * kPScaleInv;
+        lse_p[(size_t)h * N + p] = kPScaleLog2 - lse[(size_t)h * N + n] * kLog2e;
     }
 }
 
@@ -142,8 +148,8 @@ struct BwdArgs {
     const int* ptr;        // [heads][NT + 1]
     const int* ent;        // [heads][NT * NT]
     const int* src;        // [heads][N]
-    const float* lse_p;    // [heads][N] log2-scaled, block order
-    const float* di_p;     // [heads][N]  (scaled like dO)
+    const float* lse_p;    // [heads][N] 15 - LSE log2(e), block order
+    const float* di_p;     // [heads][N] -D 2^-15 (D scaled like dO)
     const uint32_t* dmax;  // [heads] max |dO| bits: outputs are divided by the dO scale
     void* out0;            // dK (dkdv) or dQ (dq), raster order
     void* out1;            // dV (dkdv)
@@ -401,6 +407,11 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             const bool valid = (m2 >> kh) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (u >> 1) & 1, a.err, 1001))) { ok = false; break; }
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1002))) { ok = false; break; }
+            // dS^T(u - 2) has been read (dK, dQ^T) before dS^T(u) overwrites it
+            if (u >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1003))) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
             uint32_t sv[32], dp[32];
             PRISM_TMEM_LD32(tmem + lane_off + 128 * b + c0, sv);
@@ -409,30 +420,36 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             // both warpgroups of this lane quarter have read dP^T before P^T overwrites it
             named_bar(2 + (warp & 3), 64);
             ++nbar;
-            if (u >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1003))) {
-                ok = false;
-                break;
-            }
-            const float* lq = sm.lse[s] + c0;
-            const float* dq = sm.di[s] + c0;
+            const float4* lq4 = reinterpret_cast<const float4*>(sm.lse[s] + c0);
+            const float4* dq4 = reinterpret_cast<const float4*>(sm.di[s] + c0);
             const uint32_t ds_s = smem_u32(sm.ds[b]);
             uint32_t pt[16];
             #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
+                // lse_p = 15 - LSE log2(e) and di_p = -D 2^-15 of the chunk's 8 queries
+                const float4 x0 = lq4[2 * ch], x1 = lq4[2 * ch + 1];
+                const float4 y0 = dq4[2 * ch], y1 = dq4[2 * ch + 1];
+                const float lq[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                const float dq[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
                 uint32_t wd[4];
                 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = ch * 8 + 2 * e;
                     float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
                     if (valid) {
-                        p0 = ex2(fmaf(__uint_as_float(sv[c]), a.scale_log2, -lq[c]));
-                        p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), a.scale_log2, -lq[c + 1]));
-                        d0 = p0 * (__uint_as_float(dp[c]) - dq[c]);
-                        d1 = p1 * (__uint_as_float(dp[c + 1]) - dq[c + 1]);
+                        // P' = 2^15 P: the dV operand, normal in fp16 down to P = 2^-29
+                        // (dV is unscaled at the end); dS = P (dP - D) = P' (dP 2^-15 - D 2^-15)
+                        float x0_, x1_;
+                        ffma2(x0_, x1_, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), a.scale_log2,
+                              a.scale_log2, lq[2 * e], lq[2 * e + 1]);
+                        p0 = ex2(x0_);
+                        p1 = ex2(x1_);
+                        float t0, t1;
+                        ffma2(t0, t1, __uint_as_float(dp[c]), __uint_as_float(dp[c + 1]), kPScaleInv, kPScaleInv,
+                              dq[2 * e], dq[2 * e + 1]);
+                        fmul2(d0, d1, p0, p1, t0, t1);
                     }
-                    // the dV operand is 2^15 P (normal in fp16 down to P = 2^-29);
-                    // dV is unscaled in the epilogue
-                    pt[ch * 4 + e] = pack_f16(p0 * kPScale, p1 * kPScale);
+                    pt[ch * 4 + e] = pack_f16(p0, p1);
                     wd[e] = pack_f16(d0, d1);
                 }
                 st_shared_v4(ds_s + swz128(r, 4 * wg + ch), wd[0], wd[1], wd[2], wd[3]);
@@ -686,10 +703,11 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                     const int c = ch * 8 + 2 * e;
                     float d0 = 0.f, d1 = 0.f;
                     if (valid) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sv[c]), a.scale_log2, -lse2));
-                        const float p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), a.scale_log2, -lse2));
-                        d0 = p0 * (__uint_as_float(dp[c]) - di);
-                        d1 = p1 * (__uint_as_float(dp[c + 1]) - di);
+                        // P' = 2^15 P and dS = P' (dP 2^-15 - D 2^-15), as in the dK/dV kernel
+                        const float p0 = ex2(fmaf(__uint_as_float(sv[c]), a.scale_log2, lse2));
+                        const float p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), a.scale_log2, lse2));
+                        d0 = p0 * fmaf(__uint_as_float(dp[c]), kPScaleInv, di);
+                        d1 = p1 * fmaf(__uint_as_float(dp[c + 1]), kPScaleInv, di);
                     }
                     wd[e] = pack_f16(d0, d1);
                 }
