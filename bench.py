@@ -48,6 +48,14 @@ def args_():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true",
                     help="skip the dense same-shape comparison (torch SDPA and all-blocks Prism)")
+    # variants of the pages' ablation and operating point (defaults: the workload's method)
+    ap.add_argument("--top-k", type=int, default=None)
+    ap.add_argument("--top-p", type=float, default=None)
+    ap.add_argument("--topk-frac", type=float, default=0.0,
+                    help="k as a fraction of each head's blocks (the pages' Top-k 95%% = 0.05)")
+    ap.add_argument("--alpha", type=float, default=0.5, help="shape-mapping exponent (1/2: the method)")
+    ap.add_argument("--shape-mode", choices=["dynamic", "isotropic", "fixed"], default="dynamic")
+    ap.add_argument("--fixed-shape", type=int, default=3, help="candidate index for --shape-mode fixed")
     return ap.parse_args()
 
 
@@ -145,7 +153,21 @@ def peaks():
 
 
 # --------------------------------------------------------- CPU oracle leg
-def oracle_head_ms(Qh, Kh, Vh, dOh, a, w, budget_s, seed=0):
+def variant_of(a):
+    """The oracle's keyword arguments for the command line's variant flags."""
+    mode = {"dynamic": 0, "isotropic": 1, "fixed": 2}[a.shape_mode]
+    return dict(alpha=a.alpha, shape_mode=mode, fixed_shape=a.fixed_shape, k_frac=a.topk_frac)
+
+
+def workload_of(a):
+    from dynamic_block_sparse_indicator_b200 import synthetic as syn
+    over = {k: v for k, v in (("top_k", a.top_k), ("top_p", a.top_p)) if v is not None}
+    if a.grid:
+        over.update(T=a.grid[0], H=a.grid[1], W=a.grid[2])
+    return syn.workload(a.workload, **over)
+
+
+def oracle_head_ms(Qh, Kh, Vh, dOh, a, w, budget_s, seed=0, variant=None):
     """The oracle on one head: full plan, then forward + backward on a seeded
     sample of query blocks until `budget_s` elapses; the attention time is
     extrapolated to the head by the share of selected pairs.  Returns
@@ -153,7 +175,7 @@ def oracle_head_ms(Qh, Kh, Vh, dOh, a, w, budget_s, seed=0):
     import numpy as np
     from oracle import prism_oracle as po
     t0 = time.perf_counter()
-    pl = po.plan_head(Qh, Kh, Vh, a, w.T, w.H, w.W, w.top_k, w.top_p, w.eps)
+    pl = po.plan_head(Qh, Kh, Vh, a, w.T, w.H, w.W, w.top_k, w.top_p, w.eps, **(variant or {}))
     t_plan = time.perf_counter() - t0
     src, st, sel = pl["src"], pl["starts"], pl["sel"]
     size = np.diff(st)
@@ -204,7 +226,8 @@ def run_reference(a, rank, world):
     import numpy as np
     import torch
     from dynamic_block_sparse_indicator_b200 import synthetic as syn
-    w = syn.workload(a.workload)
+    w = workload_of(a)
+    var = variant_of(a)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     heads = min(w.heads, a.steps + 1)
     Q, K, V = syn.make_qkv(w, device=dev, heads=heads)
@@ -213,13 +236,13 @@ def run_reference(a, rank, world):
     host = lambda t, h: t[h].to("cpu", torch.float64).numpy()
     # warm-up steps: a one-second sample on head 0
     for _ in range(a.warmup):
-        oracle_head_ms(host(Q, 0), host(K, 0), host(V, 0), host(dO, 0), amap, w, 1.0)
+        oracle_head_ms(host(Q, 0), host(K, 0), host(V, 0), host(dO, 0), amap, w, 1.0, variant=var)
     vals, desc, threads = [], "", 1
     t0 = time.perf_counter()
     for s in range(a.steps):
         h = s % heads
         ms, desc, threads = oracle_head_ms(host(Q, h), host(K, h), host(V, h), host(dO, h), amap, w,
-                                           a.cpu_seconds / 4, seed=s)
+                                           a.cpu_seconds / 4, seed=s, variant=var)
         vals.append(ms)
     wall = time.perf_counter() - t0
     v = float(np.mean(vals))
@@ -227,7 +250,8 @@ def run_reference(a, rank, world):
           "steps": a.steps, "warmup": a.warmup, "ms_per_step": v, "higher_is_better": False,
           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
           "config": {"workload": w.name(), "grid": [w.T, w.H, w.W], "tokens": w.N,
-                     "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p},
+                     "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p,
+                     "top_k_frac": a.topk_frac, "alpha": a.alpha, "shape_mode": a.shape_mode},
           "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                            "sample": desc, "wall_s": wall},
           "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
@@ -306,9 +330,10 @@ def run_prism(a, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = syn.workload(a.workload)
-    if a.grid:
-        w = syn.workload(a.workload, T=a.grid[0], H=a.grid[1], W=a.grid[2])
+    w = workload_of(a)
+    mode = {"dynamic": _lib.PRISM_SHAPE_DYNAMIC, "isotropic": _lib.PRISM_SHAPE_ISOTROPIC,
+            "fixed": _lib.PRISM_SHAPE_FIXED}[a.shape_mode]
+    variant = dict(alpha=a.alpha, shape_mode=mode, fixed_shape=a.fixed_shape, top_k_frac=a.topk_frac)
     lib = _lib.load()
     need = a.warmup + a.steps
     heads = min(w.heads, need)
@@ -319,7 +344,7 @@ def run_prism(a, rank, world, local_rank):
     dO = syn.make_dout(w, device=dev, heads=gen_heads, out_dtype=torch.bfloat16).float()
     amap = syn.make_amap(w, device=dev)
     params = _lib.make_params(w.T, w.H, w.W, 1, w.head_dim, _lib.PRISM_BF16, w.top_k, w.top_p,
-                              w.eps, out_dtype=_lib.PRISM_F32)
+                              w.eps, out_dtype=_lib.PRISM_F32, **variant)
     ws = torch.empty(_lib.workspace_bytes(params), dtype=torch.uint8, device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
     O = torch.empty(1, w.N, w.head_dim, **f32)
@@ -467,7 +492,7 @@ def run_prism(a, rank, world, local_rank):
         h = order[a.warmup]
         host = lambda t: t[h].to("cpu", torch.float64).numpy()
         ms, desc, threads = oracle_head_ms(host(Q), host(K), host(V), host(dO),
-                                           amap.cpu().numpy(), w, a.cpu_seconds)
+                                           amap.cpu().numpy(), w, a.cpu_seconds, variant=variant_of(a))
         cpu = {"value": ms, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
     if rank == 0:
         emit({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
@@ -477,6 +502,8 @@ def run_prism(a, rank, world, local_rank):
               "config": {"workload": w.name(), "grid": [w.T, w.H, w.W], "tokens": w.N,
                          "heads_in_sequence": True, "head_dim": D, "input_dtype": "bf16",
                          "output_dtype": "fp32", "top_k": w.top_k, "top_p": w.top_p,
+                         "top_k_frac": a.topk_frac, "alpha": a.alpha, "shape_mode": a.shape_mode,
+                         **({"fixed_shape": a.fixed_shape} if a.shape_mode == "fixed" else {}),
                          "l2": "inputs larger than L2 (259 MB per tensor per head)"},
               "tflops": {"fwd_bwd_selected": attn_tflops,
                          "fraction_of_peak": attn_tflops / peak},

@@ -34,12 +34,18 @@ ITEMS = {
 }
 
 
+PRISM_SHAPE_DYNAMIC = 0
+PRISM_SHAPE_ISOTROPIC = 1
+PRISM_SHAPE_FIXED = 2
+
+
 class PrismParams(C.Structure):
     _fields_ = [("T", C.c_int32), ("H", C.c_int32), ("W", C.c_int32), ("heads", C.c_int32),
                 ("head_dim", C.c_int32), ("dtype", C.c_int32), ("out_dtype", C.c_int32),
                 ("top_k", C.c_int32),
                 ("top_p", C.c_float), ("eps", C.c_float), ("tau128", C.c_float),
-                ("tau256", C.c_float)]
+                ("tau256", C.c_float), ("alpha", C.c_float), ("shape_mode", C.c_int32),
+                ("fixed_shape", C.c_int32), ("top_k_frac", C.c_float)]
 
 
 class PrismError(RuntimeError):
@@ -101,9 +107,11 @@ def status_string(st: int) -> str:
 
 
 def make_params(T, H, W, heads, head_dim, dtype, top_k, top_p, eps, tau128=0.5, tau256=0.25,
-                out_dtype=PRISM_F32):
+                out_dtype=PRISM_F32, alpha=0.5, shape_mode=PRISM_SHAPE_DYNAMIC, fixed_shape=0,
+                top_k_frac=0.0):
     return PrismParams(T, H, W, heads, head_dim, dtype, out_dtype, top_k, float(top_p),
-                       float(eps), float(tau128), float(tau256))
+                       float(eps), float(tau128), float(tau256), float(alpha), int(shape_mode),
+                       int(fixed_shape), float(top_k_frac))
 
 
 def workspace_bytes(params: PrismParams) -> int:

@@ -103,7 +103,12 @@ int validate_params(const prism_params* p) {
     if (p->out_dtype != PRISM_BF16 && p->out_dtype != PRISM_F32) return PRISM_ERR_INVALID_ARG;
     if (p->top_k < 0) return PRISM_ERR_INVALID_ARG;
     if (!(p->top_p >= 0.f && p->top_p <= 1.f)) return PRISM_ERR_INVALID_ARG;
-    if (p->top_k < 1 && p->top_p <= 0.f) return PRISM_ERR_INVALID_ARG;
+    if (!(p->top_k_frac >= 0.f && p->top_k_frac <= 1.f)) return PRISM_ERR_INVALID_ARG;
+    if (p->top_k < 1 && !(p->top_k_frac > 0.f) && p->top_p <= 0.f) return PRISM_ERR_INVALID_ARG;
+    if (!(p->alpha >= 0.f) || !std::isfinite(p->alpha)) return PRISM_ERR_INVALID_ARG;
+    if (p->shape_mode < PRISM_SHAPE_DYNAMIC || p->shape_mode > PRISM_SHAPE_FIXED) return PRISM_ERR_INVALID_ARG;
+    if (p->shape_mode == PRISM_SHAPE_FIXED && (p->fixed_shape < 0 || p->fixed_shape >= 16))
+        return PRISM_ERR_INVALID_ARG;
     if (!(p->eps > 0.f) || !std::isfinite(p->eps)) return PRISM_ERR_INVALID_ARG;
     if (!(p->tau256 >= 0.f && p->tau128 >= p->tau256 && p->tau128 <= 1e30f))
         return PRISM_ERR_INVALID_ARG;
@@ -438,16 +443,19 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restri
 }
 
 // Per head: rho normalisation, volume, closed form, snapping, block offsets.
-__device__ int snap_shape(const float g[3], int vol) {
+// Closed form with the mapping exponent alpha (the pages' method: 1/2):
+// l*_d = -alpha log2 g_d + 1/3 (S + alpha sum_d' log2 g_d'), so that
+// b_d ~ g_d^-alpha and prod b_d = B.
+__device__ int snap_shape(const float g[3], int vol, float alpha) {
     const float lg0 = log2f(g[0]), lg1 = log2f(g[1]), lg2 = log2f(g[2]);
     const float S = vol == 64 ? 6.f : (vol == 128 ? 7.f : 8.f);
-    float inner = __fadd_rn(S, __fmul_rn(0.5f, lg0));
-    inner = __fadd_rn(inner, __fmul_rn(0.5f, lg1));
-    inner = __fadd_rn(inner, __fmul_rn(0.5f, lg2));
+    float inner = __fadd_rn(S, __fmul_rn(alpha, lg0));
+    inner = __fadd_rn(inner, __fmul_rn(alpha, lg1));
+    inner = __fadd_rn(inner, __fmul_rn(alpha, lg2));
     const float third = __fdiv_rn(inner, 3.f);
-    const float e0 = __fadd_rn(__fmul_rn(-0.5f, lg0), third);
-    const float e1 = __fadd_rn(__fmul_rn(-0.5f, lg1), third);
-    const float e2 = __fadd_rn(__fmul_rn(-0.5f, lg2), third);
+    const float e0 = __fadd_rn(__fmul_rn(-alpha, lg0), third);
+    const float e1 = __fadd_rn(__fmul_rn(-alpha, lg1), third);
+    const float e2 = __fadd_rn(__fmul_rn(-alpha, lg2), third);
     const int lo = vol == 64 ? 0 : (vol == 128 ? 7 : 13);
     const int hi = vol == 64 ? 7 : (vol == 128 ? 13 : 16);
     int best = lo;
@@ -463,8 +471,34 @@ __device__ int snap_shape(const float g[3], int vol) {
     return best;
 }
 
-__global__ void __launch_bounds__(1024) k_zone_finalize(DevPlan d, float eps, float tau128,
-                                                        float tau256, int use_given_shapes) {
+// Shape id of zone m of head h from its statistics (zs: the head's zone
+// stats, mx: the head's maximum raw density).
+struct ShapeRule {
+    float eps, tau128, tau256, alpha;
+    int mode, fixed;
+};
+__device__ int zone_shape(const DevPlan& d, const float* zs, float mx, int m, const ShapeRule& rule) {
+    if (rule.mode == PRISM_SHAPE_FIXED) return rule.fixed;
+    const float rho = mx > 0.f ? __fdiv_rn(zs[m * 4 + 3], mx) : 0.f;
+    const int vol = rho < rule.tau256 ? 256 : (rho < rule.tau128 ? 128 : 64);
+    float g[3];
+    if (rule.mode == PRISM_SHAPE_ISOTROPIC) {
+        g[0] = g[1] = g[2] = 1.f;
+    } else {
+        const float s0 = zs[m * 4], s1 = zs[m * 4 + 1], s2 = zs[m * 4 + 2];
+        const float tot = __fadd_rn(__fadd_rn(s0, s1), s2);
+        float r[3];
+        if (tot > 0.f) { r[0] = __fdiv_rn(s0, tot); r[1] = __fdiv_rn(s1, tot); r[2] = __fdiv_rn(s2, tot); }
+        else { r[0] = r[1] = r[2] = 1.f / 3.f; }
+        const float ab = d.abar[m];
+        #pragma unroll
+        for (int ax = 0; ax < 3; ++ax)
+            g[ax] = __fadd_rn(__fadd_rn(r[ax], __fmul_rn(ab, d.vhat[3 * m + ax])), rule.eps);
+    }
+    return snap_shape(g, vol, rule.alpha);
+}
+
+__global__ void __launch_bounds__(1024) k_zone_finalize(DevPlan d, ShapeRule rule, int use_given_shapes) {
     __shared__ float redf[32];
     __shared__ int red[1024];
     extern __shared__ int nbz[];   // [Nz + 1]
@@ -475,21 +509,7 @@ __global__ void __launch_bounds__(1024) k_zone_finalize(DevPlan d, float eps, fl
         float mx = 0.f;
         for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) mx = fmaxf(mx, zs[m * 4 + 3]);
         mx = block_max<1024>(mx, redf);
-        for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
-            const float rho = mx > 0.f ? __fdiv_rn(zs[m * 4 + 3], mx) : 0.f;
-            const int vol = rho < tau256 ? 256 : (rho < tau128 ? 128 : 64);
-            const float s0 = zs[m * 4], s1 = zs[m * 4 + 1], s2 = zs[m * 4 + 2];
-            const float tot = __fadd_rn(__fadd_rn(s0, s1), s2);
-            float r[3];
-            if (tot > 0.f) { r[0] = __fdiv_rn(s0, tot); r[1] = __fdiv_rn(s1, tot); r[2] = __fdiv_rn(s2, tot); }
-            else { r[0] = r[1] = r[2] = 1.f / 3.f; }
-            const float ab = d.abar[m];
-            float g[3];
-            #pragma unroll
-            for (int ax = 0; ax < 3; ++ax)
-                g[ax] = __fadd_rn(__fadd_rn(r[ax], __fmul_rn(ab, d.vhat[3 * m + ax])), eps);
-            sid[m] = (uint8_t)snap_shape(g, vol);
-        }
+        for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) sid[m] = (uint8_t)zone_shape(d, zs, mx, m, rule);
         __syncthreads();
     }
     for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
@@ -632,7 +652,7 @@ constexpr int SEL_THREADS = 512;
 __device__ __forceinline__ uint32_t fkey(float x) { return __float_as_uint(x); }
 
 template <int D>
-__global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, float top_p) {
+__global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, float top_k_frac, float top_p) {
     extern __shared__ float prow[];                 // [NB] logits, then probabilities
     __shared__ float redf[SEL_THREADS / 32];
     __shared__ int redi[SEL_THREADS / 32];
@@ -675,7 +695,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, fl
     __syncthreads();
 
     // L = shortest prefix of (P desc, j asc) with mass >= p
-    const int K = min(top_k, nb);
+    // k as a fraction of the head's block count: ceil(frac * N_b) in fp32
+    const int K = min(top_k_frac > 0.f ? (int)ceilf(__fmul_rn(top_k_frac, (float)nb)) : top_k, nb);
     int L;
     if (top_p >= 1.f) L = nb;
     else if (top_p <= 0.f) L = 0;
@@ -982,6 +1003,11 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 static int g_profile_plans = 0;   // prism_profile_plans: timing state of new plans
 
+static ShapeRule shape_rule(const prism_params& p) {
+    // alpha 0 stands for the pages' 1/2
+    return ShapeRule{p.eps, p.tau128, p.tau256, p.alpha > 0.f ? p.alpha : 0.5f, p.shape_mode, p.fixed_shape};
+}
+
 static int plan_common(const prism_params* p, const void* Q, const void* K, const void* V,
                        void* workspace, size_t ws_bytes, prism_plan_s** outP) {
     int st = validate_params(p);
@@ -1084,7 +1110,7 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
         const size_t fin_smem = sizeof(int) * (g.Nz + 1);
         if (fin_smem > 48 * 1024)
             cudaFuncSetAttribute(k_zone_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
-        k_zone_finalize<<<g.heads, 1024, fin_smem, s>>>(d, p.eps, p.tau128, p.tau256, given_shapes ? 1 : 0);
+        k_zone_finalize<<<g.heads, 1024, fin_smem, s>>>(d, shape_rule(p), given_shapes ? 1 : 0);
     }
     {
         PrismProf prof(P, PRISM_STAGE_PLAN_GATHER, s);
@@ -1098,10 +1124,10 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
         const size_t sm = sizeof(float) * g.NB;
         if (g.D == 128) {
             cudaFuncSetAttribute(k_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-            k_select<128><<<dim3(g.NB, g.heads), SEL_THREADS, sm, s>>>(d, p.top_k, p.top_p);
+            k_select<128><<<dim3(g.NB, g.heads), SEL_THREADS, sm, s>>>(d, p.top_k, p.top_k_frac, p.top_p);
         } else {
             cudaFuncSetAttribute(k_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-            k_select<64><<<dim3(g.NB, g.heads), SEL_THREADS, sm, s>>>(d, p.top_k, p.top_p);
+            k_select<64><<<dim3(g.NB, g.heads), SEL_THREADS, sm, s>>>(d, p.top_k, p.top_k_frac, p.top_p);
         }
     } else {
         cudaMemcpyAsync(d.sel, given_sel, sizeof(uint32_t) * (size_t)g.heads * g.NB * g.WORDS,
@@ -1333,7 +1359,7 @@ static size_t noalloc_floats(int Nz, int heads, size_t* off_abar, size_t* off_vh
 
 // Variant of k_zone_finalize that stops at the shapes: shape id per zone and
 // the head's block count, no block offsets.
-__global__ void __launch_bounds__(1024) k_zone_shapes_static(DevPlan d, float eps, float tau128, float tau256,
+__global__ void __launch_bounds__(1024) k_zone_shapes_static(DevPlan d, ShapeRule rule,
                                                              uint8_t* __restrict__ sid_out,
                                                              int* __restrict__ nblocks_out) {
     __shared__ float redf[32];
@@ -1345,20 +1371,9 @@ __global__ void __launch_bounds__(1024) k_zone_shapes_static(DevPlan d, float ep
     mx = block_max<1024>(mx, redf);
     int blocks = 0;
     for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
-        const float rho = mx > 0.f ? __fdiv_rn(zs[m * 4 + 3], mx) : 0.f;
-        const int vol = rho < tau256 ? 256 : (rho < tau128 ? 128 : 64);
-        const float s0 = zs[m * 4], s1 = zs[m * 4 + 1], s2 = zs[m * 4 + 2];
-        const float tot = __fadd_rn(__fadd_rn(s0, s1), s2);
-        float r[3];
-        if (tot > 0.f) { r[0] = __fdiv_rn(s0, tot); r[1] = __fdiv_rn(s1, tot); r[2] = __fdiv_rn(s2, tot); }
-        else { r[0] = r[1] = r[2] = 1.f / 3.f; }
-        const float ab = d.abar[m];
-        float g[3];
-        #pragma unroll
-        for (int ax = 0; ax < 3; ++ax)
-            g[ax] = __fadd_rn(__fadd_rn(r[ax], __fmul_rn(ab, d.vhat[3 * m + ax])), eps);
-        sid_out[(size_t)h * d.Nz + m] = (uint8_t)snap_shape(g, vol);
-        blocks += 512 / vol;
+        const int s = zone_shape(d, zs, mx, m, rule);
+        sid_out[(size_t)h * d.Nz + m] = (uint8_t)s;
+        blocks += 512 / (c_shape[s][0] * c_shape[s][1] * c_shape[s][2]);
     }
     blocks = block_sum_int<1024>(blocks, redi);
     if (threadIdx.x == 0) nblocks_out[h] = blocks;
@@ -1423,6 +1438,6 @@ extern "C" int prism_zone_shapes_noalloc(const prism_params* p, const void* V, c
     else if (bf) noalloc_stats<__nv_bfloat16, 64>(g, d, V, s);
     else if (g.D == 128) noalloc_stats<float, 128>(g, d, V, s);
     else noalloc_stats<float, 64>(g, d, V, s);
-    k_zone_shapes_static<<<g.heads, 1024, 0, s>>>(d, p->eps, p->tau128, p->tau256, shape_id, nblocks);
+    k_zone_shapes_static<<<g.heads, 1024, 0, s>>>(d, shape_rule(*p), shape_id, nblocks);
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }

@@ -70,14 +70,37 @@ extern "C" {
  *             feed the statistics and the pooled means in fp32; attention runs
  *             on their bf16 rounding (round to nearest even).
  *   out_dtype element type of O, dO, dQ, dK, dV: PRISM_BF16 or PRISM_F32.
- *             The tensor-core products are bf16 with fp32 accumulation either
- *             way; fp32 outputs keep the fp32 accumulators unrounded.
+ *             The tensor-core products take fp16 operands (exact for bf16
+ *             inputs inside +-65504) with fp32 accumulation either way; fp32
+ *             outputs keep the fp32 accumulators unrounded.
  *   top_k     k of Top-k (>= 0); k >= number of blocks keeps every block.
  *   top_p     p of Top-p in [0, 1]; p >= 1 keeps every block, p <= 0 none.
- *             top_k < 1 together with top_p <= 0 is rejected (empty sets).
+ *             Empty sets (top_k < 1, top_k_frac <= 0 and top_p <= 0) are
+ *             rejected.
  *   eps       epsilon of g_d = r_{v,d} + a_bar * v_hat_{a,d} + eps.
  *   tau128, tau256   density thresholds (the pages use 0.5 and 0.25).
+ * Variants of the pages' ablation (page xyznot.com/id, Table 10) and operating
+ * point (page paper.rainbus.top: Top-k 95%, Top-p 0.2):
+ *   alpha       exponent of the shape mapping b_d ~ g_d^-alpha:
+ *               l*_d = -alpha log2 g_d + 1/3 (log2 B + alpha sum_d' log2 g_d').
+ *               0 means the pages' 1/2; must be >= 0.
+ *   shape_mode  PRISM_SHAPE_DYNAMIC (the method), PRISM_SHAPE_ISOTROPIC (g_d
+ *               taken equal on the three axes: the volume still follows rho,
+ *               the shape is the candidate nearest the cube, ties to the lower
+ *               index) or PRISM_SHAPE_FIXED (every zone takes candidate
+ *               fixed_shape, whatever its statistics: the fixed-block
+ *               comparator).
+ *   fixed_shape candidate index 0..15 for PRISM_SHAPE_FIXED, ignored otherwise.
+ *               Candidates are ordered by volume (64, 128, 256), each volume
+ *               lexicographically in (b_T, b_H, b_W): 3 = 4x4x4, 8 = 4x4x8,
+ *               13 = 4x8x8 (the candidate nearest the cube of each volume).
+ *   top_k_frac  k as a fraction of the head's block count: when > 0, each
+ *               head's k is ceil(top_k_frac * N_b) in fp32 (the pages' "Top-k
+ *               95%" sparsity keeps 5%: 0.05) and top_k is ignored; in [0, 1].
  */
+#define PRISM_SHAPE_DYNAMIC   0
+#define PRISM_SHAPE_ISOTROPIC 1
+#define PRISM_SHAPE_FIXED     2
 typedef struct prism_params {
     int32_t T, H, W;
     int32_t heads;
@@ -89,6 +112,10 @@ typedef struct prism_params {
     float   eps;
     float   tau128;
     float   tau256;
+    float   alpha;
+    int32_t shape_mode;
+    int32_t fixed_shape;
+    float   top_k_frac;
 } prism_params;
 
 /* Opaque host-side handle: a small host struct pointing into the workspace. */
@@ -110,7 +137,8 @@ PRISM_API size_t prism_plan_workspace_bytes(const prism_params* p);
  *   r_{v,d}, the audio coupling a_bar and v_hat_{a,d} from a_map, g_d, the
  *   density rho -> volume B in {64,128,256} (thresholds tau256, tau128), the
  *   closed form l*_d = -1/2 log2 g_d + 1/3 (log2 B + 1/2 sum log2 g) snapped to
- *   the nearest of the 16 candidate shapes.
+ *   the nearest of the 16 candidate shapes (alpha and shape_mode select the
+ *   ablation variants).
  *   Stage 2: reorder tokens so every block is contiguous (bf16 copies of Q,
  *   K, V in block order, kept in the workspace).
  *   Stage 3 ("Metode" 3): block means Qbar, Kbar; P_i = softmax(Qbar_i Kbar^T

@@ -166,13 +166,17 @@ def volume(rho32, tau128, tau256):
     return np.where(rho32 < t256, 256, np.where(rho32 < t128, 128, 64)).astype(np.int64)
 
 
-def ideal_log_edges(g32, vol):
-    """l*_d = -1/2 log2 g_d + 1/3 (S + 1/2 sum_d' log2 g_d'), S = log2 B (float32)."""
+def ideal_log_edges(g32, vol, alpha=0.5):
+    """l*_d = -alpha log2 g_d + 1/3 (S + alpha sum_d' log2 g_d'), S = log2 B (float32).
+
+    The pages' closed form is alpha = 1/2 ("Metode" 2); Table 10's ablation
+    varies the exponent of b_d ~ g_d^-alpha, and the product stays B.
+    """
     lg = np.log2(g32.astype(F32))
     S = np.log2(np.asarray(vol, dtype=F32))
-    half = F32(0.5)
-    inner = S + half * lg[..., 0] + half * lg[..., 1] + half * lg[..., 2]
-    return (-half * lg + (inner / F32(3.0))[..., None]).astype(F32)
+    a = F32(alpha)
+    inner = S + a * lg[..., 0] + a * lg[..., 1] + a * lg[..., 2]
+    return (-a * lg + (inner / F32(3.0))[..., None]).astype(F32)
 
 
 def snap(ell32, vol):
@@ -195,11 +199,18 @@ def snap_margin(ell64, vol):
     return ds[1] - ds[0] if len(ds) > 1 else np.inf
 
 
-def zone_shapes(V, a, T, H, W, eps, tau128=0.5, tau256=0.25):
+SHAPE_DYNAMIC, SHAPE_ISOTROPIC, SHAPE_FIXED = 0, 1, 2
+
+
+def zone_shapes(V, a, T, H, W, eps, tau128=0.5, tau256=0.25, alpha=0.5, shape_mode=SHAPE_DYNAMIC,
+                fixed_shape=0):
     """Stage one for one head: V [N, D] raster, a [T,H,W] or None.
 
     Returns dict with shape_id [Nz], B [Nz], g [Nz,3] (float32), rho [Nz]
     (float32) and the float64 decision margins rho_margin, snap_margin.
+    Variants (Table 10's ablation): alpha is the mapping exponent; the
+    isotropic mode takes g_d equal on the three axes (B still from rho); the
+    fixed mode gives every zone candidate fixed_shape.
     """
     Vz = zones_of(np.asarray(V, dtype=np.float64), T, H, W)
     r = ratio(directional_variance(Vz))
@@ -209,16 +220,26 @@ def zone_shapes(V, a, T, H, W, eps, tau128=0.5, tau256=0.25):
     else:
         abar, vhat = audio_terms(a, T, H, W)
     g32 = (r.astype(F32) + abar.astype(F32)[:, None] * vhat.astype(F32) + F32(eps)).astype(F32)
+    g64 = r + abar[:, None] * vhat + eps
+    if shape_mode == SHAPE_ISOTROPIC:
+        g32 = np.ones_like(g32)
+        g64 = np.ones_like(g64)
     rho64 = normalise_by_max(density_raw(Vz))
     rho32 = rho64.astype(F32)
     B = volume(rho32, tau128, tau256)
-    ell = ideal_log_edges(g32, B.astype(F32))
+    ell = ideal_log_edges(g32, B.astype(F32), alpha)
     sid = np.array([snap(ell[m], B[m]) for m in range(len(B))], dtype=np.int64)
-    g64 = r + abar[:, None] * vhat + eps
     lg = np.log2(g64)
-    ell64 = -0.5 * lg + (np.log2(B) + 0.5 * lg.sum(axis=1))[:, None] / 3.0
+    ell64 = -alpha * lg + (np.log2(B) + alpha * lg.sum(axis=1))[:, None] / 3.0
     rho_margin = np.minimum(np.abs(rho64 - tau128), np.abs(rho64 - tau256))
     smargin = np.array([snap_margin(ell64[m], B[m]) for m in range(len(B))])
+    if shape_mode == SHAPE_ISOTROPIC:
+        smargin = np.full(len(B), np.inf)      # the tie rule decides exactly
+    if shape_mode == SHAPE_FIXED:
+        sid = np.full(len(B), int(fixed_shape), dtype=np.int64)
+        B = np.full(len(B), int(np.prod(SHAPES[int(fixed_shape)])), dtype=np.int64)
+        rho_margin = np.full(len(B), np.inf)
+        smargin = np.full(len(B), np.inf)
     return dict(shape_id=sid, B=B, g=g32, rho=rho32, r=r, abar=abar, vhat=vhat,
                 ell=ell, rho_margin=rho_margin, snap_margin=smargin)
 
@@ -294,9 +315,18 @@ def select_row(P_row, k, p):
     return np.sort(order[:cnt]), order, cnt
 
 
-def select(Qbar, Kbar, k, p):
-    """List of selected key-block arrays for every query block, plus (s32, P32)."""
+def k_of_fraction(frac, nb):
+    """k = ceil(frac * N_b) with the product in float32 (the pages' "Top-k 95%"
+    is a sparsity: frac = 0.05 keeps 5% of the key blocks)."""
+    return int(np.ceil(F32(frac) * F32(nb)))
+
+
+def select(Qbar, Kbar, k, p, k_frac=0.0):
+    """List of selected key-block arrays for every query block, plus (s32, P32).
+    k_frac > 0 replaces k by k_of_fraction(k_frac, N_b)."""
     s, P = block_probs(Qbar, Kbar)
+    if k_frac > 0:
+        k = k_of_fraction(k_frac, P.shape[1])
     sel = [select_row(P[i], k, p)[0] for i in range(P.shape[0])]
     return sel, s, P
 
@@ -304,13 +334,14 @@ def select(Qbar, Kbar, k, p):
 # ---------------------------------------------------------------------------
 # Whole plan for one head
 # ---------------------------------------------------------------------------
-def plan_head(Q, K, V, a, T, H, W, k, p, eps, tau128=0.5, tau256=0.25, shape_id=None):
+def plan_head(Q, K, V, a, T, H, W, k, p, eps, tau128=0.5, tau256=0.25, shape_id=None, alpha=0.5,
+              shape_mode=SHAPE_DYNAMIC, fixed_shape=0, k_frac=0.0):
     """Stages one to three for one head.  Q, K, V: [N, D] raster."""
-    st = zone_shapes(V, a, T, H, W, eps, tau128, tau256)
+    st = zone_shapes(V, a, T, H, W, eps, tau128, tau256, alpha, shape_mode, fixed_shape)
     sid = st["shape_id"] if shape_id is None else np.asarray(shape_id)
     src, starts = partition(sid, T, H, W)
     Qbar, Kbar = pool(Q, src, starts), pool(K, src, starts)
-    sel, s, P = select(Qbar, Kbar, k, p)
+    sel, s, P = select(Qbar, Kbar, k, p, k_frac)
     return dict(stats=st, shape_id=sid, src=src, starts=starts, Qbar=Qbar, Kbar=Kbar,
                 sel=sel, logits=s, P=P)
 

@@ -41,9 +41,12 @@ def _oracle_plans(w, Q, K, V, a, heads):
                          w.T, w.H, w.W, w.top_k, w.top_p, w.eps) for h in range(heads)]
 
 
-def _check_plan(pl, orc, w, heads):
+def _check_plan(pl, orc, w, heads, k=None, p=None):
     """Stage-wise comparison; returns per head the set of query blocks whose
-    selection equals the oracle's exactly (None when the shapes differ)."""
+    selection equals the oracle's exactly (None when the shapes differ).
+    k (an int, or a function of the head's block count) and p default to the
+    workload's."""
+    p = w.top_p if p is None else p
     NB, WORDS, Nz, N = w.N // 64, (w.N // 64 + 31) // 32, w.zones, w.N
     sid = pl.export("shape_id").reshape(heads, Nz)
     nblocks = pl.export("nblocks")
@@ -71,9 +74,10 @@ def _check_plan(pl, orc, w, heads):
         np.testing.assert_allclose(qbar[h, :nb], o["Qbar"], rtol=1e-5, atol=1e-6)
         np.testing.assert_allclose(kbar[h, :nb], o["Kbar"], rtol=1e-5, atol=1e-6)
         gsets = parity.bits_to_sets(bits[h], nb, WORDS)
+        kk = w.top_k if k is None else (k(nb) if callable(k) else k)
         exact = set()
         for i in range(nb):
-            assert parity.selection_agrees(gsets[i], o["logits"][i], o["P"][i], w.top_k, w.top_p), \
+            assert parity.selection_agrees(gsets[i], o["logits"][i], o["P"][i], kk, p), \
                 f"head {h} row {i}: selection differs beyond the tie margin"
             if np.array_equal(gsets[i], o["sel"][i]):
                 exact.add(i)
