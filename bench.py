@@ -145,6 +145,27 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def measured_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture
+    (profiles/dram_traffic_grid72x88x160.md), or None if the kernel's sources
+    changed since (their hash no longer matches) or there is no capture."""
+    import hashlib
+    tu = {"k_bwd_dkdv": "prism_attn_bwd.cu", "k_attn_fwd": "prism_attn_fwd.cu"}.get(kernel)
+    path = os.path.join(ROOT, "profiles", "dram_traffic_grid72x88x160.md")
+    if tu is None or not os.path.exists(path):
+        return None
+    m = hashlib.sha256()
+    for f in (tu, "prism_dev.cuh", "prism_internal.h"):
+        with open(os.path.join(ROOT, "dynamic_block_sparse_indicator_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    digest = m.hexdigest()[:16]
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) == 5 and cells[0] == kernel and cells[4] == digest:
+            return float(cells[1]) + float(cells[2])
+    return None
+
+
 def peaks():
     try:
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -514,7 +535,10 @@ def run_prism(a, rank, world, local_rank):
               "roofline": {"kernel": {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv",
                                       "bwd_dq": "k_dq_finalize" if fused else "k_bwd_dq"}[dom],
                            "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                           "frac": ach / peak, "peak_source": peak_src, "traffic": None},
+                           "frac": ach / peak, "peak_source": peak_src,
+                           "traffic": measured_traffic(
+                               {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv"}.get(dom, ""))
+                           if w.N == 1013760 else None},
               "plan_kernels": plan_kernels, "dense_same_shape": dense,
               "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks})
 
