@@ -24,6 +24,12 @@ Recipe for one tensor (Q, K or V), per head and channel:
   * for the 2K workloads, 85 % of the zones (chosen by seed, never a
     localised one) are near-uniform: the smoothed field is scaled by 0.1 and
     the noise standard deviation is 0.03.
+Inputs of the audio-to-video cross-attention that produces the norm map
+(make_av_inputs): the video queries Qv are a further tensor of the recipe
+above (seed id 5); the audio keys and values Ka, Va [heads, M, D] are, per head
+and channel, white N(0,1) noise over the M audio tokens smoothed by a 1-D
+Gaussian (sigma 3 tokens, radius 9, replicate padding), divided by its std,
+plus N(0, 0.3^2) (seed ids 6 and 7).
 The audio norm map is 0.05 everywhere, raised to a Gaussian blob
 0.05 + 0.95 exp(-|x - c|^2 / (2 * 3^2)) around the centre c of every localised
 zone (blobs combine by max).  dO is N(0,1).  Seeds: workload id x 1000 +
@@ -212,11 +218,38 @@ def make_dout(w: Workload, device="cpu", heads=None, out_dtype=None) -> torch.Te
     return t
 
 
+def make_av_inputs(w: Workload, M: int, device="cpu", heads=None, out_dtype=torch.bfloat16,
+                   qk_scale: float = 1.0):
+    """Qv [heads, N, D], Ka, Va [heads, M, D] for the norm-map producer (bf16 by default)."""
+    heads = w.heads if heads is None else heads
+    loc, uniform = zone_layout(w)
+    utok = _uniform_tokens(w, uniform, device)
+    g = _gen(w.wid * 1000 + 5, device)
+    Qv = torch.empty(heads, w.N, w.head_dim, dtype=out_dtype, device=device)
+    for h in range(heads):
+        Qv[h] = (_field_one_head(w, g, loc, utok, device) * qk_scale).to(out_dtype)
+    sigma, radius = 3.0, 9
+    k = torch.arange(-radius, radius + 1, dtype=torch.float32, device=device)
+    taps = torch.exp(-(k * k) / (2 * sigma * sigma))
+    taps = taps / taps.sum()
+    out = []
+    for tid in (6, 7):
+        ga = _gen(w.wid * 1000 + tid, device)
+        x = torch.randn(heads, w.head_dim, M, generator=ga, device=device)
+        x = _blur_axis(x, 2, taps)
+        x = x / x.std(dim=2, keepdim=True).clamp_min(1e-12) if M > 1 else x
+        x = x + 0.3 * torch.randn(heads, w.head_dim, M, generator=ga, device=device)
+        if tid == 6 and qk_scale != 1.0:
+            x = x * qk_scale
+        out.append(x.transpose(1, 2).contiguous().to(out_dtype))
+    return Qv, out[0], out[1]
+
+
 def roundtrip_float(t: torch.Tensor):
     """Exact float64 numpy copy of a tensor's values (bf16 values are exact in f64)."""
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-__all__ = ["Workload", "workload", "zone_layout", "make_qkv", "make_amap", "make_dout",
+__all__ = ["Workload", "workload", "zone_layout", "make_qkv", "make_amap", "make_dout", "make_av_inputs",
            "roundtrip_float"]
 

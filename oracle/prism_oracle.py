@@ -440,3 +440,46 @@ def attention_rows(Q, K, V, src, starts, sel, rows, dO=None):
             Di = g @ O[r]
             dQ[r] = (P * (dP - Di)) @ K[keys] * sc
     return O, lse, dQ
+
+
+# ---------------------------------------------------------------------------
+# Guidance map producer: the audio-to-video cross-attention output norm.
+# Page paper.rainbus.top, section "前置知识" (the dual-branch DiT paragraph): the
+# video hidden state takes in audio through h_hat = CrossAttn(h, K_a, V_a), and
+# the L2 norm of that output measures how much audio a video position absorbed.
+# Page xyznot.com/id, section "Metode" 1: a_{t,h,w} = ||h_hat_{t,h,w}||_2, cached
+# from the previous layer (page xyznot.com/th, section on limitations: the
+# self-attention runs before the cross-attention inside a block, hence the
+# one-layer lag).  Reading (the pages print no formula for the multi-head
+# case): h_hat of a token is the concatenation over heads of
+# softmax(q_h K_{a,h}^T / sqrt(D)) V_{a,h}, taken before the output projection
+# (which needs the backbone's weights), and the norm runs over all heads'
+# channels.
+def av_cross_attn(Qv, Ka, Va):
+    """Per-head cross-attention outputs h_hat [heads, N, D] (float64).
+
+    Qv [heads, N, D]: the video tokens' queries; Ka, Va [heads, M, D]: the
+    audio tokens' keys and values.  Softmax over the M audio tokens, logits
+    scaled by 1/sqrt(D), max subtracted before exp."""
+    Qv, Ka, Va = (np.asarray(x, np.float64) for x in (Qv, Ka, Va))
+    heads, N, D = Qv.shape
+    out = np.empty((heads, N, D))
+    for h in range(heads):
+        for r0 in range(0, N, 4096):
+            s = Qv[h, r0:r0 + 4096] @ Ka[h].T / np.sqrt(D)
+            e = np.exp(s - s.max(axis=1, keepdims=True))
+            out[h, r0:r0 + 4096] = (e / e.sum(axis=1, keepdims=True)) @ Va[h]
+    return out
+
+
+def av_norm_map(Qv, Ka, Va):
+    """The guidance map a [N] = ||h_hat||_2 over the concatenated heads, and
+    h_hat [heads, N, D] (float64)."""
+    hh = av_cross_attn(Qv, Ka, Va)
+    return np.sqrt((hh * hh).sum(axis=(0, 2))), hh
+
+
+def av_norm_rows(Qv, Ka, Va, rows):
+    """a and h_hat [heads, len(rows), D] for the given token rows only."""
+    rows = np.asarray(rows)
+    return av_norm_map(np.asarray(Qv)[:, rows], Ka, Va)
