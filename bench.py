@@ -56,6 +56,9 @@ def args_():
     ap.add_argument("--alpha", type=float, default=0.5, help="shape-mapping exponent (1/2: the method)")
     ap.add_argument("--shape-mode", choices=["dynamic", "isotropic", "fixed"], default="dynamic")
     ap.add_argument("--fixed-shape", type=int, default=3, help="candidate index for --shape-mode fixed")
+    ap.add_argument("--av-tokens", type=int, default=1000,
+                    help="audio tokens of the guidance-map producer leg (the pages: under 1K)")
+    ap.add_argument("--no-av", action="store_true", help="skip the guidance-map producer leg")
     return ap.parse_args()
 
 
@@ -342,6 +345,49 @@ def dense_same_shape(Q, K, V, dO, amap, w, ws, O, lse, dQ, dK, dV, h, peak):
     return out
 
 
+def guidance_map_leg(w, M, pk, reps=5):
+    """The guidance map producer (prism_av_norm) on the layer's video grid: one
+    launch over all heads of the audio-to-video cross-attention (4 N M D flops per
+    head), timed alone with CUDA events on the launching stream, with h_hat
+    written in bf16 (the fused producer of a model) and with the map alone."""
+    import torch
+    from dynamic_block_sparse_indicator_b200 import _lib
+    from dynamic_block_sparse_indicator_b200 import synthetic as syn
+    Qv, Ka, Va = syn.make_av_inputs(w, M, device="cuda")
+    heads, N, D = Qv.shape
+    amap = torch.empty(N, dtype=torch.float32, device="cuda")
+    hh = torch.empty(heads, N, D, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    flops = 4.0 * N * M * D * heads
+    burst = pk.get("bf16_tflops") or 1590.0
+    sust = pk.get("bf16_tflops_sustained") or 1400.0
+    out = {"workload": f"grid{w.T}x{w.H}x{w.W} ({N} video tokens), {M} audio tokens, {heads} heads, "
+                       f"head_dim {D}, bf16 inputs", "flops": flops, "launches_per_call": 1}
+    for name, hbuf in (("with_hhat_bf16", hh), ("map_only", None)):
+        for _ in range(2):
+            _lib.av_norm(Qv, Ka, Va, a_map=amap, h_hat=hbuf, status=status)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            _lib.av_norm(Qv, Ka, Va, a_map=amap, h_hat=hbuf, status=status)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        tf = flops / (ms * 1e-3) / 1e12
+        out[name] = {"ms": ms, "tflops": tf, "frac_of_burst": tf / burst, "frac_of_sustained": tf / sust}
+    st, site = _lib.status_read(status)
+    if st:
+        raise RuntimeError(f"guidance map: device status {_lib.status_string(st)} at site {site}")
+    ach = out["with_hhat_bf16"]["tflops"]
+    out["roofline"] = {"kernel": "k_av_norm", "bound": "tensor", "achieved": ach, "peak": burst,
+                       "unit": "TFLOP/s", "frac": ach / burst,
+                       "peak_source": "measured burst bf16 (timed alone)" if pk else "fallback"}
+    del Qv, Ka, Va, amap, hh
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_prism(a, rank, world, local_rank):
     import numpy as np
     import torch
@@ -475,6 +521,10 @@ def run_prism(a, rank, world, local_rank):
     dense = None
     if world == 1 and not a.no_dense:
         dense = dense_same_shape(Q, K, V, dO, amap, w, ws, O, lse, dQ, dK, dV, order[a.warmup], peak)
+    # ------------------------------------- guidance map producer (next layer's a)
+    av = None
+    if world == 1 and not a.no_av:
+        av = guidance_map_leg(w, a.av_tokens, pk)
     # --------------------------------------------------- end to end (host)
     e2e = None
     if a.e2e_steps > 0:
@@ -539,7 +589,7 @@ def run_prism(a, rank, world, local_rank):
                            "traffic": measured_traffic(
                                {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv"}.get(dom, ""))
                            if w.N == 1013760 else None},
-              "plan_kernels": plan_kernels, "dense_same_shape": dense,
+              "plan_kernels": plan_kernels, "dense_same_shape": dense, "guidance_map": av,
               "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks})
 
 

@@ -88,6 +88,9 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_profile_read": (i32, [vp, C.POINTER(C.c_float), C.POINTER(C.c_int), vp]),
         "prism_launch_count": (C.c_int64, [vp]),
         "prism_zone_shapes_noalloc": (i32, [pp, vp, vp, vp, vp, vp]),
+        "prism_av_norm": (i32, [C.c_int64, C.c_int32, C.c_int32, C.c_int32, vp, vp, vp, vp, vp,
+                                C.c_int32, vp, vp]),
+        "prism_status_read": (i32, [vp, C.POINTER(C.c_int32), vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -272,3 +275,42 @@ def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None
     if st:
         raise PrismError(st, "prism_plan_import")
     return Plan(params, h, workspace, (Q, K, V, shape_id, sel_bits))
+
+
+def av_norm(Qv, Ka, Va, a_map=None, h_hat=None, hhat_dtype=None, want_hhat=False, status=None,
+            stream=None):
+    """The guidance map a [N] (fp32) = || CrossAttn(Qv, Ka, Va) ||_2 over the heads, and
+    optionally h_hat [heads, N, D].  Qv [heads, N, D], Ka, Va [heads, M, D]: contiguous
+    bf16 CUDA tensors.  `status` is a device int32[4] block (zeroed here when created);
+    read it with status_read()."""
+    import torch
+    for t in (Qv, Ka, Va):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError("Qv, Ka, Va must be contiguous 3-D bf16 CUDA tensors")
+    heads, N, D = Qv.shape
+    M = Ka.shape[1]
+    if tuple(Ka.shape) != (heads, M, D) or tuple(Va.shape) != (heads, M, D):
+        raise ValueError(f"Ka, Va must be [heads, M, D] = [{heads}, M, {D}]")
+    dev = Qv.device
+    if a_map is None:
+        a_map = torch.empty(N, dtype=torch.float32, device=dev)
+    if hhat_dtype is None:
+        hhat_dtype = PRISM_BF16 if h_hat is None or h_hat.dtype == torch.bfloat16 else PRISM_F32
+    if h_hat is None and want_hhat:
+        dt = torch.float32 if hhat_dtype == PRISM_F32 else torch.bfloat16
+        h_hat = torch.empty(heads, N, D, dtype=dt, device=dev)
+    if status is None:
+        status = torch.zeros(4, dtype=torch.int32, device=dev)
+    st = load().prism_av_norm(int(N), int(M), int(heads), int(D), _ptr(Qv), _ptr(Ka), _ptr(Va),
+                              _ptr(a_map), _ptr(h_hat), int(hhat_dtype), _ptr(status),
+                              _stream(stream))
+    if st:
+        raise PrismError(st, "prism_av_norm")
+    return a_map, h_hat, status
+
+
+def status_read(status, stream=None):
+    """(status, site) of a device status block; synchronises and clears it."""
+    site = C.c_int32(0)
+    st = load().prism_status_read(_ptr(status), C.byref(site), _stream(stream))
+    return int(st), int(site.value)

@@ -219,6 +219,47 @@ PRISM_API int prism_attn_bwd(prism_plan_t plan, const void* dO, const void* O, c
 PRISM_API int prism_zone_shapes_noalloc(const prism_params* p, const void* V, const float* a_map,
                                         uint8_t* shape_id, int32_t* nblocks, void* stream);
 
+/* ---- guidance map producer ---------------------------------------------- */
+/*
+ * prism_av_norm -- the audio-to-video cross-attention output norm that the
+ *   next layer's prism_plan() reads as a_map (page paper.rainbus.top, section
+ *   "前置知识", the dual-branch DiT paragraph: h_hat = CrossAttn(h, K_a, V_a)
+ *   and its L2 norm per video position; page xyznot.com/id, section "Metode"
+ *   1: a_{t,h,w} = ||h_hat_{t,h,w}||_2, cached from the previous layer):
+ *     h_hat[head][n] = softmax_m(Qv[head][n] . Ka[head][m] / sqrt(D)) Va[head][m]
+ *     a_map[n]       = sqrt(sum over heads and channels of h_hat[head][n][c]^2)
+ *   i.e. the norm of the heads' concatenated outputs before the output
+ *   projection (which belongs to the backbone's weights).  One launch covers
+ *   every head; the map is written once per token (no atomics).
+ * Arguments
+ *   N          video tokens (T*H*W of the map, raster order), 1 .. 2^31 - 128.
+ *   M          audio tokens, 1 .. 2^20 (the pages' audio is under 1K tokens).
+ *   heads      1 .. 4096;  head_dim 64 or 128.
+ *   Qv         device bf16 [heads][N][head_dim]: the video tokens' queries.
+ *   Ka, Va     device bf16 [heads][M][head_dim]: the audio tokens' keys, values.
+ *   a_map      device fp32 [N] (output): the map, ready for prism_plan.
+ *   h_hat      device [heads][N][head_dim] of hhat_dtype (output), or NULL to
+ *              produce the map alone.
+ *   hhat_dtype PRISM_BF16 or PRISM_F32.
+ *   dev_status device int32[4], zero before the call: a bounded device wait
+ *              that gives up records PRISM_ERR_TIMEOUT and its site there
+ *              (read and cleared by prism_status_read).
+ * Tensor-core products take the bf16 inputs as they are and a bf16 P, with
+ * fp32 accumulation and an fp32 online softmax.  All pointers 16-byte aligned.
+ * Returns PRISM_ERR_INVALID_ARG for sizes or pointers outside the above,
+ * PRISM_ERR_UNSUPPORTED without an sm_100 device, PRISM_ERR_CUDA if the launch
+ * fails; asynchronous on `stream` otherwise.
+ */
+PRISM_API int prism_av_norm(int64_t N, int32_t M, int32_t heads, int32_t head_dim, const void* Qv,
+                            const void* Ka, const void* Va, float* a_map, void* h_hat,
+                            int32_t hhat_dtype, int32_t* dev_status, void* stream);
+
+/* Synchronises `stream`, reads a device status block (int32[4], as passed to
+ * prism_av_norm), clears it, and returns its status (PRISM_OK or
+ * PRISM_ERR_TIMEOUT; PRISM_ERR_CUDA if the copy fails).  *site (if not NULL)
+ * receives the site of a timed-out wait. */
+PRISM_API int prism_status_read(int32_t* dev_status, int32_t* site, void* stream);
+
 /* ---- inspection -------------------------------------------------------- */
 #define PRISM_ITEM_SHAPE_ID   0  /* uint8  [heads][Nz]                         */
 #define PRISM_ITEM_NBLOCKS    1  /* int32  [heads]                             */

@@ -85,3 +85,19 @@ def test_no_cpu_fallback_in_package():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dp, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
+
+
+def test_av_norm_validation_without_device(lib):
+    """prism_av_norm rejects bad sizes, dtypes and pointers before touching a device."""
+    from dynamic_block_sparse_indicator_b200 import _lib
+    d = C.c_void_p(256)
+    odd = C.c_void_p(264)
+
+    def call(N=2048, M=100, heads=2, D=64, q=d, k=d, v=d, a=d, hh=None, hdt=_lib.PRISM_BF16, st=d):
+        return lib.prism_av_norm(N, M, heads, D, q, k, v, a, hh, hdt, st, None)
+
+    for bad in (dict(N=0), dict(N=1 << 31), dict(M=0), dict(M=(1 << 20) + 1), dict(heads=0),
+                dict(D=96), dict(hdt=5), dict(q=None), dict(k=None), dict(v=None), dict(a=None),
+                dict(st=None), dict(q=odd), dict(a=odd), dict(hh=odd), dict(st=odd)):
+        assert call(**bad) == _lib.PRISM_ERR_INVALID_ARG, bad
+    assert lib.prism_status_read(None, None, None) == _lib.PRISM_ERR_INVALID_ARG
