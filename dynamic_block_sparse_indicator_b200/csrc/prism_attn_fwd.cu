@@ -8,15 +8,23 @@
 //
 // Design (B200): one CTA per 128-token query tile.  The plan's tile list gives,
 // for the tile, the 128-token key tiles to visit with a 4-bit mask (which
-// 64-token query half attends to which 64-token key half).  Per key tile:
-//   TMA (128B swizzle) K (2-stage ring) and V (one buffer), fp16 block-ordered copies
-//   tcgen05.mma S = Q K^T into TMEM (double-buffered, 2 x 128 columns)
-//   8 softmax warps (2 per TMEM lane quarter, 64 keys each) read S, mask, update the
-//     running max (rescaling O in TMEM only when it grows by more than 2^8),
-//     write P = 2^(s - m) as fp16 into TMEM
-//   tcgen05.mma O += P V (P read from TMEM, V from shared memory) into TMEM
-// Warp roles: 0-7 softmax/epilogue (two warpgroups, one per 64-key half),
-// 8 TMA producer (and TMEM allocator), 9 MMA issuer.  Every barrier wait is bounded (PRISM_ERR_TIMEOUT).
+// 64-token query half attends to which 64-token key half).  The key tiles
+// alternate between two softmax warpgroups: group g takes steps j = g, g + 2,
+// ..., each thread one full query row of the step's 128 keys, with its own
+// running max and sum and its own O accumulator in TMEM.  The groups never wait
+// for each other inside the loop (no per-step exchange of row maxima), so one
+// group's exponentials overlap the other's products; the two partial outputs
+// are merged once at the end, O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / L.
+//   TMA (128B swizzle): Q once, K and V two-stage rings (fp16 block-ordered copies)
+//   tcgen05.mma S = Q K^T into TMEM (one 128-column buffer per group), issued by
+//     warp 9 as soon as the group has read its previous S (s_free)
+//   softmax: row max (exact rescale of the group's O when it grows), P = 2^15
+//     2^(s - m) as fp16 into the group's shared-memory buffer
+//   tcgen05.mma O_g += P V, issued by warp 10 (a second issuer, so a wait for P
+//     never holds back the next S)
+// Warp roles: 0-7 softmax (two warpgroups) and epilogue, 8 TMA producer (and
+// TMEM allocator), 9 QK issuer, 10 PV issuer.  Every barrier wait is bounded
+// (PRISM_ERR_TIMEOUT).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -26,7 +34,8 @@
 
 namespace prism {
 
-constexpr int FWD_STAGES = 2;
+constexpr int FWD_KST = 2;          // K ring depth
+constexpr int FWD_VST = 2;          // V ring depth
 #ifndef PRISM_RESCALE_LOG2
 #define PRISM_RESCALE_LOG2 0.0f
 #endif
@@ -36,22 +45,20 @@ constexpr int FWD_STAGES = 2;
 constexpr float kRescaleLog2 = PRISM_RESCALE_LOG2;
 constexpr float kPScaleLog2 = 15.f;   // P operand scale 2^15 (<= 32768 < fp16 max)
 constexpr int SLAB = 128 * 64 * 2;   // bytes of a 128-row x 64-column fp16 slab
+constexpr int FWD_THREADS = 352;
 
 template <int HD>
 struct FwdSmem {
     static constexpr int NSL = HD / 64;
     alignas(1024) uint8_t q[NSL][SLAB];
-    alignas(1024) uint8_t k[FWD_STAGES][NSL][SLAB];
-    alignas(1024) uint8_t v[NSL][SLAB];           // one V tile: PV_j runs long after QK_j+1
-    alignas(1024) uint8_t p[2][2][SLAB];          // [buffer][64-key slab]
+    alignas(1024) uint8_t k[FWD_KST][NSL][SLAB];
+    alignas(1024) uint8_t v[FWD_VST][NSL][SLAB];
+    alignas(1024) uint8_t p[2][2][SLAB];          // [group][64-key slab]; the epilogue's exchange reuses it
     uint64_t bar_q;
-    uint64_t k_full[FWD_STAGES], k_empty[FWD_STAGES];
-    uint64_t v_full, v_empty;
-    uint64_t s_full[2], p_full[2], pv_done[2];
-    float pmax[2][2][128];                        // [step parity][warpgroup][row] partial max
-    float psum[2][128];                           // [warpgroup][row] partial sum (epilogue)
+    uint64_t k_full[FWD_KST], k_empty[FWD_KST];
+    uint64_t v_full[FWD_VST], v_empty[FWD_VST];
+    uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
     uint32_t tmem_base;
-    int abort;
 };
 
 struct FwdArgs {
@@ -67,8 +74,96 @@ struct FwdArgs {
     int* err;
 };
 
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// max over 64 fp32 values held as bits
+__device__ __forceinline__ float max64(const uint32_t* sr) {
+    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    #pragma unroll
+    for (int c = 0; c < 64; c += 2)
+        m4[(c >> 1) & 3] = fmax3f(m4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+    return fmax3f(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+}
+
+// Pairs of P (out of every 8 pairs of a row's keys) whose 2^x runs on the FMA
+// pipe instead of the MUFU unit (16 ex2 per SM per clock take as long as the
+// tile's two products at head_dim 128).  Measured on B200 at the 1M-token head:
+// 0 of 8 -> 550 ms, 2 -> 630 ms, 3 -> 650 ms (the emulation's dependent chain
+// costs more than the MUFU time it frees), so the default is 0.
+#ifndef PRISM_FWD_EMU
+#define PRISM_FWD_EMU 0
+#endif
+constexpr int kFwdEmuPer8 = PRISM_FWD_EMU;
+
+__device__ __forceinline__ void add2f(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x for two lanes on the FMA pipe: x = n + f, n = round(x) (adding 1.5 * 2^23
+// leaves n in the low mantissa bits), 2^f on [-1/2, 1/2] by a degree-4
+// polynomial, minimax in relative error (coefficients fitted by Lawson-weighted
+// least squares; max relative error 2.7e-6 evaluated in fp32, well below the
+// 2^-11 rounding of the fp16 P it feeds), 2^n added into the exponent field.  x
+// is clamped at -126 so that field never underflows.
+__device__ __forceinline__ void exp2_poly4(float& y0, float& y1, float x0, float x1) {
+    constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+    constexpr float c0 = 0.99999928f, c1 = 0.69312179f, c2 = 0.24024744f, c3 = 0.055917863f,
+                    c4 = 0.0095700966f;
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    float t0, t1, n0, n1, f0, f1, p0, p1;
+    add2f(t0, t1, x0, x1, kRound, kRound);
+    add2f(n0, n1, t0, t1, -kRound, -kRound);
+    add2f(f0, f1, x0, x1, -n0, -n1);
+    ffma2(p0, p1, c4, c4, f0, f1, c3, c3);
+    ffma2(p0, p1, p0, p1, f0, f1, c2, c2);
+    ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// P' = 2^(s * scale_log2 + neg) for one row's 64 keys as 32 packed fp16 pairs
+// (zeros when the key half is masked); returns the sum of the values.
+__device__ __forceinline__ float exp_p64(const uint32_t* sr, bool valid, float scale_log2, float neg,
+                                         uint32_t* pk) {
+    float l2[2] = {0.f, 0.f};
+    #pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        float p0 = 0.f, p1 = 0.f;
+        if (valid) {
+            float x0, x1;
+            ffma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), scale_log2, scale_log2, neg,
+                  neg);
+            if ((e & 7) >= 8 - kFwdEmuPer8) {
+                exp2_poly4(p0, p1, x0, x1);
+            } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+            }
+        }
+        add2f(l2[0], l2[1], l2[0], l2[1], p0, p1);
+        pk[e] = pack_f16(p0, p1);
+    }
+    return l2[0] + l2[1];
+}
+
+// 32 packed pairs (64 keys) of row r into a 128B-swizzled shared-memory slab.
+__device__ __forceinline__ void store_p64(const uint32_t* pk, uint32_t slab_s, int r) {
+    #pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+        st_shared_v4(slab_s + swz128(r, ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+}
+
 template <int HD>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(FWD_THREADS, 1)
 k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, FwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -84,21 +179,17 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < FWD_STAGES; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
-        mbar_init(&sm.v_full, 1);
-        mbar_init(&sm.v_empty, 1);
+        for (int s = 0; s < FWD_KST; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
+        for (int s = 0; s < FWD_VST; ++s) { mbar_init(&sm.v_full[s], 1); mbar_init(&sm.v_empty[s], 1); }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.p_full[b], 256);
+            mbar_init(&sm.s_free[b], 128);
+            mbar_init(&sm.p_full[b], 128);
             mbar_init(&sm.pv_done[b], 1);
         }
-        sm.abort = 0;
         mbar_fence_init();
     }
-    // warps 0-7: two softmax warpgroups (same 128 query rows; warpgroup g takes
-    // the 64 keys of key half g of every tile); warp 8: TMA producer + TMEM
-    // allocator; warp 9: MMA issuer.
-    constexpr int W_PROD = 8, W_MMA = 9;
+    constexpr int W_PROD = 8, W_QK = 9, W_PV = 10;
     if (warp == W_PROD) {
         __syncwarp();
         tmem_alloc(&sm.tmem_base, 512);
@@ -107,8 +198,8 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    // TMEM columns: S double-buffered at 0 and 128, O at 256 (HD columns)
-    constexpr uint32_t TS = 0, TO = 256;
+    // TMEM columns: S of group g at 128 g; O of group g at 256 + HD g
+    constexpr uint32_t TO = 256;
     const int64_t qrow0 = (int64_t)h * a.N + (int64_t)t * 128;
 
     if (warp == W_PROD) {
@@ -119,201 +210,219 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             mbar_expect_tx(&sm.bar_q, NSL * SLAB);
             for (int c = 0; c < NSL; ++c) tma_load_2d(sm.q[c], &tm_q, &sm.bar_q, 64 * c, (int)qrow0);
             for (int j = 0; j < n; ++j) {
-                const int s = j % FWD_STAGES;
-                if (j >= FWD_STAGES &&
-                    !mbar_wait(&sm.k_empty[s], ((j / FWD_STAGES) - 1) & 1, a.err, 401)) break;
+                const int s = j % FWD_KST;
+                if (j >= FWD_KST &&
+                    !mbar_wait(&sm.k_empty[s], ((j / FWD_KST) - 1) & 1, a.err, 401)) break;
                 const int krow = (int)((int64_t)h * a.N + (int64_t)(ents[j] >> 4) * 128);
                 mbar_expect_tx(&sm.k_full[s], NSL * SLAB);
                 for (int c = 0; c < NSL; ++c) tma_load_2d(sm.k[s][c], &tm_k, &sm.k_full[s], 64 * c, krow);
             }
         } else if (lane == 1 && n > 0) {
             for (int j = 0; j < n; ++j) {
-                if (j >= 1 && !mbar_wait(&sm.v_empty, (j - 1) & 1, a.err, 402)) break;
+                const int s = j % FWD_VST;
+                if (j >= FWD_VST &&
+                    !mbar_wait(&sm.v_empty[s], ((j / FWD_VST) - 1) & 1, a.err, 402)) break;
                 const int krow = (int)((int64_t)h * a.N + (int64_t)(ents[j] >> 4) * 128);
-                mbar_expect_tx(&sm.v_full, NSL * SLAB);
-                for (int c = 0; c < NSL; ++c) tma_load_2d(sm.v[c], &tm_v, &sm.v_full, 64 * c, krow);
+                mbar_expect_tx(&sm.v_full[s], NSL * SLAB);
+                for (int c = 0; c < NSL; ++c) tma_load_2d(sm.v[s][c], &tm_v, &sm.v_full[s], 64 * c, krow);
             }
         }
-    } else if (warp == W_MMA) {
-        // ------------------------------------------------ MMA issuer
+    } else if (warp == W_QK) {
+        // ------------------------------------------------ S = Q K^T issuer
         if (lane == 0 && n > 0) {
             constexpr uint32_t idesc_qk = idesc_f16(128, 128, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_f16(128, HD, 0, 1);
-            // descriptor low words; every K step below adds an immediate
             const uint32_t qA = desc_lo(smem_u32(sm.q[0]), 16);
-            const uint32_t vT = desc_lo(smem_u32(sm.v[0]), SLAB);
-            bool ok = mbar_wait(&sm.bar_q, 0, a.err, 501);
-            for (int j = 0; ok && j <= n; ++j) {
-                if (j < n) {
-                    const int s = j % FWD_STAGES, b = j & 1;
-                    if (!mbar_wait(&sm.k_full[s], (j / FWD_STAGES) & 1, a.err, 502)) { ok = false; break; }
+            if (mbar_wait(&sm.bar_q, 0, a.err, 501)) {
+                for (int j = 0; j < n; ++j) {
+                    const int s = j % FWD_KST, b = j & 1;
+                    // group b has read S of its previous step out of TMEM
+                    if (j >= 2 && !mbar_wait(&sm.s_free[b], ((j - 2) >> 1) & 1, a.err, 505)) break;
+                    if (!mbar_wait(&sm.k_full[s], (j / FWD_KST) & 1, a.err, 502)) break;
                     tc_fence_after();
                     const uint32_t kB = desc_lo(smem_u32(sm.k[s][0]), 16);
                     #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)
-                        umma_f16(tmem + TS + 128 * b, desc_from_lo(qA + kmajor_step(kk, SLAB)),
+                        umma_f16(tmem + 128 * b, desc_from_lo(qA + kmajor_step(kk, SLAB)),
                                  desc_from_lo(kB + kmajor_step(kk, SLAB)), idesc_qk, kk > 0);
                     umma_commit(&sm.s_full[b]);
                     umma_commit(&sm.k_empty[s]);
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, b = jj & 1;
-                    if (!mbar_wait(&sm.p_full[b], (jj >> 1) & 1, a.err, 503)) { ok = false; break; }
-                    if (!mbar_wait(&sm.v_full, jj & 1, a.err, 504)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t pA = desc_lo(smem_u32(sm.p[b][0]), 16);
-                    #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_f16(tmem + TO, desc_from_lo(pA + kmajor_step(kk, SLAB)),
-                                 desc_from_lo(vT + mnmajor_step(kk)), idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&sm.pv_done[b]);
-                    umma_commit(&sm.v_empty);
-                }
             }
-            if (!ok) sm.abort = 1;
         }
-    } else {
+    } else if (warp == W_PV) {
+        // ------------------------------------------------ O_g += P V issuer
+        if (lane == 0 && n > 0) {
+            constexpr uint32_t idesc_pv = idesc_f16(128, HD, 0, 1);
+            for (int j = 0; j < n; ++j) {
+                const int s = j % FWD_VST, b = j & 1;
+                if (!mbar_wait(&sm.p_full[b], (j >> 1) & 1, a.err, 503)) break;
+                if (!mbar_wait(&sm.v_full[s], (j / FWD_VST) & 1, a.err, 504)) break;
+                tc_fence_after();
+                const uint32_t pA = desc_lo(smem_u32(sm.p[b][0]), 16);
+                const uint32_t vT = desc_lo(smem_u32(sm.v[s][0]), SLAB);
+                #pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + TO + HD * b, desc_from_lo(pA + kmajor_step(kk, SLAB)),
+                             desc_from_lo(vT + mnmajor_step(kk)), idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+                umma_commit(&sm.pv_done[b]);
+                umma_commit(&sm.v_empty[s]);
+            }
+        }
+    } else if (warp < 8) {
         // ------------------------------------------------ softmax + epilogue
-        // tcgen05.ld/st are warp-collective (.sync.aligned): every decision that
-        // guards one is made warp-uniform (__all_sync / __any_sync).  The two
-        // warps sharing a TMEM lane quarter (w and w + 4) combine their row maxima
-        // through shared memory and a 64-thread named barrier, so both take the
-        // same rescaling decisions.
-        const int wg = warp >> 2;                  // key half handled by this warpgroup
+        // tcgen05.ld/st are warp-collective: every decision that guards one is
+        // warp-uniform (__all_sync / __any_sync).
+        const int g = warp >> 2;                   // group: steps j = g, g + 2, ...
         const int r = (warp & 3) * 32 + lane;      // query row of the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int pair_bar = 1 + (warp & 3);
-        const int qh = r >> 6;                     // uniform per warp (32 | 64)
-        constexpr int OC = HD / 2;                 // O columns rescaled / written per warpgroup
-        const uint32_t ocol = TO + OC * wg;
-        float m_ref = -INFINITY, l = 0.f;          // l: this warpgroup's share of the row sum
+        const int qh = r >> 6;                     // query half (uniform per warp: 32 | 64)
+        const uint32_t scol = 128 * g;             // this group's S columns
+        const uint32_t ocol = TO + HD * g;         // this group's O columns
+        const uint32_t p_s = smem_u32(sm.p[g][0]);
+        float m_ref = -INFINITY, l = 0.f;          // running max (log2 units) and scaled sum
         bool ok = true;
-        int nbar = 0;                              // pair barriers taken in the loop
-        for (int j = 0; j < n; ++j) {
-            const int b = j & 1;
+        int cnt = 0;
+        for (int j = g; j < n; j += 2, ++cnt) {
             const int msk = ents[j] & 15;
-            const bool valid = (msk >> (qh * 2 + wg)) & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (j >> 1) & 1, a.err, 1))) { ok = false; break; }
+            const bool v0 = (msk >> (qh * 2)) & 1, v1 = (msk >> (qh * 2 + 1)) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g], (j >> 1) & 1, a.err, 1))) { ok = false; break; }
             tc_fence_after();
             uint32_t sr[64];
-            PRISM_TMEM_LD32(tmem + lane_off + TS + 128 * b + 64 * wg, (sr + 0));
-            PRISM_TMEM_LD32(tmem + lane_off + TS + 128 * b + 64 * wg + 32, (sr + 32));
-            tmem_wait_ld();
             float mx = -INFINITY;
-            if (valid) {
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                #pragma unroll
-                for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
-                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            if (v0) {
+                PRISM_TMEM_LD32(tmem + lane_off + scol, (sr + 0));
+                PRISM_TMEM_LD32(tmem + lane_off + scol + 32, (sr + 32));
+                tmem_wait_ld();
+                mx = max64(sr);
+            }
+            if (v1) {                              // key half 1 stays in registers
+                PRISM_TMEM_LD32(tmem + lane_off + scol + 64, (sr + 0));
+                PRISM_TMEM_LD32(tmem + lane_off + scol + 96, (sr + 32));
+                tmem_wait_ld();
+                mx = fmaxf(mx, max64(sr));
             }
             mx *= a.scale_log2;
-            sm.pmax[j & 1][wg][r] = mx;
-            named_bar(pair_bar, 64);
-            ++nbar;
-            mx = fmaxf(mx, sm.pmax[j & 1][wg ^ 1][r]);
+            const bool first = (cnt == 0) || (m_ref == -INFINITY);
             const float m_new = fmaxf(m_ref, mx);
-            const bool first = (j == 0) || (m_ref == -INFINITY);
-            const bool need = !first && (m_new > m_ref + kRescaleLog2);
             if (first) m_ref = m_new;
-            const bool rescale = __any_sync(0xffffffffu, need);
-            if (rescale) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err, 2))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const float f = need ? ex2(m_ref - m_new) : 1.f;
-                #pragma unroll
-                for (int c = 0; c < OC / 32; ++c) {
-                    uint32_t o[32];
-                    PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * c, o);
-                    tmem_wait_ld();
-                    #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    PRISM_TMEM_ST32(tmem + lane_off + ocol + 32 * c, o);
-                }
-                if (need) { l *= f; m_ref = m_new; }
-            }
-            if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[b], ((j - 2) >> 1) & 1, a.err, 3))) {
-                ok = false;
-                break;
-            }
+            const bool need = !first && (m_new > m_ref + kRescaleLog2);
+            const float f = need ? ex2(m_ref - m_new) : 1.f;
+            if (need) m_ref = m_new;
             // P is formed as 2^15 * 2^(s - m): the fp16 operand of the PV product then
             // holds probabilities down to 2^-29 as normal numbers (the near-uniform rows
             // of a 1M-token head sit near 1e-6, fp16's subnormal range), and the
             // 2^15 cancels in O = acc / l because l sums the same scaled values.
+            // The exponentials go to registers first: only the stores into this
+            // group's P buffer (and the rescale of O_g) wait for the previous product.
             const float neg = kPScaleLog2 - m_ref;
-            const uint32_t p_s = smem_u32(sm.p[b][wg]);
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
-            #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t w[4];
-                #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = ch * 8 + 2 * e;
-                    float p0 = 0.f, p1 = 0.f;
-                    if (valid) {
-                        p0 = ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, neg));
-                        p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, neg));
-                    }
-                    l4[e] += p0 + p1;
-                    w[e] = pack_f16(p0, p1);
-                }
-                st_shared_v4(p_s + swz128(r, ch), w[0], w[1], w[2], w[3]);
+            uint32_t pk1[32], pk0[32];
+            float lsum = exp_p64(sr, v1, a.scale_log2, neg, pk1);
+            if (v0) {                              // key half 0 again from TMEM
+                PRISM_TMEM_LD32(tmem + lane_off + scol, (sr + 0));
+                PRISM_TMEM_LD32(tmem + lane_off + scol + 32, (sr + 32));
+                tmem_wait_ld();
             }
-            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            // S has been read: the next S of this group may overwrite it
+            tc_fence_before();
+            mbar_arrive(&sm.s_free[g]);
+            lsum += exp_p64(sr, v0, a.scale_log2, neg, pk0);
+            // O_g and this group's P buffer were last used by the product of step j - 2
+            if (cnt > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g], ((j - 2) >> 1) & 1, a.err, 2))) {
+                ok = false;
+                break;
+            }
+            store_p64(pk1, p_s + SLAB, r);
+            store_p64(pk0, p_s, r);
+            const bool rescale = __any_sync(0xffffffffu, need);
+            if (rescale) {
+                tc_fence_after();
+                #pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * c, o);
+                    tmem_wait_ld();
+                    #pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        float y0, y1;
+                        fmul2(y0, y1, __uint_as_float(o[e]), __uint_as_float(o[e + 1]), f, f);
+                        o[e] = __float_as_uint(y0);
+                        o[e + 1] = __float_as_uint(y1);
+                    }
+                    PRISM_TMEM_ST32(tmem + lane_off + ocol + 32 * c, o);
+                }
+            }
+            l = fmaf(l, f, lsum);
             fence_proxy_async_smem();
             if (rescale) tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.p_full[b]);
+            mbar_arrive(&sm.p_full[g]);
         }
-        // epilogue: both warpgroups add their row sums, each writes half of O
+        // epilogue: merge the groups' partial outputs.  Each group waits for its own
+        // last product first (the PV issuer completes products in step order, so the
+        // other group's barrier is then at most one phase behind), then the other's.
+        const bool has0 = n > 0, has1 = n > 1;
+        bool fin = ok && has0;
+        for (int k = 0; k < 2 && fin; ++k) {
+            const int gg = k == 0 ? g : (g ^ 1);
+            if (n <= gg) continue;
+            const int jl = gg + 2 * ((n - 1 - gg) / 2);
+            fin = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[gg], (jl >> 1) & 1, a.err, 4));
+        }
+        // the P buffers are idle once every product has completed: exchange there
+        float* xm = reinterpret_cast<float*>(&sm.p[0][0][0]);    // [group][row] max
+        float* xl = xm + 256;                                     // [group][row] sum
+        if (fin) {
+            xm[g * 128 + r] = m_ref;
+            xl[g * 128 + r] = l;
+        }
+        named_bar(1 + (warp & 3), 64);
         const int row_perm = t * 128 + r;
         const int dst = a.src[(size_t)h * a.N + row_perm];
         const size_t orow = (size_t)h * a.N + (size_t)dst;
-        // A warp that left the loop on a failed wait still takes the pair barriers
-        // its partner will take (one per tile, then the epilogue's), so the
-        // partner is never left at a barrier.
-        for (; nbar < n; ++nbar) named_bar(pair_bar, 64);
-        bool fin = false;
-        if (ok && n > 0)
-            fin = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err, 4));
-        sm.psum[wg][r] = l;
-        named_bar(pair_bar, 64);
         if (fin) {
-            const float lt = sm.psum[0][r] + sm.psum[1][r];
-            tc_fence_after();
+            const float m0 = xm[r], m1 = has1 ? xm[128 + r] : -INFINITY;
+            const float l0 = xl[r], l1 = has1 ? xl[128 + r] : 0.f;
+            const float m = fmaxf(m0, m1);
+            const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
+            const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
+            const float lt = l0 * f0 + l1 * f1;
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const float w0 = f0 * inv, w1 = f1 * inv;
+            tc_fence_after();
+            constexpr int OC = HD / 2;             // output columns written by each group
             #pragma unroll
             for (int c = 0; c < OC / 32; ++c) {
-                uint32_t o[32];
-                PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * c, o);
+                const int c0 = OC * g + 32 * c;
+                uint32_t o0[32], o1[32];
+                PRISM_TMEM_LD32(tmem + lane_off + TO + c0, o0);
+                if (has1) PRISM_TMEM_LD32(tmem + lane_off + TO + HD + c0, o1);
                 tmem_wait_ld();
-                const int c0 = OC * wg + 32 * c;
+                float x[32];
+                #pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    x[e] = has1 ? fmaf(__uint_as_float(o0[e]), w0, __uint_as_float(o1[e]) * w1)
+                                : __uint_as_float(o0[e]) * w0;
                 if (a.out_f32) {
                     float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * HD + c0);
                     #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        op[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
-                                            __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+                    for (int e = 0; e < 8; ++e) op[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
                 } else {
                     uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + orow * HD + c0);
                     #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        op[e] = make_uint4(pack_bf16(__uint_as_float(o[8 * e]) * inv, __uint_as_float(o[8 * e + 1]) * inv),
-                                           pack_bf16(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv),
-                                           pack_bf16(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv),
-                                           pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv));
+                        op[e] = make_uint4(pack_bf16(x[8 * e], x[8 * e + 1]), pack_bf16(x[8 * e + 2], x[8 * e + 3]),
+                                           pack_bf16(x[8 * e + 4], x[8 * e + 5]), pack_bf16(x[8 * e + 6], x[8 * e + 7]));
                 }
             }
-            if (wg == 0)
-                a.lse[orow] = lt > 0.f ? (m_ref - kPScaleLog2) * 0.69314718055994531f + logf(lt) : -INFINITY;
+            if (g == 0)
+                a.lse[orow] = lt > 0.f ? (m - kPScaleLog2) * 0.69314718055994531f + logf(lt) : -INFINITY;
         } else if (n == 0) {
-            for (int c = OC * wg; c < OC * wg + OC; ++c) {
+            constexpr int OC = HD / 2;
+            for (int c = OC * g; c < OC * g + OC; ++c) {
                 if (a.out_f32) static_cast<float*>(a.O)[orow * HD + c] = 0.f;
                 else static_cast<__nv_bfloat16*>(a.O)[orow * HD + c] = __float2bfloat16(0.f);
             }
-            if (wg == 0) a.lse[orow] = -INFINITY;
+            if (g == 0) a.lse[orow] = -INFINITY;
         }
     }
     tc_fence_before();
@@ -358,7 +467,7 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
         return PRISM_ERR_CUDA;
     {
         PrismProf prof(P, PRISM_STAGE_FWD, s);
-        k_attn_fwd<HD><<<dim3(g.NT, g.heads), 320, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+        k_attn_fwd<HD><<<dim3(g.NT, g.heads), FWD_THREADS, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
     }
     P->launches += 1;
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
