@@ -24,7 +24,8 @@
 //     never holds back the next S)
 // Warp roles: 0-7 softmax (two warpgroups) and epilogue, 8 TMA producer (and
 // TMEM allocator), 9 QK issuer, 10 PV issuer.  Every barrier wait is bounded
-// (PRISM_ERR_TIMEOUT).
+// (PRISM_ERR_TIMEOUT).  Heads with more than 1,024 key tiles run in passes over
+// key-tile ranges (see kFwdKeyChunk) that carry (O, max, sum) per query row.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -46,6 +47,13 @@ constexpr float kRescaleLog2 = PRISM_RESCALE_LOG2;
 constexpr float kPScaleLog2 = 15.f;   // P operand scale 2^15 (<= 32768 < fp16 max)
 constexpr int SLAB = 128 * 64 * 2;   // bytes of a 128-row x 64-column fp16 slab
 constexpr int FWD_THREADS = 352;
+// Key tiles per pass.  Every query tile's list is walked in ascending key order;
+// over a whole 1M-token head (7,920 key tiles, 518 MB of fp16 K and V) the CTAs in
+// flight drift apart along their lists and a third of the K/V tile loads missed
+// L2.  A pass visits only 1,024 key tiles (64 MB of K and V, half of L2) for
+// every query tile, and merges its (O, max, sum) into a running state that the
+// next pass continues; the last pass writes O and LSE.
+constexpr int kFwdKeyChunk = 1024;
 
 template <int HD>
 struct FwdSmem {
@@ -59,6 +67,7 @@ struct FwdSmem {
     uint64_t v_full[FWD_VST], v_empty[FWD_VST];
     uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
     uint32_t tmem_base;
+    int e0, n;                                    // this pass's entries of the tile's list
 };
 
 struct FwdArgs {
@@ -71,8 +80,24 @@ struct FwdArgs {
     int NT;
     int out_f32;
     float scale_log2;      // log2(e) / sqrt(HD)
+    int key_lo, key_hi;    // this pass's key tiles [key_lo, key_hi)
+    int first, last;       // first pass (no state to merge), last pass (write O and LSE)
+    float* st_o;           // [heads][N][HD] running O (unnormalised, relative to 2^m), block order
+    float* st_m;           // [heads][N] running max (log2 units, P scale included)
+    float* st_l;           // [heads][N] running sum
     int* err;
 };
+
+// First index in the ascending list e[0, n) whose tile (entry >> 4) is >= key.
+__device__ __forceinline__ int fwd_lower_bound(const int* e, int n, int key) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((e[mid] >> 4) < key) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
 
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
     float r;
@@ -172,12 +197,14 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     constexpr int NSL = HD / 64;
     const int t = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int* ents = a.qt_ent + (size_t)h * a.NT * a.NT;
-    const int e0 = a.qt_ptr[(size_t)h * (a.NT + 1) + t];
-    const int n = a.qt_ptr[(size_t)h * (a.NT + 1) + t + 1] - e0;
-    ents += e0;
-
     if (threadIdx.x == 0) {
+        // this pass visits the key tiles of [key_lo, key_hi) of the tile's ascending list
+        const int p0 = a.qt_ptr[(size_t)h * (a.NT + 1) + t];
+        const int n0 = a.qt_ptr[(size_t)h * (a.NT + 1) + t + 1] - p0;
+        const int* all = a.qt_ent + (size_t)h * a.NT * a.NT + p0;
+        const int lo = fwd_lower_bound(all, n0, a.key_lo);
+        sm.e0 = p0 + lo;
+        sm.n = fwd_lower_bound(all, n0, a.key_hi) - lo;
         mbar_init(&sm.bar_q, 1);
         for (int s = 0; s < FWD_KST; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
         for (int s = 0; s < FWD_VST; ++s) { mbar_init(&sm.v_full[s], 1); mbar_init(&sm.v_empty[s], 1); }
@@ -198,6 +225,8 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    const int n = sm.n;
+    const int* ents = a.qt_ent + (size_t)h * a.NT * a.NT + sm.e0;
     // TMEM columns: S of group g at 128 g; O of group g at 256 + HD g
     constexpr uint32_t TO = 256;
     const int64_t qrow0 = (int64_t)h * a.N + (int64_t)t * 128;
@@ -361,7 +390,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // last product first (the PV issuer completes products in step order, so the
         // other group's barrier is then at most one phase behind), then the other's.
         const bool has0 = n > 0, has1 = n > 1;
-        bool fin = ok && has0;
+        bool fin = ok;
         for (int k = 0; k < 2 && fin; ++k) {
             const int gg = k == 0 ? g : (g ^ 1);
             if (n <= gg) continue;
@@ -377,32 +406,59 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         named_bar(1 + (warp & 3), 64);
         const int row_perm = t * 128 + r;
-        const int dst = a.src[(size_t)h * a.N + row_perm];
-        const size_t orow = (size_t)h * a.N + (size_t)dst;
+        const size_t prow = (size_t)h * a.N + (size_t)row_perm;   // block order (running state)
         if (fin) {
-            const float m0 = xm[r], m1 = has1 ? xm[128 + r] : -INFINITY;
-            const float l0 = xl[r], l1 = has1 ? xl[128 + r] : 0.f;
-            const float m = fmaxf(m0, m1);
-            const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
-            const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
-            const float lt = l0 * f0 + l1 * f1;
-            const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            const float w0 = f0 * inv, w1 = f1 * inv;
+            // this pass: (O_0 2^(m_0 - m_c) + O_1 2^(m_1 - m_c), l_c) relative to 2^m_c
+            const float m0 = has0 ? xm[r] : -INFINITY, m1 = has1 ? xm[128 + r] : -INFINITY;
+            const float l0 = has0 ? xl[r] : 0.f, l1 = has1 ? xl[128 + r] : 0.f;
+            const float mc = fmaxf(m0, m1);
+            const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - mc);
+            const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - mc);
+            const float lc = l0 * f0 + l1 * f1;
+            // merged with the state of the previous passes over the other key tiles
+            const float ms = a.first ? -INFINITY : a.st_m[prow];
+            const float ls = a.first ? 0.f : a.st_l[prow];
+            const float m = fmaxf(mc, ms);
+            const float fc = mc == -INFINITY ? 0.f : ex2(mc - m);
+            const float fs = ms == -INFINITY ? 0.f : ex2(ms - m);
+            const float lt = lc * fc + ls * fs;
+            const float inv = a.last ? (lt > 0.f ? 1.f / lt : 0.f) : 1.f;
+            const float w0 = f0 * fc * inv, w1 = f1 * fc * inv, ws = fs * inv;
+            const bool use_s = !a.first && ms != -INFINITY;
+            const size_t orow = a.last ? (size_t)h * a.N + (size_t)a.src[prow] : 0;
             tc_fence_after();
             constexpr int OC = HD / 2;             // output columns written by each group
             #pragma unroll
             for (int c = 0; c < OC / 32; ++c) {
                 const int c0 = OC * g + 32 * c;
                 uint32_t o0[32], o1[32];
-                PRISM_TMEM_LD32(tmem + lane_off + TO + c0, o0);
+                if (has0) PRISM_TMEM_LD32(tmem + lane_off + TO + c0, o0);
                 if (has1) PRISM_TMEM_LD32(tmem + lane_off + TO + HD + c0, o1);
                 tmem_wait_ld();
                 float x[32];
                 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    x[e] = has1 ? fmaf(__uint_as_float(o0[e]), w0, __uint_as_float(o1[e]) * w1)
-                                : __uint_as_float(o0[e]) * w0;
-                if (a.out_f32) {
+                for (int e = 0; e < 32; ++e) {
+                    float v = 0.f;
+                    if (has0) v = __uint_as_float(o0[e]) * w0;
+                    if (has1) v = fmaf(__uint_as_float(o1[e]), w1, v);
+                    x[e] = v;
+                }
+                if (use_s) {
+                    const float4* sp = reinterpret_cast<const float4*>(a.st_o + prow * HD + c0);
+                    #pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 y = sp[e];
+                        x[4 * e] = fmaf(y.x, ws, x[4 * e]);
+                        x[4 * e + 1] = fmaf(y.y, ws, x[4 * e + 1]);
+                        x[4 * e + 2] = fmaf(y.z, ws, x[4 * e + 2]);
+                        x[4 * e + 3] = fmaf(y.w, ws, x[4 * e + 3]);
+                    }
+                }
+                if (!a.last) {
+                    float4* sp = reinterpret_cast<float4*>(a.st_o + prow * HD + c0);
+                    #pragma unroll
+                    for (int e = 0; e < 8; ++e) sp[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                } else if (a.out_f32) {
                     float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * HD + c0);
                     #pragma unroll
                     for (int e = 0; e < 8; ++e) op[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
@@ -414,15 +470,14 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                            pack_bf16(x[8 * e + 4], x[8 * e + 5]), pack_bf16(x[8 * e + 6], x[8 * e + 7]));
                 }
             }
-            if (g == 0)
-                a.lse[orow] = lt > 0.f ? (m - kPScaleLog2) * 0.69314718055994531f + logf(lt) : -INFINITY;
-        } else if (n == 0) {
-            constexpr int OC = HD / 2;
-            for (int c = OC * g; c < OC * g + OC; ++c) {
-                if (a.out_f32) static_cast<float*>(a.O)[orow * HD + c] = 0.f;
-                else static_cast<__nv_bfloat16*>(a.O)[orow * HD + c] = __float2bfloat16(0.f);
+            if (g == 0) {
+                if (a.last) {
+                    a.lse[orow] = lt > 0.f ? (m - kPScaleLog2) * 0.69314718055994531f + logf(lt) : -INFINITY;
+                } else {
+                    a.st_m[prow] = m;
+                    a.st_l[prow] = lt;
+                }
             }
-            if (g == 0) a.lse[orow] = -INFINITY;
         }
     }
     tc_fence_before();
@@ -462,14 +517,26 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
     a.out_f32 = P->p.out_dtype == PRISM_F32;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
     a.err = (int*)(b + P->L.err);
+    // The running state between passes lives in buffers the backward fills only
+    // later: the fp32 dQ accumulator (O) and the per-row terms (max, sum).
+    a.st_o = (float*)(b + P->L.dq_acc);
+    a.st_m = (float*)(b + P->L.lse_p);
+    a.st_l = (float*)(b + P->L.di_p);
     const int smem = (int)sizeof(FwdSmem<HD>) + 1024;
     if (cudaFuncSetAttribute(k_attn_fwd<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
+    const int passes = (g.NT + kFwdKeyChunk - 1) / kFwdKeyChunk;
     {
         PrismProf prof(P, PRISM_STAGE_FWD, s);
-        k_attn_fwd<HD><<<dim3(g.NT, g.heads), FWD_THREADS, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+        for (int c = 0; c < passes; ++c) {
+            a.key_lo = c * kFwdKeyChunk;
+            a.key_hi = c + 1 == passes ? g.NT : (c + 1) * kFwdKeyChunk;
+            a.first = c == 0;
+            a.last = c + 1 == passes;
+            k_attn_fwd<HD><<<dim3(g.NT, g.heads), FWD_THREADS, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+        }
     }
-    P->launches += 1;
+    P->launches += passes;
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
