@@ -53,7 +53,10 @@ constexpr int FWD_THREADS = 352;
 // L2.  A pass visits only 1,024 key tiles (64 MB of K and V, half of L2) for
 // every query tile, and merges its (O, max, sum) into a running state that the
 // next pass continues; the last pass writes O and LSE.
-constexpr int kFwdKeyChunk = 1024;
+#ifndef PRISM_FWD_KEY_CHUNK
+#define PRISM_FWD_KEY_CHUNK 1024
+#endif
+constexpr int kFwdKeyChunk = PRISM_FWD_KEY_CHUNK;
 
 template <int HD>
 struct FwdSmem {
