@@ -3,12 +3,12 @@
 Heads with more than 1,024 key tiles (131,072 tokens) are processed in passes
 that each visit one range of key tiles for every query tile and carry the
 running (O, max, sum) of every query row to the next pass; the last pass writes
-O and LSE.  A 16 x 64 x 144 grid (147,456 tokens, 1,152 key tiles: two passes)
-is planned with the oracle's own shapes and selection (prism_plan_import), so
-every query row's key set is exactly the oracle's, and O and LSE are compared on
-sampled rows spread over all query tiles, the rows of the first and the last
-tile included, plus the rows with the most and the fewest selected keys in the
-last key range.
+O and LSE.  A 16 x 64 x 144 grid (147,456 tokens, 1,152 key tiles: two passes),
+at head_dim 128 and 64, is planned with the oracle's own shapes and selection
+(prism_plan_import), so every query row's key set is exactly the oracle's, and O
+and LSE are compared on sampled rows spread over all query tiles, the rows of the
+first and the last tile included, plus the rows with the most and the fewest
+selected keys in the last key range.
 """
 import numpy as np
 import pytest
@@ -22,8 +22,9 @@ from oracle import prism_oracle as po
 pytestmark = pytest.mark.gpu
 
 
-def test_two_pass_forward_matches_oracle(cuda_device):
-    w = syn.workload(2, T=16, H=64, W=144)
+@pytest.mark.parametrize("head_dim", [128, 64])
+def test_two_pass_forward_matches_oracle(head_dim, cuda_device):
+    w = syn.workload(2, T=16, H=64, W=144, head_dim=head_dim)
     assert w.N // 128 > 1024                     # more than one pass
     Q, K, V = syn.make_qkv(w, heads=1)
     a = syn.make_amap(w)
