@@ -59,6 +59,9 @@ def args_():
     ap.add_argument("--av-tokens", type=int, default=1000,
                     help="audio tokens of the guidance-map producer leg (the pages: under 1K)")
     ap.add_argument("--no-av", action="store_true", help="skip the guidance-map producer leg")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the 2K inference sweep instead of the step: forward only on grid 64x88x152, "
+                         "peaked (Q, K x3) and diffuse (x0.5) logits, Top-k 8/16/32 x Top-p 0.8/0.9/0.95")
     return ap.parse_args()
 
 
@@ -388,6 +391,59 @@ def guidance_map_leg(w, M, pk, reps=5):
     return out
 
 
+def run_sweep(a):
+    """The 2K inference sweep (workload 4: grid 64x88x152, 856,064 tokens, head_dim 128,
+    bf16, forward only), one head per point: plan + forward timed with CUDA events
+    (1 warm-up, `--steps` timed), TFLOP/s = 4 D Pi / forward time, mean selected
+    blocks per query block.  Prints one JSON line with every point."""
+    import numpy as np
+    import torch
+    from dynamic_block_sparse_indicator_b200 import _lib
+    from dynamic_block_sparse_indicator_b200 import synthetic as syn
+    pk = peaks()
+    peak = pk.get("bf16_tflops_sustained") or 1400.0
+    points = []
+    for regime, scale in (("peaked", 3.0), ("diffuse", 0.5)):
+        w0 = syn.workload(4, qk_scale=scale)
+        Q, K, V = syn.make_qkv(w0, device="cuda", heads=1)
+        amap = syn.make_amap(w0, device="cuda")
+        for k in (8, 16, 32):
+            for p in (0.8, 0.9, 0.95):
+                params = _lib.make_params(w0.T, w0.H, w0.W, 1, w0.head_dim, _lib.PRISM_BF16, k, p, w0.eps,
+                                          out_dtype=_lib.PRISM_F32)
+                pl = _lib.plan(Q, K, V, amap, params)
+                O, lse = pl.attn_fwd()
+                torch.cuda.synchronize()
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                tp, tf = 0.0, 0.0
+                for _ in range(a.steps):
+                    ev[0].record()
+                    pl = _lib.plan(Q, K, V, amap, params)
+                    ev[1].record()
+                    pl.attn_fwd(O, lse)
+                    ev[2].record()
+                    torch.cuda.synchronize()
+                    tp += ev[0].elapsed_time(ev[1])
+                    tf += ev[1].elapsed_time(ev[2])
+                st = pl.status()
+                if st:
+                    raise RuntimeError(f"device status: {_lib.status_string(st)}")
+                Pi, nb, sel = selected_pairs(pl)
+                fwd_ms = tf / a.steps
+                tfl = 4.0 * w0.head_dim * Pi / (fwd_ms * 1e-3) / 1e12
+                points.append({"regime": regime, "top_k": k, "top_p": p, "plan_ms": tp / a.steps,
+                               "fwd_ms": fwd_ms, "ms_per_head_layer": tp / a.steps + fwd_ms,
+                               "tflops": tfl, "fraction_of_sustained": tfl / peak,
+                               "blocks_per_head": nb, "mean_selected_blocks": sel,
+                               "pair_density": Pi / float(w0.N) ** 2})
+        del Q, K, V
+        torch.cuda.empty_cache()
+    emit({"mode": "sweep", "metric": "Prism sparse-attn forward ms/head-layer, 2K inference sweep",
+          "unit": "ms/head-layer", "higher_is_better": False, "data": "synthetic", "steps": a.steps,
+          "config": {"workload": "grid64x88x152_h1_d128_bf16", "tokens": 856064, "head_dim": 128},
+          "peak_tflops": peak, "sweep": points})
+
+
 def run_prism(a, rank, world, local_rank):
     import numpy as np
     import torch
@@ -608,6 +664,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=timedelta(seconds=600))
     try:
+        if a.sweep:
+            if rank == 0:
+                run_sweep(a)
+            return
         run_prism(a, rank, world, local_rank)
     finally:
         if world > 1:
