@@ -42,7 +42,7 @@ def args_():
     ap.add_argument("--workload", type=int, default=3)
     ap.add_argument("--grid", type=int, nargs=3, default=None, metavar=("T", "H", "W"),
                     help="override the grid (smaller cases for profiler captures)")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="attention sample budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -582,37 +582,70 @@ def run_prism(a, rank, world, local_rank):
     if world == 1 and not a.no_av:
         av = guidance_map_leg(w, a.av_tokens, pk)
     # --------------------------------------------------- end to end (host)
+    # Through the C ABI from pinned host buffers: every step copies its inputs
+    # (Q, K, V, dO, the map) to the device and reads its results (O, LSE, dQ, dK,
+    # dV) back.  The copies run on a side stream against two device buffer sets,
+    # so step i + 1's upload and step i's download overlap step i's kernels; the
+    # timed region runs from before the first upload to after the last download.
     e2e = None
     if a.e2e_steps > 0:
         pin = lambda t: t.cpu().pin_memory()
-        hq, hk, hv = pin(Q[:1]), pin(K[:1]), pin(V[:1])
-        hdo, ha = pin(dO[:1]), pin(amap)
-        outs = [torch.empty(1, w.N, D, dtype=torch.float32).pin_memory() for _ in range(4)]
-        hlse = torch.empty(1, w.N, dtype=torch.float32).pin_memory()
-        dq_, dk_, dv_ = (torch.empty_like(Q[:1]) for _ in range(3))
-        bufs = dict(q=dq_, k=dk_, v=dv_, do=torch.empty_like(dO[:1]), a=torch.empty_like(amap))
-        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo, ha))
-        d2h = sum(x.numel() * x.element_size() for x in outs) + hlse.numel() * 4
+        hin = dict(q=pin(Q[:1]), k=pin(K[:1]), v=pin(V[:1]), do=pin(dO[:1]), a=pin(amap))
+        f32 = dict(dtype=torch.float32, device=dev)
+        din = [{k_: torch.empty_like(v_, device=dev) for k_, v_ in hin.items()} for _ in range(2)]
+        dout = [dict(O=torch.empty(1, w.N, D, **f32), lse=torch.empty(1, w.N, **f32),
+                     dQ=torch.empty(1, w.N, D, **f32), dK=torch.empty(1, w.N, D, **f32),
+                     dV=torch.empty(1, w.N, D, **f32)) for _ in range(2)]
+        hout = [{k_: torch.empty(tuple(v_.shape), dtype=v_.dtype).pin_memory() for k_, v_ in dout[0].items()}
+                for _ in range(2)]
+        h2d = sum(x.numel() * x.element_size() for x in hin.values())
+        d2h = sum(x.numel() * x.element_size() for x in hout[0].values())
+        main, cs = torch.cuda.current_stream(), torch.cuda.Stream()
+        up = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        down = [torch.cuda.Event() for _ in range(2)]
+
+        def upload(b):
+            with torch.cuda.stream(cs):
+                for k_, v_ in hin.items():
+                    din[b][k_].copy_(v_, non_blocking=True)
+                up[b].record(cs)
+
         barrier()
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        x0.record()
-        for _ in range(a.e2e_steps):
-            bufs["q"].copy_(hq, non_blocking=True)
-            bufs["k"].copy_(hk, non_blocking=True)
-            bufs["v"].copy_(hv, non_blocking=True)
-            bufs["do"].copy_(hdo, non_blocking=True)
-            bufs["a"].copy_(ha, non_blocking=True)
-            pl = _lib.plan(bufs["q"], bufs["k"], bufs["v"], bufs["a"], params, workspace=ws)
-            pl.attn_fwd(O, lse)
-            pl.attn_bwd(bufs["do"], O, lse, dQ, dK, dV)
-            for hbuf, dbuf in zip(outs, (O, dQ, dK, dV)):
-                hbuf.copy_(dbuf, non_blocking=True)
-            hlse.copy_(lse, non_blocking=True)
-        x1.record()
+        x0.record(main)
+        cs.wait_event(x0)
+        upload(0)
+        for i in range(a.e2e_steps):
+            b = i & 1
+            main.wait_event(up[b])
+            if i >= 2:
+                main.wait_event(down[b])          # step i - 2's results have been read back
+            d, o = din[b], dout[b]
+            pl = _lib.plan(d["q"], d["k"], d["v"], d["a"], params, workspace=ws)
+            pl.attn_fwd(o["O"], o["lse"])
+            pl.attn_bwd(d["do"], o["O"], o["lse"], o["dQ"], o["dK"], o["dV"])
+            done[b].record(main)
+            if i + 1 < a.e2e_steps:
+                if i >= 1:
+                    cs.wait_event(done[b ^ 1])    # step i - 1 has finished with that input set
+                upload(b ^ 1)
+            with torch.cuda.stream(cs):
+                cs.wait_event(done[b])
+                for k_, v_ in o.items():
+                    hout[b][k_].copy_(v_, non_blocking=True)
+                down[b].record(cs)
+        main.wait_stream(cs)
+        x1.record(main)
         barrier()
+        st = pl.status()
+        if st:
+            raise RuntimeError(f"device status (end to end): {_lib.status_string(st)}")
         te = max_over_ranks(x0.elapsed_time(x1), world, dev)
         e2e = {"value": te / (a.e2e_steps * world), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "copies": "side stream, two device buffer sets: uploads and downloads overlap the kernels"}
+        del din, dout, hout, hin
     # --------------------------------------------------- CPU oracle baseline
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
