@@ -151,20 +151,32 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def measured_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture
-    (profiles/dram_traffic_grid72x88x160.md), or None if the kernel's sources
-    changed since (their hash no longer matches) or there is no capture."""
+KERNEL_TU = {"k_bwd_dkdv": "prism_attn_bwd.cu", "k_attn_fwd": "prism_attn_fwd.cu",
+             "k_av_norm": "prism_av_norm.cu"}
+
+
+def source_digest(kernel):
+    """First 16 hex digits of sha256 over the kernel's translation unit, then
+    csrc/prism_dev.cuh and csrc/prism_internal.h (None for an unknown kernel)."""
     import hashlib
-    tu = {"k_bwd_dkdv": "prism_attn_bwd.cu", "k_attn_fwd": "prism_attn_fwd.cu"}.get(kernel)
-    path = os.path.join(ROOT, "profiles", "dram_traffic_grid72x88x160.md")
-    if tu is None or not os.path.exists(path):
+    tu = KERNEL_TU.get(kernel)
+    if tu is None:
         return None
     m = hashlib.sha256()
     for f in (tu, "prism_dev.cuh", "prism_internal.h"):
         with open(os.path.join(ROOT, "dynamic_block_sparse_indicator_b200", "csrc", f), "rb") as fh:
             m.update(fh.read())
-    digest = m.hexdigest()[:16]
+    return m.hexdigest()[:16]
+
+
+def measured_traffic(kernel, path=None):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture
+    (profiles/dram_traffic_grid72x88x160.md), or None if the kernel's sources
+    changed since (their hash no longer matches) or there is no capture."""
+    path = path or os.path.join(ROOT, "profiles", "dram_traffic_grid72x88x160.md")
+    digest = source_digest(kernel)
+    if digest is None or not os.path.exists(path):
+        return None
     for line in open(path):
         cells = [c.strip() for c in line.strip().strip("|").split("|")]
         if len(cells) == 5 and cells[0] == kernel and cells[4] == digest:
@@ -385,7 +397,9 @@ def guidance_map_leg(w, M, pk, reps=5):
     ach = out["with_hhat_bf16"]["tflops"]
     out["roofline"] = {"kernel": "k_av_norm", "bound": "tensor", "achieved": ach, "peak": burst,
                        "unit": "TFLOP/s", "frac": ach / burst,
-                       "peak_source": "measured burst bf16 (timed alone)" if pk else "fallback"}
+                       "peak_source": "measured burst bf16 (timed alone)" if pk else "fallback",
+                       "traffic": measured_traffic("k_av_norm")
+                       if (w.N, M, heads, D) == (1013760, 1000, 40, 128) else None}
     del Qv, Ka, Va, amap, hh
     torch.cuda.empty_cache()
     return out
