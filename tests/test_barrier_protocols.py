@@ -1,5 +1,8 @@
 """Models of the attention kernels' mbarrier protocols, checked on the host.
 
+Covered: the forward (k_attn_fwd), the backward (k_bwd_dkdv, with and without
+the fused dQ drain) and the guidance-map producer (k_av_norm).
+
 Each kernel role (TMA producer lanes, MMA issuers, softmax groups) is written
 as the sequence of its barrier operations, in the order and with the phase
 parities the kernel source uses: ('wait', barrier, k) waits for the k-th
@@ -176,6 +179,65 @@ def test_guidance_map_protocol(heads, MT, rescale):
     roles, softmax = av_roles(heads, MT)
     for seed in range(60 if heads < 40 else 8):
         assert run(roles + [softmax(rescale)], {}, seed) is None, (heads, MT, seed)
+
+
+# ------------------------------------------------------------- backward
+def backward_roles(U, fuse=True, ST=3):
+    """k_bwd_dkdv: 64-query units of a key tile, a 3-stage Q/dO ring, S^T/dP^T
+    double-buffered in TMEM; issuer A (S^T, dP^T), issuer B (dV, dQ^T, dK),
+    softmax (P'^T into TMEM, dS^T into shared memory), dQ^T drain (fuse)."""
+    def producer():
+        yield ("arrive", "kv")
+        for u in range(U):
+            s = u % ST
+            if u >= ST:
+                yield ("wait", f"st_empty{s}", u // ST - 1)
+            yield ("arrive", f"st_full{s}")
+
+    def issuer_a():
+        yield ("wait", "kv", 0)
+        for u in range(U):
+            b = u & 1
+            yield ("wait", f"st_full{u % ST}", u // ST)
+            if u >= 2:
+                yield ("wait", f"p_full{b}", (u - 2) >> 1)
+                yield ("wait", f"dq_free{b}" if fuse else f"pd_done{b}", (u - 2) >> 1)
+            yield ("arrive", f"s_full{b}")
+
+    def issuer_b():
+        for u in range(U):
+            b = u & 1
+            yield ("wait", f"p_full{b}", u >> 1)
+            if fuse:
+                yield ("arrive", f"dq_full{b}")
+            yield ("arrive", f"pd_done{b}")
+            yield ("arrive", f"st_empty{u % ST}")
+        yield ("arrive", "acc_done")
+
+    def softmax():
+        for u in range(U):
+            b = u & 1
+            yield ("wait", f"s_full{b}", u >> 1)
+            yield ("wait", f"st_full{u % ST}", u // ST)
+            if u >= 2:
+                yield ("wait", f"pd_done{b}", (u - 2) >> 1)
+            yield ("arrive", f"p_full{b}")
+        yield ("wait", "acc_done", 0)
+
+    def drain():
+        for u in range(U):
+            b = u & 1
+            yield ("wait", f"dq_full{b}", u >> 1)
+            yield ("arrive", f"dq_free{b}")
+
+    return [producer, issuer_a, issuer_b, softmax] + ([drain] if fuse else [])
+
+
+@pytest.mark.parametrize("U", list(range(1, 10)) + [33, 100])
+@pytest.mark.parametrize("fuse", [True, False])
+def test_backward_protocol(U, fuse):
+    for seed in range(150):
+        assert run(backward_roles(U, fuse), {}, seed) is None, (U, fuse, seed)
 
 
 def test_model_catches_a_wrong_parity():
