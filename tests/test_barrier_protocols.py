@@ -1,7 +1,8 @@
 """Models of the attention kernels' mbarrier protocols, checked on the host.
 
 Covered: the forward (k_attn_fwd), the backward (k_bwd_dkdv, with and without
-the fused dQ drain) and the guidance-map producer (k_av_norm).
+the fused dQ drain; k_bwd_dq for head_dim 64) and the guidance-map producer
+(k_av_norm).
 
 Each kernel role (TMA producer lanes, MMA issuers, softmax groups) is written
 as the sequence of its barrier operations, in the order and with the phase
@@ -238,6 +239,50 @@ def backward_roles(U, fuse=True, ST=3):
 def test_backward_protocol(U, fuse):
     for seed in range(150):
         assert run(backward_roles(U, fuse), {}, seed) is None, (U, fuse, seed)
+
+
+def dq_roles(U, ST=2):
+    """k_bwd_dq (head_dim 64): one 128-query tile, 64-key units; one issuer
+    (S and dP of unit u, then dQ += dS K of unit u - 1), the softmax forms dS."""
+    def producer():
+        yield ("arrive", "q")
+        for u in range(U):
+            if u >= ST:
+                yield ("wait", f"st_empty{u % ST}", u // ST - 1)
+            yield ("arrive", f"st_full{u % ST}")
+
+    def issuer():
+        yield ("wait", "q", 0)
+        for u in range(U + 1):
+            if u < U:
+                yield ("wait", f"st_full{u % ST}", u // ST)
+                if u >= 2:
+                    yield ("wait", f"s_free{u & 1}", (u - 2) >> 1)
+                yield ("arrive", f"s_full{u & 1}")
+            if u >= 1:
+                uu = u - 1
+                yield ("wait", f"ds_full{uu & 1}", uu >> 1)
+                yield ("arrive", f"dq_done{uu & 1}")
+                yield ("arrive", f"st_empty{uu % ST}")
+
+    def softmax():
+        for u in range(U):
+            b = u & 1
+            yield ("wait", f"s_full{b}", u >> 1)
+            yield ("arrive", f"s_free{b}")
+            if u >= 2:
+                yield ("wait", f"dq_done{b}", (u - 2) >> 1)
+            yield ("arrive", f"ds_full{b}")
+        if U:
+            yield ("wait", f"dq_done{(U - 1) & 1}", (U - 1) >> 1)
+
+    return [producer, issuer, softmax]
+
+
+@pytest.mark.parametrize("U", list(range(0, 9)) + [40])
+def test_dq_protocol(U):
+    for seed in range(150):
+        assert run(dq_roles(U), {}, seed) is None, (U, seed)
 
 
 def test_model_catches_a_wrong_parity():
