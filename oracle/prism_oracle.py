@@ -43,10 +43,14 @@ notes of the repository):
 
 Parity status: the candidate set, the closed form l*, the snapping, the
 directional statistics, the selection rule and the attention (forward and
-backward) are pinned by the tests in tests/test_oracle_pins.py.  The rho
-formula and the a_bar / v_hat normalisations are readings; their code is
-pinned to hand-built fields and to a per-token brute force, the readings
-themselves are not pinned by the pages ("parity unpinned" for the reading).
+backward) are pinned by the tests in tests/test_oracle_pins.py; the block-score
+softmax (hand-worked values, torch float64), the tie margins (written-out
+candidate distances, constructed threshold ties) and closed forms of the
+statistics on hand-built fields by tests/test_oracle_selection_pins.py, with
+planted mistakes that each of those checks catches.  The rho formula and the
+a_bar / v_hat normalisations are readings: their code is pinned to closed
+forms and to a per-token brute force, the readings themselves are not fixed by
+the pages ("parity unpinned" for the reading).
 """
 from __future__ import annotations
 
@@ -199,6 +203,12 @@ def snap_margin(ell64, vol):
     return ds[1] - ds[0] if len(ds) > 1 else np.inf
 
 
+def rho_margin_of(rho64, tau128, tau256):
+    """Float64 distance of the density to the nearer volume threshold (tie margin)."""
+    rho64 = np.asarray(rho64, dtype=np.float64)
+    return np.minimum(np.abs(rho64 - tau128), np.abs(rho64 - tau256))
+
+
 SHAPE_DYNAMIC, SHAPE_ISOTROPIC, SHAPE_FIXED = 0, 1, 2
 
 
@@ -231,7 +241,7 @@ def zone_shapes(V, a, T, H, W, eps, tau128=0.5, tau256=0.25, alpha=0.5, shape_mo
     sid = np.array([snap(ell[m], B[m]) for m in range(len(B))], dtype=np.int64)
     lg = np.log2(g64)
     ell64 = -alpha * lg + (np.log2(B) + alpha * lg.sum(axis=1))[:, None] / 3.0
-    rho_margin = np.minimum(np.abs(rho64 - tau128), np.abs(rho64 - tau256))
+    rho_margin = rho_margin_of(rho64, tau128, tau256)
     smargin = np.array([snap_margin(ell64[m], B[m]) for m in range(len(B))])
     if shape_mode == SHAPE_ISOTROPIC:
         smargin = np.full(len(B), np.inf)      # the tie rule decides exactly
