@@ -422,34 +422,88 @@ def attention_bwd(Q, K, V, dO, src, starts, sel):
     return dQ, dK, dV
 
 
-def attention_rows(Q, K, V, src, starts, sel, rows, dO=None):
-    """Forward (and dQ when dO is given) for selected raster query rows only.
+def block_selection_matrix(sel, nb):
+    """Boolean [nb, nb]: entry (i, j) is True when key block j is in S_i."""
+    bsel = np.zeros((nb, nb), dtype=bool)
+    for i, js in enumerate(sel):
+        bsel[i, js] = True
+    return bsel
 
-    Returns O [len(rows), D], LSE [len(rows)] and optionally dQ [len(rows), D].
+
+def attention_rows(Q, K, V, src, starts, sel, rows, dO=None, chunk=64):
+    """Forward (and dQ when dO is given) for selected raster query rows only,
+    from the masked definition: row q attends to every key n whose block is in
+    S_block(q), with a softmax over exactly those keys.
+
+    Rows are taken `chunk` at a time against all N keys (masked logits are
+    -inf), so no key is gathered.  Returns O [len(rows), D], LSE [len(rows)]
+    and optionally dQ [len(rows), D] (float64).
     """
     Q, K, V = (np.asarray(x, np.float64) for x in (Q, K, V))
     D = Q.shape[1]
     sc = 1.0 / np.sqrt(D)
+    rows = np.asarray(rows, dtype=np.int64)
     bt = block_of_token(src, starts)
+    bsel = block_selection_matrix(sel, len(starts) - 1)
     O = np.empty((len(rows), D))
     lse = np.empty(len(rows))
     dQ = np.empty((len(rows), D)) if dO is not None else None
-    for r, q in enumerate(rows):
-        js = sel[bt[q]]
-        keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in js])
-        s = K[keys] @ Q[q] * sc
-        m = s.max()
+    for r0 in range(0, len(rows), chunk):
+        rr = rows[r0:r0 + chunk]
+        mask = bsel[bt[rr]][:, bt]                                 # [r, N]
+        s = np.where(mask, Q[rr] @ K.T * sc, -np.inf)
+        m = s.max(axis=1, keepdims=True)
         e = np.exp(s - m)
-        z = e.sum()
+        z = e.sum(axis=1, keepdims=True)
         P = e / z
-        O[r] = P @ V[keys]
-        lse[r] = m + np.log(z)
+        O[r0:r0 + len(rr)] = P @ V
+        lse[r0:r0 + len(rr)] = (m + np.log(z))[:, 0]
         if dO is not None:
-            g = np.asarray(dO[q], np.float64)
-            dP = V[keys] @ g
-            Di = g @ O[r]
-            dQ[r] = (P * (dP - Di)) @ K[keys] * sc
+            g = np.asarray(dO[rr], np.float64)
+            dP = g @ V.T
+            Di = (g * O[r0:r0 + len(rr)]).sum(axis=1, keepdims=True)
+            dQ[r0:r0 + len(rr)] = (P * (dP - Di)) @ K * sc
     return O, lse, dQ
+
+
+def attention_key_rows(Q, K, V, dO, src, starts, sel, key_rows):
+    """dK and dV [len(key_rows), D] (float64) of selected raster key rows.
+
+    Key n receives, from every query row q whose block selects block(n), the
+    terms P[q, n] dO_q (dV) and P[q, n] (dP[q, n] - D_q) Q_q / sqrt(D) (dK),
+    where P[q, .] is q's softmax over all keys of its selection (its full LSE),
+    dP[q, n] = dO_q . V_n and D_q = dO_q . O_q.  The query blocks that select
+    a sampled key's block are evaluated whole, one at a time (practical when
+    the selections are short).
+    """
+    Q, K, V, dO = (np.asarray(x, np.float64) for x in (Q, K, V, dO))
+    D = Q.shape[1]
+    sc = 1.0 / np.sqrt(D)
+    key_rows = np.asarray(key_rows, dtype=np.int64)
+    bt = block_of_token(src, starts)
+    nb = len(starts) - 1
+    bsel = block_selection_matrix(sel, nb)
+    dK = np.zeros((len(key_rows), D))
+    dV = np.zeros((len(key_rows), D))
+    kblk = bt[key_rows]
+    users = np.nonzero(bsel[:, np.unique(kblk)].any(axis=1))[0]   # query blocks that select any of them
+    for i in users:
+        qi = src[starts[i]:starts[i + 1]]
+        keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in sel[i]])
+        s = Q[qi] @ K[keys].T * sc
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        P = e / e.sum(axis=1, keepdims=True)                      # [|B_i|, |keys|]
+        Oi = P @ V[keys]
+        g = dO[qi]
+        Di = (g * Oi).sum(axis=1)
+        col = {int(n): c for c, n in enumerate(keys)}
+        for r in np.nonzero(bsel[i, kblk])[0]:
+            n = int(key_rows[r])
+            p = P[:, col[n]]
+            dV[r] += p @ g
+            dK[r] += (p * (g @ V[n] - Di)) @ Q[qi] * sc
+    return dK, dV
 
 
 # ---------------------------------------------------------------------------

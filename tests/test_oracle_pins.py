@@ -394,3 +394,28 @@ def test_tiny_workload_plan_properties():
         assert np.argmax(st["g"][m]) == 0
         b = po.SHAPES[st["shape_id"][m]]
         assert b[0] <= b[1] and b[0] <= b[2]
+
+
+@pytest.mark.parametrize("seed,k,p", [(0, 3, 0.5), (1, 1, 0.0), (2, 2, 0.9)])
+def test_key_rows_match_torch_autograd(seed, k, p):
+    """attention_key_rows gives torch's float64 autograd dK, dV of the masked
+    attention at every key row; attention_rows its O, LSE and dQ rows."""
+    Q, K, V, pl, D = _tiny_plan(seed, k, p)
+    mask = po.token_mask(pl["src"], pl["starts"], pl["sel"])
+    q, kk, v, m = _torch_masked(Q, K, V, mask)
+    for t in (q, kk, v):
+        t.requires_grad_(True)
+    out = torch.nn.functional.scaled_dot_product_attention(q[None, None], kk[None, None],
+                                                           v[None, None], attn_mask=m)[0, 0]
+    dO = np.random.default_rng(40 + seed).normal(size=Q.shape)
+    out.backward(torch.tensor(dO))
+    keys = np.arange(Q.shape[0])
+    dKr, dVr = po.attention_key_rows(Q, K, V, dO, pl["src"], pl["starts"], pl["sel"], keys)
+    np.testing.assert_allclose(dKr, kk.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(dVr, v.grad.numpy(), atol=1e-10)
+    rows = np.random.default_rng(seed).choice(Q.shape[0], 100, replace=False)
+    Or, lr, dQr = po.attention_rows(Q, K, V, pl["src"], pl["starts"], pl["sel"], rows, dO=dO, chunk=32)
+    np.testing.assert_allclose(Or, out.detach().numpy()[rows], atol=1e-10)
+    np.testing.assert_allclose(dQr, q.grad.numpy()[rows], atol=1e-10)
+    s = (q @ kk.T / np.sqrt(D)).masked_fill(~m, float("-inf"))
+    np.testing.assert_allclose(lr, torch.logsumexp(s, 1).detach().numpy()[rows], atol=1e-10)
