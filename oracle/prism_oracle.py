@@ -387,11 +387,14 @@ def attention_fwd(Q, K, V, src, starts, sel):
     for i, js in enumerate(sel):
         qi = src[starts[i]:starts[i + 1]]
         keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in js])
-        s = Q[qi] @ K[keys].T / np.sqrt(D)
+        s = Q[qi] @ K[keys].T
+        s /= np.sqrt(D)                                  # logits
         m = s.max(axis=1, keepdims=True)
-        e = np.exp(s - m)
-        z = e.sum(axis=1, keepdims=True)
-        O[qi] = (e / z) @ V[keys]
+        s -= m
+        np.exp(s, out=s)                                 # exp(logit - row max)
+        z = s.sum(axis=1, keepdims=True)
+        s /= z                                           # softmax over the row's keys
+        O[qi] = s @ V[keys]
         lse[qi] = (m + np.log(z))[:, 0]
     return O, lse
 
@@ -403,13 +406,17 @@ def block_grads(Q, K, V, dO, O, lse, src, starts, sel, i, dQ, dK, dV):
     sc = 1.0 / np.sqrt(D)
     qi = src[starts[i]:starts[i + 1]]
     keys = np.concatenate([src[starts[j]:starts[j + 1]] for j in sel[i]])
-    P = np.exp(Q[qi] @ K[keys].T * sc - lse[qi][:, None])
-    dV[keys] += P.T @ dO[qi]
-    dP = dO[qi] @ V[keys].T
-    Di = (dO[qi] * O[qi]).sum(axis=1, keepdims=True)
-    dS = P * (dP - Di)
-    dQ[qi] = dS @ K[keys] * sc
-    dK[keys] += dS.T @ Q[qi] * sc
+    Kk, Vk, Qi, g = K[keys], V[keys], Q[qi], dO[qi]
+    P = Qi @ Kk.T
+    P *= sc
+    P -= lse[qi][:, None]
+    np.exp(P, out=P)                                     # P = exp(S / sqrt(D) - LSE)
+    dV[keys] += P.T @ g
+    dS = g @ Vk.T                                        # dP
+    dS -= (g * O[qi]).sum(axis=1, keepdims=True)         # dP - D_i
+    dS *= P                                              # dS = P o (dP - D)
+    dQ[qi] = dS @ Kk * sc
+    dK[keys] += dS.T @ Qi * sc
 
 
 def attention_bwd(Q, K, V, dO, src, starts, sel):
