@@ -117,45 +117,11 @@ __device__ __forceinline__ float max64(const uint32_t* sr) {
     return fmax3f(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
 }
 
-// Pairs of P (out of every 8 pairs of a row's keys) whose 2^x runs on the FMA
-// pipe instead of the MUFU unit (16 ex2 per SM per clock take as long as the
-// tile's two products at head_dim 128).  Measured on B200 at the 1M-token head:
-// 0 of 8 -> 550 ms, 2 -> 630 ms, 3 -> 650 ms (the emulation's dependent chain
-// costs more than the MUFU time it frees), so the default is 0.
-#ifndef PRISM_FWD_EMU
-#define PRISM_FWD_EMU 0
-#endif
-constexpr int kFwdEmuPer8 = PRISM_FWD_EMU;
-
 __device__ __forceinline__ void add2f(float& d0, float& d1, float a0, float a1, float b0, float b1) {
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
         "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
-// 2^x for two lanes on the FMA pipe: x = n + f, n = round(x) (adding 1.5 * 2^23
-// leaves n in the low mantissa bits), 2^f on [-1/2, 1/2] by a degree-4
-// polynomial, minimax in relative error (coefficients fitted by Lawson-weighted
-// least squares; max relative error 2.7e-6 evaluated in fp32, well below the
-// 2^-11 rounding of the fp16 P it feeds), 2^n added into the exponent field.  x
-// is clamped at -126 so that field never underflows.
-__device__ __forceinline__ void exp2_poly4(float& y0, float& y1, float x0, float x1) {
-    constexpr float kRound = 12582912.f;   // 1.5 * 2^23
-    constexpr float c0 = 0.99999928f, c1 = 0.69312179f, c2 = 0.24024744f, c3 = 0.055917863f,
-                    c4 = 0.0095700966f;
-    x0 = fmaxf(x0, -126.f);
-    x1 = fmaxf(x1, -126.f);
-    float t0, t1, n0, n1, f0, f1, p0, p1;
-    add2f(t0, t1, x0, x1, kRound, kRound);
-    add2f(n0, n1, t0, t1, -kRound, -kRound);
-    add2f(f0, f1, x0, x1, -n0, -n1);
-    ffma2(p0, p1, c4, c4, f0, f1, c3, c3);
-    ffma2(p0, p1, p0, p1, f0, f1, c2, c2);
-    ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
-    ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // P' = 2^(s * scale_log2 + neg) for one row's 64 keys as 32 packed fp16 pairs
@@ -170,12 +136,8 @@ __device__ __forceinline__ float exp_p64(const uint32_t* sr, bool valid, float s
             float x0, x1;
             ffma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), scale_log2, scale_log2, neg,
                   neg);
-            if ((e & 7) >= 8 - kFwdEmuPer8) {
-                exp2_poly4(p0, p1, x0, x1);
-            } else {
-                p0 = ex2(x0);
-                p1 = ex2(x1);
-            }
+            p0 = ex2(x0);
+            p1 = ex2(x1);
         }
         add2f(l2[0], l2[1], l2[0], l2[1], p0, p1);
         pk[e] = pack_f16(p0, p1);

@@ -52,17 +52,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
            "r"(x), "r"(y), "r"(z) : "memory");
 }
 
-// Pairs of P (out of every 8 pairs of a row's 64 keys) whose 2^x runs on the
-// FMA pipe instead of the MUFU unit.  16 MUFU ex2 per SM per clock take as long
-// as the tile's products (128 x 128 keys x 2 products of K = 128), but measured
-// on B200 the softmax here is latency-bound rather than MUFU-bound and every
-// split tried (2, 3, 4 of 8) ran slower (24.4 - 25.2 ms against 23.7 ms at the
-// 2K layer), so the default keeps every exponential on the MUFU unit.
-#ifndef PRISM_AV_EMU
-#define PRISM_AV_EMU 0
-#endif
-constexpr int kEmuPer8 = PRISM_AV_EMU;
-
 __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -74,31 +63,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
-}
-
-// 2^x for two lanes on the FMA pipe.  x = n + f with n = round(x): adding
-// 1.5 * 2^23 leaves n in the low mantissa bits (round to nearest), so f lies in
-// [-1/2, 1/2]; 2^f is a degree-3 polynomial, minimax in relative error on that
-// interval (coefficients fitted here by Lawson-weighted least squares: max
-// relative error 7.5e-5 evaluated in fp32, far below the 2^-9 rounding of the
-// bf16 P it feeds); 2^n is added into the exponent field (the low bits of the
-// rounded sum, shifted by 23, are n << 23 exactly).  x is clamped at -126 so
-// the exponent field never underflows.
-__device__ __forceinline__ void exp2_poly(float& y0, float& y1, float x0, float x1) {
-    constexpr float kRound = 12582912.f;   // 1.5 * 2^23
-    constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261114f, c3 = 0.055171628f;
-    x0 = fmaxf(x0, -126.f);
-    x1 = fmaxf(x1, -126.f);
-    float t0, t1, n0, n1, f0, f1;
-    add2(t0, t1, x0, x1, kRound, kRound);
-    add2(n0, n1, t0, t1, -kRound, -kRound);
-    add2(f0, f1, x0, x1, -n0, -n1);
-    float p0, p1;
-    ffma2(p0, p1, c3, c3, f0, f1, c2, c2);
-    ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
-    ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 accumulate.
@@ -369,13 +333,7 @@ k_av_norm(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                     float x0, x1;
                     ffma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), a.scale_log2,
                           a.scale_log2, neg, neg);
-                    float p0, p1;
-                    if ((e & 7) >= 8 - kEmuPer8) {
-                        exp2_poly(p0, p1, x0, x1);
-                    } else {
-                        p0 = ex2(x0);
-                        p1 = ex2(x1);
-                    }
+                    const float p0 = ex2(x0), p1 = ex2(x1);
                     const int q = (e & 1) * 2;
                     add2(l4[q], l4[q + 1], l4[q], l4[q + 1], p0, p1);
                     pk[e] = pack_bf16(p0, p1);

@@ -26,10 +26,12 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "prism_internal.h"
@@ -539,9 +541,11 @@ __global__ void __launch_bounds__(1024) k_zone_finalize(DevPlan d, ShapeRule rul
 }
 
 // ================================================================ stage 2
-// The block-ordered copies are fp16: bf16 values inside +-65504 convert
-// exactly, and fp16 operands keep the tensor-core products' rounding error 8x
-// below bf16's.  A value outside the fp16 range is a device-check error.
+// The block-ordered copies are fp16: a bf16 value converts exactly when
+// 2^-14 <= |x| <= 65504 (or x = 0), smaller magnitudes round to fp16's
+// subnormal grid (absolute error at most 2^-25), and fp16 operands keep the
+// tensor-core products' rounding error 8x below bf16's.  A value beyond the
+// fp16 range (or a NaN) is a device-check error.
 constexpr float kHalfMax = 65504.f;
 
 __device__ __forceinline__ uint32_t ph2(float a, float b) {
@@ -1388,15 +1392,18 @@ static void noalloc_stats(const Geom& g, const DevPlan& d, const void* V, cudaSt
 
 // Device address of the scratch array, looked up once per device (with that
 // device current) the first time the entry point runs on it.
+// The lookup runs once per device under a std::once_flag, so host threads
+// making their first calls on one device at the same time do not race on the
+// cache; a failed lookup leaves nullptr and the call reports PRISM_ERR_CUDA.
 static float* noalloc_scratch_ptr(int dev) {
-    static float* ptrs[64] = {};
+    static std::once_flag once[64];
+    static std::atomic<float*> ptrs[64];
     if (dev < 0 || dev >= 64) return nullptr;
-    if (!ptrs[dev]) {
+    std::call_once(once[dev], [dev] {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<float*>(p);
-    }
-    return ptrs[dev];
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess) ptrs[dev].store(static_cast<float*>(p));
+    });
+    return ptrs[dev].load();
 }
 
 }  // namespace prism

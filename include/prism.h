@@ -68,11 +68,16 @@ extern "C" {
  *   head_dim  D, 64 or 128.
  *   dtype     element type of Q, K, V: PRISM_BF16 or PRISM_F32.  fp32 inputs
  *             feed the statistics and the pooled means in fp32; attention runs
- *             on their bf16 rounding (round to nearest even).
+ *             on their fp16 rounding (round to nearest even).
  *   out_dtype element type of O, dO, dQ, dK, dV: PRISM_BF16 or PRISM_F32.
- *             The tensor-core products take fp16 operands (exact for bf16
- *             inputs inside +-65504) with fp32 accumulation either way; fp32
- *             outputs keep the fp32 accumulators unrounded.
+ *             The tensor-core products take fp16 operands with fp32
+ *             accumulation either way; fp32 outputs keep the fp32 accumulators
+ *             unrounded.  A bf16 input converts to fp16 exactly when
+ *             2^-14 <= |x| <= 65504 (or x = 0); smaller magnitudes round to
+ *             fp16's subnormal grid (absolute error at most 2^-25), and a value
+ *             beyond 65504 (or a NaN) makes the plan report
+ *             PRISM_ERR_DEVICE_CHECK.  dO is scaled per head by an exact power
+ *             of two before its conversion, so its magnitude does not matter.
  *   top_k     k of Top-k (>= 0); k >= number of blocks keeps every block.
  *   top_p     p of Top-p in [0, 1]; p >= 1 keeps every block, p <= 0 none.
  *             Empty sets (top_k < 1, top_k_frac <= 0 and top_p <= 0) are
@@ -139,7 +144,7 @@ PRISM_API size_t prism_plan_workspace_bytes(const prism_params* p);
  *   closed form l*_d = -1/2 log2 g_d + 1/3 (log2 B + 1/2 sum log2 g) snapped to
  *   the nearest of the 16 candidate shapes (alpha and shape_mode select the
  *   ablation variants).
- *   Stage 2: reorder tokens so every block is contiguous (bf16 copies of Q,
+ *   Stage 2: reorder tokens so every block is contiguous (fp16 copies of Q,
  *   K, V in block order, kept in the workspace).
  *   Stage 3 ("Metode" 3): block means Qbar, Kbar; P_i = softmax(Qbar_i Kbar^T
  *   / sqrt(D)); S_i = Top-k(P_i, k) U Top-p(P_i, p) as per-query-block CSR
@@ -176,8 +181,8 @@ PRISM_API int prism_plan_import(const prism_params* p, const void* Q, const void
 /*
  * prism_attn_fwd -- stages 4-5: for every query token q of block i,
  *   O_q = softmax_n(q . k_n / sqrt(D)) v_n over the tokens n of the key
- *   blocks in S_i (fp32 online softmax, bf16 tensor-core products), written
- *   back in raster order (inverse permutation).
+ *   blocks in S_i (fp32 online softmax, fp16 tensor-core products with fp32
+ *   accumulation), written back in raster order (inverse permutation).
  *   O    device [heads][N][head_dim] of `out_dtype`.
  *   lse  device fp32 [heads][N], log-sum-exp of the scaled logits, raster order.
  */

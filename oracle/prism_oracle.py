@@ -458,18 +458,22 @@ def attention_rows(Q, K, V, src, starts, sel, rows, dO=None, chunk=64):
     for r0 in range(0, len(rows), chunk):
         rr = rows[r0:r0 + chunk]
         mask = bsel[bt[rr]][:, bt]                                 # [r, N]
-        s = np.where(mask, Q[rr] @ K.T * sc, -np.inf)
-        m = s.max(axis=1, keepdims=True)
-        e = np.exp(s - m)
-        z = e.sum(axis=1, keepdims=True)
-        P = e / z
+        P = Q[rr] @ K.T
+        P *= sc
+        P[~mask] = -np.inf                                         # keys outside the selection
+        m = P.max(axis=1, keepdims=True)
+        P -= m
+        np.exp(P, out=P)
+        z = P.sum(axis=1, keepdims=True)
+        P /= z                                                     # softmax over the selected keys
         O[r0:r0 + len(rr)] = P @ V
         lse[r0:r0 + len(rr)] = (m + np.log(z))[:, 0]
         if dO is not None:
             g = np.asarray(dO[rr], np.float64)
-            dP = g @ V.T
-            Di = (g * O[r0:r0 + len(rr)]).sum(axis=1, keepdims=True)
-            dQ[r0:r0 + len(rr)] = (P * (dP - Di)) @ K * sc
+            dS = g @ V.T                                           # dP
+            dS -= (g * O[r0:r0 + len(rr)]).sum(axis=1, keepdims=True)
+            dS *= P                                                # P o (dP - D)
+            dQ[r0:r0 + len(rr)] = dS @ K * sc
     return O, lse, dQ
 
 

@@ -4,7 +4,8 @@ The 2K training layer (grid 72x88x160, 1,013,760 tokens, head_dim 128, bf16,
 Top-k 16, Top-p 0.9), one head planned at a time, fp32 outputs:
   * the plan (shapes, block offsets, permutation, every selected set) against
     the oracle's full plan of the head, with the near-tie rules;
-  * O, LSE and dQ on sampled query rows against the oracle row by row;
+  * O, LSE and dQ on 320 sampled query rows (64 query blocks spread over the
+    grid, the first and the last included) against the oracle;
   * dV and dK through identities that hold at any size: the rows of dV sum to
     the rows of dO (each row's softmax weights sum to one) and the rows of dK
     sum to zero (each query row's dS sums to zero).  The identities are checked
@@ -39,17 +40,23 @@ def run(cuda_device):
     host = lambda t: t[0].double().cpu().numpy()
     q, k, v, g = host(Q), host(K), host(V), host(dO)
     orc = po.plan_head(q, k, v, a.cpu().numpy(), w.T, w.H, w.W, w.top_k, w.top_p, w.eps)
-    return dict(w=w, pl=pl, q=q, k=k, v=v, g=g, orc=orc, O=host(O), lse=lse[0].double().cpu().numpy(),
+    return dict(w=w, pl=pl, q=q, k=k, v=v, g=g, a=a.cpu().numpy(), orc=orc, O=host(O),
+                lse=lse[0].double().cpu().numpy(),
                 dQ=host(dQ), dK=host(dK), dV=host(dV))
 
 
 def test_fullsize_plan(run):
     w, pl, o = run["w"], run["pl"], run["orc"]
     NB, WORDS = w.N // 64, (w.N // 64 + 31) // 32
-    ok, tie, bad = parity.shapes_agree(pl.export("shape_id"), o["stats"])
+    gsid = pl.export("shape_id")
+    ok, tie, bad = parity.shapes_agree(gsid, o["stats"])
     assert not bad
     if tie:
-        pytest.skip(f"accepted near-tie shapes in zones {tie}: downstream stages differ legitimately")
+        # shapes differ only at near-ties: the downstream stages are compared
+        # against the oracle run on the GPU's accepted shapes
+        o = po.plan_head(run["q"], run["k"], run["v"], run["a"], w.T, w.H, w.W, w.top_k, w.top_p, w.eps,
+                         shape_id=gsid)
+        run["orc"] = o
     nb = len(o["starts"]) - 1
     assert pl.export("nblocks")[0] == nb
     np.testing.assert_array_equal(pl.export("blk_start")[:nb + 1], o["starts"])
@@ -70,9 +77,12 @@ def test_fullsize_sampled_rows(run):
         pytest.skip("plan comparison did not run")
     nb = len(o["starts"]) - 1
     rng = np.random.default_rng(3)
-    blocks = [i for i in rng.permutation(nb) if np.array_equal(gsets[i], o["sel"][i])][:6]
-    rows = np.array([o["src"][o["starts"][i] + int(rng.integers(o["starts"][i + 1] - o["starts"][i]))]
-                     for i in blocks])
+    exact = [i for i in range(nb) if np.array_equal(gsets[i], o["sel"][i])]
+    blocks = set(rng.choice(exact, 62, replace=False).tolist())
+    blocks |= {exact[0], exact[-1]}                      # the first and the last query block
+    # 5 rows per block: 320 rows spread over the query tiles
+    rows = np.concatenate([rng.choice(o["src"][o["starts"][i]:o["starts"][i + 1]], 5, replace=False)
+                           for i in sorted(blocks)])
     Oo, lo, dQo = po.attention_rows(run["q"], run["k"], run["v"], o["src"], o["starts"], o["sel"], rows,
                                     dO=run["g"])
     for got, want, nm in ((run["O"][rows], Oo, "O"), (run["dQ"][rows], dQo, "dQ")):
