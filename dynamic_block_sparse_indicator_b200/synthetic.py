@@ -30,6 +30,9 @@ above (seed id 5); the audio keys and values Ka, Va [heads, M, D] are, per head
 and channel, white N(0,1) noise over the M audio tokens smoothed by a 1-D
 Gaussian (sigma 3 tokens, radius 9, replicate padding), divided by its std,
 plus N(0, 0.3^2) (seed ids 6 and 7).
+Shot cuts (optional, `shot_cuts`): from each listed frame on, the recipe's field
+is replaced by a fresh draw (a new shot); local cuts (`local_cuts`, (zt, zh, zw,
+local frame)): the same inside one zone from a local frame on.
 The audio norm map is 0.05 everywhere, raised to a Gaussian blob
 0.05 + 0.95 exp(-|x - c|^2 / (2 * 3^2)) around the centre c of every localised
 zone (blobs combine by max).  dO is N(0,1).  Seeds: workload id x 1000 +
@@ -61,6 +64,8 @@ class Workload:
     uniform_frac: float = 0.0
     qk_scale: float = 1.0
     fixed_zones: list = field(default_factory=list)  # explicit (zt, zh, zw, axis)
+    shot_cuts: list = field(default_factory=list)    # global frames where a new shot starts
+    local_cuts: list = field(default_factory=list)   # (zt, zh, zw, local frame): a zone changes content
 
     @property
     def N(self) -> int:
@@ -137,8 +142,8 @@ def _blur_axis(x: torch.Tensor, dim: int, taps: torch.Tensor) -> torch.Tensor:
     return y.reshape(shp).movedim(-1, dim)
 
 
-def _field_one_head(w: Workload, g: torch.Generator, loc, uniform_tok, device) -> torch.Tensor:
-    """One head of one tensor: [N, D] float32 in raster token order."""
+def _base_field(w: Workload, g: torch.Generator, uniform_tok, device) -> torch.Tensor:
+    """Smoothed unit-std field plus noise (near-uniform zones damped): [D, T, H, W]."""
     D, T, H, W = w.head_dim, w.T, w.H, w.W
     sigma, radius = 3.0, 9
     k = torch.arange(-radius, radius + 1, dtype=torch.float32, device=device)
@@ -151,9 +156,25 @@ def _field_one_head(w: Workload, g: torch.Generator, loc, uniform_tok, device) -
     noise = torch.randn(D, T, H, W, generator=g, device=device)
     if uniform_tok is not None:
         u = uniform_tok.view(1, T, H, W)
-        x = torch.where(u, x * 0.1, x) + torch.where(u, noise * 0.03, noise * 0.3)
-    else:
-        x = x + 0.3 * noise
+        return torch.where(u, x * 0.1, x) + torch.where(u, noise * 0.03, noise * 0.3)
+    return x + 0.3 * noise
+
+
+def _field_one_head(w: Workload, g: torch.Generator, loc, uniform_tok, device) -> torch.Tensor:
+    """One head of one tensor: [N, D] float32 in raster token order.
+
+    Shot cuts: from each cut frame on, every frame is a fresh draw of the base
+    field (a new shot).  Local cuts: inside one zone, from a local frame on, the
+    tokens are a fresh draw (content that changes abruptly in one region, as in
+    a fast zoom)."""
+    D, T, H, W = w.head_dim, w.T, w.H, w.W
+    x = _base_field(w, g, uniform_tok, device)
+    for c in sorted(w.shot_cuts):
+        x[:, c:] = _base_field(w, g, uniform_tok, device)[:, c:]
+    for (zt, zh, zw, tl) in w.local_cuts:
+        y = _base_field(w, g, uniform_tok, device)
+        sl = (slice(None), slice(8 * zt + tl, 8 * zt + 8), slice(8 * zh, 8 * zh + 8), slice(8 * zw, 8 * zw + 8))
+        x[sl] = y[sl]
     for (zt, zh, zw, ax) in loc:
         comp = torch.randn(D, 8, generator=g, device=device)
         sl = (slice(None), slice(8 * zt, 8 * zt + 8), slice(8 * zh, 8 * zh + 8),

@@ -82,8 +82,16 @@ def candidate_shapes():
 SHAPES = candidate_shapes()
 
 
-def shapes_of_volume(vol):
-    return [(i, s) for i, s in enumerate(SHAPES) if s[0] * s[1] * s[2] == vol]
+def shapes_of_volume(vol, L=Z):
+    """Candidates of volume vol whose time edge b_T divides a region of L frames
+    (every candidate for a whole 8-frame zone)."""
+    return [(i, s) for i, s in enumerate(SHAPES) if s[0] * s[1] * s[2] == vol and L % s[0] == 0]
+
+
+def max_volume(L):
+    """Largest candidate volume that tiles a region of L frames (256 for 8 and 4
+    frames, 128 for 2 and 6: those take b_T = 2 only)."""
+    return max(s[0] * s[1] * s[2] for s in SHAPES if L % s[0] == 0)
 
 
 # ---------------------------------------------------------------------------
@@ -183,10 +191,11 @@ def ideal_log_edges(g32, vol, alpha=0.5):
     return (-a * lg + (inner / F32(3.0))[..., None]).astype(F32)
 
 
-def snap(ell32, vol):
-    """Shape id of the candidate of volume vol nearest (squared log2 distance) to l*."""
+def snap(ell32, vol, L=Z):
+    """Shape id of the candidate of volume vol nearest (squared log2 distance) to l*
+    (among those that tile a region of L frames)."""
     best, best_d = -1, None
-    for sid, s in shapes_of_volume(int(vol)):
+    for sid, s in shapes_of_volume(int(vol), L):
         e = np.log2(np.asarray(s, dtype=F32))
         d = (e - ell32).astype(F32)
         dist = F32(d[0] * d[0]) + F32(d[1] * d[1])
@@ -196,10 +205,10 @@ def snap(ell32, vol):
     return best
 
 
-def snap_margin(ell64, vol):
+def snap_margin(ell64, vol, L=Z):
     """Float64 gap between the two smallest snap distances (tie margin)."""
     ds = sorted(float(np.sum((np.log2(np.asarray(s, float)) - ell64) ** 2))
-                for _, s in shapes_of_volume(int(vol)))
+                for _, s in shapes_of_volume(int(vol), L))
     return ds[1] - ds[0] if len(ds) > 1 else np.inf
 
 
@@ -213,16 +222,19 @@ SHAPE_DYNAMIC, SHAPE_ISOTROPIC, SHAPE_FIXED = 0, 1, 2
 
 
 def zone_shapes(V, a, T, H, W, eps, tau128=0.5, tau256=0.25, alpha=0.5, shape_mode=SHAPE_DYNAMIC,
-                fixed_shape=0):
+                fixed_shape=0, cut_ratio=0.0):
     """Stage one for one head: V [N, D] raster, a [T,H,W] or None.
 
     Returns dict with shape_id [Nz], B [Nz], g [Nz,3] (float32), rho [Nz]
     (float32) and the float64 decision margins rho_margin, snap_margin.
     Variants (Table 10's ablation): alpha is the mapping exponent; the
     isotropic mode takes g_d equal on the three axes (B still from rho); the
-    fixed mode gives every zone candidate fixed_shape.
+    fixed mode gives every zone candidate fixed_shape.  cut_ratio > 0 turns on
+    the adaptive temporal boundaries (zone_shapes_cut); 0 keeps every zone whole.
     """
     Vz = zones_of(np.asarray(V, dtype=np.float64), T, H, W)
+    if cut_ratio > 0:
+        return zone_shapes_cut(Vz, a, T, H, W, eps, tau128, tau256, alpha, shape_mode, cut_ratio)
     r = ratio(directional_variance(Vz))
     if a is None:
         abar = np.zeros(Vz.shape[0])
@@ -250,43 +262,171 @@ def zone_shapes(V, a, T, H, W, eps, tau128=0.5, tau256=0.25, alpha=0.5, shape_mo
         B = np.full(len(B), int(np.prod(SHAPES[int(fixed_shape)])), dtype=np.int64)
         rho_margin = np.full(len(B), np.inf)
         smargin = np.full(len(B), np.inf)
+    nz = len(B)
     return dict(shape_id=sid, B=B, g=g32, rho=rho32, r=r, abar=abar, vhat=vhat,
-                ell=ell, rho_margin=rho_margin, snap_margin=smargin)
+                ell=ell, rho_margin=rho_margin, snap_margin=smargin,
+                cut=np.zeros(nz, np.int64), shape_id2=np.full(nz, -1, np.int64), cut_margin=np.full(nz, np.inf))
+
+
+# ---------------------------------------------------------------------------
+# Adaptive temporal zone boundaries.  Page paper.rainbus.top, section
+# "独立分析的弱点" item (1) and section "未来方向" (the authors' first
+# direction): a macro-zone with a fixed 8-frame window that spans a shot cut or
+# a fast zoom mixes unrelated content under one block shape; detect the cut from
+# frame differences and split the zone there (page xyznot.com/th, limitations,
+# names the same failure mode).  Reading (the pages give no formula):
+#   * per zone and head, the frame-difference energy e_t = mean over the zone's
+#     64 tokens and D channels of (V[t+1] - V[t])^2, t = 0..6;
+#   * a cut follows the largest e_t* (lowest t on ties) when e_t* exceeds
+#     cut_ratio times the median of the seven energies (float32 decision);
+#   * the boundary t* + 1 snaps to the nearest of {2, 4, 6} (3 and 5 to 4): the
+#     time edges of the candidate blocks are 2, 4 or 8, so a part must hold an
+#     even number of frames;
+#   * each part (frames [0, c) and [c, 8)) is a region planned like a zone:
+#     its own directional variances (the T profile has the part's length),
+#     density (its frames and frame differences) and audio terms; rho and a_bar
+#     are normalised by their maxima over the head's regions; the volume is
+#     capped at the largest that tiles the part (128 for 2 or 6 frames) and the
+#     shape is the nearest candidate whose b_T divides the part's length.
+# ---------------------------------------------------------------------------
+CUT_SNAP = {1: 2, 2: 2, 3: 4, 4: 4, 5: 4, 6: 6, 7: 6}
+
+
+def frame_diff_energy(Vz):
+    """e_t = mean over the zone's 64 tokens and D channels of (V[t+1] - V[t])^2: [Nz, 7] float64."""
+    Vz = np.asarray(Vz, dtype=np.float64)
+    d = Vz[:, 1:] - Vz[:, :-1]
+    return (d * d).mean(axis=(2, 3, 4))
+
+
+def zone_cuts(e, cut_ratio):
+    """Split position per zone (0 = whole zone, else 2, 4 or 6) and a relative
+    float64 margin of the decision (distance of e_t* to the threshold and to
+    the runner-up energy; infinite for a zone without frame changes)."""
+    e = np.asarray(e, dtype=np.float64)
+    e32 = e.astype(F32)
+    cut = np.zeros(e.shape[0], np.int64)
+    margin = np.full(e.shape[0], np.inf)
+    for m in range(e.shape[0]):
+        t = int(np.argmax(e32[m]))
+        med = np.sort(e32[m])[3]
+        if e32[m, t] > F32(F32(cut_ratio) * med):
+            cut[m] = CUT_SNAP[t + 1]
+        srt = np.sort(e[m])
+        if srt[-1] > 0:
+            margin[m] = min(abs(srt[-1] - cut_ratio * srt[3]), srt[-1] - srt[-2]) / srt[-1]
+    return cut, margin
+
+
+def zone_regions(cut):
+    """[(zone, t0, t1)] in zone order, parts in time order."""
+    out = []
+    for m, c in enumerate(cut):
+        out += [(m, 0, Z)] if c == 0 else [(m, 0, int(c)), (m, int(c), Z)]
+    return out
+
+
+def region_audio(az, regions):
+    """Audio terms of each region: zone-style mean and directional slice variances."""
+    araw, vhat = np.empty(len(regions)), np.zeros((len(regions), 3))
+    for k, (m, t0, t1) in enumerate(regions):
+        x = az[m, t0:t1]                                        # [L, 8, 8]
+        mean = x.mean()
+        sig = np.array([((x.mean(axis=p) - mean) ** 2).mean() for p in ((1, 2), (0, 2), (0, 1))])
+        araw[k] = mean
+        if sig.sum() > 0:
+            vhat[k] = sig / sig.sum()
+    return araw, vhat
+
+
+def zone_shapes_cut(Vz, a, T, H, W, eps, tau128, tau256, alpha, shape_mode, cut_ratio):
+    """Stage one with adaptive temporal boundaries (see the reading above)."""
+    e = frame_diff_energy(Vz)
+    cut, cut_margin = zone_cuts(e, cut_ratio)
+    regions = zone_regions(cut)
+    sig = np.stack([directional_variance(Vz[m:m + 1, t0:t1])[0] for m, t0, t1 in regions])
+    rraw = np.array([density_raw(Vz[m:m + 1, t0:t1])[0] for m, t0, t1 in regions])
+    r = ratio(sig)
+    if a is None:
+        abar, vhat = np.zeros(len(regions)), np.zeros((len(regions), 3))
+    else:
+        a64 = np.asarray(a, dtype=np.float32).astype(np.float64)
+        araw, vhat = region_audio(zones_of(a64.reshape(-1, 1), T, H, W)[..., 0], regions)
+        abar = normalise_by_max(araw)
+    g32 = (r.astype(F32) + abar.astype(F32)[:, None] * vhat.astype(F32) + F32(eps)).astype(F32)
+    g64 = r + abar[:, None] * vhat + eps
+    if shape_mode == SHAPE_ISOTROPIC:
+        g32, g64 = np.ones_like(g32), np.ones_like(g64)
+    rho64 = normalise_by_max(rraw)
+    rho32 = rho64.astype(F32)
+    L = np.array([t1 - t0 for _, t0, t1 in regions])
+    B = np.minimum(volume(rho32, tau128, tau256), [max_volume(x) for x in L])
+    ell = ideal_log_edges(g32, B.astype(F32), alpha)
+    rsid = np.array([snap(ell[k], B[k], L[k]) for k in range(len(regions))], dtype=np.int64)
+    lg = np.log2(g64)
+    ell64 = -alpha * lg + (np.log2(B) + alpha * lg.sum(axis=1))[:, None] / 3.0
+    rmargin = rho_margin_of(rho64, tau128, tau256)
+    smargin = np.array([snap_margin(ell64[k], B[k], L[k]) for k in range(len(regions))])
+    if shape_mode == SHAPE_ISOTROPIC:
+        smargin = np.full(len(regions), np.inf)
+    nz = Vz.shape[0]
+    sid, sid2 = np.zeros(nz, np.int64), np.full(nz, -1, np.int64)
+    zr, zs = np.full(nz, np.inf), np.full(nz, np.inf)
+    for k, (m, t0, _t1) in enumerate(regions):
+        if t0 == 0:
+            sid[m] = rsid[k]
+        else:
+            sid2[m] = rsid[k]
+        zr[m] = min(zr[m], rmargin[k])
+        zs[m] = min(zs[m], smargin[k])
+    return dict(shape_id=sid, shape_id2=sid2, cut=cut, cut_margin=cut_margin, energy=e,
+                rho_margin=zr, snap_margin=zs, regions=regions, region_shape=rsid, region_B=B,
+                region_rho=rho32, region_g=g32, region_r=r, region_abar=abar, region_vhat=vhat,
+                region_L=L)
 
 
 # ---------------------------------------------------------------------------
 # Stage 2: token reorder (Algorithm 1 stage two)
 # ---------------------------------------------------------------------------
-def _local_order(shape):
-    """Zone-local raster indices (lt*64 + lh*8 + lw) in block-contiguous order."""
+def _local_order(shape, t0=0, L=Z):
+    """Zone-local raster indices (lt*64 + lh*8 + lw) of frames [t0, t0 + L) in
+    block-contiguous order."""
     bt, bh, bw = shape
     out = []
-    for kt in range(Z // bt):
+    for kt in range(L // bt):
         for kh in range(Z // bh):
             for kw in range(Z // bw):
                 for lt in range(bt):
                     for lh in range(bh):
                         for lw in range(bw):
-                            out.append(((kt * bt + lt) * Z + kh * bh + lh) * Z + kw * bw + lw)
+                            out.append(((t0 + kt * bt + lt) * Z + kh * bh + lh) * Z + kw * bw + lw)
     return np.array(out, dtype=np.int64)
 
 
 _LOCAL = [_local_order(s) for s in SHAPES]
 
 
-def partition(shape_id, T, H, W):
-    """src [N] (raster token of each permuted position) and block starts [N_b + 1]."""
+def partition(shape_id, T, H, W, cut=None, shape_id2=None):
+    """src [N] (raster token of each permuted position) and block starts [N_b + 1].
+
+    With cuts, zone m's frames [0, c) take shape_id[m] and frames [c, 8)
+    shape_id2[m]; the first part's blocks come first."""
     zh_n, zw_n = H // Z, W // Z
     src = np.empty(T * H * W, dtype=np.int64)
     starts = [0]
     for m, sid in enumerate(shape_id):
         zt, rem = divmod(m, zh_n * zw_n)
         zh, zw = divmod(rem, zw_n)
-        loc = _LOCAL[int(sid)]
-        lt, lh, lw = loc // 64, (loc // 8) % 8, loc % 8
-        src[512 * m: 512 * (m + 1)] = ((zt * Z + lt) * H + zh * Z + lh) * W + zw * Z + lw
-        vol = int(np.prod(SHAPES[int(sid)]))
-        starts.extend(512 * m + vol * (k + 1) for k in range(512 // vol))
+        c = 0 if cut is None else int(cut[m])
+        parts = [(0, Z, int(sid))] if c == 0 else [(0, c, int(sid)), (c, Z, int(shape_id2[m]))]
+        pos = 512 * m
+        for t0, t1, s in parts:
+            loc = _LOCAL[s] if t1 - t0 == Z else _local_order(SHAPES[s], t0, t1 - t0)
+            lt, lh, lw = loc // 64, (loc // 8) % 8, loc % 8
+            src[pos: pos + len(loc)] = ((zt * Z + lt) * H + zh * Z + lh) * W + zw * Z + lw
+            vol = int(np.prod(SHAPES[s]))
+            starts.extend(pos + vol * (k + 1) for k in range(len(loc) // vol))
+            pos += len(loc)
     return src, np.array(starts, dtype=np.int64)
 
 
@@ -345,15 +485,18 @@ def select(Qbar, Kbar, k, p, k_frac=0.0):
 # Whole plan for one head
 # ---------------------------------------------------------------------------
 def plan_head(Q, K, V, a, T, H, W, k, p, eps, tau128=0.5, tau256=0.25, shape_id=None, alpha=0.5,
-              shape_mode=SHAPE_DYNAMIC, fixed_shape=0, k_frac=0.0):
-    """Stages one to three for one head.  Q, K, V: [N, D] raster."""
-    st = zone_shapes(V, a, T, H, W, eps, tau128, tau256, alpha, shape_mode, fixed_shape)
+              shape_mode=SHAPE_DYNAMIC, fixed_shape=0, k_frac=0.0, cut_ratio=0.0, cut=None, shape_id2=None):
+    """Stages one to three for one head.  Q, K, V: [N, D] raster.  shape_id (and,
+    with adaptive boundaries, cut and shape_id2) replace stage one's result."""
+    st = zone_shapes(V, a, T, H, W, eps, tau128, tau256, alpha, shape_mode, fixed_shape, cut_ratio)
     sid = st["shape_id"] if shape_id is None else np.asarray(shape_id)
-    src, starts = partition(sid, T, H, W)
+    cut = st["cut"] if cut is None else np.asarray(cut)
+    sid2 = st["shape_id2"] if shape_id2 is None else np.asarray(shape_id2)
+    src, starts = partition(sid, T, H, W, cut, sid2)
     Qbar, Kbar = pool(Q, src, starts), pool(K, src, starts)
     sel, s, P = select(Qbar, Kbar, k, p, k_frac)
-    return dict(stats=st, shape_id=sid, src=src, starts=starts, Qbar=Qbar, Kbar=Kbar,
-                sel=sel, logits=s, P=P)
+    return dict(stats=st, shape_id=sid, cut=cut, shape_id2=sid2, src=src, starts=starts, Qbar=Qbar,
+                Kbar=Kbar, sel=sel, logits=s, P=P)
 
 
 def block_of_token(src, starts):

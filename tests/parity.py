@@ -6,13 +6,21 @@ where |rho - tau| or the gap between the two nearest candidates is below
 1e-5; a selected set may differ only in blocks whose logit lies within 1e-5
 of the boundary block's logit, and its size only as far as moving p by 1e-5
 moves the Top-p prefix.  Attention outputs and gradients from bf16 inputs
-must reach relative L2 <= 1e-2 and max-abs <= 3e-2 against the oracle.
+must reach relative L2 <= 1e-2 and max-abs <= 3e-2 against the oracle
+(gradients: max-abs 3e-2 plus half a bf16 ulp of the element, close_grad).
 """
 import numpy as np
 
 TIE = 1e-5
 REL_L2 = 1e-2
 MAX_ABS = 3e-2
+# Gradients: the max-abs bar holds at unit scale; an element of magnitude |g|
+# may in addition carry half an ulp of the pages' 16-bit operand format (bf16:
+# 2^-9 |g|).  The backward is linear in dO, so a purely absolute bar would
+# depend on the caller's scale of dO; the operating point's dK reaches 170 at
+# unit-variance dO, where one fp16 rounding of a dominant dS term (2^-12
+# relative) alone is 0.04.
+GRAD_RTOL = 2.0 ** -9
 
 
 def bits_to_sets(words, nb, nwords):
@@ -32,15 +40,24 @@ def sets_to_bits(sel, nb_max, nwords):
     return out
 
 
-def shapes_agree(gpu_sid, st):
-    """(exact matches, accepted near-tie mismatches, bad zones)."""
+def shapes_agree(gpu_sid, st, gpu_cut=None, gpu_sid2=None):
+    """(exact matches, accepted near-tie mismatches, bad zones).  With adaptive
+    temporal boundaries the split position and the second part's shape are
+    compared too; a split decision may differ only where the oracle's relative
+    cut margin is below the tie bound."""
     bad, tie = [], []
+    cut_m = st.get("cut_margin")
     for m, (g, o) in enumerate(zip(gpu_sid, st["shape_id"])):
-        if int(g) != int(o):
-            if st["rho_margin"][m] < TIE or st["snap_margin"][m] < TIE:
-                tie.append(m)
-            else:
-                bad.append(m)
+        same = int(g) == int(o)
+        if gpu_cut is not None:
+            same = same and int(gpu_cut[m]) == int(st["cut"][m])
+            if same and int(st["cut"][m]):
+                same = int(gpu_sid2[m]) == int(st["shape_id2"][m])
+        if not same:
+            near = st["rho_margin"][m] < TIE or st["snap_margin"][m] < TIE
+            if cut_m is not None and cut_m[m] < TIE:
+                near = True
+            (tie if near else bad).append(m)
     return len(gpu_sid) - len(bad) - len(tie), tie, bad
 
 
@@ -78,3 +95,16 @@ def close(a, b, rel=REL_L2, mabs=MAX_ABS):
     rl2 = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
     ma = float(np.max(np.abs(a - b))) if a.size else 0.0
     return rl2 <= rel and ma <= mabs, rl2, ma
+
+
+def close_grad(a, b, rel=REL_L2, mabs=MAX_ABS, rtol=GRAD_RTOL):
+    """Gradient comparison: relative L2 <= rel over the tensor and, per element,
+    |a - b| <= mabs + rtol |b|.  Returns (ok, relL2, max-abs, worst ratio of an
+    element's error to its bound)."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    rl2 = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
+    err = np.abs(a - b)
+    ma = float(err.max()) if a.size else 0.0
+    worst = float((err / (mabs + rtol * np.abs(b))).max()) if a.size else 0.0
+    return rl2 <= rel and worst <= 1.0, rl2, ma, worst

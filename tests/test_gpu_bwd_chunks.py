@@ -17,7 +17,8 @@ every key's set of attending queries is exactly the oracle's:
     sampled key rows (the first and the last key tile, and keys of 64-, 128- and
     256-token blocks spread over the grid) computed one by one by the oracle,
     O and dQ on sampled query rows.
-Tolerances: relative L2 <= 1e-2 and max-abs <= 3e-2 (tests/parity.py).
+Tolerances (tests/parity.py): relative L2 <= 1e-2 and max-abs <= 3e-2; for the
+gradients max-abs 3e-2 plus half a bf16 ulp of each element.
 """
 import numpy as np
 import pytest
@@ -59,6 +60,11 @@ def _assert_close(got, want, what):
     assert good, f"{what}: relL2 {rl2:.2e} maxabs {ma:.2e}"
 
 
+def _assert_grad(got, want, what):
+    good, rl2, ma, worst = parity.close_grad(got, want)
+    assert good, f"{what}: relL2 {rl2:.2e} maxabs {ma:.2e} (worst element at {worst:.2f} of its bound)"
+
+
 @pytest.mark.parametrize("case", ["p06_2chunks", "operating_point_3chunks"])
 def test_multichunk_backward_full(case, cuda_device):
     if case == "p06_2chunks":
@@ -75,7 +81,7 @@ def test_multichunk_backward_full(case, cuda_device):
     np.testing.assert_allclose(r["lse"], lo, atol=2e-2, rtol=1e-3)
     ref = po.attention_bwd(r["q"], r["k"], r["v"], r["g"], o["src"], o["starts"], o["sel"])
     for got, want, nm in zip((r["dQ"], r["dK"], r["dV"]), ref, ("dQ", "dK", "dV")):
-        _assert_close(got, want, f"{case} {nm}")
+        _assert_grad(got, want, f"{case} {nm}")
         # per-key rows: no key tile's rows land elsewhere or cancel
         rows = np.linalg.norm(got - want, axis=1) / np.maximum(np.linalg.norm(want, axis=1), 1e-3)
         assert np.quantile(rows, 0.999) < 0.05, f"{case} {nm}: worst rows {np.sort(rows)[-5:]}"
@@ -115,10 +121,10 @@ def test_fullsize_backward_sampled_key_rows(wid, k, cuda_device):
     vols = np.diff(o["starts"])[po.block_of_token(o["src"], o["starts"])[keys]]
     assert {64, 128, 256} & set(vols.tolist())
     dKo, dVo = po.attention_key_rows(r["q"], r["k"], r["v"], r["g"], o["src"], o["starts"], o["sel"], keys)
-    _assert_close(r["dK"][keys], dKo, f"workload {wid} dK key rows")
-    _assert_close(r["dV"][keys], dVo, f"workload {wid} dV key rows")
+    _assert_grad(r["dK"][keys], dKo, f"workload {wid} dK key rows")
+    _assert_grad(r["dV"][keys], dVo, f"workload {wid} dV key rows")
     rows = _sample_query_rows(o, rng)
     Oo, lo, dQo = po.attention_rows(r["q"], r["k"], r["v"], o["src"], o["starts"], o["sel"], rows, dO=r["g"])
     _assert_close(r["O"][rows], Oo, f"workload {wid} O rows")
-    _assert_close(r["dQ"][rows], dQo, f"workload {wid} dQ rows")
+    _assert_grad(r["dQ"][rows], dQo, f"workload {wid} dQ rows")
     np.testing.assert_allclose(r["lse"][rows], lo, atol=2e-2, rtol=1e-3)

@@ -209,8 +209,8 @@ def test_imported_oracle_plan_backward(name, cuda_device):
         qa, ka, va = _attn_inputs(w, Q, K, V, h)
         ref = po.attention_bwd(qa, ka, va, dO[h].double().numpy(), o["src"], o["starts"], o["sel"])
         for got, want, nm in zip((dQ, dK, dV), ref, ("dQ", "dK", "dV")):
-            good, rl2, ma = parity.close(got[h].double().cpu().numpy(), want)
-            assert good, f"{name} head {h} {nm}: relL2 {rl2:.2e} maxabs {ma:.2e}"
+            good, rl2, ma, worst = parity.close_grad(got[h].double().cpu().numpy(), want)
+            assert good, f"{name} head {h} {nm}: relL2 {rl2:.2e} maxabs {ma:.2e} worst {worst:.2f}"
 
 
 def test_full_pipeline_backward_tiny(cuda_device):
@@ -238,8 +238,8 @@ def test_full_pipeline_backward_tiny(cuda_device):
             assert good, f"head {h} O vs {what} inputs: relL2 {rl2:.2e} maxabs {ma:.2e}"
             ref = po.attention_bwd(*inputs, dO[h].double().numpy(), o["src"], o["starts"], o["sel"])
             for got, want, nm in zip((dQ, dK, dV), ref, ("dQ", "dK", "dV")):
-                good, rl2, ma = parity.close(got[h].double().cpu().numpy(), want)
-                assert good, f"head {h} {nm} vs {what} inputs: relL2 {rl2:.2e} maxabs {ma:.2e}"
+                good, rl2, ma, worst = parity.close_grad(got[h].double().cpu().numpy(), want)
+                assert good, f"head {h} {nm} vs {what} inputs: relL2 {rl2:.2e} maxabs {ma:.2e} worst {worst:.2f}"
 
 
 def test_tiny_magnitude_values_follow_the_fp16_bound(cuda_device):

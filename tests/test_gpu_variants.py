@@ -105,7 +105,7 @@ def test_operating_point_backward(cuda_device):
         ref = po.attention_bwd(*_attn_inputs(W, Q, K, V, h), dO[h].double().numpy(), o["src"],
                                o["starts"], o["sel"])
         for got, want, nm in zip((dQ, dK, dV), ref, ("dQ", "dK", "dV")):
-            good, rl2, ma = parity.close(got[h].double().cpu().numpy(), want)
-            assert good, f"head {h} {nm}: relL2 {rl2:.2e} maxabs {ma:.2e}"
+            good, rl2, ma, worst = parity.close_grad(got[h].double().cpu().numpy(), want)
+            assert good, f"head {h} {nm}: relL2 {rl2:.2e} maxabs {ma:.2e} worst {worst:.2f}"
         compared += 1
     assert compared >= 1, "no head whose whole selection matched the oracle"

@@ -35,3 +35,13 @@ def test_selection_mismatch_needs_a_near_tie():
     s2 = s[0].copy()
     s2[order[3]] = s2[order[2]]
     assert parity.selection_agrees(np.sort(np.r_[order[:2], order[3]]), s2, P[0], 3, 0.0)
+
+
+def test_gradient_rule_adds_half_a_bf16_ulp_per_element():
+    ref = np.array([0.5, 170.0, -80.0])
+    # 0.04 off on the element of 170: inside 3e-2 + 170 / 512
+    assert parity.close_grad(ref + [0.0, 0.04, 0.0], ref)[0]
+    # 0.04 off on the element of 0.5: outside 3e-2 + 0.5 / 512
+    assert not parity.close_grad(ref + [0.04, 0.0, 0.0], ref)[0]
+    # a relative error of 2^-8 (a whole bf16 ulp) on the large element fails
+    assert not parity.close_grad(ref * [1, 1 + 2.0 ** -8, 1] + [0, 0.03, 0], ref)[0]
