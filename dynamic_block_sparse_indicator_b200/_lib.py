@@ -31,6 +31,8 @@ ITEMS = {
     "sel_bits": (3, np.uint32), "row_ptr": (4, np.int32), "col_idx": (5, np.int32),
     "col_ptr": (6, np.int32), "row_idx": (7, np.int32), "qbar": (8, np.float32),
     "kbar": (9, np.float32), "src": (10, np.int32), "zone_stats": (11, np.float32),
+    "zone_cut": (12, np.uint8), "shape_id2": (13, np.uint8), "zone_energy": (14, np.float32),
+    "region_stats": (15, np.float32),
 }
 
 
@@ -45,7 +47,7 @@ class PrismParams(C.Structure):
                 ("top_k", C.c_int32),
                 ("top_p", C.c_float), ("eps", C.c_float), ("tau128", C.c_float),
                 ("tau256", C.c_float), ("alpha", C.c_float), ("shape_mode", C.c_int32),
-                ("fixed_shape", C.c_int32), ("top_k_frac", C.c_float)]
+                ("fixed_shape", C.c_int32), ("top_k_frac", C.c_float), ("cut_ratio", C.c_float)]
 
 
 class PrismError(RuntimeError):
@@ -73,6 +75,7 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_plan_workspace_bytes": (sz, [pp]),
         "prism_plan": (i32, [pp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import": (i32, [pp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
+        "prism_plan_import_cuts": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_attn_fwd": (i32, [vp, vp, vp, vp]),
         "prism_attn_bwd": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
         "prism_plan_item_bytes": (sz, [vp, i32]),
@@ -111,10 +114,10 @@ def status_string(st: int) -> str:
 
 def make_params(T, H, W, heads, head_dim, dtype, top_k, top_p, eps, tau128=0.5, tau256=0.25,
                 out_dtype=PRISM_F32, alpha=0.5, shape_mode=PRISM_SHAPE_DYNAMIC, fixed_shape=0,
-                top_k_frac=0.0):
+                top_k_frac=0.0, cut_ratio=0.0):
     return PrismParams(T, H, W, heads, head_dim, dtype, out_dtype, top_k, float(top_p),
                        float(eps), float(tau128), float(tau256), float(alpha), int(shape_mode),
-                       int(fixed_shape), float(top_k_frac))
+                       int(fixed_shape), float(top_k_frac), float(cut_ratio))
 
 
 def workspace_bytes(params: PrismParams) -> int:
@@ -260,8 +263,11 @@ def plan(Q, K, V, a_map, params: PrismParams, workspace=None, stream=None) -> Pl
     return Plan(params, h, workspace, (Q, K, V, a_map))
 
 
-def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None, stream=None) -> Plan:
-    """A plan from given shape ids [heads, Nz] (uint8) and selection bitmap (int32/uint32 words)."""
+def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None, stream=None,
+                zone_cut=None, shape_id2=None) -> Plan:
+    """A plan from given shape ids [heads, Nz] (uint8) and selection bitmap (int32/uint32 words);
+    with adaptive temporal boundaries also the split frames zone_cut and the second parts'
+    shapes shape_id2 ([heads, Nz] uint8 each)."""
     import torch
     lib = load()
     _check_inputs(Q, K, V, params)
@@ -269,12 +275,17 @@ def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
     h = C.c_void_p()
-    st = lib.prism_plan_import(C.byref(params), _ptr(Q), _ptr(K), _ptr(V), _ptr(shape_id),
-                               _ptr(sel_bits), _ptr(workspace), workspace.numel(), _stream(stream),
-                               C.byref(h))
+    if zone_cut is None:
+        st = lib.prism_plan_import(C.byref(params), _ptr(Q), _ptr(K), _ptr(V), _ptr(shape_id),
+                                   _ptr(sel_bits), _ptr(workspace), workspace.numel(), _stream(stream),
+                                   C.byref(h))
+    else:
+        st = lib.prism_plan_import_cuts(C.byref(params), _ptr(Q), _ptr(K), _ptr(V), _ptr(shape_id),
+                                        _ptr(zone_cut), _ptr(shape_id2), _ptr(sel_bits), _ptr(workspace),
+                                        workspace.numel(), _stream(stream), C.byref(h))
     if st:
         raise PrismError(st, "prism_plan_import")
-    return Plan(params, h, workspace, (Q, K, V, shape_id, sel_bits))
+    return Plan(params, h, workspace, (Q, K, V, shape_id, sel_bits, zone_cut, shape_id2))
 
 
 def av_norm(Qv, Ka, Va, a_map=None, h_hat=None, hhat_dtype=None, want_hhat=False, status=None,

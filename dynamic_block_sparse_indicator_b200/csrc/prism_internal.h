@@ -29,7 +29,13 @@ struct Layout {
     size_t araw;                        // double[Nz]  zone mean of the audio map
     size_t abar, vhat;                  // float[Nz], float[Nz][3]
     size_t zstat;                       // float[heads][Nz][4]
-    size_t shape_id;                    // uint8[heads][Nz]
+    size_t shape_id;                    // uint8[heads][Nz]   (first part's shape when split)
+    size_t zdiff;                       // float[heads][Nz][7] frame-difference energies
+    size_t zcut;                        // uint8[heads][Nz]   split frame: 0, 2, 4, 6
+    size_t shape_id2;                   // uint8[heads][Nz]   second part's shape (255: none)
+    size_t rstat;                       // float[heads][Nz][2][4] statistics of the parts
+    size_t araw_seg;                    // double[Nz][3][2]   audio means of the six possible parts
+    size_t vhat_seg;                    // float[Nz][3][2][3] their v_hat
     size_t zone_off;                    // int32[heads][Nz + 1]  first block of each zone
     size_t nblocks;                     // int32[heads]
     size_t blk_start;                   // int32[heads][NB + 1]
@@ -63,6 +69,7 @@ struct prism_plan_s {
     size_t ws_bytes;
     int device;
     int has_audio;
+    int has_cuts;             // adaptive temporal boundaries in force (computed or imported)
     CUtensorMap tm_q, tm_k, tm_v, tm_do;       // 2D [heads*N, D] fp16, 128-row boxes, 128B swizzle
     CUtensorMap tm_q64, tm_k64, tm_v64, tm_do64;  // the same with 64-row boxes
     CUtensorMap tm_dq;                            // fp32 dQ accumulator, 32-row boxes, no swizzle

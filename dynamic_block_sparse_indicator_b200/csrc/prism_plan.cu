@@ -64,6 +64,12 @@ Layout make_layout(const Geom& g) {
     L.vhat = take(sizeof(float) * g.Nz * 3);
     L.zstat = take(sizeof(float) * H * g.Nz * 4);
     L.shape_id = take(H * g.Nz);
+    L.zdiff = take(sizeof(float) * H * g.Nz * 7);
+    L.zcut = take(H * g.Nz);
+    L.shape_id2 = take(H * g.Nz);
+    L.rstat = take(sizeof(float) * H * g.Nz * 8);
+    L.araw_seg = take(sizeof(double) * g.Nz * 6);
+    L.vhat_seg = take(sizeof(float) * g.Nz * 18);
     L.zone_off = take(sizeof(int) * H * (g.Nz + 1));
     L.nblocks = take(sizeof(int) * H);
     L.blk_start = take(sizeof(int) * H * (NB + 1));
@@ -112,6 +118,8 @@ int validate_params(const prism_params* p) {
     if (p->shape_mode == PRISM_SHAPE_FIXED && (p->fixed_shape < 0 || p->fixed_shape >= 16))
         return PRISM_ERR_INVALID_ARG;
     if (!(p->eps > 0.f) || !std::isfinite(p->eps)) return PRISM_ERR_INVALID_ARG;
+    if (!(p->cut_ratio >= 0.f) || !std::isfinite(p->cut_ratio)) return PRISM_ERR_INVALID_ARG;
+    if (p->cut_ratio > 0.f && p->shape_mode == PRISM_SHAPE_FIXED) return PRISM_ERR_INVALID_ARG;
     if (!(p->tau256 >= 0.f && p->tau128 >= p->tau256 && p->tau128 <= 1e30f))
         return PRISM_ERR_INVALID_ARG;
     const int64_t N = (int64_t)p->T * p->H * p->W;
@@ -141,6 +149,12 @@ struct DevPlan {
     float* vhat;
     float* zstat;
     uint8_t* shape_id;
+    float* zdiff;          // adaptive temporal boundaries (null when cut_ratio = 0)
+    uint8_t* zcut;
+    uint8_t* shape_id2;
+    float* rstat;
+    double* araw_seg;
+    float* vhat_seg;
     int* zone_off;
     int* nblocks;
     int* blk_start;
@@ -176,6 +190,14 @@ static DevPlan dev_plan(const prism_plan_s* P) {
     d.vhat = (float*)(b + L.vhat);
     d.zstat = (float*)(b + L.zstat);
     d.shape_id = (uint8_t*)(b + L.shape_id);
+    if (P->has_cuts) {
+        d.zdiff = (float*)(b + L.zdiff);
+        d.zcut = (uint8_t*)(b + L.zcut);
+        d.shape_id2 = (uint8_t*)(b + L.shape_id2);
+        d.rstat = (float*)(b + L.rstat);
+        d.araw_seg = (double*)(b + L.araw_seg);
+        d.vhat_seg = (float*)(b + L.vhat_seg);
+    }
     d.zone_off = (int*)(b + L.zone_off);
     d.nblocks = (int*)(b + L.nblocks);
     d.blk_start = (int*)(b + L.blk_start);
@@ -307,6 +329,46 @@ __global__ void __launch_bounds__(256) k_audio_zone(DevPlan d, const float* __re
     }
 }
 
+// Audio terms of the six parts a split can make (frames [0, c) and [c, 8) for
+// c = 2, 4, 6), head independent: the zone reading applied to each part (mean
+// of the map over the part; slice means along T (c or 8 - c slices), H and W
+// (8 each); their variances around the part's mean; v_hat = variance / sum).
+__global__ void __launch_bounds__(256) k_audio_seg(DevPlan d, const float* __restrict__ amap) {
+    const int m = blockIdx.x;
+    const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
+    __shared__ double v[512];
+    for (int i = threadIdx.x; i < 512; i += 256) {
+        const int lt = i >> 6, lh = (i >> 3) & 7, lw = i & 7;
+        const int64_t n = ((int64_t)(8 * zt + lt) * d.H + 8 * zh + lh) * d.W + 8 * zw + lw;
+        v[i] = (double)amap[n];
+    }
+    __syncthreads();
+    if (threadIdx.x < 6) {
+        const int ci = threadIdx.x >> 1, part = threadIdx.x & 1, c = 2 * (ci + 1);
+        const int t0 = part ? c : 0, t1 = part ? 8 : c, L = t1 - t0;
+        double st[8], sh[8], sw[8], tot = 0.0;
+        for (int i = 0; i < 8; ++i) st[i] = sh[i] = sw[i] = 0.0;
+        for (int lt = t0; lt < t1; ++lt)
+            for (int lh = 0; lh < 8; ++lh)
+                for (int lw = 0; lw < 8; ++lw) {
+                    const double x = v[(lt << 6) | (lh << 3) | lw];
+                    st[lt - t0] += x; sh[lh] += x; sw[lw] += x; tot += x;
+                }
+        const double mean = tot / (64.0 * L);
+        double sig[3] = {0.0, 0.0, 0.0};
+        for (int i = 0; i < L; ++i) { const double e = st[i] / 64.0 - mean; sig[0] += e * e; }
+        for (int i = 0; i < 8; ++i) {
+            const double eh = sh[i] / (8.0 * L) - mean, ew = sw[i] / (8.0 * L) - mean;
+            sig[1] += eh * eh; sig[2] += ew * ew;
+        }
+        sig[0] /= L; sig[1] /= 8.0; sig[2] /= 8.0;
+        const double s3 = sig[0] + sig[1] + sig[2];
+        const int k = m * 6 + threadIdx.x;
+        d.araw_seg[k] = mean;
+        for (int ax = 0; ax < 3; ++ax) d.vhat_seg[k * 3 + ax] = s3 > 0.0 ? (float)(sig[ax] / s3) : 0.f;
+    }
+}
+
 __global__ void __launch_bounds__(1024) k_audio_norm(DevPlan d) {
     __shared__ double red[32];
     double mx = 0.0;
@@ -346,31 +408,49 @@ struct Pair<float> {
     }
 };
 
-template <typename T, int D>
-__global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restrict__ V) {
+// MODE 0: statistics of whole zones.  MODE 1: the same, plus the zone's
+// frame-difference energies e_t = mean over its 64 tokens and D channels of
+// (V[t+1] - V[t])^2 and its split decision (adaptive temporal boundaries).
+// MODE 2: statistics of the two parts of every split zone (grid z = part),
+// over the part's frames [t0, t1) only.
+template <typename T, int D, int MODE>
+__global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restrict__ V, float cut_ratio) {
     constexpr int CP = D / 2;            // channel pairs
     constexpr int G = 256 / CP;          // groups
     constexpr int RPG = 8 / G;           // h-rows per group
-    constexpr int NV = 26;               // ST[8] SQ[8] SW[8] Dsum Dsq
+    constexpr int NE = MODE == 1 ? 7 : 0;
+    constexpr int NV = 26 + NE;          // ST[8] SQ[8] SW[8] Dsum Dsq (+ E[7])
     extern __shared__ float zs_dyn[];    // [G][D][NV]
     float (*red)[D][NV] = reinterpret_cast<float (*)[D][NV]>(zs_dyn);
     __shared__ float shs[D][8];
     __shared__ float cst[D][4];
+    __shared__ float cse[MODE == 1 ? D : 1][8];
+    __shared__ float ez[8];
     const int m = blockIdx.x, h = blockIdx.y;
+    int t0 = 0, t1 = 8;
+    if (MODE == 2) {
+        const int c = d.zcut[(size_t)h * d.Nz + m];
+        if (c == 0) return;
+        t0 = blockIdx.z ? c : 0;
+        t1 = blockIdx.z ? 8 : c;
+    }
+    const int L = t1 - t0;
     const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
     const int cp = threadIdx.x % CP, grp = threadIdx.x / CP;
     const T* Vh = V + (size_t)h * d.N * D;
     auto tok = [&](int lt, int lh, int lw) -> int64_t {
         return ((int64_t)(8 * zt + lt) * d.H + 8 * zh + lh) * d.W + 8 * zw + lw;
     };
-    const float2 ref = Pair<T>::load(Vh + tok(0, 0, 0) * D + 2 * cp);
-    float ST[2][8], SQ[2][8], SW[2][8], SH[2][RPG], Ds[2], Dq[2];
+    const float2 ref = Pair<T>::load(Vh + tok(t0, 0, 0) * D + 2 * cp);
+    float ST[2][8], SQ[2][8], SW[2][8], SH[2][RPG], Ds[2], Dq[2], Et[2][NE > 0 ? NE : 1];
     #pragma unroll
     for (int c = 0; c < 2; ++c) {
         #pragma unroll
         for (int i = 0; i < 8; ++i) ST[c][i] = SQ[c][i] = SW[c][i] = 0.f;
         #pragma unroll
         for (int i = 0; i < RPG; ++i) SH[c][i] = 0.f;
+        #pragma unroll
+        for (int i = 0; i < (NE > 0 ? NE : 1); ++i) Et[c][i] = 0.f;
         Ds[c] = Dq[c] = 0.f;
     }
     #pragma unroll
@@ -378,7 +458,10 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restri
         const int lh = grp * RPG + rr;
         float prev[2][8];
         #pragma unroll
+        for (int i = 0; i < 8; ++i) prev[0][i] = prev[1][i] = 0.f;
+        #pragma unroll
         for (int lt = 0; lt < 8; ++lt) {
+            if (MODE == 2 && (lt < t0 || lt >= t1)) continue;
             float2 x[8];
             #pragma unroll
             for (int lw = 0; lw < 8; ++lw) x[lw] = Pair<T>::load(Vh + tok(lt, lh, lw) * D + 2 * cp);
@@ -389,10 +472,11 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restri
                 SQ[0][lt] += v0 * v0; SQ[1][lt] += v1 * v1;
                 SW[0][lw] += v0; SW[1][lw] += v1;
                 SH[0][rr] += v0; SH[1][rr] += v1;
-                if (lt > 0) {
+                if (lt > t0) {
                     const float d0 = v0 - prev[0][lw], d1 = v1 - prev[1][lw];
                     Ds[0] += d0; Ds[1] += d1;
                     Dq[0] += d0 * d0; Dq[1] += d1 * d1;
+                    if (MODE == 1) { Et[0][(lt - 1) % 7] += d0 * d0; Et[1][(lt - 1) % 7] += d1 * d1; }
                 }
                 prev[0][lw] = v0; prev[1][lw] = v1;
             }
@@ -405,42 +489,87 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restri
         for (int i = 0; i < 8; ++i) { r[i] = ST[c][i]; r[8 + i] = SQ[c][i]; r[16 + i] = SW[c][i]; }
         r[24] = Ds[c]; r[25] = Dq[c];
         #pragma unroll
+        for (int i = 0; i < NE; ++i) r[26 + i] = Et[c][i];
+        #pragma unroll
         for (int rr = 0; rr < RPG; ++rr) shs[2 * cp + c][grp * RPG + rr] = SH[c][rr];
     }
     __syncthreads();
+    // per-part divisors: a whole zone (L = 8) divides by the same constants 64, 8, 448
+    const float n_plane = 8.f * (float)L, n_len = (float)L, n_diff = 64.f * (float)(L - 1);
     if (threadIdx.x < D) {
         const int c = threadIdx.x;
-        float st[8], sq[8], sw[8], ds = 0.f, dq = 0.f;
+        float st[8], sq[8], sw[8], ds = 0.f, dq = 0.f, et[NE > 0 ? NE : 1];
         #pragma unroll
         for (int i = 0; i < 8; ++i) st[i] = sq[i] = sw[i] = 0.f;
+        #pragma unroll
+        for (int i = 0; i < (NE > 0 ? NE : 1); ++i) et[i] = 0.f;
         for (int g = 0; g < G; ++g) {
             const float* r = red[g][c];
             #pragma unroll
             for (int i = 0; i < 8; ++i) { st[i] += r[i]; sq[i] += r[8 + i]; sw[i] += r[16 + i]; }
             ds += r[24]; dq += r[25];
+            #pragma unroll
+            for (int i = 0; i < NE; ++i) et[i] += r[26 + i];
         }
         float zsum = 0.f;
         #pragma unroll
         for (int i = 0; i < 8; ++i) zsum += st[i];
-        const float mu = zsum / 512.f;
+        const float mu = zsum / (64.f * n_len);
         float vt = 0.f, vh = 0.f, vw = 0.f, sp = 0.f;
         #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float et = st[i] / 64.f - mu, eh = shs[c][i] / 64.f - mu, ew = sw[i] / 64.f - mu;
-            vt += et * et; vh += eh * eh; vw += ew * ew;
-            const float fm = st[i] / 64.f;
-            sp += sq[i] / 64.f - fm * fm;
+            const float eh = shs[c][i] / n_plane - mu, ew = sw[i] / n_plane - mu;
+            vh += eh * eh; vw += ew * ew;
+            if (i >= t0 && i < t1) {
+                const float et_ = st[i] / 64.f - mu;
+                vt += et_ * et_;
+                const float fm = st[i] / 64.f;
+                sp += sq[i] / 64.f - fm * fm;
+            }
         }
-        const float dm = ds / 448.f;
-        const float temporal = dq / 448.f - dm * dm;
-        cst[c][0] = vt / 8.f; cst[c][1] = vh / 8.f; cst[c][2] = vw / 8.f;
-        cst[c][3] = sp / 8.f + temporal;
+        const float dm = ds / n_diff;
+        const float temporal = dq / n_diff - dm * dm;
+        cst[c][0] = vt / n_len; cst[c][1] = vh / 8.f; cst[c][2] = vw / 8.f;
+        cst[c][3] = sp / n_len + temporal;
+        #pragma unroll
+        for (int i = 0; i < NE; ++i) cse[c][i] = et[i];
     }
     __syncthreads();
     if (threadIdx.x < 4) {
         float s = 0.f;
         for (int c = 0; c < D; ++c) s += cst[c][threadIdx.x];
-        d.zstat[((size_t)h * d.Nz + m) * 4 + threadIdx.x] = s / (float)D;
+        if (MODE == 2)
+            d.rstat[(((size_t)h * d.Nz + m) * 2 + blockIdx.z) * 4 + threadIdx.x] = s / (float)D;
+        else
+            d.zstat[((size_t)h * d.Nz + m) * 4 + threadIdx.x] = s / (float)D;
+    }
+    if (MODE == 1) {
+        if (threadIdx.x >= 32 && threadIdx.x < 32 + 7) {
+            const int t = threadIdx.x - 32;
+            float s = 0.f;
+            for (int c = 0; c < D; ++c) s += cse[c][t];
+            const float e = s / (64.f * (float)D);
+            ez[t] = e;
+            d.zdiff[((size_t)h * d.Nz + m) * 7 + t] = e;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // largest energy (lowest t on ties) against cut_ratio x the median of the seven
+            int tm = 0;
+            float srt[7];
+            for (int t = 0; t < 7; ++t) {
+                srt[t] = ez[t];
+                if (ez[t] > ez[tm]) tm = t;
+            }
+            for (int i = 1; i < 7; ++i)
+                for (int j = i; j > 0 && srt[j - 1] > srt[j]; --j) { const float x = srt[j]; srt[j] = srt[j - 1]; srt[j - 1] = x; }
+            int cut = 0;
+            if (ez[tm] > __fmul_rn(cut_ratio, srt[3])) {
+                const int bnd = tm + 1;                           // boundary frame 1..7
+                cut = bnd <= 2 ? 2 : (bnd <= 5 ? 4 : 6);         // nearest of 2, 4, 6; 3 and 5 to 4
+            }
+            d.zcut[(size_t)h * d.Nz + m] = (uint8_t)cut;
+        }
     }
 }
 
@@ -448,7 +577,7 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restri
 // Closed form with the mapping exponent alpha (the pages' method: 1/2):
 // l*_d = -alpha log2 g_d + 1/3 (S + alpha sum_d' log2 g_d'), so that
 // b_d ~ g_d^-alpha and prod b_d = B.
-__device__ int snap_shape(const float g[3], int vol, float alpha) {
+__device__ int snap_shape(const float g[3], int vol, float alpha, int L = 8) {
     const float lg0 = log2f(g[0]), lg1 = log2f(g[1]), lg2 = log2f(g[2]);
     const float S = vol == 64 ? 6.f : (vol == 128 ? 7.f : 8.f);
     float inner = __fadd_rn(S, __fmul_rn(alpha, lg0));
@@ -460,15 +589,17 @@ __device__ int snap_shape(const float g[3], int vol, float alpha) {
     const float e2 = __fadd_rn(__fmul_rn(-alpha, lg2), third);
     const int lo = vol == 64 ? 0 : (vol == 128 ? 7 : 13);
     const int hi = vol == 64 ? 7 : (vol == 128 ? 13 : 16);
-    int best = lo;
+    // candidates whose time edge divides the region's L frames (all for a whole zone)
+    int best = -1;
     float bd = 0.f;
     for (int s = lo; s < hi; ++s) {
+        if (L % c_shape[s][0]) continue;
         const float d0 = __fsub_rn((float)c_log2shape[s][0], e0);
         const float d1 = __fsub_rn((float)c_log2shape[s][1], e1);
         const float d2 = __fsub_rn((float)c_log2shape[s][2], e2);
         float dist = __fadd_rn(__fmul_rn(d0, d0), __fmul_rn(d1, d1));
         dist = __fadd_rn(dist, __fmul_rn(d2, d2));
-        if (s == lo || dist < bd) { best = s; bd = dist; }
+        if (best < 0 || dist < bd) { best = s; bd = dist; }
     }
     return best;
 }
@@ -540,6 +671,150 @@ __global__ void __launch_bounds__(1024) k_zone_finalize(DevPlan d, ShapeRule rul
     for (int j = nb + threadIdx.x; j <= d.NB; j += blockDim.x) bs[j] = (int)d.N;
 }
 
+// Shape of one part of a split zone (or a whole zone, L = 8) from its
+// statistics st = (sigma2_T, sigma2_H, sigma2_W, rho_raw), the head's maximum
+// density mx, its audio coupling ab and v_hat vh.  The volume is capped at the
+// largest that tiles L frames (b_T in {2, 4, 8} must divide L: 128 for 2 or 6).
+__device__ int region_shape(const float* st, float mx, float ab, const float* vh, int L, const ShapeRule& rule) {
+    const float rho = mx > 0.f ? __fdiv_rn(st[3], mx) : 0.f;
+    int vol = rho < rule.tau256 ? 256 : (rho < rule.tau128 ? 128 : 64);
+    if ((L == 2 || L == 6) && vol == 256) vol = 128;
+    float g[3];
+    if (rule.mode == PRISM_SHAPE_ISOTROPIC) {
+        g[0] = g[1] = g[2] = 1.f;
+    } else {
+        const float tot = __fadd_rn(__fadd_rn(st[0], st[1]), st[2]);
+        float r[3];
+        if (tot > 0.f) { r[0] = __fdiv_rn(st[0], tot); r[1] = __fdiv_rn(st[1], tot); r[2] = __fdiv_rn(st[2], tot); }
+        else { r[0] = r[1] = r[2] = 1.f / 3.f; }
+        #pragma unroll
+        for (int ax = 0; ax < 3; ++ax) g[ax] = __fadd_rn(__fadd_rn(r[ax], __fmul_rn(ab, vh[ax])), rule.eps);
+    }
+    return snap_shape(g, vol, rule.alpha, L);
+}
+
+// A split frame outside {0, 2, 4, 6} (an imported plan's mistake) is read as 4
+// everywhere, so every index stays inside its zone; finalize reports it.
+__device__ __forceinline__ int sane_cut(int c) { return (c == 0 || c == 2 || c == 4 || c == 6) ? c : 4; }
+
+// Parts of zone m (at most two): first frame, length, shape.
+__device__ __forceinline__ int zone_parts(const DevPlan& d, int h, int m, int* t0, int* len, int* sh) {
+    const size_t k = (size_t)h * d.Nz + m;
+    const int c = sane_cut(d.zcut[k]);
+    if (c == 0) { t0[0] = 0; len[0] = 8; sh[0] = d.shape_id[k]; return 1; }
+    t0[0] = 0; len[0] = c; sh[0] = d.shape_id[k];
+    t0[1] = c; len[1] = 8 - c; sh[1] = d.shape_id2[k];
+    return 2;
+}
+
+// Volume of a part's blocks; a shape id out of range, a split frame other than
+// 0, 2, 4, 6, a b_T that does not divide the part's length or a volume that
+// does not tile it sets *bad, and the part is tiled with 128-token blocks so
+// that every later index stays inside the zone (64 L is a multiple of 128).
+__device__ __forceinline__ int part_vol(int sh, int len, int c, bool* bad) {
+    *bad = sh >= 16 || (c != 0 && c != 2 && c != 4 && c != 6);
+    if (*bad) return 128;
+    const int vol = c_shape[sh][0] * c_shape[sh][1] * c_shape[sh][2];
+    *bad = (len % c_shape[sh][0]) != 0 || ((64 * len) % vol) != 0;
+    return *bad ? 128 : vol;
+}
+
+// Finalize with adaptive temporal boundaries: rho and a_bar normalised over
+// the head's zones and parts, one shape per part, block offsets and the
+// 64-token tile -> block map with each split zone's first part first.
+__global__ void __launch_bounds__(1024) k_zone_finalize_cut(DevPlan d, ShapeRule rule, int use_given_shapes,
+                                                            int has_audio) {
+    __shared__ float redf[32];
+    __shared__ double redd[32];
+    __shared__ int red[1024];
+    extern __shared__ int nbz[];   // [Nz + 1]
+    const int h = blockIdx.x;
+    const float* zs = d.zstat + (size_t)h * d.Nz * 4;
+    const float* rs = d.rstat + (size_t)h * d.Nz * 8;
+    const uint8_t* cut = d.zcut + (size_t)h * d.Nz;
+    uint8_t* sid = d.shape_id + (size_t)h * d.Nz;
+    uint8_t* sid2 = d.shape_id2 + (size_t)h * d.Nz;
+    if (!use_given_shapes) {
+        float mx = 0.f;
+        double ma = 0.0;
+        for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+            const int c = cut[m];
+            if (c == 0) {
+                mx = fmaxf(mx, zs[m * 4 + 3]);
+                if (has_audio) ma = fmax(ma, d.araw[m]);
+            } else {
+                for (int p = 0; p < 2; ++p) {
+                    mx = fmaxf(mx, rs[(m * 2 + p) * 4 + 3]);
+                    if (has_audio) ma = fmax(ma, d.araw_seg[m * 6 + (c / 2 - 1) * 2 + p]);
+                }
+            }
+        }
+        mx = block_max<1024>(mx, redf);
+        for (int o = 16; o > 0; o >>= 1) ma = fmax(ma, __shfl_xor_sync(0xffffffffu, ma, o));
+        if ((threadIdx.x & 31) == 0) redd[threadIdx.x >> 5] = ma;
+        __syncthreads();
+        ma = redd[0];
+        for (int i = 1; i < 32; ++i) ma = fmax(ma, redd[i]);
+        const float zero3[3] = {0.f, 0.f, 0.f};
+        for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+            const int c = cut[m];
+            if (c == 0) {
+                const float ab = has_audio && ma > 0.0 ? (float)(d.araw[m] / ma) : 0.f;
+                sid[m] = (uint8_t)region_shape(zs + m * 4, mx, ab, has_audio ? d.vhat + 3 * m : zero3, 8, rule);
+                sid2[m] = 255;
+            } else {
+                for (int p = 0; p < 2; ++p) {
+                    const int k = m * 6 + (c / 2 - 1) * 2 + p;
+                    const float ab = has_audio && ma > 0.0 ? (float)(d.araw_seg[k] / ma) : 0.f;
+                    const int s = region_shape(rs + (m * 2 + p) * 4, mx, ab, has_audio ? d.vhat_seg + 3 * k : zero3,
+                                               p ? 8 - c : c, rule);
+                    (p ? sid2 : sid)[m] = (uint8_t)s;
+                }
+            }
+        }
+        __syncthreads();
+    }
+    // blocks per zone; a part whose shape cannot tile it is a device-check error
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+        int t0[2], len[2], sh[2];
+        const int np = zone_parts(d, h, m, t0, len, sh);
+        int nb = 0;
+        if (sane_cut(cut[m]) != cut[m]) dev_fail(d.err, PRISM_ERR_DEVICE_CHECK);
+        for (int p = 0; p < np; ++p) {
+            bool bad;
+            const int vol = part_vol(sh[p], len[p], sane_cut(cut[m]), &bad);
+            if (bad) dev_fail(d.err, PRISM_ERR_DEVICE_CHECK);
+            nb += 64 * len[p] / vol;
+        }
+        nbz[m] = nb;
+    }
+    __syncthreads();
+    block_exclusive_scan_inplace(nbz, d.Nz, red);
+    int* zoff = d.zone_off + (size_t)h * (d.Nz + 1);
+    int* bs = d.blk_start + (size_t)h * (d.NB + 1);
+    int* t64 = d.t64_blk + (size_t)h * d.NB;
+    for (int m = threadIdx.x; m <= d.Nz; m += blockDim.x) zoff[m] = nbz[m];
+    const int nbt = nbz[d.Nz];
+    if (threadIdx.x == 0) d.nblocks[h] = nbt;
+    for (int m = threadIdx.x; m < d.Nz; m += blockDim.x) {
+        int t0[2], len[2], sh[2];
+        const int np = zone_parts(d, h, m, t0, len, sh);
+        int j = nbz[m];
+        for (int p = 0; p < np; ++p) {
+            bool bad;
+            const int v = part_vol(sh[p], len[p], sane_cut(cut[m]), &bad);
+            const int pos0 = 512 * m + 64 * t0[p];
+            const int cnt = 64 * len[p] / v;
+            for (int k = 0; k < cnt; ++k, ++j) {
+                const int st = pos0 + k * v;
+                bs[j] = st;
+                for (int u = 0; u < v / 64; ++u) t64[st / 64 + u] = j;
+            }
+        }
+    }
+    for (int j = nbt + threadIdx.x; j <= d.NB; j += blockDim.x) bs[j] = (int)d.N;
+}
+
 // ================================================================ stage 2
 // The block-ordered copies are fp16: a bf16 value converts exactly when
 // 2^-14 <= |x| <= 65504 (or x = 0), smaller magnitudes round to fp16's
@@ -568,9 +843,23 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
     const int* bs = d.blk_start + (size_t)h * (d.NB + 1);
     const int start = bs[j], vol = bs[j + 1] - start;
     const int m = start >> 9;
-    const int s = d.shape_id[(size_t)h * d.Nz + m];
+    // the block's part of the zone: frames [toff, toff + L), first slot 512 m + 64 toff
+    int s, toff = 0, rlo = start - 512 * m;
+    if (d.zcut) {
+        int t0[2], len[2], sh[2];
+        const int np = zone_parts(d, h, m, t0, len, sh);
+        const int p = (np == 2 && rlo >= 64 * t0[1]) ? 1 : 0;
+        bool bad;
+        part_vol(sh[p], len[p], sane_cut(d.zcut[(size_t)h * d.Nz + m]), &bad);
+        s = bad ? 7 : sh[p];                     // 2 x 8 x 8 tiles any part (device-check error set)
+        toff = t0[p];
+        rlo -= 64 * t0[p];
+    } else {
+        s = d.shape_id[(size_t)h * d.Nz + m];
+        s = s < 16 ? s : 0;
+    }
     const int bt = c_shape[s][0], bh = c_shape[s][1], bw = c_shape[s][2];
-    const int kin = (start - 512 * m) / vol;
+    const int kin = rlo / vol;
     const int nkw = 8 / bw, nkh = 8 / bh;
     const int kw = kin % nkw, kh = (kin / nkw) % nkh, kt = kin / (nkw * nkh);
     const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
@@ -582,7 +871,7 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
     const size_t hoff = (size_t)h * d.N * D;
     for (int r = rl; r < vol; r += RP) {
         const int lw = r % bw, lh = (r / bw) % bh, lt = r / (bw * bh);
-        const int64_t n = ((int64_t)(8 * zt + kt * bt + lt) * d.H + 8 * zh + kh * bh + lh) * d.W +
+        const int64_t n = ((int64_t)(8 * zt + toff + kt * bt + lt) * d.H + 8 * zh + kh * bh + lh) * d.W +
                           8 * zw + kw * bw + lw;
         const size_t so = hoff + (size_t)n * D + (size_t)c * EPC;
         const size_t dst = hoff + (size_t)(start + r) * D + (size_t)c * EPC;
@@ -1054,8 +1343,17 @@ template <typename T, int D>
 static void launch_stats(prism_plan_s* P, const DevPlan& d, const void* V, cudaStream_t s) {
     const Geom& g = P->g;
     const int sm = (256 / (D / 2)) * D * 26 * (int)sizeof(float);
-    cudaFuncSetAttribute(k_zone_stats<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    k_zone_stats<T, D><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V);
+    if (!P->has_cuts) {
+        cudaFuncSetAttribute(k_zone_stats<T, D, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V, 0.f);
+        return;
+    }
+    // whole zones with their energies and split decisions, then the parts of the split zones
+    const int sm1 = (256 / (D / 2)) * D * 33 * (int)sizeof(float);
+    cudaFuncSetAttribute(k_zone_stats<T, D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
+    k_zone_stats<T, D, 1><<<dim3(g.Nz, g.heads), 256, sm1, s>>>(d, (const T*)V, P->p.cut_ratio);
+    cudaFuncSetAttribute(k_zone_stats<T, D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    k_zone_stats<T, D, 2><<<dim3(g.Nz, g.heads, 2), 256, sm, s>>>(d, (const T*)V, 0.f);
 }
 
 template <typename T, int D>
@@ -1085,10 +1383,12 @@ static void launch_lists(prism_plan_s* P, const DevPlan& d, cudaStream_t s) {
 }
 
 static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V, const float* amap,
-                    const uint8_t* given_shapes, const uint32_t* given_sel, cudaStream_t s) {
-    // kernels launched below: audio 1-2, stats 1, finalize 1, gather 1, select (or
+                    const uint8_t* given_shapes, const uint32_t* given_sel, cudaStream_t s,
+                    const uint8_t* given_cut = nullptr, const uint8_t* given_sid2 = nullptr) {
+    // kernels launched below: audio 1-3, stats 1-2, finalize 1, gather 1, select (or
     // mask + popcount) 1-2, lists 12
-    P->launches += (given_shapes ? 0 : (amap ? 3 : 2)) + 2 + (given_sel ? 2 : 1) + 12;
+    const int cut_extra = P->has_cuts && !given_shapes ? 1 + (amap ? 1 : 0) : 0;
+    P->launches += (given_shapes ? 0 : (amap ? 3 : 2)) + cut_extra + 2 + (given_sel ? 2 : 1) + 12;
     const Geom& g = P->g;
     const prism_params& p = P->p;
     DevPlan d = dev_plan(P);
@@ -1099,6 +1399,7 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
         if (amap) {
             k_audio_zone<<<g.Nz, 256, 0, s>>>(d, amap);
             k_audio_norm<<<1, 1024, 0, s>>>(d);
+            if (P->has_cuts) k_audio_seg<<<g.Nz, 256, 0, s>>>(d, amap);
         } else {
             k_audio_none<<<(g.Nz + 255) / 256, 256, 0, s>>>(d);
         }
@@ -1108,13 +1409,24 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
         else launch_stats<float, 64>(P, d, V, s);
     } else {
         cudaMemcpyAsync(d.shape_id, given_shapes, (size_t)g.heads * g.Nz, cudaMemcpyDeviceToDevice, s);
+        if (P->has_cuts) {
+            cudaMemcpyAsync(d.zcut, given_cut, (size_t)g.heads * g.Nz, cudaMemcpyDeviceToDevice, s);
+            cudaMemcpyAsync(d.shape_id2, given_sid2, (size_t)g.heads * g.Nz, cudaMemcpyDeviceToDevice, s);
+        }
     }
     {
         PrismProf prof(P, PRISM_STAGE_PLAN_SHAPES, s);
         const size_t fin_smem = sizeof(int) * (g.Nz + 1);
-        if (fin_smem > 48 * 1024)
-            cudaFuncSetAttribute(k_zone_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
-        k_zone_finalize<<<g.heads, 1024, fin_smem, s>>>(d, shape_rule(p), given_shapes ? 1 : 0);
+        if (P->has_cuts) {
+            if (fin_smem > 48 * 1024)
+                cudaFuncSetAttribute(k_zone_finalize_cut, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
+            k_zone_finalize_cut<<<g.heads, 1024, fin_smem, s>>>(d, shape_rule(p), given_shapes ? 1 : 0,
+                                                               amap ? 1 : 0);
+        } else {
+            if (fin_smem > 48 * 1024)
+                cudaFuncSetAttribute(k_zone_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fin_smem);
+            k_zone_finalize<<<g.heads, 1024, fin_smem, s>>>(d, shape_rule(p), given_shapes ? 1 : 0);
+        }
     }
     {
         PrismProf prof(P, PRISM_STAGE_PLAN_GATHER, s);
@@ -1167,7 +1479,27 @@ extern "C" int prism_plan(const prism_params* p, const void* Q, const void* K, c
     int st = plan_common(p, Q, K, V, workspace, ws_bytes, &P);
     if (st) return st;
     P->has_audio = a_map != nullptr;
+    P->has_cuts = p->cut_ratio > 0.f;
     st = run_plan(P, Q, K, V, a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+    if (st) { delete P; return st; }
+    *out = P;
+    return PRISM_OK;
+}
+
+extern "C" int prism_plan_import_cuts(const prism_params* p, const void* Q, const void* K, const void* V,
+                                      const uint8_t* shape_id, const uint8_t* zone_cut, const uint8_t* shape_id2,
+                                      const uint32_t* sel, void* workspace, size_t ws_bytes, void* stream,
+                                      prism_plan_t* out) {
+    if (!out) return PRISM_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!shape_id || !sel || !aligned16(sel)) return PRISM_ERR_INVALID_ARG;
+    if ((zone_cut == nullptr) != (shape_id2 == nullptr)) return PRISM_ERR_INVALID_ARG;
+    prism_plan_s* P = nullptr;
+    int st = plan_common(p, Q, K, V, workspace, ws_bytes, &P);
+    if (st) return st;
+    P->has_audio = 0;
+    P->has_cuts = zone_cut != nullptr;
+    st = run_plan(P, Q, K, V, nullptr, shape_id, sel, static_cast<cudaStream_t>(stream), zone_cut, shape_id2);
     if (st) { delete P; return st; }
     *out = P;
     return PRISM_OK;
@@ -1176,17 +1508,7 @@ extern "C" int prism_plan(const prism_params* p, const void* Q, const void* K, c
 extern "C" int prism_plan_import(const prism_params* p, const void* Q, const void* K, const void* V,
                                  const uint8_t* shape_id, const uint32_t* sel, void* workspace,
                                  size_t ws_bytes, void* stream, prism_plan_t* out) {
-    if (!out) return PRISM_ERR_INVALID_ARG;
-    *out = nullptr;
-    if (!shape_id || !sel || !aligned16(sel)) return PRISM_ERR_INVALID_ARG;
-    prism_plan_s* P = nullptr;
-    int st = plan_common(p, Q, K, V, workspace, ws_bytes, &P);
-    if (st) return st;
-    P->has_audio = 0;
-    st = run_plan(P, Q, K, V, nullptr, shape_id, sel, static_cast<cudaStream_t>(stream));
-    if (st) { delete P; return st; }
-    *out = P;
-    return PRISM_OK;
+    return prism_plan_import_cuts(p, Q, K, V, shape_id, nullptr, nullptr, sel, workspace, ws_bytes, stream, out);
 }
 
 extern "C" size_t prism_plan_item_bytes(prism_plan_t P, int item) {
@@ -1206,6 +1528,10 @@ extern "C" size_t prism_plan_item_bytes(prism_plan_t P, int item) {
         case PRISM_ITEM_KBAR: return 4 * H * NB * g.D;
         case PRISM_ITEM_SRC: return 4 * H * (size_t)g.N;
         case PRISM_ITEM_ZONE_STATS: return 4 * H * g.Nz * 4;
+        case PRISM_ITEM_ZONE_CUT: return P->has_cuts ? H * g.Nz : 0;
+        case PRISM_ITEM_SHAPE_ID2: return P->has_cuts ? H * g.Nz : 0;
+        case PRISM_ITEM_ZONE_ENERGY: return P->has_cuts ? 4 * H * g.Nz * 7 : 0;
+        case PRISM_ITEM_REGION_STATS: return P->has_cuts ? 4 * H * g.Nz * 8 : 0;
         default: return 0;
     }
 }
@@ -1229,6 +1555,10 @@ extern "C" int prism_plan_export(prism_plan_t P, int item, void* host_dst, size_
         case PRISM_ITEM_KBAR: off = L.kbar; break;
         case PRISM_ITEM_SRC: off = L.src; break;
         case PRISM_ITEM_ZONE_STATS: off = L.zstat; break;
+        case PRISM_ITEM_ZONE_CUT: off = L.zcut; break;
+        case PRISM_ITEM_SHAPE_ID2: off = L.shape_id2; break;
+        case PRISM_ITEM_ZONE_ENERGY: off = L.zdiff; break;
+        case PRISM_ITEM_REGION_STATS: off = L.rstat; break;
         default: return PRISM_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1386,8 +1716,8 @@ __global__ void __launch_bounds__(1024) k_zone_shapes_static(DevPlan d, ShapeRul
 template <typename T, int D>
 static void noalloc_stats(const Geom& g, const DevPlan& d, const void* V, cudaStream_t s) {
     const int sm = (256 / (D / 2)) * D * 26 * (int)sizeof(float);
-    cudaFuncSetAttribute(k_zone_stats<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    k_zone_stats<T, D><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V);
+    cudaFuncSetAttribute(k_zone_stats<T, D, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V, 0.f);
 }
 
 // Device address of the scratch array, looked up once per device (with that
@@ -1413,6 +1743,7 @@ extern "C" int prism_zone_shapes_noalloc(const prism_params* p, const void* V, c
     using namespace prism;
     int st = validate_params(p);
     if (st) return st;
+    if (p->cut_ratio != 0.f) return PRISM_ERR_INVALID_ARG;   // whole zones only
     if (!V || !shape_id || !nblocks || !aligned16(V) || (a_map && !aligned16(a_map)))
         return PRISM_ERR_INVALID_ARG;
     st = check_device();

@@ -102,6 +102,23 @@ extern "C" {
  *   top_k_frac  k as a fraction of the head's block count: when > 0, each
  *               head's k is ceil(top_k_frac * N_b) in fp32 (the pages' "Top-k
  *               95%" sparsity keeps 5%: 0.05) and top_k is ignored; in [0, 1].
+ * Adaptive temporal zone boundaries (page paper.rainbus.top, section
+ * "独立分析的弱点" item (1) and section "未来方向": split a macro-zone where a
+ * shot cut shows in the frame differences):
+ *   cut_ratio   0 keeps every zone whole (the pages' method).  When > 0, per
+ *               zone and head the frame-difference energies e_t (mean over the
+ *               zone's 64 tokens and D channels of (V[t+1] - V[t])^2, t = 0..6,
+ *               fp32) are formed; a cut follows the largest e_t (lowest t on
+ *               ties) when it exceeds cut_ratio times their median; the
+ *               boundary snaps to the nearest of frames 2, 4, 6 (3 and 5 to 4),
+ *               and each part is planned like a zone: its own statistics,
+ *               volume capped at what its length tiles (128 for 2 or 6 frames),
+ *               shape among the candidates whose b_T divides its length; rho
+ *               and a_bar are normalised over the head's zones and parts.  The
+ *               first part's blocks come first in the zone.  Must be >= 0 and
+ *               finite; not allowed with PRISM_SHAPE_FIXED.  Smooth content
+ *               stays below 2 and a shot cut is typically above 3.5: 2.5 is a
+ *               reasonable value.
  */
 #define PRISM_SHAPE_DYNAMIC   0
 #define PRISM_SHAPE_ISOTROPIC 1
@@ -121,6 +138,7 @@ typedef struct prism_params {
     int32_t shape_mode;
     int32_t fixed_shape;
     float   top_k_frac;
+    float   cut_ratio;
 } prism_params;
 
 /* Opaque host-side handle: a small host struct pointing into the workspace. */
@@ -179,6 +197,20 @@ PRISM_API int prism_plan_import(const prism_params* p, const void* Q, const void
                       void* workspace, size_t ws_bytes, void* stream, prism_plan_t* out);
 
 /*
+ * prism_plan_import_cuts -- prism_plan_import for plans with adaptive temporal
+ * boundaries: zone_cut (device uint8 [heads][Nz], 0, 2, 4 or 6) gives each
+ * zone's split frame and shape_id2 (device uint8 [heads][Nz]) the shape of the
+ * part after it; shape_id then holds the first part's shape.  A shape whose
+ * b_T does not divide its part's length, or a volume its part cannot tile, is
+ * reported as PRISM_ERR_DEVICE_CHECK by prism_get_status.  NULL zone_cut (and
+ * shape_id2) is prism_plan_import.
+ */
+PRISM_API int prism_plan_import_cuts(const prism_params* p, const void* Q, const void* K, const void* V,
+                                     const uint8_t* shape_id, const uint8_t* zone_cut,
+                                     const uint8_t* shape_id2, const uint32_t* sel, void* workspace,
+                                     size_t ws_bytes, void* stream, prism_plan_t* out);
+
+/*
  * prism_attn_fwd -- stages 4-5: for every query token q of block i,
  *   O_q = softmax_n(q . k_n / sqrt(D)) v_n over the tokens n of the key
  *   blocks in S_i (fp32 online softmax, fp16 tensor-core products with fp32
@@ -209,6 +241,7 @@ PRISM_API int prism_attn_bwd(prism_plan_t plan, const void* dO, const void* O, c
  *   device fp32 [T][H][W] or NULL).  Outputs (device, caller-allocated):
  *     shape_id  uint8 [heads][Nz], the candidate index per zone and head;
  *     nblocks   int32 [heads], blocks of the head (sum over zones of 512 / B).
+ *   Whole zones only: p->cut_ratio must be 0 (PRISM_ERR_INVALID_ARG otherwise).
  *   Scratch: a file-scope static device array of 4 MiB (2^20 floats) that
  *   every GPU loading the library holds until the process exits.  Its use is
  *   2*Nz + Nz + 3*Nz + 4*heads*Nz floats (each part rounded up to 64 floats);
@@ -278,7 +311,11 @@ PRISM_API int prism_status_read(int32_t* dev_status, int32_t* site, void* stream
 #define PRISM_ITEM_KBAR       9  /* fp32   [heads][N/64][head_dim]             */
 #define PRISM_ITEM_SRC       10  /* int32  [heads][N] raster token of each permuted slot */
 #define PRISM_ITEM_ZONE_STATS 11 /* fp32   [heads][Nz][4] sigma2_T, sigma2_H, sigma2_W, rho_raw */
-#define PRISM_ITEM_COUNT     12
+#define PRISM_ITEM_ZONE_CUT  12  /* uint8  [heads][Nz] split frame (0 = whole zone, 2, 4 or 6) */
+#define PRISM_ITEM_SHAPE_ID2 13  /* uint8  [heads][Nz] shape of the part after the split (255 if none) */
+#define PRISM_ITEM_ZONE_ENERGY 14 /* fp32  [heads][Nz][7] frame-difference energies e_t */
+#define PRISM_ITEM_REGION_STATS 15 /* fp32 [heads][Nz][2][4] the parts' statistics (split zones) */
+#define PRISM_ITEM_COUNT     16
 
 /* Bytes of an item (0 for an unknown item). */
 PRISM_API size_t prism_plan_item_bytes(prism_plan_t plan, int item);
