@@ -953,8 +953,10 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, fl
     const int i = blockIdx.x, h = blockIdx.y;
     const int nb = d.nblocks[h];
     int* rowcnt = d.row_ptr + (size_t)h * (d.NB + 1);
-    if (i >= nb) {
+    if (i >= nb) {                                  // rows past the head's blocks: empty
         if (threadIdx.x == 0) rowcnt[i] = 0;
+        uint32_t* row = d.sel + ((size_t)h * d.NB + i) * d.WORDS;
+        for (int w = threadIdx.x; w < d.WORDS; w += SEL_THREADS) row[w] = 0u;
         return;
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -37,11 +37,15 @@ def test_selection_mismatch_needs_a_near_tie():
     assert parity.selection_agrees(np.sort(np.r_[order[:2], order[3]]), s2, P[0], 3, 0.0)
 
 
-def test_gradient_rule_adds_half_a_bf16_ulp_per_element():
+def test_gradient_rule_adds_half_a_bf16_ulp_of_the_tensor_scale():
     ref = np.array([0.5, 170.0, -80.0])
-    # 0.04 off on the element of 170: inside 3e-2 + 170 / 512
-    assert parity.close_grad(ref + [0.0, 0.04, 0.0], ref)[0]
-    # 0.04 off on the element of 0.5: outside 3e-2 + 0.5 / 512
-    assert not parity.close_grad(ref + [0.04, 0.0, 0.0], ref)[0]
-    # a relative error of 2^-8 (a whole bf16 ulp) on the large element fails
-    assert not parity.close_grad(ref * [1, 1 + 2.0 ** -8, 1] + [0, 0.03, 0], ref)[0]
+    # 0.3 off anywhere: inside 3e-2 + 170 / 512
+    assert parity.close_grad(ref + [0.3, 0.0, 0.0], ref)[0]
+    assert parity.close_grad(ref + [0.0, 0.3, 0.0], ref)[0]
+    # 0.4 off: outside it
+    assert not parity.close_grad(ref + [0.4, 0.0, 0.0], ref)[0]
+    # on a unit-scale tensor the bar is the plain 3e-2 (plus 2^-9)
+    small = np.array([0.5, -1.0, 0.25])
+    assert not parity.close_grad(small + [0.04, 0.0, 0.0], small)[0]
+    # the relative-L2 bar still applies
+    assert not parity.close_grad(ref * 1.02, ref)[0]
