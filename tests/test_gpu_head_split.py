@@ -8,7 +8,8 @@ ranks) must reproduce the one-call plan bit for bit and the one-call outputs:
 O and LSE bit for bit (each query tile is reduced in one fixed order), dK and
 dV bit for bit on a one-chunk grid (each key tile's sums stay in TMEM and are
 added once into zeroed accumulators), and dQ to fp32 rounding (its partial sums
-from different key tiles are reduce-added in the order the CTAs finish).  The
+from different key tiles are reduce-added in the order the CTAs finish: within
+1e-5 of the tensor's largest magnitude).  The
 two "ranks" run one after the other on the same GPU; nothing waits on the other.
 """
 import numpy as np
@@ -66,6 +67,8 @@ def test_two_head_shards_equal_one_call(wid, grid, cuda_device):
         for got, want, nm in zip(outs, whole, ("O", "LSE", "dQ", "dK", "dV")):
             g, r = got.cpu(), want[sl].cpu()
             if nm == "dQ":
-                torch.testing.assert_close(g, r, rtol=1e-5, atol=1e-6, msg=f"rank {rank} dQ")
+                # fp32 sums of the key tiles' partial dQ, in the order the CTAs finish
+                diff, scale = (g - r).abs().max().item(), r.abs().max().item()
+                assert diff <= 1e-5 * scale, f"rank {rank} dQ: max diff {diff:.3e} at scale {scale:.3e}"
             else:
                 assert torch.equal(g, r), f"rank {rank} {nm}: max diff {(g - r).abs().max().item():.3e}"
