@@ -32,7 +32,7 @@ ITEMS = {
     "col_ptr": (6, np.int32), "row_idx": (7, np.int32), "qbar": (8, np.float32),
     "kbar": (9, np.float32), "src": (10, np.int32), "zone_stats": (11, np.float32),
     "zone_cut": (12, np.uint8), "shape_id2": (13, np.uint8), "zone_energy": (14, np.float32),
-    "region_stats": (15, np.float32),
+    "region_stats": (15, np.float32), "list_offsets": (16, np.int64),
 }
 
 
@@ -73,6 +73,9 @@ def load(path: str | None = None) -> C.CDLL:
     pp = C.POINTER(PrismParams)
     sig = {
         "prism_plan_workspace_bytes": (sz, [pp]),
+        "prism_plan_core_bytes": (sz, [pp]),
+        "prism_plan_list_bytes": (i32, [vp, C.POINTER(sz), vp]),
+        "prism_plan_attach_lists": (i32, [vp, vp, sz, vp]),
         "prism_plan": (i32, [pp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import": (i32, [pp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import_cuts": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
@@ -121,7 +124,13 @@ def make_params(T, H, W, heads, head_dim, dtype, top_k, top_p, eps, tau128=0.5, 
 
 
 def workspace_bytes(params: PrismParams) -> int:
+    """Workspace of a plan ready in one call (index lists at their dense bound)."""
     return int(load().prism_plan_workspace_bytes(C.byref(params)))
+
+
+def core_bytes(params: PrismParams) -> int:
+    """Workspace without the index lists (they go to a second buffer sized after planning)."""
+    return int(load().prism_plan_core_bytes(C.byref(params)))
 
 
 def _ptr(t):
@@ -137,10 +146,11 @@ def _stream(stream):
 class Plan:
     """A plan handle plus the device buffers it points into (kept alive here)."""
 
-    def __init__(self, params, handle, workspace, inputs):
+    def __init__(self, params, handle, workspace, inputs, lists=None):
         self.params = params
         self._h = handle
         self._ws = workspace
+        self._lists = lists            # the index lists' buffer of a two-call plan
         self._inputs = inputs          # Q, K, V must outlive the plan
 
     @property
@@ -245,12 +255,28 @@ def _check_inputs(Q, K, V, params):
                              f"got {tuple(t.shape)}")
 
 
-def plan(Q, K, V, a_map, params: PrismParams, workspace=None, stream=None) -> Plan:
-    """Stages 1-3 on the GPU.  Q, K, V: [heads, N, D] CUDA tensors (raster order)."""
+def _attach_lists(lib, h, device, stream):
+    """Size and build a two-call plan's index lists in a buffer of their own."""
+    import torch
+    nbytes = C.c_size_t(0)
+    st = lib.prism_plan_list_bytes(h, C.byref(nbytes), _stream(stream))
+    if st:
+        raise PrismError(st, "prism_plan_list_bytes")
+    lists = torch.empty(max(int(nbytes.value), 16), dtype=torch.uint8, device=device)
+    st = lib.prism_plan_attach_lists(h, _ptr(lists), lists.numel(), _stream(stream))
+    if st:
+        raise PrismError(st, "prism_plan_attach_lists")
+    return lists
+
+
+def plan(Q, K, V, a_map, params: PrismParams, workspace=None, stream=None, compact=False) -> Plan:
+    """Stages 1-3 on the GPU.  Q, K, V: [heads, N, D] CUDA tensors (raster order).
+    compact=True plans with the core workspace and sizes the index lists from
+    their counts (one stream synchronisation) instead of their dense bound."""
     import torch
     lib = load()
     _check_inputs(Q, K, V, params)
-    need = workspace_bytes(params)
+    need = core_bytes(params) if compact else workspace_bytes(params)
     if need == 0:
         raise PrismError(PRISM_ERR_INVALID_ARG, "prism_plan_workspace_bytes")
     if workspace is None:
@@ -260,18 +286,25 @@ def plan(Q, K, V, a_map, params: PrismParams, workspace=None, stream=None) -> Pl
                         workspace.numel(), _stream(stream), C.byref(h))
     if st:
         raise PrismError(st, "prism_plan")
-    return Plan(params, h, workspace, (Q, K, V, a_map))
+    lists = None
+    if workspace.numel() < workspace_bytes(params):
+        try:
+            lists = _attach_lists(lib, h, Q.device, stream)
+        except PrismError:
+            lib.prism_plan_destroy(h)
+            raise
+    return Plan(params, h, workspace, (Q, K, V, a_map), lists)
 
 
 def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None, stream=None,
-                zone_cut=None, shape_id2=None) -> Plan:
+                zone_cut=None, shape_id2=None, compact=False) -> Plan:
     """A plan from given shape ids [heads, Nz] (uint8) and selection bitmap (int32/uint32 words);
     with adaptive temporal boundaries also the split frames zone_cut and the second parts'
     shapes shape_id2 ([heads, Nz] uint8 each)."""
     import torch
     lib = load()
     _check_inputs(Q, K, V, params)
-    need = workspace_bytes(params)
+    need = core_bytes(params) if compact else workspace_bytes(params)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
     h = C.c_void_p()
@@ -285,7 +318,14 @@ def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None
                                         workspace.numel(), _stream(stream), C.byref(h))
     if st:
         raise PrismError(st, "prism_plan_import")
-    return Plan(params, h, workspace, (Q, K, V, shape_id, sel_bits, zone_cut, shape_id2))
+    lists = None
+    if workspace.numel() < workspace_bytes(params):
+        try:
+            lists = _attach_lists(lib, h, Q.device, stream)
+        except PrismError:
+            lib.prism_plan_destroy(h)
+            raise
+    return Plan(params, h, workspace, (Q, K, V, shape_id, sel_bits, zone_cut, shape_id2), lists)
 
 
 def av_norm(Qv, Ka, Va, a_map=None, h_hat=None, hhat_dtype=None, want_hhat=False, status=None,

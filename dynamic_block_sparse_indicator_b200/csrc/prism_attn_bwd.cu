@@ -36,6 +36,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "prism_dev.cuh"
 #include "prism_internal.h"
 
@@ -84,16 +86,16 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, cons
                                                  const float* __restrict__ lse,
                                                  const int* __restrict__ src, const uint32_t* dmax,
                                                  __half* __restrict__ dOp, float* __restrict__ lse_p,
-                                                 float* __restrict__ di_p, int64_t N, int HD, int* err) {
+                                                 float* __restrict__ di_p, int64_t N, int HD, int h0, int* err) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t p = (int64_t)blockIdx.x * 8 + warp;
-    const int h = blockIdx.y;
+    const int h = h0 + blockIdx.y;                   // dOp holds the head group [h0, h0 + gridDim.y)
     if (p >= N) return;
     const float sc = ldexpf(1.f, -dscale_exp(dmax[h], err));
     const int64_t n = src[(size_t)h * N + p];
     const OT* dr = dO + ((size_t)h * N + n) * HD;
     const OT* orow = O + ((size_t)h * N + n) * HD;
-    __half* out = dOp + ((size_t)h * N + p) * HD;
+    __half* out = dOp + ((size_t)(h - h0) * N + p) * HD;
     float acc = 0.f;
     for (int c = lane; c < HD; c += 32) {
         const float g = (float)dr[c];
@@ -146,7 +148,10 @@ __device__ __forceinline__ int count_units(const int* ents, int n, int own_is_ke
 
 struct BwdArgs {
     const int* ptr;        // [heads][NT + 1]
-    const int* ent;        // [heads][NT * NT]
+    const int* lbase;      // index lists; head h's tile list starts at lbase + ent_off[h]
+    const int64_t* ent_off;
+    int h0;                // first head of the launch's group: the dO copy and the
+                           // accumulators hold heads h0, h0 + 1, ... (rows (h - h0) N + ...)
     const int* src;        // [heads][N]
     const float* lse_p;    // [heads][N] 15 - LSE log2(e), block order
     const float* di_p;     // [heads][N] -D 2^-15 (D scaled like dO)
@@ -245,12 +250,12 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     // one CTA per (key tile t, chunk c of CQ query tiles): the grid runs chunk
     // after chunk, so the dQ accumulator rows and the Q / dO tiles that all CTAs
     // in flight touch are one chunk's (about 32 MB), resident in L2
-    const int t = blockIdx.x, c = blockIdx.y, h = blockIdx.z;
+    const int t = blockIdx.x, c = blockIdx.y, h = a.h0 + blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         const int p0 = a.ptr[(size_t)h * (a.NT + 1) + t];
         const int n0 = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - p0;
-        const int* all = a.ent + (size_t)h * a.NT * a.NT + p0;
+        const int* all = a.lbase + a.ent_off[h] + p0;
         const int lo = tiles_lower_bound(all, n0, c * a.CQ);
         const int hi = tiles_lower_bound(all, n0, (c + 1) * a.CQ);
         sm.e0 = p0 + lo;
@@ -260,7 +265,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     __syncthreads();
     const int e0 = sm.e0, ne = sm.ne, U = sm.U;
     if (U == 0) return;                            // nothing selected in this chunk
-    const int* ents = a.ent + (size_t)h * a.NT * a.NT + e0;
+    const int* ents = a.lbase + a.ent_off[h] + e0;
     // TMEM columns: buffer b = [128b, 128b + 128): S^T at 128b, dP^T at 128b + 64.
     // The softmax writes P^T (fp16 pairs) over the first half of dP^T; dQ^T of
     // the unit then overwrites all 64 dP^T columns after dV has read P^T (the
@@ -294,7 +299,8 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int64_t hrow = (int64_t)h * a.N;
+    const int64_t hrow = (int64_t)h * a.N;               // Q, K, V copies and per-row terms
+    const int64_t grow = (int64_t)(h - a.h0) * a.N;      // dO copy and accumulators (head group)
 
     if (warp == W_PROD) {
         if (lane == 0 && U > 0) {
@@ -311,10 +317,11 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 if (u >= DKDV_STAGES &&
                     !mbar_wait(&sm.st_empty[s], ((u / DKDV_STAGES) - 1) & 1, a.err, 1401)) break;
                 const int64_t qrow = hrow + (int64_t)r64 * 64;
+                const int64_t grow_q = grow + (int64_t)r64 * 64;
                 mbar_expect_tx(&sm.st_full[s], 2 * NSL * SLAB64 + 2 * 256);
                 for (int c = 0; c < NSL; ++c) {
                     tma_load_2d(sm.q[s][c], &tm_q64, &sm.st_full[s], 64 * c, (int)qrow);
-                    tma_load_2d(sm.dO[s][c], &tm_do64, &sm.st_full[s], 64 * c, (int)qrow);
+                    tma_load_2d(sm.dO[s][c], &tm_do64, &sm.st_full[s], 64 * c, (int)grow_q);
                 }
                 bulk_load(sm.lse[s], a.lse_p + qrow, 256, &sm.st_full[s]);
                 bulk_load(sm.di[s], a.di_p + qrow, 256, &sm.st_full[s]);
@@ -488,7 +495,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                tma_reduce_add_2d(wg ? &tm_dk : &tm_dv, stage, 0, (int)(hrow + (int64_t)t * 128 + 32 * (warp & 3)));
+                tma_reduce_add_2d(wg ? &tm_dk : &tm_dv, stage, 0, (int)(grow + (int64_t)t * 128 + 32 * (warp & 3)));
                 bulk_commit();
                 bulk_wait0();
             }
@@ -512,7 +519,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.dq_free[b]);
-            const int64_t qrow = hrow + (int64_t)r64 * 64;
+            const int64_t qrow = grow + (int64_t)r64 * 64;      // the group's dQ accumulator
             #pragma unroll
             for (int pass = 0; pass < 2; ++pass) {
                 if (leader) bulk_wait_read0();      // the previous reduce has read the stage
@@ -545,14 +552,14 @@ template <typename OT>
 __global__ void __launch_bounds__(256) k_acc_finalize(const float* __restrict__ acc0, float scale0, OT* __restrict__ out0,
                                                       const float* __restrict__ acc1, float scale1,
                                                       OT* __restrict__ out1, const int* __restrict__ src,
-                                                      const uint32_t* dmax, int64_t N, int HD, int* err) {
+                                                      const uint32_t* dmax, int64_t N, int HD, int h0, int* err) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t p = (int64_t)blockIdx.x * 8 + warp;
-    const int h = blockIdx.y;
+    const int h = h0 + blockIdx.y;                   // accumulators hold the head group from h0
     if (p >= N) return;
     const float unscale = ldexpf(1.f, dscale_exp(dmax[h], err));
     const int64_t n = src[(size_t)h * N + p];
-    const size_t ir = ((size_t)h * N + p) * HD, orow = ((size_t)h * N + n) * HD;
+    const size_t ir = ((size_t)(h - h0) * N + p) * HD, orow = ((size_t)h * N + n) * HD;
     for (int c = lane; c < HD; c += 32) out0[orow + c] = (OT)(acc0[ir + c] * (scale0 * unscale));
     if (acc1)
         for (int c = lane; c < HD; c += 32) out1[orow + c] = (OT)(acc1[ir + c] * (scale1 * unscale));
@@ -582,11 +589,11 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     DqSmem<HD>& sm = *reinterpret_cast<DqSmem<HD>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NSL = HD / 64;
-    const int t = blockIdx.x, h = blockIdx.y;
+    const int t = blockIdx.x, h = a.h0 + blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e0 = a.ptr[(size_t)h * (a.NT + 1) + t];
     const int ne = a.ptr[(size_t)h * (a.NT + 1) + t + 1] - e0;
-    const int* ents = a.ent + (size_t)h * a.NT * a.NT + e0;
+    const int* ents = a.lbase + a.ent_off[h] + e0;
     const int U = count_units(ents, ne, 0);
     constexpr uint32_t TS = 0, TDP = 128, TDQ = 256;
 
@@ -606,15 +613,17 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int64_t hrow = (int64_t)h * a.N;
+    const int64_t hrow = (int64_t)h * a.N;                  // Q, K, V copies, per-row terms
+    const int64_t grow = (int64_t)(h - a.h0) * a.N;         // the head group's dO copy
 
     if (warp == 4) {
         if (lane == 0 && U > 0) {
             const int qrow = (int)(hrow + (int64_t)t * 128);
+            const int dorow = (int)(grow + (int64_t)t * 128);
             mbar_expect_tx(&sm.bar_q, 2 * NSL * SLAB128);
             for (int c = 0; c < NSL; ++c) {
                 tma_load_2d(sm.q[c], &tm_q, &sm.bar_q, 64 * c, qrow);
-                tma_load_2d(sm.dO[c], &tm_do, &sm.bar_q, 64 * c, qrow);
+                tma_load_2d(sm.dO[c], &tm_do, &sm.bar_q, 64 * c, dorow);
             }
             HalfIter it{ents, ne, 0, 0, 0};
             int r64, m2;
@@ -752,21 +761,14 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     float* di_p = (float*)(b + P->L.di_p);
     uint32_t* dmax = (uint32_t*)(b + P->L.dmax);
     int* err = (int*)(b + P->L.err);
+    const bool f32 = P->p.out_dtype == PRISM_F32;
     cudaMemsetAsync(dmax, 0, sizeof(uint32_t) * g.heads, s);
-    const dim3 gmax(296, g.heads);
-    const dim3 gpre((unsigned)((g.N + 7) / 8), g.heads);
-    P->launches += 4;
     {
-    PrismProf prof(P, PRISM_STAGE_BWD_PRE, s);
-    if (P->p.out_dtype == PRISM_F32) {
-        k_bwd_absmax<float><<<gmax, 256, 0, s>>>((const float*)dO, dmax, g.N * HD);
-        k_bwd_pre<float><<<gpre, 256, 0, s>>>((const float*)dO, (const float*)O, lse, src, dmax, dOp, lse_p,
-                                              di_p, g.N, HD, err);
-    } else {
-        k_bwd_absmax<__nv_bfloat16><<<gmax, 256, 0, s>>>((const __nv_bfloat16*)dO, dmax, g.N * HD);
-        k_bwd_pre<__nv_bfloat16><<<gpre, 256, 0, s>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)O, lse,
-                                                      src, dmax, dOp, lse_p, di_p, g.N, HD, err);
-    }
+        PrismProf prof(P, PRISM_STAGE_BWD_PRE, s);
+        const dim3 gmax(296, g.heads);
+        if (f32) k_bwd_absmax<float><<<gmax, 256, 0, s>>>((const float*)dO, dmax, g.N * HD);
+        else k_bwd_absmax<__nv_bfloat16><<<gmax, 256, 0, s>>>((const __nv_bfloat16*)dO, dmax, g.N * HD);
+        P->launches += 1;
     }
     BwdArgs a{};
     a.src = src;
@@ -775,66 +777,83 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     a.dmax = dmax;
     a.N = g.N;
     a.NT = g.NT;
-    a.out_f32 = P->p.out_dtype == PRISM_F32;
+    a.out_f32 = f32;
     a.scale_log2 = kLog2e / sqrtf((float)HD);
     a.inv_sqrt_d = 1.f / sqrtf((float)HD);
     a.err = err;
-    // dK, dV (and for head_dim 128 dQ) per key tile over the transposed lists
+    a.lbase = (const int*)P->lists;
+    const int64_t* loff = (const int64_t*)(b + P->L.loff);
     constexpr bool FUSE = HD == 128;
-    a.ptr = (const int*)(b + P->L.kt_ptr);
-    a.ent = (const int*)(b + P->L.kt_ent);
-    a.out0 = dK;
-    a.out1 = dV;
     static_assert(epilogue_fits<HD, FUSE>(), "dK/dV staging does not fit in the Q/dO/dS buffers");
     float* dq_acc = (float*)(b + P->L.dq_acc);
     float* dk_acc = (float*)(b + P->L.dk_acc);
     float* dv_acc = (float*)(b + P->L.dv_acc);
-    const size_t acc_bytes = sizeof(float) * (size_t)g.heads * g.N * HD;
     const int sm1 = (int)sizeof(DkdvSmem<HD, FUSE>) + 1024;
+    const int sm2 = (int)sizeof(DqSmem<HD>) + 1024;
     if (cudaFuncSetAttribute(k_bwd_dkdv<HD, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1) != cudaSuccess)
+        return PRISM_ERR_CUDA;
+    if (!FUSE &&
+        cudaFuncSetAttribute(k_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2) != cudaSuccess)
         return PRISM_ERR_CUDA;
     // chunks of kChunkTiles query tiles (65536 tokens): about 32 MB of dQ
     // accumulator per chunk, so the reduce-adds of the CTAs in flight stay in L2
     a.CQ = kChunkTiles;
     const unsigned chunks = (unsigned)((g.NT + kChunkTiles - 1) / kChunkTiles);
-    const dim3 gfin((unsigned)((g.N + 7) / 8), g.heads);
-    P->launches += 1;
-    {
-        PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
-        if (FUSE) cudaMemsetAsync(dq_acc, 0, acc_bytes, s);
-        cudaMemsetAsync(dk_acc, 0, acc_bytes, s);
-        cudaMemsetAsync(dv_acc, 0, acc_bytes, s);
-        k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, chunks, g.heads), FUSE ? 480 : 352, sm1, s>>>(
-            P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, P->tm_dk, P->tm_dv, a);
-        if (a.out_f32)
-            k_acc_finalize<float><<<gfin, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (float*)dK, dv_acc, 1.f / kPScale,
-                                                       (float*)dV, src, dmax, g.N, HD, err);
-        else
-            k_acc_finalize<__nv_bfloat16><<<gfin, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (__nv_bfloat16*)dK, dv_acc,
-                                                               1.f / kPScale, (__nv_bfloat16*)dV, src, dmax, g.N,
-                                                               HD, err);
-    }
-    if (FUSE) {
-        PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
-        if (a.out_f32)
-            k_acc_finalize<float><<<gfin, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (float*)dQ, nullptr, 0.f, nullptr,
-                                                       src, dmax, g.N, HD, err);
-        else
-            k_acc_finalize<__nv_bfloat16><<<gfin, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (__nv_bfloat16*)dQ, nullptr,
-                                                               0.f, nullptr, src, dmax, g.N, HD, err);
-        return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
-    }
-    // dQ per query tile over the forward lists (head_dim 64)
-    a.ptr = (const int*)(b + P->L.qt_ptr);
-    a.ent = (const int*)(b + P->L.qt_ent);
-    a.out0 = dQ;
-    a.out1 = nullptr;
-    const int sm2 = (int)sizeof(DqSmem<HD>) + 1024;
-    if (cudaFuncSetAttribute(k_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2) != cudaSuccess)
-        return PRISM_ERR_CUDA;
-    {
-        PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
-        k_bwd_dq<HD><<<dim3(g.NT, g.heads), 192, sm2, s>>>(P->tm_q, P->tm_do, P->tm_k64, P->tm_v64, a);
+    // the dO copy and the accumulators hold one group of heads: the groups run in turn
+    for (int h0 = 0; h0 < g.heads; h0 += g.GH) {
+        const int nh = std::min(g.GH, g.heads - h0);
+        const size_t acc_bytes = sizeof(float) * (size_t)nh * g.N * HD;
+        const dim3 grows((unsigned)((g.N + 7) / 8), nh);
+        a.h0 = h0;
+        {
+            PrismProf prof(P, PRISM_STAGE_BWD_PRE, s);
+            if (f32)
+                k_bwd_pre<float><<<grows, 256, 0, s>>>((const float*)dO, (const float*)O, lse, src, dmax, dOp, lse_p,
+                                                       di_p, g.N, HD, h0, err);
+            else
+                k_bwd_pre<__nv_bfloat16><<<grows, 256, 0, s>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)O,
+                                                               lse, src, dmax, dOp, lse_p, di_p, g.N, HD, h0, err);
+        }
+        // dK, dV (and for head_dim 128 dQ) per key tile over the transposed lists
+        a.ptr = (const int*)(b + P->L.kt_ptr);
+        a.ent_off = loff + LIST_BWD * (size_t)g.heads;
+        a.out0 = dK;
+        a.out1 = dV;
+        {
+            PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
+            if (FUSE) cudaMemsetAsync(dq_acc, 0, acc_bytes, s);
+            cudaMemsetAsync(dk_acc, 0, acc_bytes, s);
+            cudaMemsetAsync(dv_acc, 0, acc_bytes, s);
+            k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, chunks, nh), FUSE ? 480 : 352, sm1, s>>>(
+                P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, P->tm_dk, P->tm_dv, a);
+            if (f32)
+                k_acc_finalize<float><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (float*)dK, dv_acc, 1.f / kPScale,
+                                                            (float*)dV, src, dmax, g.N, HD, h0, err);
+            else
+                k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (__nv_bfloat16*)dK, dv_acc,
+                                                                    1.f / kPScale, (__nv_bfloat16*)dV, src, dmax,
+                                                                    g.N, HD, h0, err);
+        }
+        {
+            PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
+            if (FUSE) {
+                if (f32)
+                    k_acc_finalize<float><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (float*)dQ, nullptr, 0.f,
+                                                                nullptr, src, dmax, g.N, HD, h0, err);
+                else
+                    k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (__nv_bfloat16*)dQ,
+                                                                        nullptr, 0.f, nullptr, src, dmax, g.N, HD,
+                                                                        h0, err);
+            } else {
+                // dQ per query tile over the forward lists (head_dim 64)
+                a.ptr = (const int*)(b + P->L.qt_ptr);
+                a.ent_off = loff + LIST_FWD * (size_t)g.heads;
+                a.out0 = dQ;
+                a.out1 = nullptr;
+                k_bwd_dq<HD><<<dim3(g.NT, nh), 192, sm2, s>>>(P->tm_q, P->tm_do, P->tm_k64, P->tm_v64, a);
+            }
+        }
+        P->launches += 4;
     }
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }

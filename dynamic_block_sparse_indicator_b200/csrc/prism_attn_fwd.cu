@@ -30,6 +30,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "prism_dev.cuh"
 #include "prism_internal.h"
 
@@ -75,7 +77,9 @@ struct FwdSmem {
 
 struct FwdArgs {
     const int* qt_ptr;     // [heads][NT + 1]
-    const int* qt_ent;     // [heads][NT * NT]
+    const int* lbase;      // index lists; head h's tile list starts at lbase + qt_off[h]
+    const int64_t* qt_off; // [heads]
+    int h0;                // first head of this launch (grid y = heads h0, h0 + 1, ...)
     const int* src;        // [heads][N]
     void* O;               // [heads][N][HD] raster order
     float* lse;            // [heads][N]
@@ -85,7 +89,7 @@ struct FwdArgs {
     float scale_log2;      // log2(e) / sqrt(HD)
     int key_lo, key_hi;    // this pass's key tiles [key_lo, key_hi)
     int first, last;       // first pass (no state to merge), last pass (write O and LSE)
-    float* st_o;           // [heads][N][HD] running O (unnormalised, relative to 2^m), block order
+    float* st_o;           // [group heads][N][HD] running O (unnormalised, relative to 2^m), block order
     float* st_m;           // [heads][N] running max (log2 units, P scale included)
     float* st_l;           // [heads][N] running sum
     int* err;
@@ -160,13 +164,13 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     FwdSmem<HD>& sm = *reinterpret_cast<FwdSmem<HD>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NSL = HD / 64;
-    const int t = blockIdx.x, h = blockIdx.y;
+    const int t = blockIdx.x, h = a.h0 + blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         // this pass visits the key tiles of [key_lo, key_hi) of the tile's ascending list
         const int p0 = a.qt_ptr[(size_t)h * (a.NT + 1) + t];
         const int n0 = a.qt_ptr[(size_t)h * (a.NT + 1) + t + 1] - p0;
-        const int* all = a.qt_ent + (size_t)h * a.NT * a.NT + p0;
+        const int* all = a.lbase + a.qt_off[h] + p0;
         const int lo = fwd_lower_bound(all, n0, a.key_lo);
         sm.e0 = p0 + lo;
         sm.n = fwd_lower_bound(all, n0, a.key_hi) - lo;
@@ -191,7 +195,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int n = sm.n;
-    const int* ents = a.qt_ent + (size_t)h * a.NT * a.NT + sm.e0;
+    const int* ents = a.lbase + a.qt_off[h] + sm.e0;
     // TMEM columns: S of group g at 128 g; O of group g at 256 + HD g
     constexpr uint32_t TO = 256;
     const int64_t qrow0 = (int64_t)h * a.N + (int64_t)t * 128;
@@ -371,7 +375,8 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         named_bar(1 + (warp & 3), 64);
         const int row_perm = t * 128 + r;
-        const size_t prow = (size_t)h * a.N + (size_t)row_perm;   // block order (running state)
+        const size_t prow = (size_t)h * a.N + (size_t)row_perm;   // block order (running max, sum)
+        const size_t grow = (size_t)(h - a.h0) * a.N + (size_t)row_perm;   // the group's running O
         if (fin) {
             // this pass: (O_0 2^(m_0 - m_c) + O_1 2^(m_1 - m_c), l_c) relative to 2^m_c
             const float m0 = has0 ? xm[r] : -INFINITY, m1 = has1 ? xm[128 + r] : -INFINITY;
@@ -409,7 +414,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     x[e] = v;
                 }
                 if (use_s) {
-                    const float4* sp = reinterpret_cast<const float4*>(a.st_o + prow * HD + c0);
+                    const float4* sp = reinterpret_cast<const float4*>(a.st_o + grow * HD + c0);
                     #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float4 y = sp[e];
@@ -420,7 +425,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     }
                 }
                 if (!a.last) {
-                    float4* sp = reinterpret_cast<float4*>(a.st_o + prow * HD + c0);
+                    float4* sp = reinterpret_cast<float4*>(a.st_o + grow * HD + c0);
                     #pragma unroll
                     for (int e = 0; e < 8; ++e) sp[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
                 } else if (a.out_f32) {
@@ -473,7 +478,8 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
     FwdArgs a;
     char* b = P->ws;
     a.qt_ptr = (const int*)(b + P->L.qt_ptr);
-    a.qt_ent = (const int*)(b + P->L.qt_ent);
+    a.lbase = (const int*)P->lists;
+    a.qt_off = (const int64_t*)(b + P->L.loff) + LIST_FWD * (size_t)g.heads;
     a.src = (const int*)(b + P->L.src);
     a.O = O;
     a.lse = lse;
@@ -491,17 +497,24 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
     if (cudaFuncSetAttribute(k_attn_fwd<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PRISM_ERR_CUDA;
     const int passes = (g.NT + kFwdKeyChunk - 1) / kFwdKeyChunk;
+    // one pass: every head in one launch (no running state); several passes: the
+    // running O lives in a head group's scratch, so the groups run one after another
+    const int gh = passes == 1 ? g.heads : g.GH;
     {
         PrismProf prof(P, PRISM_STAGE_FWD, s);
-        for (int c = 0; c < passes; ++c) {
-            a.key_lo = c * kFwdKeyChunk;
-            a.key_hi = c + 1 == passes ? g.NT : (c + 1) * kFwdKeyChunk;
-            a.first = c == 0;
-            a.last = c + 1 == passes;
-            k_attn_fwd<HD><<<dim3(g.NT, g.heads), FWD_THREADS, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+        for (int h0 = 0; h0 < g.heads; h0 += gh) {
+            const int nh = std::min(gh, g.heads - h0);
+            a.h0 = h0;
+            for (int c = 0; c < passes; ++c) {
+                a.key_lo = c * kFwdKeyChunk;
+                a.key_hi = c + 1 == passes ? g.NT : (c + 1) * kFwdKeyChunk;
+                a.first = c == 0;
+                a.last = c + 1 == passes;
+                k_attn_fwd<HD><<<dim3(g.NT, nh), FWD_THREADS, smem, s>>>(P->tm_q, P->tm_k, P->tm_v, a);
+                P->launches += 1;
+            }
         }
     }
-    P->launches += passes;
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 

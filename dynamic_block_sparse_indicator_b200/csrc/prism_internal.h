@@ -21,7 +21,12 @@ struct Geom {
     int NB;               // max blocks per head = N / 64
     int NT;               // 128-token tiles per head = N / 128
     int WORDS;            // 32-bit words per selection-bitmap row = ceil(NB / 32)
+    int GH;               // heads per group of the forward-state / gradient scratch
+    int SEL_ROWS;         // CTAs of the selection kernel when a block row is staged in global memory (0: shared)
 };
+
+// Kinds of index lists (offset tables loff[kind][heads], in ints from the list base).
+enum { LIST_CSR = 0, LIST_CSC = 1, LIST_FWD = 2, LIST_BWD = 3, LIST_KINDS = 4 };
 
 // Byte offsets of the workspace regions (each 256-byte aligned).
 struct Layout {
@@ -43,16 +48,20 @@ struct Layout {
     size_t src;                         // int32[heads][N]        raster token of each slot
     size_t qbar, kbar;                  // float[heads][NB][D]
     size_t sel, selT;                   // uint32[heads][NB][WORDS]
-    size_t row_ptr, col_idx;            // int32[heads][NB + 1], int32[heads][NB * NB]
-    size_t col_ptr, row_idx;            // CSC
-    size_t qt_ptr, qt_ent;              // int32[heads][NT + 1], int32[heads][NT * NT]
-    size_t kt_ptr, kt_ent;              // (forward / backward tile lists)
-    size_t qp, kp, vp, dop;             // fp16[heads][N][D] block-ordered copies
+    size_t row_ptr, col_ptr;            // int32[heads][NB + 1]  CSR / CSC row pointers
+    size_t qt_ptr, kt_ptr;              // int32[heads][NT + 1]  forward / backward tile-list pointers
+    size_t loff;                        // int64[LIST_KINDS][heads] list offsets (ints from the list base)
+    size_t selrow;                      // float[SEL_ROWS][NB + NB/32 + 1]: staged block rows (SEL_ROWS > 0)
+    size_t qp, kp, vp;                  // fp16[heads][N][D] block-ordered copies
+    size_t dop;                         // fp16[GH][N][D] block-ordered dO of a head group
     size_t lse_p, di_p;                 // float[heads][N] (backward, block order)
     size_t dmax;                        // uint32[heads]: max |dO| bits (backward scaling)
-    size_t dq_acc;                      // float[heads][N][D]: dQ accumulated in block order
-    size_t dk_acc, dv_acc;              // float[heads][N][D]: dK, dV accumulated in block order
-    size_t total;
+    size_t dq_acc;                      // float[GH][N][D]: dQ (and the forward's pass state) of a head group
+    size_t dk_acc, dv_acc;              // float[GH][N][D]: dK, dV of a head group, block order
+    size_t core;                        // bytes up to here: everything but the index lists
+    size_t col_idx, row_idx;            // lists inside the workspace (one-call plans):
+    size_t qt_ent, kt_ent;              // int32[heads][NB * NB] x 2, int32[heads][NT * NT] x 2
+    size_t total;                       // core + the lists at their dense bound
 };
 
 Geom make_geom(const prism_params* p);
@@ -70,10 +79,15 @@ struct prism_plan_s {
     int device;
     int has_audio;
     int has_cuts;             // adaptive temporal boundaries in force (computed or imported)
+    char* lists;              // base of the index lists: inside ws (one-call) or the caller's list buffer
+    int lists_ready;          // lists built (attention calls need them)
+    int64_t list_len[prism::LIST_KINDS];  // ints per kind over all heads (packed lists)
+    std::vector<int64_t> loff_host;       // [LIST_KINDS][heads] offsets uploaded to L.loff
     CUtensorMap tm_q, tm_k, tm_v, tm_do;       // 2D [heads*N, D] fp16, 128-row boxes, 128B swizzle
     CUtensorMap tm_q64, tm_k64, tm_v64, tm_do64;  // the same with 64-row boxes
-    CUtensorMap tm_dq;                            // fp32 dQ accumulator, 32-row boxes, no swizzle
+    CUtensorMap tm_dq;                            // fp32 dQ accumulator [GH*N, D], 32-row boxes, no swizzle
     CUtensorMap tm_dk, tm_dv;                     // fp32 dK, dV accumulators, the same boxes
+    // tm_do / tm_do64 cover the head group's dO copy: [GH*N, D]
     int64_t launches;                             // kernels launched so far
     int profile;                                  // per-stage event timing on?
     struct Timed { int stage; cudaEvent_t a, b; };

@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -41,6 +42,14 @@ namespace prism {
 // ------------------------------------------------------------------ geometry
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The selection kernel stages one query block's row of block probabilities in
+// shared memory up to kSelSmemRow blocks (192 KB); longer rows (grids above
+// 3.1M tokens, e.g. a native 4K layer) go to a global-memory row per CTA of a
+// grid-stride launch of kSelGlobalCtas CTAs.
+constexpr int kSelSmemRow = 48 * 1024;
+constexpr int kSelGlobalCtas = 296;
+constexpr int kMaxBlocks = 1 << 18;          // N / 64 limit: 16.7M tokens per head
+
 Geom make_geom(const prism_params* p) {
     Geom g{};
     g.T = p->T; g.H = p->H; g.W = p->W; g.heads = p->heads; g.D = p->head_dim; g.dtype = p->dtype;
@@ -50,6 +59,13 @@ Geom make_geom(const prism_params* p) {
     g.NB = (int)(g.N / 64);
     g.NT = (int)(g.N / 128);
     g.WORDS = (g.NB + 31) / 32;
+    // The forward's pass state and the backward's fp32 accumulators and fp16 dO
+    // are sized for a group of heads walked in sequence: at least 2M tokens per
+    // group (about 16K query tiles per launch, many waves on 148 SMs), one head
+    // at a time above that (the 1M-token layer: two heads, 3.6 GB instead of
+    // 72 GB for 40 heads).
+    g.GH = (int)std::min<int64_t>(p->heads, std::max<int64_t>(1, ((int64_t)1 << 21) / g.N));
+    g.SEL_ROWS = g.NB > kSelSmemRow ? kSelGlobalCtas : 0;
     return g;
 }
 
@@ -58,6 +74,7 @@ Layout make_layout(const Geom& g) {
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
     const size_t H = (size_t)g.heads, NB = (size_t)g.NB, NT = (size_t)g.NT, N = (size_t)g.N;
+    const size_t GH = (size_t)g.GH;
     L.err = take(16);
     L.araw = take(sizeof(double) * g.Nz);
     L.abar = take(sizeof(float) * g.Nz);
@@ -80,23 +97,26 @@ Layout make_layout(const Geom& g) {
     L.sel = take(sizeof(uint32_t) * H * NB * g.WORDS);
     L.selT = take(sizeof(uint32_t) * H * NB * g.WORDS);
     L.row_ptr = take(sizeof(int) * H * (NB + 1));
-    L.col_idx = take(sizeof(int) * H * NB * NB);
     L.col_ptr = take(sizeof(int) * H * (NB + 1));
-    L.row_idx = take(sizeof(int) * H * NB * NB);
     L.qt_ptr = take(sizeof(int) * H * (NT + 1));
-    L.qt_ent = take(sizeof(int) * H * NT * NT);
     L.kt_ptr = take(sizeof(int) * H * (NT + 1));
-    L.kt_ent = take(sizeof(int) * H * NT * NT);
+    L.loff = take(sizeof(int64_t) * LIST_KINDS * H);
+    L.selrow = take(sizeof(float) * (size_t)g.SEL_ROWS * (NB + NB / 32 + 1));
     L.qp = take(2 * H * N * g.D);
     L.kp = take(2 * H * N * g.D);
     L.vp = take(2 * H * N * g.D);
-    L.dop = take(2 * H * N * g.D);
+    L.dop = take(2 * GH * N * g.D);
     L.lse_p = take(sizeof(float) * H * N);
     L.di_p = take(sizeof(float) * H * N);
     L.dmax = take(sizeof(uint32_t) * H);
-    L.dq_acc = take(sizeof(float) * H * N * g.D);
-    L.dk_acc = take(sizeof(float) * H * N * g.D);
-    L.dv_acc = take(sizeof(float) * H * N * g.D);
+    L.dq_acc = take(sizeof(float) * GH * N * g.D);
+    L.dk_acc = take(sizeof(float) * GH * N * g.D);
+    L.dv_acc = take(sizeof(float) * GH * N * g.D);
+    L.core = off;
+    L.col_idx = take(sizeof(int) * H * NB * NB);
+    L.row_idx = take(sizeof(int) * H * NB * NB);
+    L.qt_ent = take(sizeof(int) * H * NT * NT);
+    L.kt_ent = take(sizeof(int) * H * NT * NT);
     L.total = off;
     return L;
 }
@@ -123,8 +143,7 @@ int validate_params(const prism_params* p) {
     if (!(p->tau256 >= 0.f && p->tau128 >= p->tau256 && p->tau128 <= 1e30f))
         return PRISM_ERR_INVALID_ARG;
     const int64_t N = (int64_t)p->T * p->H * p->W;
-    // one query-block row of block probabilities is staged in shared memory
-    if (N / 64 > 48 * 1024) return PRISM_ERR_INVALID_ARG;
+    if (N / 64 > kMaxBlocks) return PRISM_ERR_INVALID_ARG;
     if ((int64_t)p->heads * N >= (int64_t)1 << 31) return PRISM_ERR_INVALID_ARG;
     return PRISM_OK;
 }
@@ -165,13 +184,13 @@ struct DevPlan {
     uint32_t* sel;
     uint32_t* selT;
     int* row_ptr;
-    int* col_idx;
     int* col_ptr;
-    int* row_idx;
     int* qt_ptr;
-    int* qt_ent;
     int* kt_ptr;
-    int* kt_ent;
+    int* lbase;            // index lists: kind k of head h starts at lbase + loff[k * heads + h]
+    int64_t* loff;
+    float* selrow;         // staged block rows of the selection (SEL_ROWS > 0)
+    int SEL_ROWS;
     __half* qp;
     __half* kp;
     __half* vp;
@@ -208,13 +227,13 @@ static DevPlan dev_plan(const prism_plan_s* P) {
     d.sel = (uint32_t*)(b + L.sel);
     d.selT = (uint32_t*)(b + L.selT);
     d.row_ptr = (int*)(b + L.row_ptr);
-    d.col_idx = (int*)(b + L.col_idx);
     d.col_ptr = (int*)(b + L.col_ptr);
-    d.row_idx = (int*)(b + L.row_idx);
     d.qt_ptr = (int*)(b + L.qt_ptr);
-    d.qt_ent = (int*)(b + L.qt_ent);
     d.kt_ptr = (int*)(b + L.kt_ptr);
-    d.kt_ent = (int*)(b + L.kt_ent);
+    d.lbase = (int*)P->lists;
+    d.loff = (int64_t*)(b + L.loff);
+    d.selrow = (float*)(b + L.selrow);
+    d.SEL_ROWS = g.SEL_ROWS;
     d.qp = (__half*)(b + L.qp);
     d.kp = (__half*)(b + L.kp);
     d.vp = (__half*)(b + L.vp);
@@ -944,20 +963,19 @@ constexpr int SEL_THREADS = 512;
 
 __device__ __forceinline__ uint32_t fkey(float x) { return __float_as_uint(x); }
 
+// One query block's row: prow holds the row's logits then probabilities (NB
+// floats), tiecnt the per-word tie counts (NB / 32 + 1 ints); both in shared or
+// global memory.  Called by every thread of the CTA.
 template <int D>
-__global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, float top_k_frac, float top_p) {
-    extern __shared__ float prow[];                 // [NB] logits, then probabilities
-    __shared__ float redf[SEL_THREADS / 32];
-    __shared__ int redi[SEL_THREADS / 32];
-    __shared__ int tiecnt[48 * 1024 / 32 + 1];
-    const int i = blockIdx.x, h = blockIdx.y;
+__device__ void select_row(const DevPlan& d, int i, int h, float* prow, int* tiecnt, float* redf, int* redi,
+                           int top_k, float top_k_frac, float top_p) {
     const int nb = d.nblocks[h];
     int* rowcnt = d.row_ptr + (size_t)h * (d.NB + 1);
     if (i >= nb) {                                  // rows past the head's blocks: empty
         if (threadIdx.x == 0) rowcnt[i] = 0;
         uint32_t* row = d.sel + ((size_t)h * d.NB + i) * d.WORDS;
         for (int w = threadIdx.x; w < d.WORDS; w += SEL_THREADS) row[w] = 0u;
-        return;
+        return;                                     // uniform: i and h are the CTA's
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int PL = D / 32;
@@ -1085,6 +1103,32 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, fl
     if (threadIdx.x == 0) rowcnt[i] = cnt;
 }
 
+// One CTA per (query block, head), the row staged in shared memory.
+template <int D>
+__global__ void __launch_bounds__(SEL_THREADS) k_select(DevPlan d, int top_k, float top_k_frac, float top_p) {
+    extern __shared__ float prow[];                 // [NB] row, then [NB / 32 + 1] tie counts
+    __shared__ float redf[SEL_THREADS / 32];
+    __shared__ int redi[SEL_THREADS / 32];
+    select_row<D>(d, blockIdx.x, blockIdx.y, prow, reinterpret_cast<int*>(prow + d.NB), redf, redi, top_k,
+                  top_k_frac, top_p);
+}
+
+// Rows longer than shared memory holds: a grid-stride loop over (query block,
+// head), each CTA staging its rows in its own slice of global scratch (read
+// back from L2 by the bisections).
+template <int D>
+__global__ void __launch_bounds__(SEL_THREADS) k_select_global(DevPlan d, int top_k, float top_k_frac, float top_p) {
+    __shared__ float redf[SEL_THREADS / 32];
+    __shared__ int redi[SEL_THREADS / 32];
+    float* prow = d.selrow + (size_t)blockIdx.x * (d.NB + d.NB / 32 + 1);
+    int* tiecnt = reinterpret_cast<int*>(prow + d.NB);
+    const int64_t rows = (int64_t)d.NB * d.heads;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        select_row<D>(d, (int)(r % d.NB), (int)(r / d.NB), prow, tiecnt, redf, redi, top_k, top_k_frac, top_p);
+        __syncthreads();                            // the row's scratch is reused by the next row
+    }
+}
+
 // Bitmap popcount per row (used for imported selections and for the transpose).
 __global__ void k_row_popc(const uint32_t* __restrict__ bits, int* __restrict__ cnt, const int* nblocks,
                            int NB, int WORDS) {
@@ -1144,15 +1188,15 @@ __global__ void __launch_bounds__(1024) k_scan_heads(int* a, int n) {
 
 // Bitmap rows -> ascending index lists (CSR from sel, CSC from selT).
 __global__ void k_fill_lists(const uint32_t* __restrict__ bits, const int* __restrict__ ptr,
-                             int* __restrict__ idx, const int* nblocks, int NB, int WORDS,
-                             int* err) {
+                             int* __restrict__ lbase, const int64_t* __restrict__ loff, const int* nblocks,
+                             int NB, int WORDS, int* err) {
     const int i = blockIdx.x, h = blockIdx.y;
     const int nb = nblocks[h];
     if (i >= nb) return;
     const int lane = threadIdx.x;
     const uint32_t* r = bits + ((size_t)h * NB + i) * WORDS;
     const int* p = ptr + (size_t)h * (NB + 1);
-    int* out = idx + (size_t)h * NB * NB;
+    int* out = lbase + loff[h];
     int base = p[i];
     const int end = p[i + 1];
     const int nw = (nb + 31) / 32;
@@ -1190,8 +1234,8 @@ __device__ __forceinline__ int bit_of(const uint32_t* rowbits, int j) {
 template <bool FILL>
 __global__ void __launch_bounds__(256) k_tile_lists(const uint32_t* __restrict__ bits,
                                                     const int* __restrict__ t64, int* ptr,
-                                                    int* ent, int NB, int NT, int WORDS,
-                                                    int transposed, int* err) {
+                                                    int* lbase, const int64_t* __restrict__ loff, int NB, int NT,
+                                                    int WORDS, int transposed, int* err) {
     __shared__ int red[256];
     const int t = blockIdx.x, h = blockIdx.y;
     const int* tb = t64 + (size_t)h * NB;
@@ -1231,7 +1275,7 @@ __global__ void __launch_bounds__(256) k_tile_lists(const uint32_t* __restrict__
     }
     int pos = p[t] + red[threadIdx.x] - cnt;
     const int end = p[t + 1];
-    int* e = ent + (size_t)h * NT * NT;
+    int* e = lbase + loff[h];
     for (int o = c0; o < c1; ++o) {
         const int mk = mask_of(o);
         if (mk) {
@@ -1314,7 +1358,9 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
     if (st) return st;
     Geom g = make_geom(p);
     Layout L = make_layout(g);
-    if (ws_bytes < L.total) return PRISM_ERR_WORKSPACE;
+    // a workspace with room for the lists at their dense bound plans in one call;
+    // one with room for the core alone leaves the lists to prism_plan_attach_lists
+    if (ws_bytes < L.core) return PRISM_ERR_WORKSPACE;
     prism_plan_s* P = new (std::nothrow) prism_plan_s();
     if (!P) return PRISM_ERR_CUDA;
     P->p = *p;
@@ -1323,19 +1369,22 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
     P->ws = static_cast<char*>(workspace);
     P->ws_bytes = ws_bytes;
     P->profile = g_profile_plans;
+    P->lists = ws_bytes >= L.total ? P->ws + L.col_idx : nullptr;
+    P->lists_ready = 0;
     cudaGetDevice(&P->device);
-    const int64_t rows = (int64_t)g.heads * g.N;
+    const int64_t rows = (int64_t)g.heads * g.N;      // Q, K, V copies: every head
+    const int64_t grows = (int64_t)g.GH * g.N;        // dO copy and accumulators: one head group
     st = make_tmap(&P->tm_q, P->ws + L.qp, rows, g.D, 128);
     if (!st) st = make_tmap(&P->tm_k, P->ws + L.kp, rows, g.D, 128);
     if (!st) st = make_tmap(&P->tm_v, P->ws + L.vp, rows, g.D, 128);
-    if (!st) st = make_tmap(&P->tm_do, P->ws + L.dop, rows, g.D, 128);
+    if (!st) st = make_tmap(&P->tm_do, P->ws + L.dop, grows, g.D, 128);
     if (!st) st = make_tmap(&P->tm_q64, P->ws + L.qp, rows, g.D, 64);
     if (!st) st = make_tmap(&P->tm_k64, P->ws + L.kp, rows, g.D, 64);
     if (!st) st = make_tmap(&P->tm_v64, P->ws + L.vp, rows, g.D, 64);
-    if (!st) st = make_tmap(&P->tm_do64, P->ws + L.dop, rows, g.D, 64);
-    if (!st) st = make_tmap_f32(&P->tm_dq, P->ws + L.dq_acc, rows, g.D, 32);
-    if (!st) st = make_tmap_f32(&P->tm_dk, P->ws + L.dk_acc, rows, g.D, 32);
-    if (!st) st = make_tmap_f32(&P->tm_dv, P->ws + L.dv_acc, rows, g.D, 32);
+    if (!st) st = make_tmap(&P->tm_do64, P->ws + L.dop, grows, g.D, 64);
+    if (!st) st = make_tmap_f32(&P->tm_dq, P->ws + L.dq_acc, grows, g.D, 32);
+    if (!st) st = make_tmap_f32(&P->tm_dk, P->ws + L.dk_acc, grows, g.D, 32);
+    if (!st) st = make_tmap_f32(&P->tm_dv, P->ws + L.dv_acc, grows, g.D, 32);
     if (st) { delete P; return st; }
     *outP = P;
     return PRISM_OK;
@@ -1365,23 +1414,36 @@ static void launch_gather(prism_plan_s* P, const DevPlan& d, const void* Q, cons
     k_gather_pool<T, D><<<dim3(g.NB, g.heads), 256, 0, s>>>(d, (const T*)Q, (const T*)K, (const T*)V);
 }
 
-static void launch_lists(prism_plan_s* P, const DevPlan& d, cudaStream_t s) {
+// Counts and pointers of the index lists (CSR rows already counted by the
+// selection or the imported bitmap's popcount; the CSC from the transpose; the
+// forward and backward tile lists per 128-token tile), each scanned per head:
+// ptr[h][n] then holds the head's list length.
+static void launch_list_counts(prism_plan_s* P, const DevPlan& d, cudaStream_t s) {
     const Geom& g = P->g;
-    // CSR from sel (row counts already in row_ptr[0..NB))
     k_scan_heads<<<g.heads, 1024, 0, s>>>(d.row_ptr, g.NB);
-    k_fill_lists<<<dim3(g.NB, g.heads), 32, 0, s>>>(d.sel, d.row_ptr, d.col_idx, d.nblocks, g.NB, g.WORDS, d.err);
-    // transpose and CSC
     k_transpose_bits<<<dim3(g.WORDS, g.WORDS, g.heads), 32, 0, s>>>(d);
     k_row_popc<<<dim3((g.NB + 255) / 256, g.heads), 256, 0, s>>>(d.selT, d.col_ptr, d.nblocks, g.NB, g.WORDS);
     k_scan_heads<<<g.heads, 1024, 0, s>>>(d.col_ptr, g.NB);
-    k_fill_lists<<<dim3(g.NB, g.heads), 32, 0, s>>>(d.selT, d.col_ptr, d.row_idx, d.nblocks, g.NB, g.WORDS, d.err);
-    // tile lists (forward from sel, backward from selT)
-    k_tile_lists<false><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.sel, d.t64_blk, d.qt_ptr, d.qt_ent, g.NB, g.NT, g.WORDS, 0, d.err);
+    k_tile_lists<false><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.sel, d.t64_blk, d.qt_ptr, nullptr, nullptr, g.NB, g.NT,
+                                                             g.WORDS, 0, d.err);
     k_scan_heads<<<g.heads, 1024, 0, s>>>(d.qt_ptr, g.NT);
-    k_tile_lists<true><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.sel, d.t64_blk, d.qt_ptr, d.qt_ent, g.NB, g.NT, g.WORDS, 0, d.err);
-    k_tile_lists<false><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.selT, d.t64_blk, d.kt_ptr, d.kt_ent, g.NB, g.NT, g.WORDS, 1, d.err);
+    k_tile_lists<false><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.selT, d.t64_blk, d.kt_ptr, nullptr, nullptr, g.NB, g.NT,
+                                                             g.WORDS, 1, d.err);
     k_scan_heads<<<g.heads, 1024, 0, s>>>(d.kt_ptr, g.NT);
-    k_tile_lists<true><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.selT, d.t64_blk, d.kt_ptr, d.kt_ent, g.NB, g.NT, g.WORDS, 1, d.err);
+}
+
+// The lists themselves, at the offsets in d.loff.
+static void launch_list_fill(prism_plan_s* P, const DevPlan& d, cudaStream_t s) {
+    const Geom& g = P->g;
+    const int64_t H = g.heads;
+    k_fill_lists<<<dim3(g.NB, g.heads), 32, 0, s>>>(d.sel, d.row_ptr, d.lbase, d.loff + LIST_CSR * H, d.nblocks,
+                                                    g.NB, g.WORDS, d.err);
+    k_fill_lists<<<dim3(g.NB, g.heads), 32, 0, s>>>(d.selT, d.col_ptr, d.lbase, d.loff + LIST_CSC * H, d.nblocks,
+                                                    g.NB, g.WORDS, d.err);
+    k_tile_lists<true><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.sel, d.t64_blk, d.qt_ptr, d.lbase, d.loff + LIST_FWD * H,
+                                                            g.NB, g.NT, g.WORDS, 0, d.err);
+    k_tile_lists<true><<<dim3(g.NT, g.heads), 256, 0, s>>>(d.selT, d.t64_blk, d.kt_ptr, d.lbase, d.loff + LIST_BWD * H,
+                                                            g.NB, g.NT, g.WORDS, 1, d.err);
 }
 
 static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V, const float* amap,
@@ -1439,8 +1501,13 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
     }
     PrismProf prof_sel(P, PRISM_STAGE_PLAN_SELECT, s);
     if (!given_sel) {
-        const size_t sm = sizeof(float) * g.NB;
-        if (g.D == 128) {
+        const size_t sm = sizeof(float) * ((size_t)g.NB + g.NB / 32 + 1);
+        if (g.SEL_ROWS > 0) {
+            if (g.D == 128)
+                k_select_global<128><<<g.SEL_ROWS, SEL_THREADS, 0, s>>>(d, p.top_k, p.top_k_frac, p.top_p);
+            else
+                k_select_global<64><<<g.SEL_ROWS, SEL_THREADS, 0, s>>>(d, p.top_k, p.top_k_frac, p.top_p);
+        } else if (g.D == 128) {
             cudaFuncSetAttribute(k_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
             k_select<128><<<dim3(g.NB, g.heads), SEL_THREADS, sm, s>>>(d, p.top_k, p.top_k_frac, p.top_p);
         } else {
@@ -1456,9 +1523,44 @@ static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V
     prof_sel.close();
     {
         PrismProf prof(P, PRISM_STAGE_PLAN_LISTS, s);
-        launch_lists(P, d, s);
+        launch_list_counts(P, d, s);
+        if (P->lists) {
+            // one-call plan: every head's lists at their dense bound inside the workspace
+            const Layout& L = P->L;
+            const int64_t H = g.heads, nb2 = (int64_t)g.NB * g.NB, nt2 = (int64_t)g.NT * g.NT;
+            const int64_t base[LIST_KINDS] = {0, (int64_t)(L.row_idx - L.col_idx) / 4,
+                                              (int64_t)(L.qt_ent - L.col_idx) / 4, (int64_t)(L.kt_ent - L.col_idx) / 4};
+            const int64_t stride[LIST_KINDS] = {nb2, nb2, nt2, nt2};
+            P->loff_host.assign(LIST_KINDS * H, 0);
+            for (int k = 0; k < LIST_KINDS; ++k) {
+                for (int64_t h = 0; h < H; ++h) P->loff_host[k * H + h] = base[k] + h * stride[k];
+                P->list_len[k] = H * stride[k];
+            }
+            cudaMemcpyAsync(P->ws + L.loff, P->loff_host.data(), sizeof(int64_t) * LIST_KINDS * H,
+                            cudaMemcpyHostToDevice, s);
+            launch_list_fill(P, d, s);
+            P->lists_ready = 1;
+        }
     }
     return cuda_status(cudaGetLastError());
+}
+
+// Lengths of the four index lists of every head (synchronises the stream):
+// the totals the per-head scans left in the last pointer of each head.
+static int read_list_lengths(prism_plan_s* P, cudaStream_t s, std::vector<int>* len) {
+    const Geom& g = P->g;
+    const Layout& L = P->L;
+    const size_t H = g.heads;
+    len->assign(LIST_KINDS * H, 0);
+    const size_t ptr_off[LIST_KINDS] = {L.row_ptr, L.col_ptr, L.qt_ptr, L.kt_ptr};
+    const size_t n[LIST_KINDS] = {(size_t)g.NB, (size_t)g.NB, (size_t)g.NT, (size_t)g.NT};
+    for (int k = 0; k < LIST_KINDS; ++k) {
+        const char* src = P->ws + ptr_off[k] + sizeof(int) * n[k];      // ptr[h][n] of head 0
+        if (cudaMemcpy2DAsync(len->data() + k * H, sizeof(int), src, sizeof(int) * (n[k] + 1), sizeof(int), H,
+                              cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return PRISM_ERR_CUDA;
+    }
+    return cudaStreamSynchronize(s) == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
 }  // namespace prism
@@ -1469,6 +1571,55 @@ using namespace prism;
 extern "C" size_t prism_plan_workspace_bytes(const prism_params* p) {
     if (validate_params(p) != PRISM_OK) return 0;
     return make_layout(make_geom(p)).total;
+}
+
+extern "C" size_t prism_plan_core_bytes(const prism_params* p) {
+    if (validate_params(p) != PRISM_OK) return 0;
+    return make_layout(make_geom(p)).core;
+}
+
+extern "C" int prism_plan_list_bytes(prism_plan_t P, size_t* bytes, void* stream) {
+    if (!P || !bytes) return PRISM_ERR_INVALID_ARG;
+    *bytes = 0;
+    if (P->lists_ready) return PRISM_OK;
+    std::vector<int> len;
+    const int st = read_list_lengths(P, static_cast<cudaStream_t>(stream), &len);
+    if (st) return st;
+    // packed: kind after kind, heads in order inside each kind
+    const int64_t H = P->g.heads;
+    P->loff_host.assign(LIST_KINDS * H, 0);
+    int64_t pos = 0;
+    for (int k = 0; k < LIST_KINDS; ++k) {
+        const int64_t k0 = pos;
+        for (int64_t h = 0; h < H; ++h) {
+            P->loff_host[k * H + h] = pos;
+            pos += len[k * H + h];
+        }
+        P->list_len[k] = pos - k0;
+    }
+    *bytes = sizeof(int) * (size_t)std::max<int64_t>(pos, 1);
+    return PRISM_OK;
+}
+
+extern "C" int prism_plan_attach_lists(prism_plan_t P, void* lists, size_t bytes, void* stream) {
+    if (!P || !lists || !aligned16(lists)) return PRISM_ERR_INVALID_ARG;
+    if (P->lists_ready) return PRISM_ERR_INVALID_ARG;
+    if (P->loff_host.empty()) return PRISM_ERR_INVALID_ARG;          // prism_plan_list_bytes first
+    int64_t need = 0;
+    for (int k = 0; k < LIST_KINDS; ++k) need += P->list_len[k];
+    if (bytes < sizeof(int) * (size_t)std::max<int64_t>(need, 1)) return PRISM_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    P->lists = static_cast<char*>(lists);
+    const DevPlan d = dev_plan(P);
+    cudaMemcpyAsync(P->ws + P->L.loff, P->loff_host.data(), sizeof(int64_t) * P->loff_host.size(),
+                    cudaMemcpyHostToDevice, s);
+    {
+        PrismProf prof(P, PRISM_STAGE_PLAN_LISTS, s);
+        launch_list_fill(P, d, s);
+    }
+    P->launches += 4;
+    P->lists_ready = 1;
+    return cuda_status(cudaGetLastError());
 }
 
 extern "C" int prism_plan(const prism_params* p, const void* Q, const void* K, const void* V,
@@ -1523,9 +1674,10 @@ extern "C" size_t prism_plan_item_bytes(prism_plan_t P, int item) {
         case PRISM_ITEM_BLK_START: return 4 * H * (NB + 1);
         case PRISM_ITEM_SEL_BITS: return 4 * H * NB * g.WORDS;
         case PRISM_ITEM_ROW_PTR: return 4 * H * (NB + 1);
-        case PRISM_ITEM_COL_IDX: return 4 * H * NB * NB;
+        case PRISM_ITEM_COL_IDX: return P->lists_ready ? 4 * (size_t)P->list_len[LIST_CSR] : 0;
         case PRISM_ITEM_COL_PTR: return 4 * H * (NB + 1);
-        case PRISM_ITEM_ROW_IDX: return 4 * H * NB * NB;
+        case PRISM_ITEM_ROW_IDX: return P->lists_ready ? 4 * (size_t)P->list_len[LIST_CSC] : 0;
+        case PRISM_ITEM_LIST_OFFSETS: return P->lists_ready ? 8 * LIST_KINDS * H : 0;
         case PRISM_ITEM_QBAR: return 4 * H * NB * g.D;
         case PRISM_ITEM_KBAR: return 4 * H * NB * g.D;
         case PRISM_ITEM_SRC: return 4 * H * (size_t)g.N;
@@ -1543,6 +1695,20 @@ extern "C" int prism_plan_export(prism_plan_t P, int item, void* host_dst, size_
     const size_t need = prism_plan_item_bytes(P, item);
     if (need == 0 || bytes != need) return PRISM_ERR_INVALID_ARG;
     const Layout& L = P->L;
+    const int64_t H = P->g.heads;
+    if (item == PRISM_ITEM_LIST_OFFSETS) {       // host copy: each head's offset inside its kind's list
+        int64_t* out = static_cast<int64_t*>(host_dst);
+        for (int k = 0; k < LIST_KINDS; ++k)
+            for (int64_t h = 0; h < H; ++h) out[k * H + h] = P->loff_host[k * H + h] - P->loff_host[k * H];
+        return PRISM_OK;
+    }
+    if (item == PRISM_ITEM_COL_IDX || item == PRISM_ITEM_ROW_IDX) {
+        const int k = item == PRISM_ITEM_COL_IDX ? LIST_CSR : LIST_CSC;
+        cudaStream_t s = static_cast<cudaStream_t>(stream);
+        if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
+        const char* src = P->lists + sizeof(int) * (size_t)P->loff_host[k * H];
+        return cudaMemcpy(host_dst, src, bytes, cudaMemcpyDeviceToHost) == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+    }
     size_t off;
     switch (item) {
         case PRISM_ITEM_SHAPE_ID: off = L.shape_id; break;
@@ -1550,9 +1716,7 @@ extern "C" int prism_plan_export(prism_plan_t P, int item, void* host_dst, size_
         case PRISM_ITEM_BLK_START: off = L.blk_start; break;
         case PRISM_ITEM_SEL_BITS: off = L.sel; break;
         case PRISM_ITEM_ROW_PTR: off = L.row_ptr; break;
-        case PRISM_ITEM_COL_IDX: off = L.col_idx; break;
         case PRISM_ITEM_COL_PTR: off = L.col_ptr; break;
-        case PRISM_ITEM_ROW_IDX: off = L.row_idx; break;
         case PRISM_ITEM_QBAR: off = L.qbar; break;
         case PRISM_ITEM_KBAR: off = L.kbar; break;
         case PRISM_ITEM_SRC: off = L.src; break;
@@ -1652,14 +1816,14 @@ extern "C" const char* prism_status_string(int st) {
 extern "C" const char* prism_version(void) { return "prism-b200 0.1 sm_100a"; }
 
 extern "C" int prism_attn_fwd(prism_plan_t P, void* O, float* lse, void* stream) {
-    if (!P || !O || !lse) return PRISM_ERR_INVALID_ARG;
+    if (!P || !O || !lse || !P->lists_ready) return PRISM_ERR_INVALID_ARG;
     if (!aligned16(O) || !aligned16(lse)) return PRISM_ERR_INVALID_ARG;
     return prism_launch_attn_fwd(P, O, lse, stream);
 }
 
 extern "C" int prism_attn_bwd(prism_plan_t P, const void* dO, const void* O, const float* lse,
                               void* dQ, void* dK, void* dV, void* stream) {
-    if (!P || !dO || !O || !lse || !dQ || !dK || !dV) return PRISM_ERR_INVALID_ARG;
+    if (!P || !dO || !O || !lse || !dQ || !dK || !dV || !P->lists_ready) return PRISM_ERR_INVALID_ARG;
     if (!aligned16(dO) || !aligned16(O) || !aligned16(lse) || !aligned16(dQ) || !aligned16(dK) ||
         !aligned16(dV))
         return PRISM_ERR_INVALID_ARG;

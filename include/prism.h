@@ -145,12 +145,29 @@ typedef struct prism_params {
 typedef struct prism_plan_s* prism_plan_t;
 
 /*
- * Bytes of device workspace prism_plan() needs for `p` (an upper bound: the
- * block count and the number of selected pairs are data dependent; the bound
- * assumes N/64 blocks per head and every pair selected).  Returns 0 when `p`
- * is invalid.
+ * Workspace.  The plan's index lists (the CSR key-block lists of S_i, their
+ * transpose, and the per-128-token-tile lists the attention kernels walk) are
+ * data dependent.  Two ways to hold them:
+ *   one call   a workspace of prism_plan_workspace_bytes(p) bytes holds the
+ *              lists at their dense bound (N/64 blocks per head, every pair
+ *              selected: 2 (N/64)^2 + 2 (N/128)^2 ints per head, 2.5 GB for one
+ *              1M-token head); prism_plan() returns a plan ready for attention.
+ *   two calls  a workspace of prism_plan_core_bytes(p) bytes (the rest: block-
+ *              ordered Q, K, V copies, statistics, bitmaps, and a head group's
+ *              forward-state and gradient scratch) makes prism_plan() stop after
+ *              counting the lists; prism_plan_list_bytes() then gives their exact
+ *              size (it synchronises the stream) and prism_plan_attach_lists()
+ *              builds them in a second buffer the caller allocates and keeps
+ *              alive with the workspace.  A 40-head 1M-token layer needs about
+ *              62 GB this way at the 2K workload's 92% pair density.
+ * Both return 0 when `p` is invalid.  Scratch that only the forward and the
+ * backward use (the forward's state between key-range passes, the fp32 dQ, dK,
+ * dV accumulators, the fp16 dO copy) is sized for a group of heads those calls
+ * walk one group after another: heads of at least 2M tokens together, one head
+ * at a time for larger heads.
  */
 PRISM_API size_t prism_plan_workspace_bytes(const prism_params* p);
+PRISM_API size_t prism_plan_core_bytes(const prism_params* p);
 
 /*
  * prism_plan -- stages 1-3 of Algorithm 1 for every head.
@@ -172,7 +189,9 @@ PRISM_API size_t prism_plan_workspace_bytes(const prism_params* p);
  *   a_map      device fp32 [T][H][W], the cached audio-to-video cross-attention
  *              output norm of the previous layer, shared by all heads; NULL for
  *              the first layer (then g_d = r_{v,d} + eps).
- *   workspace  device, >= prism_plan_workspace_bytes(p) bytes, 256-B aligned.
+ *   workspace  device, 256-B aligned: >= prism_plan_workspace_bytes(p) bytes for
+ *              a plan ready at once, >= prism_plan_core_bytes(p) to attach the
+ *              lists later (prism_plan_attach_lists).
  *   stream     cudaStream_t.
  *   out        receives the plan handle (host memory, freed by
  *              prism_plan_destroy).  Left NULL on error.
@@ -209,6 +228,19 @@ PRISM_API int prism_plan_import_cuts(const prism_params* p, const void* Q, const
                                      const uint8_t* shape_id, const uint8_t* zone_cut,
                                      const uint8_t* shape_id2, const uint32_t* sel, void* workspace,
                                      size_t ws_bytes, void* stream, prism_plan_t* out);
+
+/*
+ * prism_plan_list_bytes -- for a plan made with a core-only workspace: the
+ *   bytes its index lists need (0 once they are built).  Synchronises `stream`
+ *   (reads each head's list lengths).
+ * prism_plan_attach_lists -- builds the lists in `lists` (device, 16-byte
+ *   aligned, >= prism_plan_list_bytes bytes, kept alive by the caller as long
+ *   as the plan); asynchronous on `stream`.  prism_attn_fwd / prism_attn_bwd
+ *   return PRISM_ERR_INVALID_ARG for a plan whose lists are not built;
+ *   PRISM_ERR_WORKSPACE if `bytes` is too small.
+ */
+PRISM_API int prism_plan_list_bytes(prism_plan_t plan, size_t* bytes, void* stream);
+PRISM_API int prism_plan_attach_lists(prism_plan_t plan, void* lists, size_t bytes, void* stream);
 
 /*
  * prism_attn_fwd -- stages 4-5: for every query token q of block i,
@@ -304,9 +336,9 @@ PRISM_API int prism_status_read(int32_t* dev_status, int32_t* site, void* stream
 #define PRISM_ITEM_BLK_START  2  /* int32  [heads][N/64 + 1] (first nblocks+1)  */
 #define PRISM_ITEM_SEL_BITS   3  /* uint32 [heads][N/64][ceil(N/64 / 32)]       */
 #define PRISM_ITEM_ROW_PTR    4  /* int32  [heads][N/64 + 1]  CSR              */
-#define PRISM_ITEM_COL_IDX    5  /* int32  [heads][(N/64)^2]  CSR (row_ptr'd)  */
+#define PRISM_ITEM_COL_IDX    5  /* int32  CSR key blocks: row i of head h at LIST_OFFSETS[0][h] + row_ptr[h][i] */
 #define PRISM_ITEM_COL_PTR    6  /* int32  [heads][N/64 + 1]  CSC              */
-#define PRISM_ITEM_ROW_IDX    7  /* int32  [heads][(N/64)^2]  CSC              */
+#define PRISM_ITEM_ROW_IDX    7  /* int32  CSC query blocks: column j of head h at LIST_OFFSETS[1][h] + col_ptr[h][j] */
 #define PRISM_ITEM_QBAR       8  /* fp32   [heads][N/64][head_dim]             */
 #define PRISM_ITEM_KBAR       9  /* fp32   [heads][N/64][head_dim]             */
 #define PRISM_ITEM_SRC       10  /* int32  [heads][N] raster token of each permuted slot */
@@ -315,7 +347,9 @@ PRISM_API int prism_status_read(int32_t* dev_status, int32_t* site, void* stream
 #define PRISM_ITEM_SHAPE_ID2 13  /* uint8  [heads][Nz] shape of the part after the split (255 if none) */
 #define PRISM_ITEM_ZONE_ENERGY 14 /* fp32  [heads][Nz][7] frame-difference energies e_t */
 #define PRISM_ITEM_REGION_STATS 15 /* fp32 [heads][Nz][2][4] the parts' statistics (split zones) */
-#define PRISM_ITEM_COUNT     16
+#define PRISM_ITEM_LIST_OFFSETS 16 /* int64 [4][heads]: head h's first entry in the CSR, CSC,
+                                      forward and backward tile lists */
+#define PRISM_ITEM_COUNT     17
 
 /* Bytes of an item (0 for an unknown item). */
 PRISM_API size_t prism_plan_item_bytes(prism_plan_t plan, int item);

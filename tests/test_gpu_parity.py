@@ -56,9 +56,10 @@ def _check_plan(pl, orc, w, heads, k=None, p=None):
     kbar = pl.export("kbar").reshape(heads, NB, w.head_dim)
     bits = pl.export("sel_bits").reshape(heads, NB, WORDS)
     row_ptr = pl.export("row_ptr").reshape(heads, NB + 1)
-    col_idx = pl.export("col_idx").reshape(heads, NB * NB)
+    col_idx = pl.export("col_idx")
+    loff = pl.export("list_offsets").reshape(4, heads)
     col_ptr = pl.export("col_ptr").reshape(heads, NB + 1)
-    row_idx = pl.export("row_idx").reshape(heads, NB * NB)
+    row_idx = pl.export("row_idx")
     exact_rows = []
     for h in range(heads):
         o = orc[h]
@@ -83,13 +84,15 @@ def _check_plan(pl, orc, w, heads, k=None, p=None):
                 exact.add(i)
         # CSR rows = the bitmap rows; CSC = the transpose
         for i in range(nb):
-            np.testing.assert_array_equal(col_idx[h, row_ptr[h, i]:row_ptr[h, i + 1]], gsets[i])
+            np.testing.assert_array_equal(col_idx[loff[0, h] + row_ptr[h, i]:loff[0, h] + row_ptr[h, i + 1]],
+                                          gsets[i])
         cols = [[] for _ in range(nb)]
         for i in range(nb):
             for j in gsets[i]:
                 cols[j].append(i)
         for j in range(nb):
-            np.testing.assert_array_equal(row_idx[h, col_ptr[h, j]:col_ptr[h, j + 1]], cols[j])
+            np.testing.assert_array_equal(row_idx[loff[1, h] + col_ptr[h, j]:loff[1, h] + col_ptr[h, j + 1]],
+                                          cols[j])
         exact_rows.append(exact)
     return exact_rows
 
@@ -116,12 +119,19 @@ CASES = {
 }
 
 
-@pytest.mark.parametrize("name", list(CASES))
-def test_plan_and_forward_match_oracle(name, cuda_device):
+PLAN_RUNS = [(n, False) for n in CASES] + [("tiny_fp32_d64", True), ("grid16x32x32_bf16_d128", True)]
+
+
+@pytest.mark.parametrize("name,compact", PLAN_RUNS)
+def test_plan_and_forward_match_oracle(name, compact, cuda_device):
+    """compact: the workspace holds the core only and the index lists go to a
+    buffer sized from their counts (prism_plan_list_bytes / attach_lists)."""
     w, heads, audio = CASES[name]
     Q, K, V, a = _inputs(w, heads, audio)
     Qd, Kd, Vd, ad = _to_dev(Q, K, V, a)
-    pl = _lib.plan(Qd, Kd, Vd, ad, _params(w, heads))
+    pl = _lib.plan(Qd, Kd, Vd, ad, _params(w, heads), compact=compact)
+    if compact:
+        assert pl._ws.numel() < _lib.workspace_bytes(_params(w, heads)) and pl._lists is not None
     O, lse = pl.attn_fwd()
     torch.cuda.synchronize()
     assert pl.status() == 0
