@@ -59,6 +59,8 @@ def args_():
     ap.add_argument("--av-tokens", type=int, default=1000,
                     help="audio tokens of the guidance-map producer leg (the pages: under 1K)")
     ap.add_argument("--no-av", action="store_true", help="skip the guidance-map producer leg")
+    ap.add_argument("--no-op", action="store_true",
+                    help="skip the leg at the pages' operating point (k = 5%% of the blocks, Top-p 0.2)")
     ap.add_argument("--sweep", action="store_true",
                     help="the 2K inference sweep instead of the step: forward only on grid 64x88x152, "
                          "peaked (Q, K x3) and diffuse (x0.5) logits, Top-k 8/16/32 x Top-p 0.8/0.9/0.95")
@@ -251,6 +253,49 @@ def oracle_head_ms(Qh, Kh, Vh, dOh, a, w, budget_s, seed=0, variant=None):
             f"{len(sel)} query blocks ({100 * pi_s / pairs.sum():.2f}% of the selected pairs), "
             f"attention time extrapolated by pair share")
     return 1e3 * (t_plan + t_attn), desc, threads
+
+
+def operating_point_leg(Q, K, V, dO, amap, w, h, peak, steps=3):
+    """The pages' operating point (k = 5% of each head's blocks, Top-p 0.2; page
+    paper.rainbus.top, "方法步骤详情") on one head of the same workload: plan +
+    forward + backward per head-layer, 1 warm-up and `steps` timed steps (CUDA
+    events), TFLOP/s over the selected pairs' 14 D Pi flops of the attention."""
+    import torch
+    from dynamic_block_sparse_indicator_b200 import _lib
+    prm = _lib.make_params(w.T, w.H, w.W, 1, w.head_dim, _lib.PRISM_BF16, 0, 0.2, w.eps,
+                           out_dtype=_lib.PRISM_F32, top_k_frac=0.05)
+    sl = slice(h, h + 1)
+    ws = torch.empty(_lib.core_bytes(prm), dtype=torch.uint8, device=Q.device)
+
+    def run(prof):
+        pl = _lib.plan(Q[sl], K[sl], V[sl], amap, prm, workspace=ws, compact=True)
+        if prof:
+            pl.profile(True)
+        O, lse = pl.attn_fwd()
+        pl.attn_bwd(dO[sl], O, lse)
+        return pl
+
+    pl = run(False)
+    Pi, nb, sel = selected_pairs(pl)
+    del pl
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stage = {}
+    e0.record()
+    plans = [run(True) for _ in range(steps)]
+    e1.record()
+    torch.cuda.synchronize()
+    for pl in plans:
+        for k, (ms, _n) in pl.profile_read().items():
+            stage[k] = stage.get(k, 0.0) + ms / steps
+    ms = e0.elapsed_time(e1) / steps
+    attn = stage["fwd"] + stage["bwd_pre"] + stage["bwd_dkdv"] + stage["bwd_dq"]
+    tf = 14 * w.head_dim * Pi / (attn * 1e-3) / 1e12
+    return {"top_k_frac": 0.05, "top_p": 0.2, "ms_per_head_layer": ms,
+            "stages_ms": {k: stage[k] for k in ("fwd", "bwd_dkdv", "bwd_dq")},
+            "attention_tflops": tf, "frac_of_sustained": tf / peak, "selected_pairs": Pi,
+            "pair_density": Pi / float(w.N) ** 2, "mean_selected_blocks": sel, "blocks_per_head": nb,
+            "note": "plan with the core workspace and index lists sized from their counts"}
 
 
 # ------------------------------------------------------------- main paths
@@ -587,6 +632,10 @@ def run_prism(a, rank, world, local_rank):
         "lists": {"ms": per_head("plan_lists")},
         "hbm_peak_GB/s": hbm, "peak_source": "measured" if pk.get("hbm_gbs") else "fallback",
     }
+    # ------------------------------------------------- the pages' operating point
+    op = None
+    if world == 1 and not a.no_op:
+        op = operating_point_leg(Q, K, V, dO, amap, w, order[a.warmup], peak)
     # ------------------------------------------- dense attention of the same shape
     dense = None
     if world == 1 and not a.no_dense:
@@ -668,6 +717,14 @@ def run_prism(a, rank, world, local_rank):
         ms, desc, threads = oracle_head_ms(host(Q), host(K), host(V), host(dO),
                                            amap.cpu().numpy(), w, a.cpu_seconds, variant=variant_of(a))
         cpu = {"value": ms, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        try:                                      # the same on one core
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                ms1, desc1, _ = oracle_head_ms(host(Q), host(K), host(V), host(dO), amap.cpu().numpy(), w,
+                                               a.cpu_seconds / 2, variant=variant_of(a))
+            cpu["single_core"] = {"value": ms1, "unit": UNIT, "cores": 1, "sample": desc1}
+        except ImportError:
+            cpu["single_core"] = None
     if rank == 0:
         emit({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
               "warmup": a.warmup, "ms_per_step": elapsed_max / a.steps, "higher_is_better": False,
@@ -692,7 +749,8 @@ def run_prism(a, rank, world, local_rank):
                            "traffic": measured_traffic(
                                {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv"}.get(dom, ""))
                            if w.N == 1013760 else None},
-              "plan_kernels": plan_kernels, "dense_same_shape": dense, "guidance_map": av,
+              "plan_kernels": plan_kernels, "dense_same_shape": dense, "operating_point": op,
+              "guidance_map": av,
               "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks})
 
 

@@ -12,6 +12,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libprism.so")
+# the checking build: every gather / scatter / list index bounds-checked on the
+# device (a failed check is PRISM_ERR_DEVICE_CHECK, the access skipped)
+LIB_CHECKS = os.path.join(HERE, "libprism_checks.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
          "-Xcompiler", "-fvisibility=hidden"]
@@ -21,27 +24,29 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib=LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
     deps.append(os.path.join(HERE, "..", "include", "prism.h"))
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build_library(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build_library(force: bool = False, verbose: bool = False, checks: bool = False) -> str:
+    lib = LIB_CHECKS if checks else LIB
+    if not force and not _stale(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp"
-    cmd = [nvcc, *ARCH, *FLAGS, "-DPRISM_BUILD", "-o", tmp, *sources()]
+    tmp = lib + ".tmp"
+    cmd = [nvcc, *ARCH, *FLAGS, "-DPRISM_BUILD", *(["-DPRISM_CHECKS=1"] if checks else []), "-o", tmp,
+           *sources()]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build_library(force="--force" in sys.argv, verbose=True))
+    print(build_library(force="--force" in sys.argv, verbose=True, checks="--checks" in sys.argv))

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, cons
     if (p >= N) return;
     const float sc = ldexpf(1.f, -dscale_exp(dmax[h], err));
     const int64_t n = src[(size_t)h * N + p];
+    if (prism_bad_index(err, n >= 0 && n < N)) return;
     const OT* dr = dO + ((size_t)h * N + n) * HD;
     const OT* orow = O + ((size_t)h * N + n) * HD;
     __half* out = dOp + ((size_t)(h - h0) * N + p) * HD;
@@ -314,6 +315,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             int r64, m2;
             for (int u = 0; it.next(r64, m2); ++u) {
                 const int s = u % DKDV_STAGES;
+                if (prism_bad_index(a.err, r64 >= 0 && r64 < 2 * a.NT)) r64 = 0;   // checking build
                 if (u >= DKDV_STAGES &&
                     !mbar_wait(&sm.st_empty[s], ((u / DKDV_STAGES) - 1) & 1, a.err, 1401)) break;
                 const int64_t qrow = hrow + (int64_t)r64 * 64;
@@ -559,6 +561,7 @@ __global__ void __launch_bounds__(256) k_acc_finalize(const float* __restrict__ 
     if (p >= N) return;
     const float unscale = ldexpf(1.f, dscale_exp(dmax[h], err));
     const int64_t n = src[(size_t)h * N + p];
+    if (prism_bad_index(err, n >= 0 && n < N)) return;
     const size_t ir = ((size_t)(h - h0) * N + p) * HD, orow = ((size_t)h * N + n) * HD;
     for (int c = lane; c < HD; c += 32) out0[orow + c] = (OT)(acc0[ir + c] * (scale0 * unscale));
     if (acc1)
@@ -631,6 +634,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                 const int s = u % BWD_STAGES;
                 if (u >= BWD_STAGES &&
                     !mbar_wait(&sm.st_empty[s], ((u / BWD_STAGES) - 1) & 1, a.err, 2401)) break;
+                if (prism_bad_index(a.err, r64 >= 0 && r64 < 2 * a.NT)) r64 = 0;   // checking build
                 const int krow = (int)(hrow + (int64_t)r64 * 64);
                 mbar_expect_tx(&sm.st_full[s], 2 * NSL * SLAB64);
                 for (int c = 0; c < NSL; ++c) {
@@ -726,7 +730,9 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
             tc_fence_before();
             mbar_arrive(&sm.ds_full[b]);
         }
-        const size_t orow = (size_t)hrow + (size_t)a.src[prow];
+        int srow = a.src[prow];
+        if (prism_bad_index(a.err, srow >= 0 && srow < a.N)) srow = 0;               // checking build
+        const size_t orow = (size_t)hrow + (size_t)srow;
         bool fin = false;
         if (ok && U > 0)
             fin = __all_sync(0xffffffffu, mbar_wait(&sm.dq_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, 2004));

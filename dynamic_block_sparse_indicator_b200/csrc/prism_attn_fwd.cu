@@ -211,7 +211,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 const int s = j % FWD_KST;
                 if (j >= FWD_KST &&
                     !mbar_wait(&sm.k_empty[s], ((j / FWD_KST) - 1) & 1, a.err, 401)) break;
-                const int krow = (int)((int64_t)h * a.N + (int64_t)(ents[j] >> 4) * 128);
+                int kt = ents[j] >> 4;
+                if (prism_bad_index(a.err, kt >= 0 && kt < a.NT)) kt = 0;           // checking build
+                const int krow = (int)((int64_t)h * a.N + (int64_t)kt * 128);
                 mbar_expect_tx(&sm.k_full[s], NSL * SLAB);
                 for (int c = 0; c < NSL; ++c) tma_load_2d(sm.k[s][c], &tm_k, &sm.k_full[s], 64 * c, krow);
             }
@@ -220,7 +222,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 const int s = j % FWD_VST;
                 if (j >= FWD_VST &&
                     !mbar_wait(&sm.v_empty[s], ((j / FWD_VST) - 1) & 1, a.err, 402)) break;
-                const int krow = (int)((int64_t)h * a.N + (int64_t)(ents[j] >> 4) * 128);
+                int kt = ents[j] >> 4;
+                if (prism_bad_index(a.err, kt >= 0 && kt < a.NT)) kt = 0;           // checking build
+                const int krow = (int)((int64_t)h * a.N + (int64_t)kt * 128);
                 mbar_expect_tx(&sm.v_full[s], NSL * SLAB);
                 for (int c = 0; c < NSL; ++c) tma_load_2d(sm.v[s][c], &tm_v, &sm.v_full[s], 64 * c, krow);
             }
@@ -395,7 +399,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const float inv = a.last ? (lt > 0.f ? 1.f / lt : 0.f) : 1.f;
             const float w0 = f0 * fc * inv, w1 = f1 * fc * inv, ws = fs * inv;
             const bool use_s = !a.first && ms != -INFINITY;
-            const size_t orow = a.last ? (size_t)h * a.N + (size_t)a.src[prow] : 0;
+            int srow = a.last ? a.src[prow] : 0;
+            if (prism_bad_index(a.err, srow >= 0 && srow < a.N)) srow = 0;         // checking build
+            const size_t orow = a.last ? (size_t)h * a.N + (size_t)srow : 0;
             tc_fence_after();
             constexpr int OC = HD / 2;             // output columns written by each group
             #pragma unroll

@@ -451,8 +451,11 @@ extern "C" int prism_av_norm(int64_t N, int32_t M, int32_t heads, int32_t head_d
     if (major != 10 || minor != 0) return PRISM_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int f32 = hhat_dtype == PRISM_F32;
-    return head_dim == 128 ? launch<128>(N, M, heads, Qv, Ka, Va, a_map, h_hat, f32, dev_status, s)
-                           : launch<64>(N, M, heads, Qv, Ka, Va, a_map, h_hat, f32, dev_status, s);
+    nvtxRangePushA("prism av norm");
+    const int st = head_dim == 128 ? launch<128>(N, M, heads, Qv, Ka, Va, a_map, h_hat, f32, dev_status, s)
+                                   : launch<64>(N, M, heads, Qv, Ka, Va, a_map, h_hat, f32, dev_status, s);
+    nvtxRangePop();
+    return st;
 }
 
 extern "C" int prism_status_read(int32_t* dev_status, int32_t* site, void* stream) {

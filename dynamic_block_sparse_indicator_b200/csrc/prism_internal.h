@@ -8,10 +8,28 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <vector>
 
 namespace prism {
+
+// Bounds checks of the gather / scatter / list indices, compiled in with
+// -DPRISM_CHECKS=1 (the library's checking build): a failed check records
+// PRISM_ERR_DEVICE_CHECK in the plan's error word and the caller skips the
+// access; no trap.  Off by default (the checks cost registers in hot loops).
+#ifndef PRISM_CHECKS
+#define PRISM_CHECKS 0
+#endif
+#if defined(__CUDACC__)
+__device__ __forceinline__ bool prism_bad_index(int* err, bool in_bounds) {
+    if (PRISM_CHECKS && !in_bounds) {
+        atomicCAS(err, 0, PRISM_ERR_DEVICE_CHECK);
+        return true;
+    }
+    return false;
+}
+#endif
 
 // Geometry derived from prism_params.
 struct Geom {
@@ -94,22 +112,38 @@ struct prism_plan_s {
     std::vector<Timed> timed;                     // pending event pairs
 };
 
-// Event pair around one launch when profiling is on.
+// Names of the stages as NVTX ranges (a profiler's timeline shows each launch
+// group under the stage that issued it).
+inline const char* prism_stage_name(int stage) {
+    static const char* names[PRISM_STAGE_COUNT] = {
+        "prism fwd", "prism bwd pre", "prism bwd dK dV", "prism bwd dQ", "prism plan stats",
+        "prism plan shapes", "prism plan gather", "prism plan select", "prism plan lists"};
+    return stage >= 0 && stage < PRISM_STAGE_COUNT ? names[stage] : "prism";
+}
+
+// Around one stage's launches: an NVTX range always, and an event pair on the
+// stream when profiling is on.
 struct PrismProf {
     prism_plan_s* P;
     int stage;
     cudaStream_t s;
     cudaEvent_t a = nullptr, b = nullptr;
+    bool open = true;
     PrismProf(prism_plan_s* P_, int stage_, cudaStream_t s_) : P(P_), stage(stage_), s(s_) {
+        nvtxRangePushA(prism_stage_name(stage));
         if (P->profile && cudaEventCreate(&a) == cudaSuccess && cudaEventCreate(&b) == cudaSuccess)
             cudaEventRecord(a, s);
     }
-    // records the closing event now (idempotent; the destructor calls it)
+    // ends the range and records the closing event now (idempotent; the destructor calls it)
     void close() {
         if (a && b) {
             cudaEventRecord(b, s);
             P->timed.push_back({stage, a, b});
             a = b = nullptr;
+        }
+        if (open) {
+            nvtxRangePop();
+            open = false;
         }
     }
     ~PrismProf() { close(); }

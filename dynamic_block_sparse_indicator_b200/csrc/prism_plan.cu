@@ -892,6 +892,7 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
         const int lw = r % bw, lh = (r / bw) % bh, lt = r / (bw * bh);
         const int64_t n = ((int64_t)(8 * zt + toff + kt * bt + lt) * d.H + 8 * zh + kh * bh + lh) * d.W +
                           8 * zw + kw * bw + lw;
+        if (prism_bad_index(d.err, n >= 0 && n < d.N && start + r < d.N)) continue;
         const size_t so = hoff + (size_t)n * D + (size_t)c * EPC;
         const size_t dst = hoff + (size_t)(start + r) * D + (size_t)c * EPC;
         if (c == 0) d.src[(size_t)h * d.N + start + r] = (int)n;
