@@ -79,7 +79,10 @@ def test_forty_heads_at_one_million_tokens_in_one_call(cuda_device):
     assert heads == 40
     prm = _params(w, heads, out_dtype=_lib.PRISM_BF16)
     core = _lib.core_bytes(prm)
-    assert _lib.workspace_bytes(prm) > 180e9 > core            # the dense bound would not fit
+    # Q, K, V, dO, O, dQ, dK, dV in bf16 and the LSE: with the lists at their dense
+    # bound the workspace would not fit beside them on a 180 GB GPU
+    tensors = 8 * heads * w.N * w.head_dim * 2 + 4 * heads * w.N
+    assert _lib.workspace_bytes(prm) + tensors > 180e9
     Q, K, V = syn.make_qkv(w, device="cuda")
     dO = syn.make_dout(w, device="cuda", out_dtype=torch.bfloat16)
     a = syn.make_amap(w, device="cuda")
@@ -89,6 +92,7 @@ def test_forty_heads_at_one_million_tokens_in_one_call(cuda_device):
     torch.cuda.synchronize()
     assert pl.status() == _lib.PRISM_OK
     used = core + pl._lists.numel()
+    assert used + tensors < 180e9
     keep = {h: [t[h].clone() for t in (O, lse, dQ, dK, dV)] for h in (0, heads - 1)}
     items = {k: pl.export(k) for k in ("shape_id", "src")}
     del pl, O, lse, dQ, dK, dV
