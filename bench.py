@@ -330,8 +330,13 @@ def run_reference(a, rank, world):
         vals.append(ms)
     wall = time.perf_counter() - t0
     v = float(np.mean(vals))
+    # value: the oracle's time for a whole head-layer, extrapolated from each
+    # step's bounded sample (a full 1M-token head takes the oracle hours);
+    # ms_per_step: what each step actually took, so steps x ms_per_step is the
+    # timed region this run really spent
     emit({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
-          "steps": a.steps, "warmup": a.warmup, "ms_per_step": v, "higher_is_better": False,
+          "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * wall / max(a.steps, 1),
+          "value_extrapolated_from_sample": True, "higher_is_better": False,
           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
           "config": {"workload": w.name(), "grid": [w.T, w.H, w.W], "tokens": w.N,
                      "head_dim": w.head_dim, "top_k": w.top_k, "top_p": w.top_p,
