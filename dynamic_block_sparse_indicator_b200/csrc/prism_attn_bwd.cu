@@ -86,7 +86,8 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, cons
                                                  const float* __restrict__ lse,
                                                  const int* __restrict__ src, const uint32_t* dmax,
                                                  __half* __restrict__ dOp, float* __restrict__ lse_p,
-                                                 float* __restrict__ di_p, int64_t N, int HD, int h0, int* err) {
+                                                 float* __restrict__ di_p, int64_t N, int HD, int h0,
+                                                 const uint32_t* __restrict__ qkv_max, int* err) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t p = (int64_t)blockIdx.x * 8 + warp;
     const int h = h0 + blockIdx.y;                   // dOp holds the head group [h0, h0 + gridDim.y)
@@ -105,11 +106,13 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, cons
     }
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     // stored for the softmax of the backward kernels, which form P' = 2^15 P as
-    // ex2(s * log2(e)/sqrt(d) + lse_p) and dS = P' (dP 2^-15 + di_p) with one
-    // fused multiply-add each: lse_p = 15 - LSE log2(e), di_p = -D 2^-15 (D in
-    // the dO scale)
+    // ex2(s * log2(e)/sqrt(d) + lse_p) and dS' = P' (dP_copy 2^-30 + di_p) with one
+    // fused multiply-add each: lse_p = 15 - LSE log2(e), di_p = -D 2^-15 2^-ev with
+    // D in the dO scale and 2^ev = 2^(15 - sv) the V copy's scale, so that dS' =
+    // dS 2^-E 2^-ev: normalised by dO's and V's magnitudes whatever they are (dP
+    // of the copies carries 2^sv, and 2^-30 = 2^-15 2^-sv 2^-ev)
     if (lane == 0) {
-        di_p[(size_t)h * N + p] = -acc * sc * kPScaleInv;
+        di_p[(size_t)h * N + p] = -acc * sc * ldexpf(kPScaleInv, qkv_shift(qkv_max[h * 3 + 2]) - 15);
         lse_p[(size_t)h * N + p] = kPScaleLog2 - lse[(size_t)h * N + n] * kLog2e;
     }
 }
@@ -163,6 +166,7 @@ struct BwdArgs {
     int NT;
     int out_f32;
     float scale_log2;      // log2(e) / sqrt(d)
+    const uint32_t* qkv_max;  // [heads][3]: the copies' per-head scales (qkv_shift)
     float inv_sqrt_d;
     int CQ;                // query tiles per chunk of the dK/dV grid
     int* err;
@@ -302,6 +306,10 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     const uint32_t tmem = sm.tmem_base;
     const int64_t hrow = (int64_t)h * a.N;               // Q, K, V copies and per-row terms
     const int64_t grow = (int64_t)(h - a.h0) * a.N;      // dO copy and accumulators (head group)
+    // the copies carry Q 2^sq, K 2^sk, V 2^sv: the logit scale and dP undo them
+    // (dK and dQ are unscaled when the accumulators are finalised)
+    const float scale_log2 = ldexpf(a.scale_log2, -(qkv_shift(a.qkv_max[h * 3]) + qkv_shift(a.qkv_max[h * 3 + 1])));
+    constexpr float pinv = kPScaleInv * kPScaleInv;      // 2^-30: dS' = dS 2^-E 2^-ev (see k_bwd_pre)
 
     if (warp == W_PROD) {
         if (lane == 0 && U > 0) {
@@ -449,12 +457,12 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                         // P' = 2^15 P: the dV operand, normal in fp16 down to P = 2^-29
                         // (dV is unscaled at the end); dS = P (dP - D) = P' (dP 2^-15 - D 2^-15)
                         float x0_, x1_;
-                        ffma2(x0_, x1_, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), a.scale_log2,
-                              a.scale_log2, lq[2 * e], lq[2 * e + 1]);
+                        ffma2(x0_, x1_, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), scale_log2,
+                              scale_log2, lq[2 * e], lq[2 * e + 1]);
                         p0 = ex2(x0_);
                         p1 = ex2(x1_);
                         float t0, t1;
-                        ffma2(t0, t1, __uint_as_float(dp[c]), __uint_as_float(dp[c + 1]), kPScaleInv, kPScaleInv,
+                        ffma2(t0, t1, __uint_as_float(dp[c]), __uint_as_float(dp[c + 1]), pinv, pinv,
                               dq[2 * e], dq[2 * e + 1]);
                         fmul2(d0, d1, p0, p1, t0, t1);
                     }
@@ -554,12 +562,17 @@ template <typename OT>
 __global__ void __launch_bounds__(256) k_acc_finalize(const float* __restrict__ acc0, float scale0, OT* __restrict__ out0,
                                                       const float* __restrict__ acc1, float scale1,
                                                       OT* __restrict__ out1, const int* __restrict__ src,
-                                                      const uint32_t* dmax, int64_t N, int HD, int h0, int* err) {
+                                                      const uint32_t* dmax, int64_t N, int HD, int h0,
+                                                      const uint32_t* __restrict__ qkv_max, int which0, int* err) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t p = (int64_t)blockIdx.x * 8 + warp;
     const int h = h0 + blockIdx.y;                   // accumulators hold the head group from h0
     if (p >= N) return;
     const float unscale = ldexpf(1.f, dscale_exp(dmax[h], err));
+    // acc0 came from dS' (normalised by V's scale 2^ev) and the Q copy (dK) or the K
+    // copy (dQ): undo both
+    if (which0 >= 0)
+        scale0 = ldexpf(scale0, 15 - qkv_shift(qkv_max[h * 3 + 2]) - qkv_shift(qkv_max[h * 3 + which0]));
     const int64_t n = src[(size_t)h * N + p];
     if (prism_bad_index(err, n >= 0 && n < N)) return;
     const size_t ir = ((size_t)(h - h0) * N + p) * HD, orow = ((size_t)h * N + n) * HD;
@@ -618,6 +631,10 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
     const uint32_t tmem = sm.tmem_base;
     const int64_t hrow = (int64_t)h * a.N;                  // Q, K, V copies, per-row terms
     const int64_t grow = (int64_t)(h - a.h0) * a.N;         // the head group's dO copy
+    // the copies' scales: logits, dP and dQ (= dS K_copy 2^-sk) undo them
+    const int sk = qkv_shift(a.qkv_max[h * 3 + 1]), ev = 15 - qkv_shift(a.qkv_max[h * 3 + 2]);
+    const float scale_log2 = ldexpf(a.scale_log2, -(qkv_shift(a.qkv_max[h * 3]) + sk));
+    constexpr float pinv = kPScaleInv * kPScaleInv;      // 2^-30: dS' = dS 2^-E 2^-ev (see k_bwd_pre)
 
     if (warp == 4) {
         if (lane == 0 && U > 0) {
@@ -717,10 +734,10 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                     float d0 = 0.f, d1 = 0.f;
                     if (valid) {
                         // P' = 2^15 P and dS = P' (dP 2^-15 - D 2^-15), as in the dK/dV kernel
-                        const float p0 = ex2(fmaf(__uint_as_float(sv[c]), a.scale_log2, lse2));
-                        const float p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), a.scale_log2, lse2));
-                        d0 = p0 * fmaf(__uint_as_float(dp[c]), kPScaleInv, di);
-                        d1 = p1 * fmaf(__uint_as_float(dp[c + 1]), kPScaleInv, di);
+                        const float p0 = ex2(fmaf(__uint_as_float(sv[c]), scale_log2, lse2));
+                        const float p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), scale_log2, lse2));
+                        d0 = p0 * fmaf(__uint_as_float(dp[c]), pinv, di);
+                        d1 = p1 * fmaf(__uint_as_float(dp[c + 1]), pinv, di);
                     }
                     wd[e] = pack_f16(d0, d1);
                 }
@@ -744,7 +761,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                 uint32_t o[32];
                 PRISM_TMEM_LD32(tmem + lane_off + TDQ + 32 * c, o);
                 tmem_wait_ld();
-                store_row(a.out0, orow, HD, 32 * c, o, a.inv_sqrt_d * unscale, a.out_f32);
+                store_row(a.out0, orow, HD, 32 * c, o, ldexpf(a.inv_sqrt_d * unscale, ev - sk), a.out_f32);
             }
         } else if (U == 0) {
             zero_row(a.out0, orow, HD, a.out_f32);
@@ -786,6 +803,7 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     a.out_f32 = f32;
     a.scale_log2 = kLog2e / sqrtf((float)HD);
     a.inv_sqrt_d = 1.f / sqrtf((float)HD);
+    a.qkv_max = (const uint32_t*)(b + P->L.qkv_max);
     a.err = err;
     a.lbase = (const int*)P->lists;
     const int64_t* loff = (const int64_t*)(b + P->L.loff);
@@ -815,10 +833,11 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
             PrismProf prof(P, PRISM_STAGE_BWD_PRE, s);
             if (f32)
                 k_bwd_pre<float><<<grows, 256, 0, s>>>((const float*)dO, (const float*)O, lse, src, dmax, dOp, lse_p,
-                                                       di_p, g.N, HD, h0, err);
+                                                       di_p, g.N, HD, h0, a.qkv_max, err);
             else
                 k_bwd_pre<__nv_bfloat16><<<grows, 256, 0, s>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)O,
-                                                               lse, src, dmax, dOp, lse_p, di_p, g.N, HD, h0, err);
+                                                               lse, src, dmax, dOp, lse_p, di_p, g.N, HD, h0,
+                                                               a.qkv_max, err);
         }
         // dK, dV (and for head_dim 128 dQ) per key tile over the transposed lists
         a.ptr = (const int*)(b + P->L.kt_ptr);
@@ -834,22 +853,22 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
                 P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, P->tm_dk, P->tm_dv, a);
             if (f32)
                 k_acc_finalize<float><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (float*)dK, dv_acc, 1.f / kPScale,
-                                                            (float*)dV, src, dmax, g.N, HD, h0, err);
+                                                            (float*)dV, src, dmax, g.N, HD, h0, a.qkv_max, 0, err);
             else
                 k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (__nv_bfloat16*)dK, dv_acc,
                                                                     1.f / kPScale, (__nv_bfloat16*)dV, src, dmax,
-                                                                    g.N, HD, h0, err);
+                                                                    g.N, HD, h0, a.qkv_max, 0, err);
         }
         {
             PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
             if (FUSE) {
                 if (f32)
                     k_acc_finalize<float><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (float*)dQ, nullptr, 0.f,
-                                                                nullptr, src, dmax, g.N, HD, h0, err);
+                                                                nullptr, src, dmax, g.N, HD, h0, a.qkv_max, 1, err);
                 else
                     k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (__nv_bfloat16*)dQ,
                                                                         nullptr, 0.f, nullptr, src, dmax, g.N, HD,
-                                                                        h0, err);
+                                                                        h0, a.qkv_max, 1, err);
             } else {
                 // dQ per query tile over the forward lists (head_dim 64)
                 a.ptr = (const int*)(b + P->L.qt_ptr);

@@ -87,6 +87,7 @@ struct FwdArgs {
     int NT;
     int out_f32;
     float scale_log2;      // log2(e) / sqrt(HD)
+    const uint32_t* qkv_max;  // [heads][3]: the copies' per-head scales (qkv_shift)
     int key_lo, key_hi;    // this pass's key tiles [key_lo, key_hi)
     int first, last;       // first pass (no state to merge), last pass (write O and LSE)
     float* st_o;           // [group heads][N][HD] running O (unnormalised, relative to 2^m), block order
@@ -195,6 +196,10 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int n = sm.n;
+    // the copies carry Q 2^sq, K 2^sk, V 2^sv: the logits' scale and O undo them
+    const int sq = qkv_shift(a.qkv_max[h * 3]), sk = qkv_shift(a.qkv_max[h * 3 + 1]);
+    const float scale_log2 = ldexpf(a.scale_log2, -(sq + sk));
+    const float o_unscale = ldexpf(1.f, -qkv_shift(a.qkv_max[h * 3 + 2]));
     const int* ents = a.lbase + a.qt_off[h] + sm.e0;
     // TMEM columns: S of group g at 128 g; O of group g at 256 + HD g
     constexpr uint32_t TO = 256;
@@ -303,7 +308,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 tmem_wait_ld();
                 mx = fmaxf(mx, max64(sr));
             }
-            mx *= a.scale_log2;
+            mx *= scale_log2;
             const bool first = (cnt == 0) || (m_ref == -INFINITY);
             const float m_new = fmaxf(m_ref, mx);
             if (first) m_ref = m_new;
@@ -318,7 +323,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             // group's P buffer (and the rescale of O_g) wait for the previous product.
             const float neg = kPScaleLog2 - m_ref;
             uint32_t pk1[32], pk0[32];
-            float lsum = exp_p64(sr, v1, a.scale_log2, neg, pk1);
+            float lsum = exp_p64(sr, v1, scale_log2, neg, pk1);
             if (v0) {                              // key half 0 again from TMEM
                 PRISM_TMEM_LD32(tmem + lane_off + scol, (sr + 0));
                 PRISM_TMEM_LD32(tmem + lane_off + scol + 32, (sr + 32));
@@ -327,7 +332,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             // S has been read: the next S of this group may overwrite it
             tc_fence_before();
             mbar_arrive(&sm.s_free[g]);
-            lsum += exp_p64(sr, v0, a.scale_log2, neg, pk0);
+            lsum += exp_p64(sr, v0, scale_log2, neg, pk0);
             // O_g and this group's P buffer were last used by the product of step j - 2
             if (cnt > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g], ((j - 2) >> 1) & 1, a.err, 2))) {
                 ok = false;
@@ -396,7 +401,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const float fc = mc == -INFINITY ? 0.f : ex2(mc - m);
             const float fs = ms == -INFINITY ? 0.f : ex2(ms - m);
             const float lt = lc * fc + ls * fs;
-            const float inv = a.last ? (lt > 0.f ? 1.f / lt : 0.f) : 1.f;
+            const float inv = a.last ? (lt > 0.f ? o_unscale / lt : 0.f) : 1.f;
             const float w0 = f0 * fc * inv, w1 = f1 * fc * inv, ws = fs * inv;
             const bool use_s = !a.first && ms != -INFINITY;
             int srow = a.last ? a.src[prow] : 0;
@@ -493,6 +498,7 @@ static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
     a.NT = g.NT;
     a.out_f32 = P->p.out_dtype == PRISM_F32;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+    a.qkv_max = (const uint32_t*)(b + P->L.qkv_max);
     a.err = (int*)(b + P->L.err);
     // The running state between passes lives in buffers the backward fills only
     // later: the fp32 dQ accumulator (O) and the per-row terms (max, sum).

@@ -31,6 +31,22 @@ __device__ __forceinline__ bool prism_bad_index(int* err, bool in_bounds) {
 }
 #endif
 
+// Per-head input scaling of the fp16 tensor-core copies: Q, K and V of a head
+// are multiplied by exact powers of two 2^shift chosen so that the head's
+// largest magnitude lies in [2^14, 2^15) (below fp16's maximum 65504), so
+// inputs of any finite magnitude keep fp16's relative precision down to 2^-28
+// of the head's maximum.  max_bits holds the head's max |x| as float bits; the
+// kernels undo the shifts exactly (logit scale, O, dQ, dK, dP).
+#if defined(__CUDACC__)
+__device__ __forceinline__ int qkv_shift(uint32_t max_bits) {
+    const float m = __uint_as_float(max_bits);
+    if (!(m > 0.f) || !(m <= 3.402823466e38f)) return 0;    // zero, or not finite (device-checked)
+    int e;
+    frexpf(m, &e);                                          // m in [2^(e-1), 2^e)
+    return 15 - e;
+}
+#endif
+
 // Geometry derived from prism_params.
 struct Geom {
     int T, H, W, heads, D, dtype;
@@ -70,7 +86,8 @@ struct Layout {
     size_t qt_ptr, kt_ptr;              // int32[heads][NT + 1]  forward / backward tile-list pointers
     size_t loff;                        // int64[LIST_KINDS][heads] list offsets (ints from the list base)
     size_t selrow;                      // float[SEL_ROWS][NB + NB/32 + 1]: staged block rows (SEL_ROWS > 0)
-    size_t qp, kp, vp;                  // fp16[heads][N][D] block-ordered copies
+    size_t qkv_max;                     // uint32[heads][3]: max |Q|, |K|, |V| bits (the copies' scaling)
+    size_t qp, kp, vp;                  // fp16[heads][N][D] block-ordered copies, scaled by 2^shift
     size_t dop;                         // fp16[GH][N][D] block-ordered dO of a head group
     size_t lse_p, di_p;                 // float[heads][N] (backward, block order)
     size_t dmax;                        // uint32[heads]: max |dO| bits (backward scaling)

@@ -102,6 +102,7 @@ Layout make_layout(const Geom& g) {
     L.kt_ptr = take(sizeof(int) * H * (NT + 1));
     L.loff = take(sizeof(int64_t) * LIST_KINDS * H);
     L.selrow = take(sizeof(float) * (size_t)g.SEL_ROWS * (NB + NB / 32 + 1));
+    L.qkv_max = take(sizeof(uint32_t) * H * 3);
     L.qp = take(2 * H * N * g.D);
     L.kp = take(2 * H * N * g.D);
     L.vp = take(2 * H * N * g.D);
@@ -191,6 +192,7 @@ struct DevPlan {
     int64_t* loff;
     float* selrow;         // staged block rows of the selection (SEL_ROWS > 0)
     int SEL_ROWS;
+    uint32_t* qkv_max;     // [heads][3] max |Q|, |K|, |V| bits
     __half* qp;
     __half* kp;
     __half* vp;
@@ -233,6 +235,7 @@ static DevPlan dev_plan(const prism_plan_s* P) {
     d.lbase = (int*)P->lists;
     d.loff = (int64_t*)(b + L.loff);
     d.selrow = (float*)(b + L.selrow);
+    d.qkv_max = (uint32_t*)(b + L.qkv_max);
     d.SEL_ROWS = g.SEL_ROWS;
     d.qp = (__half*)(b + L.qp);
     d.kp = (__half*)(b + L.kp);
@@ -835,12 +838,39 @@ __global__ void __launch_bounds__(1024) k_zone_finalize_cut(DevPlan d, ShapeRule
 }
 
 // ================================================================ stage 2
-// The block-ordered copies are fp16: a bf16 value converts exactly when
-// 2^-14 <= |x| <= 65504 (or x = 0), smaller magnitudes round to fp16's
-// subnormal grid (absolute error at most 2^-25), and fp16 operands keep the
-// tensor-core products' rounding error 8x below bf16's.  A value beyond the
-// fp16 range (or a NaN) is a device-check error.
-constexpr float kHalfMax = 65504.f;
+// The block-ordered copies are fp16 (their products' rounding error is 8x below
+// bf16's), each head's Q, K and V scaled by an exact power of two that puts the
+// head's largest magnitude in [2^14, 2^15) (qkv_shift): any finite input keeps
+// fp16's relative precision down to 2^-28 of its head's maximum, and a bf16
+// value converts exactly unless it is that small.  A non-finite input is a
+// device-check error.
+
+// Largest magnitude of each head's Q, K and V (float bits, atomicMax: the bits
+// of non-negative floats order like the values; a NaN's bits exceed infinity's).
+template <typename T>
+__global__ void __launch_bounds__(256) k_qkv_absmax(const T* __restrict__ Q, const T* __restrict__ K,
+                                                    const T* __restrict__ V, uint32_t* __restrict__ mx,
+                                                    int64_t n_per_head, int* err) {
+    const int h = blockIdx.y;
+    const size_t off = (size_t)h * n_per_head;
+    float m[3] = {0.f, 0.f, 0.f};
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_per_head;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float q = fabsf((float)Q[off + i]), k = fabsf((float)K[off + i]), v = fabsf((float)V[off + i]);
+        m[0] = (q > m[0] || q != q) ? q : m[0];
+        m[1] = (k > m[1] || k != k) ? k : m[1];
+        m[2] = (v > m[2] || v != v) ? v : m[2];
+    }
+    #pragma unroll
+    for (int t = 0; t < 3; ++t) {
+        uint32_t b = __float_as_uint(m[t]);
+        for (int o = 16; o > 0; o >>= 1) b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
+        if ((threadIdx.x & 31) == 0) {
+            if (!(b <= 0x7f7fffffu)) atomicCAS(err, 0, PRISM_ERR_DEVICE_CHECK);      // inf or NaN
+            atomicMax(mx + h * 3 + t, b);
+        }
+    }
+}
 
 __device__ __forceinline__ uint32_t ph2(float a, float b) {
     __half2 v = __floats2half2_rn(a, b);
@@ -883,10 +913,12 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
     const int kw = kin % nkw, kh = (kin / nkw) % nkh, kt = kin / (nkw * nkh);
     const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
     const int c = threadIdx.x % CPR, rl = threadIdx.x / CPR;
+    // the copies' exact power-of-two scales (the pooled means use the inputs as they are)
+    const float sq = ldexpf(1.f, qkv_shift(d.qkv_max[h * 3])), sk = ldexpf(1.f, qkv_shift(d.qkv_max[h * 3 + 1])),
+                sv = ldexpf(1.f, qkv_shift(d.qkv_max[h * 3 + 2]));
     float aq[EPC], ak[EPC];
     #pragma unroll
     for (int e = 0; e < EPC; ++e) aq[e] = ak[e] = 0.f;
-    float amax = 0.f;
     const size_t hoff = (size_t)h * d.N * D;
     for (int r = rl; r < vol; r += RP) {
         const int lw = r % bw, lh = (r / bw) % bh, lt = r / (bw * bh);
@@ -923,15 +955,14 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
         uint32_t oq[EPC / 2], ok[EPC / 2], ov[EPC / 2];
         #pragma unroll
         for (int e = 0; e < EPC / 2; ++e) {
-            oq[e] = ph2(fq[2 * e], fq[2 * e + 1]);
-            ok[e] = ph2(fk[2 * e], fk[2 * e + 1]);
-            ov[e] = ph2(fv[2 * e], fv[2 * e + 1]);
+            oq[e] = ph2(fq[2 * e] * sq, fq[2 * e + 1] * sq);
+            ok[e] = ph2(fk[2 * e] * sk, fk[2 * e + 1] * sk);
+            ov[e] = ph2(fv[2 * e] * sv, fv[2 * e + 1] * sv);
         }
         #pragma unroll
         for (int e = 0; e < EPC; ++e) {
             aq[e] += fq[e];
             ak[e] += fk[e];
-            amax = fmaxf(amax, fmaxf(fabsf(fq[e]), fmaxf(fabsf(fk[e]), fabsf(fv[e]))));
         }
         if constexpr (EPC == 8) {
             *reinterpret_cast<uint4*>(d.qp + dst) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
@@ -943,7 +974,6 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
             *reinterpret_cast<uint2*>(d.vp + dst) = make_uint2(ov[0], ov[1]);
         }
     }
-    if (!(amax <= kHalfMax)) dev_fail(d.err, PRISM_ERR_DEVICE_CHECK);   // also catches NaN
     #pragma unroll
     for (int e = 0; e < EPC; ++e) { pq[rl][c * EPC + e] = aq[e]; pk[rl][c * EPC + e] = ak[e]; }
     __syncthreads();
@@ -1412,6 +1442,9 @@ template <typename T, int D>
 static void launch_gather(prism_plan_s* P, const DevPlan& d, const void* Q, const void* K,
                           const void* V, cudaStream_t s) {
     const Geom& g = P->g;
+    cudaMemsetAsync(d.qkv_max, 0, sizeof(uint32_t) * 3 * g.heads, s);
+    k_qkv_absmax<T><<<dim3(296, g.heads), 256, 0, s>>>((const T*)Q, (const T*)K, (const T*)V, d.qkv_max,
+                                                        g.N * D, d.err);
     k_gather_pool<T, D><<<dim3(g.NB, g.heads), 256, 0, s>>>(d, (const T*)Q, (const T*)K, (const T*)V);
 }
 
@@ -1450,10 +1483,10 @@ static void launch_list_fill(prism_plan_s* P, const DevPlan& d, cudaStream_t s) 
 static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V, const float* amap,
                     const uint8_t* given_shapes, const uint32_t* given_sel, cudaStream_t s,
                     const uint8_t* given_cut = nullptr, const uint8_t* given_sid2 = nullptr) {
-    // kernels launched below: audio 1-3, stats 1-2, finalize 1, gather 1, select (or
-    // mask + popcount) 1-2, lists 12
+    // kernels launched below: audio 1-3, stats 1-2, finalize 1, max + gather 2, select
+    // (or mask + popcount) 1-2, list counts 8, list fill 4 (here in one-call plans)
     const int cut_extra = P->has_cuts && !given_shapes ? 1 + (amap ? 1 : 0) : 0;
-    P->launches += (given_shapes ? 0 : (amap ? 3 : 2)) + cut_extra + 2 + (given_sel ? 2 : 1) + 12;
+    P->launches += (given_shapes ? 0 : (amap ? 3 : 2)) + cut_extra + 3 + (given_sel ? 2 : 1) + 8 + (P->lists ? 4 : 0);
     const Geom& g = P->g;
     const prism_params& p = P->p;
     DevPlan d = dev_plan(P);

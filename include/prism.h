@@ -72,12 +72,14 @@ extern "C" {
  *   out_dtype element type of O, dO, dQ, dK, dV: PRISM_BF16 or PRISM_F32.
  *             The tensor-core products take fp16 operands with fp32
  *             accumulation either way; fp32 outputs keep the fp32 accumulators
- *             unrounded.  A bf16 input converts to fp16 exactly when
- *             2^-14 <= |x| <= 65504 (or x = 0); smaller magnitudes round to
- *             fp16's subnormal grid (absolute error at most 2^-25), and a value
- *             beyond 65504 (or a NaN) makes the plan report
- *             PRISM_ERR_DEVICE_CHECK.  dO is scaled per head by an exact power
- *             of two before its conversion, so its magnitude does not matter.
+ *             unrounded.  Each head's Q, K, V and dO are multiplied by exact
+ *             powers of two before their fp16 conversion (Q, K, V: the head's
+ *             largest magnitude into [2^14, 2^15); dO: into [0.5, 1)), and the
+ *             kernels undo the factors exactly: any finite input magnitude is
+ *             accepted, a bf16 value converts exactly unless it lies below
+ *             2^-28 of its head's largest (then it rounds to fp16's subnormal
+ *             grid), and a non-finite input makes the plan report
+ *             PRISM_ERR_DEVICE_CHECK.
  *   top_k     k of Top-k (>= 0); k >= number of blocks keeps every block.
  *   top_p     p of Top-p in [0, 1]; p >= 1 keeps every block, p <= 0 none.
  *             Empty sets (top_k < 1, top_k_frac <= 0 and top_p <= 0) are

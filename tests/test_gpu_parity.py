@@ -252,31 +252,43 @@ def test_full_pipeline_backward_tiny(cuda_device):
                 assert good, f"head {h} {nm} vs {what} inputs: relL2 {rl2:.2e} maxabs {ma:.2e} worst {worst:.2f}"
 
 
-def test_tiny_magnitude_values_follow_the_fp16_bound(cuda_device):
-    """V of magnitude ~1e-6 (bf16 values below fp16's normal range, 2^-14):
-    the tensor-core copies round them to fp16's subnormal grid.  O matches the
-    oracle fed that rounding at the usual bar, and the oracle fed the exact bf16
-    values to within the documented conversion error (at most 2^-25 per value,
-    hence per O element, since each row's softmax weights sum to one) plus the
-    kernel's relative rounding."""
-    w = syn.workload(2, T=8, H=16, W=16)
+def _scaled_run(w, scales):
+    """Plan from the oracle (imported), forward and backward on Q, K, V scaled by
+    exact powers of two; returns the inputs as given and the outputs."""
     Q, K, V = syn.make_qkv(w, heads=1)
-    V = (V.float() * 2.0 ** -20).to(torch.bfloat16)
-    assert float(V.float().abs().max()) < 2.0 ** -14
+    Q, K, V = ((x.float() * f).to(torch.bfloat16) for x, f in zip((Q, K, V), scales))
+    dO = _dout(w, 1)
     q, k, v = (x[0].double().numpy() for x in (Q, K, V))
     o = po.plan_head(q, k, v, None, w.T, w.H, w.W, w.top_k, w.top_p, w.eps)
     NB, WORDS = w.N // 64, (w.N // 64 + 31) // 32
     sid = torch.from_numpy(o["shape_id"].astype(np.uint8)[None]).cuda()
     bits = torch.from_numpy(parity.sets_to_bits(o["sel"], NB, WORDS)[None].view(np.int32)).cuda()
     pl = _lib.plan_import(Q.cuda(), K.cuda(), V.cuda(), sid, bits, _params(w, 1))
-    O, _ = pl.attn_fwd()
+    O, lse = pl.attn_fwd()
+    grads = pl.attn_bwd(dO.cuda(), O, lse)
     torch.cuda.synchronize()
     assert pl.status() == 0
-    O = O[0].double().cpu().numpy()
-    v16 = V[0].to(torch.float16).double().numpy()
-    O16, _ = po.attention_fwd(q, k, v16, o["src"], o["starts"], o["sel"])
-    good, rl2, ma = parity.close(O, O16)
-    assert good, f"O vs fp16-rounded V: relL2 {rl2:.2e} maxabs {ma:.2e}"
-    Oe, _ = po.attention_fwd(q, k, v, o["src"], o["starts"], o["sel"])
-    bound = 2.0 ** -25 + 4e-3 * np.abs(Oe).max()
-    assert np.abs(O - Oe).max() <= bound, f"max |O - O_exact| {np.abs(O - Oe).max():.3e} > {bound:.3e}"
+    host = lambda t: t[0].double().cpu().numpy()
+    return (q, k, v, dO[0].double().numpy(), o), host(O), [host(t) for t in grads]
+
+
+@pytest.mark.parametrize("name,scales", [
+    ("tiny_V", (1.0, 1.0, 2.0 ** -20)),                  # V ~ 1e-6: below fp16's normal range
+    ("huge_V_tiny_Q_huge_K", (2.0 ** -20, 2.0 ** 20, 2.0 ** 20)),   # |K|, |V| ~ 1e6: beyond fp16's 65504
+])
+def test_any_input_magnitude_keeps_the_bar(name, scales, cuda_device):
+    """The fp16 copies are scaled per head by exact powers of two, so inputs far
+    below fp16's normal range or far beyond its largest value meet the usual bar
+    against the oracle on the exact inputs.  Q 2^a, K 2^-a leaves the logits
+    unchanged; O scales with V, dS with V, so dQ with K and V, dK with Q and V,
+    and dV not at all (compared at unit scale)."""
+    w = syn.workload(2, T=8, H=16, W=16)
+    (q, k, v, g, o), O, (dQ, dK, dV) = _scaled_run(w, scales)
+    sq, sk, sv = scales
+    Oo, _ = po.attention_fwd(q, k, v, o["src"], o["starts"], o["sel"])
+    good, rl2, ma = parity.close(O / sv, Oo / sv)
+    assert good, f"{name} O: relL2 {rl2:.2e} maxabs {ma:.2e} (at unit scale)"
+    rQ, rK, rV = po.attention_bwd(q, k, v, g, o["src"], o["starts"], o["sel"])
+    for got, want, f, nm in ((dQ, rQ, sk * sv, "dQ"), (dK, rK, sq * sv, "dK"), (dV, rV, 1.0, "dV")):
+        good, rl2, ma, worst = parity.close_grad(got / f, want / f)
+        assert good, f"{name} {nm}: relL2 {rl2:.2e} maxabs {ma:.2e} (at unit scale)"
