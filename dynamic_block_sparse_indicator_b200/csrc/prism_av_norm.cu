@@ -11,25 +11,22 @@
 // so the work is a dense contraction of 4 N M D flops per head, tensor-bound.
 //
 // Design (B200): one CTA per 128 video tokens walks every head and every
-// 128-token tile of the audio keys; the sum of squares of the normalised
-// outputs accumulates in registers over the heads, so the map is written once
-// per token with no atomics and no second pass.
-//   Two softmax warpgroups take alternate heads (group g: heads g, g + 2, ...),
-//     each thread one video token (TMEM lane) with all 128 keys of a step, its
-//     own running max and sum (O rescaled in TMEM only when the max grows by
-//     more than 2^8) and its group's O accumulator: the groups never exchange
-//     anything inside the walk, so one group's exponentials overlap the other
-//     group's products.  The steps interleave a pair of heads tile by tile.
+// 128-token tile of the audio keys ("steps" j = head * MT + key tile); the sum
+// of squares of the normalised outputs accumulates in registers over the heads,
+// so the map is written once per token with no atomics and no second pass.
 //   TMA (128B swizzle, 3-D maps [heads][rows][D] whose out-of-range rows read
-//     as zeros): Q of each group's head, K and V tiles (two-stage rings);
-//   tcgen05.mma S = Q K^T into the group's 128 TMEM columns; the softmax
-//     writes P = 2^(s - m) as bf16 over the S columns it has read;
-//   tcgen05.mma O_g += P V with P read from TMEM, V from shared memory.  At a
-//     head's end the group reads O_g into registers, frees the accumulator
-//     for its next head at once, then normalises, squares and stores.
-// Warp roles: 0-7 softmax and epilogue (two groups), 8 TMA producer (and TMEM
-// allocator), 9 MMA issuer.  Every barrier wait is bounded (PRISM_ERR_TIMEOUT
-// with a site).
+//     as zeros): Q of the head (two buffers: the next head's Q loads while this
+//     head's keys stream), K and V tiles (two-stage rings each);
+//   tcgen05.mma S = Q K^T into TMEM (two buffers of 128 columns);
+//   8 softmax warps (two warpgroups, one per 64-key half; TMEM lane = video
+//     token) mask the keys past M, keep a running max per row (O is rescaled
+//     in TMEM only when the max grows by more than 2^8), write P = 2^(s - m)
+//     as bf16 into TMEM over the S columns they have read;
+//   tcgen05.mma O += P V with P read from TMEM, V from shared memory, into one
+//     of two O accumulators (heads alternate), so the softmax warps normalise
+//     and square one head's O while the next head's products run.
+// Warp roles: 0-7 softmax and epilogue, 8 TMA producer (and TMEM allocator),
+// 9 MMA issuer.  Every barrier wait is bounded (PRISM_ERR_TIMEOUT with a site).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -74,49 +71,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// Max over the first kv (0..64) of a row's 64 logits held as bits.
-__device__ __forceinline__ float row_max(const uint32_t* sr, int kv) {
-    if (kv >= 64) {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        #pragma unroll
-        for (int c = 0; c < 64; c += 2)
-            m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-        return fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
-    }
-    float mx = -INFINITY;
-    #pragma unroll
-    for (int c = 0; c < 64; ++c)
-        if (c < kv) mx = fmaxf(mx, __uint_as_float(sr[c]));
-    return mx;
-}
-
-// P = 2^(s * scale_log2 + neg) of a row's 64 keys as 32 packed bf16 pairs (zero
-// past the first kv keys); returns the sum of the values.
-__device__ __forceinline__ float exp_half(const uint32_t* sr, int kv, float scale_log2, float neg, uint32_t* pk) {
-    float l4[4] = {0.f, 0.f, 0.f, 0.f};      // two packed pairs of partial sums
-    if (kv >= 64) {
-        #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            float x0, x1;
-            ffma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), scale_log2, scale_log2, neg,
-                  neg);
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            const int q = (e & 1) * 2;
-            add2(l4[q], l4[q + 1], l4[q], l4[q + 1], p0, p1);
-            pk[e] = pack_bf16(p0, p1);
-        }
-    } else {
-        #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const float p0 = 2 * e < kv ? ex2(fmaf(__uint_as_float(sr[2 * e]), scale_log2, neg)) : 0.f;
-            const float p1 = 2 * e + 1 < kv ? ex2(fmaf(__uint_as_float(sr[2 * e + 1]), scale_log2, neg)) : 0.f;
-            l4[e & 3] += p0 + p1;
-            pk[e] = pack_bf16(p0, p1);
-        }
-    }
-    return (l4[0] + l4[1]) + (l4[2] + l4[3]);
-}
-
 template <int HD>
 struct Smem {
     static constexpr int NSL = HD / 64;
@@ -126,8 +80,10 @@ struct Smem {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[STAGES], k_empty[STAGES];
     uint64_t v_full[STAGES], v_empty[STAGES];
-    uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];   // [group]
-    float pn[2][128];          // [group][row] sum of squares over the group's heads
+    uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+    float pmax[2][2][128];     // [step parity][warpgroup][row] partial row max
+    float psum[2][128];        // [warpgroup][row] partial row sum of the finished head
+    float pn[2][128];          // [warpgroup][row] partial sum of squares over the heads
     uint32_t tmem_base;
 };
 
@@ -140,22 +96,6 @@ struct Args {
     float scale_log2;   // log2(e) / sqrt(HD)
     int* err;
 };
-
-// Step j of the CTA's walk -> (head, key tile).  The two softmax groups take
-// alternate heads (group g: heads g, g + 2, ...); the steps interleave a pair
-// of heads tile by tile (head 2p tile 0, head 2p + 1 tile 0, head 2p tile 1,
-// ...), and an odd last head runs its tiles alone.
-__device__ __forceinline__ void step_of(int j, int MT, int heads, int& h, int& kt) {
-    const int full = (heads >> 1) * 2 * MT;
-    if (j < full) {
-        const int p = j / (2 * MT), rem = j - p * 2 * MT;
-        kt = rem >> 1;
-        h = 2 * p + (rem & 1);
-    } else {
-        kt = j - full;
-        h = heads - 1;
-    }
-}
 
 template <int HD>
 __global__ void __launch_bounds__(320, 1)
@@ -173,9 +113,9 @@ k_av_norm(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             mbar_init(&sm.q_full[i], 1);
             mbar_init(&sm.q_empty[i], 1);
             mbar_init(&sm.s_full[i], 1);
-            mbar_init(&sm.p_full[i], 128);
+            mbar_init(&sm.p_full[i], 256);
             mbar_init(&sm.pv_done[i], 1);
-            mbar_init(&sm.o_free[i], 128);
+            mbar_init(&sm.o_free[i], 256);
         }
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.k_full[s], 1);
@@ -194,8 +134,7 @@ k_av_norm(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    // TMEM columns: group g's S (then its bf16 P over the first 64 columns) at
-    // 128 g, group g's O at 256 + HD g
+    // TMEM columns: S (then P over its first 64 columns) at 0 and 128; O at 256 and 256 + HD
     constexpr uint32_t TO = 256;
 
     if (warp == W_PROD) {
@@ -204,8 +143,7 @@ k_av_norm(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (lane == 0) {
             tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
             for (int j = 0; j < J; ++j) {
-                int h, kt;
-                step_of(j, MT, a.heads, h, kt);
+                const int h = j / MT, kt = j - h * MT;
                 if (kt == 0) {
                     const int qb = h & 1;
                     if (h >= 2 && !mbar_wait(&sm.q_empty[qb], ((h >> 1) - 1) & 1, a.err, 2401)) break;
@@ -219,8 +157,7 @@ k_av_norm(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             }
         } else if (lane == 1) {
             for (int j = 0; j < J; ++j) {
-                int h, kt;
-                step_of(j, MT, a.heads, h, kt);
+                const int h = j / MT, kt = j - h * MT;
                 const int s = j % STAGES;
                 if (j >= STAGES && !mbar_wait(&sm.v_empty[s], ((j / STAGES) - 1) & 1, a.err, 2403)) break;
                 mbar_expect_tx(&sm.v_full[s], NSL * SLAB);
@@ -229,166 +166,90 @@ k_av_norm(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------ MMA issuer
-        // S(j) = Q K(j)^T into group g(j)'s S buffer and O_g += P(j) V(j) from the
-        // bf16 P written over that buffer.  One thread's MMAs run in issue order:
-        // every S(j) is issued after the PV of group g(j)'s previous step, so it
-        // overwrites P only once that product has read it.  n_p[g] counts group g's
-        // steps (the phases of its barriers), hc[g] its heads.
+        // Iteration j issues S(j) = Q K(j)^T, then O += P(j-1) V(j-1).  One thread's
+        // MMAs run in issue order, so S(j + 1) overwrites the P(j - 1) columns only
+        // after O += P(j - 1) V has read them.
         if (lane == 0) {
             constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t id_pv = idesc_bf16(128, HD, 0, 1);
-            int n_p[2] = {0, 0};
-            bool ok = true;
-            auto issue_s = [&](int j) {
-                int h, kt;
-                step_of(j, MT, a.heads, h, kt);
-                const int g = h & 1, s = j % STAGES;
-                if (kt == 0 && !mbar_wait(&sm.q_full[g], (h >> 1) & 1, a.err, 2501)) return false;
-                if (!mbar_wait(&sm.k_full[s], (j / STAGES) & 1, a.err, 2502)) return false;
-                tc_fence_after();
-                const uint32_t qA = desc_lo(smem_u32(sm.q[g][0]), 16);
-                const uint32_t kB = desc_lo(smem_u32(sm.k[s][0]), 16);
-                #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    umma_f16(tmem + 128 * g, desc_from_lo(qA + kmajor_step(kk, SLAB)),
-                             desc_from_lo(kB + kmajor_step(kk, SLAB)), id_qk, kk > 0);
-                umma_commit(&sm.s_full[g]);
-                umma_commit(&sm.k_empty[s]);
-                if (kt == MT - 1) umma_commit(&sm.q_empty[g]);
-                return true;
-            };
-            auto issue_pv = [&](int j) {
-                int h, kt;
-                step_of(j, MT, a.heads, h, kt);
-                const int g = h & 1, s = j % STAGES;
-                if (!mbar_wait(&sm.p_full[g], n_p[g] & 1, a.err, 2503)) return false;
-                if (!mbar_wait(&sm.v_full[s], (j / STAGES) & 1, a.err, 2504)) return false;
-                // the first product of the group's next head overwrites O_g: the
-                // group's epilogue must have read the previous head's O first
-                if (kt == 0 && h >= 2 && !mbar_wait(&sm.o_free[g], ((h >> 1) - 1) & 1, a.err, 2505)) return false;
-                tc_fence_after();
-                const uint32_t vT = desc_lo(smem_u32(sm.v[s][0]), SLAB);
-                #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16_ts(tmem + TO + HD * g, tmem + 128 * g + 8 * kk, desc_from_lo(vT + mnmajor_step(kk)),
-                                id_pv, (kt > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&sm.pv_done[g]);
-                umma_commit(&sm.v_empty[s]);
-                ++n_p[g];
-                return true;
-            };
-            for (int j = 0; ok && j <= J; ++j) {
-                // S(j) and PV(j - 1): PV first when both belong to one group (an odd
-                // last head), so S(j) never overwrites a P that is still to be read
-                int hj = 0, hp = 0, kt_;
-                if (j < J) step_of(j, MT, a.heads, hj, kt_);
-                if (j >= 1) step_of(j - 1, MT, a.heads, hp, kt_);
-                const bool same = j >= 1 && j < J && (hj & 1) == (hp & 1);
-                if (same) ok = issue_pv(j - 1) && issue_s(j);
-                else {
-                    if (j < J) ok = issue_s(j);
-                    if (ok && j >= 1) ok = issue_pv(j - 1);
+            for (int j = 0; j <= J; ++j) {
+                if (j < J) {
+                    const int h = j / MT, kt = j - h * MT;
+                    const int s = j % STAGES, b = j & 1, qb = h & 1;
+                    if (kt == 0 && !mbar_wait(&sm.q_full[qb], (h >> 1) & 1, a.err, 2501)) break;
+                    if (!mbar_wait(&sm.k_full[s], (j / STAGES) & 1, a.err, 2502)) break;
+                    tc_fence_after();
+                    const uint32_t qA = desc_lo(smem_u32(sm.q[qb][0]), 16);
+                    const uint32_t kB = desc_lo(smem_u32(sm.k[s][0]), 16);
+                    #pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        umma_f16(tmem + 128 * b, desc_from_lo(qA + kmajor_step(kk, SLAB)),
+                                 desc_from_lo(kB + kmajor_step(kk, SLAB)), id_qk, kk > 0);
+                    umma_commit(&sm.s_full[b]);
+                    umma_commit(&sm.k_empty[s]);
+                    if (kt == MT - 1) umma_commit(&sm.q_empty[qb]);
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, hh = jj / MT, kt = jj - hh * MT;
+                    const int s = jj % STAGES, b = jj & 1, ob = hh & 1;
+                    if (!mbar_wait(&sm.p_full[b], (jj >> 1) & 1, a.err, 2503)) break;
+                    if (!mbar_wait(&sm.v_full[s], (jj / STAGES) & 1, a.err, 2504)) break;
+                    // the first product of head hh overwrites the O of head hh - 2
+                    if (kt == 0 && hh >= 2 && !mbar_wait(&sm.o_free[ob], ((hh >> 1) - 1) & 1, a.err, 2505)) break;
+                    tc_fence_after();
+                    const uint32_t vT = desc_lo(smem_u32(sm.v[s][0]), SLAB);
+                    #pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16_ts(tmem + TO + HD * ob, tmem + 128 * b + 8 * kk, desc_from_lo(vT + mnmajor_step(kk)),
+                                    id_pv, (kt > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&sm.pv_done[b]);
+                    umma_commit(&sm.v_empty[s]);
                 }
             }
         }
     } else {
         // ------------------------------------------------ softmax + epilogue
-        // Group g (warps 4g .. 4g + 3) takes heads g, g + 2, ...: a thread is one
-        // video token (TMEM lane) with all 128 keys of every step of its group,
-        // its own running max and sum, and the group's O accumulator, so the
-        // groups never wait for each other inside the walk.  O is rescaled only
-        // when the running max grows by more than 2^8 (bf16 P keeps fp32's
-        // exponent range).  tcgen05.ld/st are warp-collective: every decision
-        // guarding one is warp-uniform.
-        const int g = warp >> 2;
+        // tcgen05.ld/st are warp-collective: every decision guarding one is
+        // warp-uniform.  The two warps sharing a TMEM lane quarter (w, w + 4)
+        // exchange row maxima and sums through shared memory and a 64-thread
+        // named barrier.
+        const int wg = warp >> 2;
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t scol = 128 * g, ocol = TO + HD * g;
+        const int pair_bar = 1 + (warp & 3);
+        constexpr int OC = HD / 2;                 // O columns per warpgroup
         const int64_t row = (int64_t)t * 128 + r;
         const bool row_ok = row < a.N;
-        float nsq = 0.f;
+        float m_ref = -INFINITY, l = 0.f, nsq = 0.f;
         bool ok = true;
-        int c = 0;                                  // the group's steps so far (barrier phases)
-        for (int h = g; ok && h < a.heads; h += 2) {
-            float m_ref = -INFINITY, l = 0.f;
-            for (int kt = 0; kt < MT; ++kt, ++c) {
-                const int kv0 = min(max(a.M - kt * 128, 0), 64);          // valid keys of half 0 (uniform)
-                const int kv1 = min(max(a.M - kt * 128 - 64, 0), 64);     // and of half 1
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[g], c & 1, a.err, 2002))) { ok = false; break; }
-                tc_fence_after();
-                uint32_t sr[64];
-                float mx = -INFINITY;
-                PRISM_TMEM_LD32(tmem + lane_off + scol, (sr + 0));
-                PRISM_TMEM_LD32(tmem + lane_off + scol + 32, (sr + 32));
-                tmem_wait_ld();
-                mx = row_max(sr, kv0);
-                PRISM_TMEM_LD32(tmem + lane_off + scol + 64, (sr + 0));  // half 1 stays in registers
-                PRISM_TMEM_LD32(tmem + lane_off + scol + 96, (sr + 32));
-                tmem_wait_ld();
-                mx = fmaxf(mx, row_max(sr, kv1));
-                mx *= a.scale_log2;
-                if (kt == 0) {
-                    m_ref = mx;                     // a new head: its first tile sets the reference
-                } else {
-                    const float m_new = fmaxf(m_ref, mx);
-                    const bool need = m_new > m_ref + kRescaleLog2;
-                    if (__any_sync(0xffffffffu, need)) {
-                        // O_g holds the products up to this group's previous step
-                        if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g], (c - 1) & 1, a.err, 2003))) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const float f = need ? ex2(m_ref - m_new) : 1.f;
-                        #pragma unroll
-                        for (int cc = 0; cc < HD / 32; ++cc) {
-                            uint32_t o[32];
-                            PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * cc, o);
-                            tmem_wait_ld();
-                            #pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                            PRISM_TMEM_ST32(tmem + lane_off + ocol + 32 * cc, o);
-                        }
-                        if (need) { l *= f; m_ref = m_new; }
-                    }
-                }
-                const float neg = -m_ref;
-                uint32_t pk1[32], pk0[32];
-                l += exp_half(sr, kv1, a.scale_log2, neg, pk1);
-                PRISM_TMEM_LD32(tmem + lane_off + scol, (sr + 0));       // half 0 again
-                PRISM_TMEM_LD32(tmem + lane_off + scol + 32, (sr + 32));
-                tmem_wait_ld();
-                l += exp_half(sr, kv0, a.scale_log2, neg, pk0);
-                // P (bf16, two keys per column) over the S columns just read
-                PRISM_TMEM_ST32(tmem + lane_off + scol, pk0);
-                PRISM_TMEM_ST32(tmem + lane_off + scol + 32, pk1);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sm.p_full[g]);
-            }
-            if (!ok) break;
-            // epilogue of head h: O_g into registers, the accumulator freed at once
-            // for the group's next head, then normalised, squared and stored
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[g], (c - 1) & 1, a.err, 2001))) { ok = false; break; }
+        int nbar = 0;                              // pair barriers taken so far
+
+        // Normalise head hp's O (buffer hp & 1, complete once PV of step jl is
+        // done), add its squares to nsq, write h_hat if asked, free the buffer.
+        auto epilogue = [&](int hp, int jl, float l_hp) {
+            bool fin = ok && __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[jl & 1], (jl >> 1) & 1, a.err, 2001));
+            sm.psum[wg][r] = l_hp;
+            named_bar(pair_bar, 64);
+            ++nbar;
+            if (!fin) { ok = false; return; }
             tc_fence_after();
-            uint32_t o[HD];
-            #pragma unroll
-            for (int cc = 0; cc < HD / 32; ++cc) PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * cc, (o + 32 * cc));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.o_free[g]);
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float lt = sm.psum[0][r] + sm.psum[1][r];
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const uint32_t ocol = TO + HD * (hp & 1) + OC * wg;
             float acc = 0.f;
             #pragma unroll
-            for (int cc = 0; cc < HD / 32; ++cc) {
+            for (int c = 0; c < OC / 32; ++c) {
+                uint32_t o[32];
+                PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * c, o);
+                tmem_wait_ld();
                 float x[32];
                 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    x[e] = __uint_as_float(o[32 * cc + e]) * inv;
+                    x[e] = __uint_as_float(o[e]) * inv;
                     acc = fmaf(x[e], x[e], acc);
                 }
                 if (a.hhat && row_ok) {
-                    const size_t base = ((size_t)h * a.N + (size_t)row) * HD + 32 * cc;
+                    const size_t base = ((size_t)hp * a.N + (size_t)row) * HD + OC * wg + 32 * c;
                     if (a.hhat_f32) {
                         float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.hhat) + base);
                         #pragma unroll
@@ -403,12 +264,105 @@ k_av_norm(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                 }
             }
             nsq += acc;
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[hp & 1]);
+        };
+
+        for (int j = 0; j < J; ++j) {
+            const int h = j / MT, kt = j - h * MT, b = j & 1;
+            const int kvalid = a.M - kt * 128 - 64 * wg;     // valid keys of this half (warp-uniform)
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (j >> 1) & 1, a.err, 2002))) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[64];
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64 * wg, (sr + 0));
+            PRISM_TMEM_LD32(tmem + lane_off + 128 * b + 64 * wg + 32, (sr + 32));
+            tmem_wait_ld();
+            float mx = -INFINITY;
+            if (kvalid >= 64) {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                #pragma unroll
+                for (int c = 0; c < 64; c += 2)
+                    m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+            } else {
+                #pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (c < kvalid) mx = fmaxf(mx, __uint_as_float(sr[c]));
+            }
+            mx *= a.scale_log2;
+            sm.pmax[j & 1][wg][r] = mx;
+            // both warpgroups have read their S columns past this barrier, so P may
+            // overwrite the first 64 of them
+            named_bar(pair_bar, 64);
+            ++nbar;
+            mx = fmaxf(mx, sm.pmax[j & 1][wg ^ 1][r]);
+            float l_done = 0.f;
+            if (kt == 0) {                 // a new head: its first tile sets the reference
+                l_done = l;
+                l = 0.f;
+                m_ref = mx;
+            } else {
+                const float m_new = fmaxf(m_ref, mx);
+                const bool need = m_new > m_ref + kRescaleLog2;
+                if (__any_sync(0xffffffffu, need)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err, 2003))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float f = need ? ex2(m_ref - m_new) : 1.f;
+                    const uint32_t ocol = TO + HD * (h & 1) + OC * wg;
+                    #pragma unroll
+                    for (int c = 0; c < OC / 32; ++c) {
+                        uint32_t o[32];
+                        PRISM_TMEM_LD32(tmem + lane_off + ocol + 32 * c, o);
+                        tmem_wait_ld();
+                        #pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                        PRISM_TMEM_ST32(tmem + lane_off + ocol + 32 * c, o);
+                    }
+                    if (need) { l *= f; m_ref = m_new; }
+                }
+            }
+            const float neg = -m_ref;
+            uint32_t pk[32];
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};      // two packed pairs of partial sums
+            if (kvalid >= 64) {
+                #pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float x0, x1;
+                    ffma2(x0, x1, __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]), a.scale_log2,
+                          a.scale_log2, neg, neg);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    const int q = (e & 1) * 2;
+                    add2(l4[q], l4[q + 1], l4[q], l4[q + 1], p0, p1);
+                    pk[e] = pack_bf16(p0, p1);
+                }
+            } else {
+                #pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = 2 * e < kvalid ? ex2(fmaf(__uint_as_float(sr[2 * e]), a.scale_log2, neg)) : 0.f;
+                    const float p1 = 2 * e + 1 < kvalid ? ex2(fmaf(__uint_as_float(sr[2 * e + 1]), a.scale_log2, neg)) : 0.f;
+                    l4[e & 3] += p0 + p1;
+                    pk[e] = pack_bf16(p0, p1);
+                }
+            }
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            PRISM_TMEM_ST32(tmem + lane_off + 128 * b + 32 * wg, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_full[b]);
+            if (kt == 0 && h > 0) epilogue(h - 1, j - 1, l_done);
+            if (!ok) break;
         }
-        // the two groups' sums of squares of each token meet once (every warp
-        // takes this barrier, on success or after a failed wait)
-        sm.pn[g][r] = nsq;
-        named_bar(1 + (warp & 3), 64);
-        if (ok && g == 0 && row_ok) a.amap[row] = sqrtf(sm.pn[0][r] + sm.pn[1][r]);
+        // A warp that left the loop on a failed wait still takes every pair
+        // barrier its partner will take: one per step, one per head epilogue.
+        const int nbar_loop = J + a.heads - 1;
+        for (; nbar < nbar_loop; ++nbar) named_bar(pair_bar, 64);
+        epilogue(a.heads - 1, J - 1, l);           // the last head (takes one more barrier)
+        sm.pn[wg][r] = nsq;
+        named_bar(pair_bar, 64);
+        if (ok && wg == 0 && row_ok) a.amap[row] = sqrtf(sm.pn[0][r] + sm.pn[1][r]);
     }
     tc_fence_before();
     __syncthreads();
