@@ -56,6 +56,11 @@ def args_():
     ap.add_argument("--alpha", type=float, default=0.5, help="shape-mapping exponent (1/2: the method)")
     ap.add_argument("--shape-mode", choices=["dynamic", "isotropic", "fixed"], default="dynamic")
     ap.add_argument("--fixed-shape", type=int, default=3, help="candidate index for --shape-mode fixed")
+    ap.add_argument("--cut-ratio", type=float, default=0.0,
+                    help="adaptive temporal zone boundaries: split a zone where its largest frame-difference "
+                         "energy exceeds this multiple of the median (0: whole zones, the method)")
+    ap.add_argument("--shot-cuts", type=int, nargs="*", default=[],
+                    help="frames where the synthetic fields start a new shot")
     ap.add_argument("--av-tokens", type=int, default=1000,
                     help="audio tokens of the guidance-map producer leg (the pages: under 1K)")
     ap.add_argument("--no-av", action="store_true", help="skip the guidance-map producer leg")
@@ -197,7 +202,8 @@ def peaks():
 def variant_of(a):
     """The oracle's keyword arguments for the command line's variant flags."""
     mode = {"dynamic": 0, "isotropic": 1, "fixed": 2}[a.shape_mode]
-    return dict(alpha=a.alpha, shape_mode=mode, fixed_shape=a.fixed_shape, k_frac=a.topk_frac)
+    return dict(alpha=a.alpha, shape_mode=mode, fixed_shape=a.fixed_shape, k_frac=a.topk_frac,
+                cut_ratio=a.cut_ratio)
 
 
 def workload_of(a):
@@ -205,6 +211,8 @@ def workload_of(a):
     over = {k: v for k, v in (("top_k", a.top_k), ("top_p", a.top_p)) if v is not None}
     if a.grid:
         over.update(T=a.grid[0], H=a.grid[1], W=a.grid[2])
+    if a.shot_cuts:
+        over.update(shot_cuts=list(a.shot_cuts))
     return syn.workload(a.workload, **over)
 
 
@@ -520,7 +528,8 @@ def run_prism(a, rank, world, local_rank):
     w = workload_of(a)
     mode = {"dynamic": _lib.PRISM_SHAPE_DYNAMIC, "isotropic": _lib.PRISM_SHAPE_ISOTROPIC,
             "fixed": _lib.PRISM_SHAPE_FIXED}[a.shape_mode]
-    variant = dict(alpha=a.alpha, shape_mode=mode, fixed_shape=a.fixed_shape, top_k_frac=a.topk_frac)
+    variant = dict(alpha=a.alpha, shape_mode=mode, fixed_shape=a.fixed_shape, top_k_frac=a.topk_frac,
+                   cut_ratio=a.cut_ratio)
     lib = _lib.load()
     need = a.warmup + a.steps
     heads = min(w.heads, need)
@@ -739,6 +748,7 @@ def run_prism(a, rank, world, local_rank):
                          "heads_in_sequence": True, "head_dim": D, "input_dtype": "bf16",
                          "output_dtype": "fp32", "top_k": w.top_k, "top_p": w.top_p,
                          "top_k_frac": a.topk_frac, "alpha": a.alpha, "shape_mode": a.shape_mode,
+                         **({"cut_ratio": a.cut_ratio, "shot_cuts": list(a.shot_cuts)} if a.cut_ratio else {}),
                          **({"fixed_shape": a.fixed_shape} if a.shape_mode == "fixed" else {}),
                          "l2": "inputs larger than L2 (259 MB per tensor per head)"},
               "tflops": {"fwd_bwd_selected": attn_tflops,
