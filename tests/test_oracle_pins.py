@@ -419,3 +419,27 @@ def test_key_rows_match_torch_autograd(seed, k, p):
     np.testing.assert_allclose(dQr, q.grad.numpy()[rows], atol=1e-10)
     s = (q @ kk.T / np.sqrt(D)).masked_fill(~m, float("-inf"))
     np.testing.assert_allclose(lr, torch.logsumexp(s, 1).detach().numpy()[rows], atol=1e-10)
+
+
+def test_token_order_inside_a_block_affects_no_result():
+    """Reading 6 (tokens inside a block in raster order) is free: any order of the
+    tokens inside each block gives the same pooled means, block scores,
+    selection, O, LSE and gradients in raster order."""
+    Q, K, V, pl, D = _tiny_plan(3, 3, 0.6)
+    src, st, sel = pl["src"], pl["starts"], pl["sel"]
+    rng = np.random.default_rng(8)
+    src2 = src.copy()
+    for i in range(len(st) - 1):
+        src2[st[i]:st[i + 1]] = rng.permutation(src[st[i]:st[i + 1]])
+    assert not np.array_equal(src2, src)
+    for X in (Q, K):
+        np.testing.assert_allclose(po.pool(X, src2, st), po.pool(X, src, st), atol=1e-12)
+    sel2, s2, _ = po.select(po.pool(Q, src2, st), po.pool(K, src2, st), 3, 0.6)
+    assert [x.tolist() for x in sel2] == [x.tolist() for x in sel]
+    O, lse = po.attention_fwd(Q, K, V, src, st, sel)
+    O2, lse2 = po.attention_fwd(Q, K, V, src2, st, sel)
+    np.testing.assert_allclose(O2, O, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse, atol=1e-12)
+    dO = rng.normal(size=Q.shape)
+    for g2, g in zip(po.attention_bwd(Q, K, V, dO, src2, st, sel), po.attention_bwd(Q, K, V, dO, src, st, sel)):
+        np.testing.assert_allclose(g2, g, atol=1e-10)
