@@ -176,18 +176,26 @@ def source_digest(kernel):
     return m.hexdigest()[:16]
 
 
-def measured_traffic(kernel, path=None):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture
-    (profiles/dram_traffic_grid72x88x160.md), or None if the kernel's sources
-    changed since (their hash no longer matches) or there is no capture."""
-    path = path or os.path.join(ROOT, "profiles", "dram_traffic_grid72x88x160.md")
+TRAFFIC_PROFILE = "dram_traffic_k_bwd_dkdv_grid16x64x144.md"
+
+
+def measured_traffic(kernel, pairs, path=None):
+    """DRAM bytes of one launch of `kernel` at `pairs` selected token pairs,
+    scaled from the committed one-launch ncu capture on a small grid (the table
+    in profiles/dram_traffic_k_bwd_dkdv_grid16x64x144.md gives the captured
+    bytes and the captured grid's selected pairs) by the ratio of selected pairs
+    (the kernel's traffic per launch follows its work: every unit loads one Q/dO
+    tile and every (key tile, chunk) one K/V tile and one dK/dV reduce).  None
+    if the kernel's sources changed since the capture (their hash no longer
+    matches) or there is no capture."""
+    path = path or os.path.join(ROOT, "profiles", TRAFFIC_PROFILE)
     digest = source_digest(kernel)
     if digest is None or not os.path.exists(path):
         return None
     for line in open(path):
         cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) == 5 and cells[0] == kernel and cells[4] == digest:
-            return float(cells[1]) + float(cells[2])
+        if len(cells) == 6 and cells[0] == kernel and cells[5] == digest:
+            return (float(cells[1]) + float(cells[2])) * float(pairs) / float(cells[4])
     return None
 
 
@@ -762,8 +770,10 @@ def run_prism(a, rank, world, local_rank):
                            "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                            "frac": ach / peak, "peak_source": peak_src,
                            "traffic": measured_traffic(
-                               {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv"}.get(dom, ""))
-                           if w.N == 1013760 else None},
+                               {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv"}.get(dom, ""), Pi),
+                           "traffic_note": "DRAM bytes per launch from a one-launch ncu capture on grid "
+                                           "16x64x144, scaled by selected pairs (profiles/" + TRAFFIC_PROFILE
+                                           + "); null once the kernel changed since"},
               "plan_kernels": plan_kernels, "dense_same_shape": dense, "operating_point": op,
               "guidance_map": av,
               "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks})
