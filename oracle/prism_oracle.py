@@ -39,7 +39,8 @@ notes of the repository):
   * selection: logits Qbar_i . Kbar_j / sqrt(D), softmax over all key blocks,
     order (P descending, j ascending); Top-p keeps the shortest prefix whose
     float32 running sum reaches p (p >= 1 keeps all, p <= 0 none); the union
-    with Top-k of the same order is the first max(k, L) blocks.
+    with Top-k of the same order is the first max(k, L) blocks;
+  * adaptive temporal boundaries (optional): see zone_shapes_cut.
 
 Parity status: the candidate set, the closed form l*, the snapping, the
 directional statistics, the selection rule and the attention (forward and
@@ -47,10 +48,14 @@ backward) are pinned by the tests in tests/test_oracle_pins.py; the block-score
 softmax (hand-worked values, torch float64), the tie margins (written-out
 candidate distances, constructed threshold ties) and closed forms of the
 statistics on hand-built fields by tests/test_oracle_selection_pins.py, with
-planted mistakes that each of those checks catches.  The rho formula and the
-a_bar / v_hat normalisations are readings: their code is pinned to closed
-forms and to a per-token brute force, the readings themselves are not fixed by
-the pages ("parity unpinned" for the reading).
+planted mistakes that each of those checks catches; the adaptive temporal
+boundaries by tests/test_oracle_cuts.py (closed-form energies, hard cuts at
+every frame, per-token brute force on the parts, the partition's invariants);
+the order of tokens inside a block by invariance (no result depends on it).
+The rho formula, the a_bar / v_hat normalisations and the cut detector are
+readings: their code is pinned to closed forms and to a per-token brute force,
+the readings themselves are not fixed by the pages ("parity unpinned" for the
+reading).
 """
 from __future__ import annotations
 
