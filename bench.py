@@ -176,27 +176,30 @@ def source_digest(kernel):
     return m.hexdigest()[:16]
 
 
-TRAFFIC_PROFILE = "dram_traffic_k_bwd_dkdv_grid16x64x144.md"
+TRAFFIC_PROFILE = "dram_traffic_k_bwd_dkdv_grid16x64x144_grid16x64x288.md"
 
 
 def measured_traffic(kernel, pairs, path=None):
     """DRAM bytes of one launch of `kernel` at `pairs` selected token pairs,
-    scaled from the committed one-launch ncu capture on a small grid (the table
-    in profiles/dram_traffic_k_bwd_dkdv_grid16x64x144.md gives the captured
+    scaled from the committed one-launch ncu captures on small grids (the table
+    in profiles/dram_traffic_k_bwd_dkdv_grid16x64x144_grid16x64x288.md gives the captured
     bytes and the captured grid's selected pairs) by the ratio of selected pairs
     (the kernel's traffic per launch follows its work: every unit loads one Q/dO
-    tile and every (key tile, chunk) one K/V tile and one dK/dV reduce).  None
+    tile and every (key tile, chunk) one K/V tile and one dK/dV reduce); of
+    several captures the one on the largest grid (most selected pairs).  None
     if the kernel's sources changed since the capture (their hash no longer
     matches) or there is no capture."""
     path = path or os.path.join(ROOT, "profiles", TRAFFIC_PROFILE)
     digest = source_digest(kernel)
     if digest is None or not os.path.exists(path):
         return None
+    best = None                       # the capture with the most selected pairs
     for line in open(path):
         cells = [c.strip() for c in line.strip().strip("|").split("|")]
         if len(cells) == 6 and cells[0] == kernel and cells[5] == digest:
-            return (float(cells[1]) + float(cells[2])) * float(pairs) / float(cells[4])
-    return None
+            row = (float(cells[4]), float(cells[1]) + float(cells[2]))
+            best = row if best is None or row[0] > best[0] else best
+    return None if best is None else best[1] * float(pairs) / best[0]
 
 
 def peaks():
@@ -464,8 +467,7 @@ def guidance_map_leg(w, M, pk, reps=5):
     out["roofline"] = {"kernel": "k_av_norm", "bound": "tensor", "achieved": ach, "peak": burst,
                        "unit": "TFLOP/s", "frac": ach / burst,
                        "peak_source": "measured burst bf16 (timed alone)" if pk else "fallback",
-                       "traffic": measured_traffic("k_av_norm")
-                       if (w.N, M, heads, D) == (1013760, 1000, 40, 128) else None}
+                       "traffic": None, "traffic_note": "no DRAM capture of this kernel"}
     del Qv, Ka, Va, amap, hh
     torch.cuda.empty_cache()
     return out
@@ -772,7 +774,7 @@ def run_prism(a, rank, world, local_rank):
                            "traffic": measured_traffic(
                                {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv"}.get(dom, ""), Pi),
                            "traffic_note": "DRAM bytes per launch from a one-launch ncu capture on grid "
-                                           "16x64x144, scaled by selected pairs (profiles/" + TRAFFIC_PROFILE
+                                           "16x64x288, scaled by selected pairs (profiles/" + TRAFFIC_PROFILE
                                            + "); null once the kernel changed since"},
               "plan_kernels": plan_kernels, "dense_same_shape": dense, "operating_point": op,
               "guidance_map": av,
