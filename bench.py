@@ -638,12 +638,13 @@ def run_prism(a, rank, world, local_rank):
     attn_tflops = 14 * D * Pi / (attn_ms * 1e-3) / 1e12
     value = elapsed_max / (a.steps * world)
     # plan kernels against their own bounds: HBM for the statistics (one read of
-    # V) and the gather (Q, K, V read, fp16 copies written); plain ALU for the
-    # block scores (2 D N_b^2 flops + N_b^2 exp)
+    # V) and the gather stage (Q, K, V read once for the per-head power-of-two
+    # scales, then read again and written as the scaled fp16 copies); plain ALU
+    # for the block scores (2 D N_b^2 flops + N_b^2 exp)
     hbm = pk.get("hbm_gbs") or 6650.0
     per_head = lambda k: stage_ms[k] / a.steps
     stats_bytes = 2.0 * D * w.N + 4.0 * w.N
-    gather_bytes = 12.0 * D * w.N
+    gather_bytes = 18.0 * D * w.N
     plan_kernels = {
         "stats": {"ms": per_head("plan_stats"), "bytes": stats_bytes,
                   "GB/s": stats_bytes / (per_head("plan_stats") * 1e-3) / 1e9 if per_head("plan_stats") else None},
@@ -773,8 +774,8 @@ def run_prism(a, rank, world, local_rank):
                            "frac": ach / peak, "peak_source": peak_src,
                            "traffic": measured_traffic(
                                {"fwd": "k_attn_fwd", "bwd_dkdv": "k_bwd_dkdv"}.get(dom, ""), Pi),
-                           "traffic_note": "DRAM bytes per launch from a one-launch ncu capture on grid "
-                                           "16x64x288, scaled by selected pairs (profiles/" + TRAFFIC_PROFILE
+                           "traffic_note": "DRAM bytes per launch from a one-launch ncu capture on a small "
+                                           "grid, scaled by selected pairs (profiles/" + TRAFFIC_PROFILE
                                            + "); null once the kernel changed since"},
               "plan_kernels": plan_kernels, "dense_same_shape": dense, "operating_point": op,
               "guidance_map": av,

@@ -32,7 +32,7 @@ ITEMS = {
     "col_ptr": (6, np.int32), "row_idx": (7, np.int32), "qbar": (8, np.float32),
     "kbar": (9, np.float32), "src": (10, np.int32), "zone_stats": (11, np.float32),
     "zone_cut": (12, np.uint8), "shape_id2": (13, np.uint8), "zone_energy": (14, np.float32),
-    "region_stats": (15, np.float32), "list_offsets": (16, np.int64),
+    "region_stats": (15, np.float32), "list_offsets": (16, np.int64), "qkv_max": (17, np.uint32),
 }
 
 

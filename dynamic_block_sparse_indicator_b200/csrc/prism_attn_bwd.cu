@@ -18,12 +18,14 @@
 //               the 64-row query halves of that range of the key tile's
 //               transposed list; S^T = K Q^T and dP^T = V dO^T into TMEM
 //               (double-buffered), softmax warps form P^T (into TMEM, over
-//               dP^T) and dS^T (fp16 shared memory), dV += P^T dO and
-//               dK += dS^T Q accumulate in TMEM and are TMA reduce-added into
-//               fp32 accumulators at the end of the chunk.  For head_dim 128
-//               the same CTA also forms dQ^T = K^T dS^T per unit and TMA
-//               reduce-adds it into an fp32 accumulator.  The grid runs chunk
-//               by chunk, so the dQ rows being accumulated stay in L2.
+//               dP^T) and dS^T (into TMEM, over S^T), dV += P^T dO and
+//               dK += dS^T Q accumulate in TMEM with their A operands read
+//               from TMEM, and are TMA reduce-added into fp32 accumulators at
+//               the end of the chunk.  For head_dim 128 the same CTA also
+//               forms dQ^T = K^T dS^T per unit (dS^T also in shared memory, as
+//               its B operand) and adds it into an fp32 accumulator with
+//               coalesced L2 reductions.  The grid runs chunk by chunk, so the
+//               dQ rows being accumulated stay in L2.
 //   k_acc_finalize  scales the accumulators and scatters them to raster order.
 //   k_bwd_dq    (head_dim 64) one CTA per 128-row query tile; iterates the
 //               64-key halves of the forward list; S = Q K^T, dP = dO V^T,
@@ -55,21 +57,24 @@ constexpr float kPScaleInv = 1.f / 32768.f;
 constexpr int kDsShift = 7;                 // dS' = dS 2^(kDsShift - E - ev): see k_bwd_pre
 
 // --------------------------------------------------------------- preprocess
+// max |dO| per head (fp32 bits, see fold_abs): one pass over 16-byte chunks (dO
+// is 16-byte aligned and a head holds N x head_dim values).
 template <typename OT>
 __global__ void __launch_bounds__(256) k_bwd_absmax(const OT* __restrict__ dO, uint32_t* dmax, int64_t n_per_head) {
     const int h = blockIdx.y;
-    const OT* x = dO + (size_t)h * n_per_head;
-    float m = 0.f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_per_head;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const float v = fabsf((float)x[i]);
-        m = (v > m || v != v) ? v : m;                    // keeps a NaN
+    const uint4* x = reinterpret_cast<const uint4*>(dO + (size_t)h * n_per_head);
+    const int64_t n16 = n_per_head * (int64_t)sizeof(OT) / 16;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    uint32_t m = 0u;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + stride < n16; i += 2 * stride) {         // two chunks in flight
+        const uint4 a = __ldg(x + i), b = __ldg(x + i + stride);
+        m = fold_abs<OT>(fold_abs<OT>(m, a), b);
     }
-    for (int o = 16; o > 0; o >>= 1) {
-        const float y = __shfl_xor_sync(0xffffffffu, m, o);
-        m = (y > m || y != y) ? y : m;
-    }
-    if ((threadIdx.x & 31) == 0) atomicMax(dmax + h, __float_as_uint(m));  // |x| bits order like values
+    if (i < n16) m = fold_abs<OT>(m, __ldg(x + i));
+    uint32_t b = abs_bits<OT>(m);
+    for (int o = 16; o > 0; o >>= 1) b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(dmax + h, b);
 }
 
 // Exponent E with max |dO| in [2^(E-1), 2^E); dO is multiplied by 2^-E.
@@ -165,6 +170,7 @@ struct BwdArgs {
     const uint32_t* dmax;  // [heads] max |dO| bits: outputs are divided by the dO scale
     void* out0;            // dK (dkdv) or dQ (dq), raster order
     void* out1;            // dV (dkdv)
+    float* dq_acc;         // (dkdv, head_dim 128) fp32 dQ accumulator, block order, head group
     int64_t N;
     int NT;
     int out_f32;
@@ -214,10 +220,12 @@ __device__ __forceinline__ void zero_row(void* base, size_t row, int HD, int out
 
 // ------------------------------------------------------------------- dK, dV
 // FUSE (head_dim 128): the same CTA also forms dQ^T = K^T dS^T for every
-// 64-query unit into the TMEM columns that S^T just vacated; a drain warpgroup
-// (warps 10-13) moves it through shared memory and TMA reduce-adds it into an
-// fp32 dQ accumulator in block order, so dQ costs one more MMA instead of a
-// second kernel that recomputes S and dP.
+// 64-query unit into the TMEM columns of dP^T; a drain warpgroup (warps 10-13)
+// adds it from registers into an fp32 dQ accumulator in block order with
+// coalesced reductions in L2, so dQ costs one more MMA instead of a second
+// kernel that recomputes S and dP.  Shared-memory bandwidth is what this
+// kernel runs at (the tensor cores read every operand from it), so dS^T also
+// goes to TMEM, where it is the A operand of dK, and dQ^T is not staged.
 template <int HD, bool FUSE>
 struct DkdvSmem {
     static constexpr int NSL = HD / 64;
@@ -225,8 +233,7 @@ struct DkdvSmem {
     alignas(1024) uint8_t v[NSL][SLAB128];
     alignas(1024) uint8_t q[DKDV_STAGES][NSL][SLAB64];
     alignas(1024) uint8_t dO[DKDV_STAGES][NSL][SLAB64];
-    alignas(1024) uint8_t ds[2][SLAB128];     // dS^T [128 keys][64 queries] (P^T lives in TMEM)
-    alignas(1024) float stage_dq[FUSE ? 32 * HD : 4];   // [32 queries][HD] fp32
+    alignas(1024) uint8_t ds[2][SLAB128];     // dS^T [128 keys][64 queries]: the B operand of dQ^T
     alignas(16) float lse[DKDV_STAGES][64];
     alignas(16) float di[DKDV_STAGES][64];
     uint64_t bar_kv;
@@ -242,15 +249,14 @@ struct DkdvSmem {
 template <int HD, bool FUSE>
 constexpr bool epilogue_fits() {
     using S = DkdvSmem<HD, FUSE>;
-    return offsetof(S, stage_dq) - offsetof(S, q) >= 8 * 32 * HD * sizeof(float);
+    return offsetof(S, lse) - offsetof(S, q) >= 8 * 32 * HD * sizeof(float);
 }
 
 template <int HD, bool FUSE>
 __global__ void __launch_bounds__(FUSE ? 480 : 352, 1)
 k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
            const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
-           const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
-           const __grid_constant__ CUtensorMap tm_dv, BwdArgs a) {
+           const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv, BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     DkdvSmem<HD, FUSE>& sm = *reinterpret_cast<DkdvSmem<HD, FUSE>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -275,10 +281,11 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     if (U == 0) return;                            // nothing selected in this chunk
     const int* ents = a.lbase + a.ent_off[h] + e0;
     // TMEM columns: buffer b = [128b, 128b + 128): S^T at 128b, dP^T at 128b + 64.
-    // The softmax writes P^T (fp16 pairs) over the first half of dP^T; dQ^T of
-    // the unit then overwrites all 64 dP^T columns after dV has read P^T (the
-    // MMAs of one issuer run in order), so the next S^T into the buffer does not
-    // wait for the dQ drain -- only the next dP^T does.  dV at 256, dK at 256 + HD.
+    // The softmax writes dS^T (fp16 pairs) over the first half of S^T and P^T
+    // over the first half of dP^T; dQ^T of the unit then overwrites all 64 dP^T
+    // columns after dV has read P^T (the MMAs of one issuer run in order), so
+    // the next S^T into the buffer waits for dK (which reads dS^T there), not
+    // for the dQ drain -- only the next dP^T does.  dV at 256, dK at 256 + HD.
     constexpr uint32_t TDV = 256, TDK = 256 + HD;
 
     if (threadIdx.x == 0) {
@@ -350,8 +357,9 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             for (int u = 0; ok && u < U; ++u) {
                 const int s = u % DKDV_STAGES, b = u & 1;
                 if (!mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1502)) break;
-                // the softmax is done with unit u - 2: S^T(u - 2) has been read
-                if (u >= 2 && !mbar_wait(&sm.p_full[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
+                // S^T(u) overwrites dS^T(u - 2): wait until dK(u - 2) has read it
+                // (pd_done follows p_full: the softmax has also read S^T(u - 2))
+                if (u >= 2 && !mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1503)) break;
                 tc_fence_after();
                 const uint32_t qB = desc_lo(smem_u32(sm.q[s][0]), 16), doB = desc_lo(smem_u32(sm.dO[s][0]), 16);
                 #pragma unroll
@@ -374,7 +382,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             }
         }
     } else if (warp == W_MMB) {
-        // ------------------------------------------------ dV, dQ^T and dK issuer
+        // ------------------------------------------------ dV, dK and dQ^T issuer
         if (lane == 0 && U > 0) {
             constexpr uint32_t id_acc = idesc_f16(128, HD, 0, 1);
             constexpr uint32_t id_dq = idesc_f16(128, 64, 1, 1);
@@ -382,33 +390,33 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             int u = 0;
             for (; u < U; ++u) {
                 const int b = u & 1, s = u % DKDV_STAGES;
-                // P^T (TMEM) and dS^T (shared memory) of unit u are complete
+                // P^T and dS^T of unit u are in TMEM (and dS^T in shared memory)
                 if (!mbar_wait(&sm.p_full[b], (u >> 1) & 1, a.err, 1504)) break;
                 tc_fence_after();
-                const uint32_t dsA = desc_lo(smem_u32(sm.ds[b]), 16);          // dS^T, K-major
-                const uint32_t dsT = desc_lo(smem_u32(sm.ds[b]), SLAB128);     // dS^T as MN-major B
                 const uint32_t qT = desc_lo(smem_u32(sm.q[s][0]), SLAB64);
                 const uint32_t doT = desc_lo(smem_u32(sm.dO[s][0]), SLAB64);
-                // dV += P^T dO with P^T (fp16) read from TMEM over the dP^T columns
+                // dV += P^T dO with P^T (fp16) read from TMEM over the dP^T columns,
+                // dK += dS^T Q with dS^T (fp16) read from TMEM over the S^T columns
                 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ts(tmem + TDV, tmem + 128 * b + 64 + 8 * kk, desc_from_lo(doT + mnmajor_step(kk)),
                                 id_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                #pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16_ts(tmem + TDK, tmem + 128 * b + 8 * kk, desc_from_lo(qT + mnmajor_step(kk)),
+                                id_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&sm.pd_done[b]);
+                umma_commit(&sm.st_empty[s]);     // Q / dO of stage s are read
                 if (FUSE) {
                     // dQ^T [HD x 64 queries] = K^T [HD x 128 keys] . dS^T [128 keys x 64 queries],
                     // over the dP^T columns (after dV above has read P^T there)
+                    const uint32_t dsT = desc_lo(smem_u32(sm.ds[b]), SLAB128);     // dS^T as MN-major B
                     #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16(tmem + 128 * b + 64, desc_from_lo(kT + mnmajor_step(kk)),
                                  desc_from_lo(dsT + mnmajor_step(kk)), id_dq, kk > 0);
                     umma_commit(&sm.dq_full[b]);
                 }
-                #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + TDK, desc_from_lo(dsA + kmajor_step(kk, SLAB128)),
-                             desc_from_lo(qT + mnmajor_step(kk)), id_acc, (u > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&sm.pd_done[b]);
-                umma_commit(&sm.st_empty[s]);
             }
             if (u == U) umma_commit(&sm.acc_done);   // dV and dK are final
         }
@@ -427,8 +435,10 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             const bool valid = (m2 >> kh) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (u >> 1) & 1, a.err, 1001))) { ok = false; break; }
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.st_full[s], (u / DKDV_STAGES) & 1, a.err, 1002))) { ok = false; break; }
-            // dS^T(u - 2) has been read (dK, dQ^T) before dS^T(u) overwrites it
-            if (u >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.pd_done[b], ((u - 2) >> 1) & 1, a.err, 1003))) {
+            // dQ^T(u - 2) has read dS^T(u - 2) in shared memory before dS^T(u) overwrites
+            // it (the TMEM copies are safe: S^T(u) was written there after dK(u - 2))
+            if (FUSE && u >= 2 &&
+                !__all_sync(0xffffffffu, mbar_wait(&sm.dq_full[b], ((u - 2) >> 1) & 1, a.err, 1003))) {
                 ok = false;
                 break;
             }
@@ -443,7 +453,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             const float4* lq4 = reinterpret_cast<const float4*>(sm.lse[s] + c0);
             const float4* dq4 = reinterpret_cast<const float4*>(sm.di[s] + c0);
             const uint32_t ds_s = smem_u32(sm.ds[b]);
-            uint32_t pt[16];
+            uint32_t pt[16], dst[16];
             #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 // lse_p = 15 - LSE log2(e) and di_p = -D 2^-15 of the chunk's 8 queries
@@ -451,7 +461,7 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 const float4 y0 = dq4[2 * ch], y1 = dq4[2 * ch + 1];
                 const float lq[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
                 const float dq[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-                uint32_t wd[4];
+                uint32_t* wd = dst + 4 * ch;
                 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = ch * 8 + 2 * e;
@@ -472,10 +482,11 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     pt[ch * 4 + e] = pack_f16(p0, p1);
                     wd[e] = pack_f16(d0, d1);
                 }
-                st_shared_v4(ds_s + swz128(r, 4 * wg + ch), wd[0], wd[1], wd[2], wd[3]);
+                if (FUSE) st_shared_v4(ds_s + swz128(r, 4 * wg + ch), wd[0], wd[1], wd[2], wd[3]);
             }
             PRISM_TMEM_ST16(tmem + lane_off + 128 * b + 64 + 16 * wg, pt);
-            fence_proxy_async_smem();
+            PRISM_TMEM_ST16(tmem + lane_off + 128 * b + 16 * wg, dst);
+            if (FUSE) fence_proxy_async_smem();
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
@@ -516,13 +527,14 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         }
     } else if (FUSE && warp >= 10) {
         // ---------------------------------------------- dQ drain (warps 10-13)
-        const int d = (warp & 3) * 32 + lane;       // head-dim row of dQ^T = TMEM lane
+        // thread = head-dim row d of dQ^T (TMEM lane); each of the 64 columns is
+        // one query: a warp's reduction covers 32 adjacent floats of that query's
+        // accumulator row (one 128-byte line)
+        const int d = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const bool leader = (warp & 3) == 0 && lane == 0;
         HalfIter it{ents, ne, 0, 0, 1};
         int r64, m2;
-        int u = 0;                                  // units drained
-        for (; it.next(r64, m2); ++u) {
+        for (int u = 0; it.next(r64, m2); ++u) {
             const int b = u & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.dq_full[b], (u >> 1) & 1, a.err, 3001))) break;
             tc_fence_after();
@@ -532,25 +544,11 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.dq_free[b]);
-            const int64_t qrow = grow + (int64_t)r64 * 64;      // the group's dQ accumulator
+            if (prism_bad_index(a.err, r64 >= 0 && r64 < 2 * a.NT)) continue;   // checking build
+            float* dst = a.dq_acc + (grow + (int64_t)r64 * 64) * HD + d;
             #pragma unroll
-            for (int pass = 0; pass < 2; ++pass) {
-                if (leader) bulk_wait_read0();      // the previous reduce has read the stage
-                named_bar(1, 128);
-                #pragma unroll
-                for (int qq = 0; qq < 32; ++qq) sm.stage_dq[qq * HD + d] = __uint_as_float(v[pass * 32 + qq]);
-                fence_proxy_async_smem();
-                named_bar(1, 128);
-                if (leader) {
-                    tma_reduce_add_2d(&tm_dq, sm.stage_dq, 0, (int)(qrow + 32 * pass));
-                    bulk_commit();
-                }
-            }
+            for (int qq = 0; qq < 64; ++qq) red_add_f32(dst + (size_t)qq * HD, __uint_as_float(v[qq]));
         }
-        // after a failed wait, the four barriers of every undrained unit, which
-        // the other drain warps may still take
-        for (int k = 4 * u; k < 4 * U; ++k) named_bar(1, 128);
-        if (leader) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
@@ -814,6 +812,7 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     constexpr bool FUSE = HD == 128;
     static_assert(epilogue_fits<HD, FUSE>(), "dK/dV staging does not fit in the Q/dO/dS buffers");
     float* dq_acc = (float*)(b + P->L.dq_acc);
+    a.dq_acc = dq_acc;
     float* dk_acc = (float*)(b + P->L.dk_acc);
     float* dv_acc = (float*)(b + P->L.dv_acc);
     const int sm1 = (int)sizeof(DkdvSmem<HD, FUSE>) + 1024;
@@ -854,7 +853,7 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
             cudaMemsetAsync(dk_acc, 0, acc_bytes, s);
             cudaMemsetAsync(dv_acc, 0, acc_bytes, s);
             k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, chunks, nh), FUSE ? 480 : 352, sm1, s>>>(
-                P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dq, P->tm_dk, P->tm_dv, a);
+                P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dk, P->tm_dv, a);
             if (f32)
                 k_acc_finalize<float><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (float*)dK, dv_acc, 1.f / kPScale,
                                                             (float*)dV, src, dmax, g.N, HD, h0, a.qkv_max, 0, err);

@@ -116,6 +116,32 @@ __device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, const void* 
     asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];"
                  :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(src)), "r"(x), "r"(y) : "memory");
 }
+// Running maximum magnitude over a 16-byte chunk of 16- or 32-bit floats: a
+// magnitude is the value's bits with the sign cleared, so the maximum is an
+// integer maximum (per 16-bit half for bf16; a NaN's bits exceed infinity's).
+// abs_bits turns the result into fp32 bits (a bf16's bits shifted left by 16).
+template <typename T>
+__device__ __forceinline__ uint32_t fold_abs(uint32_t m, const uint4& x) {
+    static_assert(sizeof(T) == 2 || sizeof(T) == 4, "16- or 32-bit values");
+    if (sizeof(T) == 2) {
+        constexpr uint32_t mask = 0x7fff7fffu;
+        m = __vmaxu2(m, x.x & mask);
+        m = __vmaxu2(m, x.y & mask);
+        m = __vmaxu2(m, x.z & mask);
+        return __vmaxu2(m, x.w & mask);
+    }
+    constexpr uint32_t mask = 0x7fffffffu;
+    return max(max(m, x.x & mask), max(max(x.y & mask, x.z & mask), x.w & mask));
+}
+template <typename T>
+__device__ __forceinline__ uint32_t abs_bits(uint32_t m) {
+    return sizeof(T) == 2 ? max(m & 0xffffu, m >> 16) << 16 : m;
+}
+
+// Fire-and-forget fp32 add into global memory, performed in L2.
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" :: "l"(p), "f"(v) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk group has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

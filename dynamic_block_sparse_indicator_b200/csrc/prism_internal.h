@@ -120,7 +120,6 @@ struct prism_plan_s {
     std::vector<int64_t> loff_host;       // [LIST_KINDS][heads] offsets uploaded to L.loff
     CUtensorMap tm_q, tm_k, tm_v, tm_do;       // 2D [heads*N, D] fp16, 128-row boxes, 128B swizzle
     CUtensorMap tm_q64, tm_k64, tm_v64, tm_do64;  // the same with 64-row boxes
-    CUtensorMap tm_dq;                            // fp32 dQ accumulator [GH*N, D], 32-row boxes, no swizzle
     CUtensorMap tm_dk, tm_dv;                     // fp32 dK, dV accumulators, the same boxes
     // tm_do / tm_do64 cover the head group's dO copy: [GH*N, D]
     int64_t launches;                             // kernels launched so far

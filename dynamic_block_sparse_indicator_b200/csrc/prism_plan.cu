@@ -35,6 +35,7 @@
 #include <mutex>
 #include <new>
 
+#include "prism_dev.cuh"
 #include "prism_internal.h"
 
 namespace prism {
@@ -847,23 +848,37 @@ __global__ void __launch_bounds__(1024) k_zone_finalize_cut(DevPlan d, ShapeRule
 
 // Largest magnitude of each head's Q, K and V (float bits, atomicMax: the bits
 // of non-negative floats order like the values; a NaN's bits exceed infinity's).
+// One pass over 16-byte chunks (the inputs are 16-byte aligned and a head holds
+// N x D elements, a multiple of 16 bytes); see fold_abs.
 template <typename T>
 __global__ void __launch_bounds__(256) k_qkv_absmax(const T* __restrict__ Q, const T* __restrict__ K,
                                                     const T* __restrict__ V, uint32_t* __restrict__ mx,
                                                     int64_t n_per_head, int* err) {
+    static_assert(sizeof(T) == 2 || sizeof(T) == 4, "16- or 32-bit inputs");
     const int h = blockIdx.y;
-    const size_t off = (size_t)h * n_per_head;
-    float m[3] = {0.f, 0.f, 0.f};
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_per_head;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const float q = fabsf((float)Q[off + i]), k = fabsf((float)K[off + i]), v = fabsf((float)V[off + i]);
-        m[0] = (q > m[0] || q != q) ? q : m[0];
-        m[1] = (k > m[1] || k != k) ? k : m[1];
-        m[2] = (v > m[2] || v != v) ? v : m[2];
+    const int64_t n16 = n_per_head * (int64_t)sizeof(T) / 16;
+    const uint4* q = reinterpret_cast<const uint4*>(Q + (size_t)h * n_per_head);
+    const uint4* k = reinterpret_cast<const uint4*>(K + (size_t)h * n_per_head);
+    const uint4* v = reinterpret_cast<const uint4*>(V + (size_t)h * n_per_head);
+    uint32_t m[3] = {0u, 0u, 0u};
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + stride < n16; i += 2 * stride) {     // two chunks of each tensor in flight
+        const uint4 q0 = __ldg(q + i), q1 = __ldg(q + i + stride);
+        const uint4 k0 = __ldg(k + i), k1 = __ldg(k + i + stride);
+        const uint4 v0 = __ldg(v + i), v1 = __ldg(v + i + stride);
+        m[0] = fold_abs<T>(fold_abs<T>(m[0], q0), q1);
+        m[1] = fold_abs<T>(fold_abs<T>(m[1], k0), k1);
+        m[2] = fold_abs<T>(fold_abs<T>(m[2], v0), v1);
+    }
+    if (i < n16) {
+        m[0] = fold_abs<T>(m[0], __ldg(q + i));
+        m[1] = fold_abs<T>(m[1], __ldg(k + i));
+        m[2] = fold_abs<T>(m[2], __ldg(v + i));
     }
     #pragma unroll
     for (int t = 0; t < 3; ++t) {
-        uint32_t b = __float_as_uint(m[t]);
+        uint32_t b = abs_bits<T>(m[t]);
         for (int o = 16; o > 0; o >>= 1) b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
         if ((threadIdx.x & 31) == 0) {
             if (!(b <= 0x7f7fffffu)) atomicCAS(err, 0, PRISM_ERR_DEVICE_CHECK);      // inf or NaN
@@ -1413,7 +1428,6 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
     if (!st) st = make_tmap(&P->tm_k64, P->ws + L.kp, rows, g.D, 64);
     if (!st) st = make_tmap(&P->tm_v64, P->ws + L.vp, rows, g.D, 64);
     if (!st) st = make_tmap(&P->tm_do64, P->ws + L.dop, grows, g.D, 64);
-    if (!st) st = make_tmap_f32(&P->tm_dq, P->ws + L.dq_acc, grows, g.D, 32);
     if (!st) st = make_tmap_f32(&P->tm_dk, P->ws + L.dk_acc, grows, g.D, 32);
     if (!st) st = make_tmap_f32(&P->tm_dv, P->ws + L.dv_acc, grows, g.D, 32);
     if (st) { delete P; return st; }
@@ -1720,6 +1734,7 @@ extern "C" size_t prism_plan_item_bytes(prism_plan_t P, int item) {
         case PRISM_ITEM_SHAPE_ID2: return P->has_cuts ? H * g.Nz : 0;
         case PRISM_ITEM_ZONE_ENERGY: return P->has_cuts ? 4 * H * g.Nz * 7 : 0;
         case PRISM_ITEM_REGION_STATS: return P->has_cuts ? 4 * H * g.Nz * 8 : 0;
+        case PRISM_ITEM_QKV_MAX: return 4 * H * 3;
         default: return 0;
     }
 }
@@ -1759,6 +1774,7 @@ extern "C" int prism_plan_export(prism_plan_t P, int item, void* host_dst, size_
         case PRISM_ITEM_SHAPE_ID2: off = L.shape_id2; break;
         case PRISM_ITEM_ZONE_ENERGY: off = L.zdiff; break;
         case PRISM_ITEM_REGION_STATS: off = L.rstat; break;
+        case PRISM_ITEM_QKV_MAX: off = L.qkv_max; break;
         default: return PRISM_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);

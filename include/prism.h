@@ -351,7 +351,9 @@ PRISM_API int prism_status_read(int32_t* dev_status, int32_t* site, void* stream
 #define PRISM_ITEM_REGION_STATS 15 /* fp32 [heads][Nz][2][4] the parts' statistics (split zones) */
 #define PRISM_ITEM_LIST_OFFSETS 16 /* int64 [4][heads]: head h's first entry in the CSR, CSC,
                                       forward and backward tile lists */
-#define PRISM_ITEM_COUNT     17
+#define PRISM_ITEM_QKV_MAX   17  /* uint32 [heads][3]: fp32 bits of max |Q|, |K|, |V| of each head,
+                                      which set the copies' power-of-two scales */
+#define PRISM_ITEM_COUNT     18
 
 /* Bytes of an item (0 for an unknown item). */
 PRISM_API size_t prism_plan_item_bytes(prism_plan_t plan, int item);

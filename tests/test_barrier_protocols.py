@@ -185,8 +185,10 @@ def test_guidance_map_protocol(heads, MT, rescale):
 # ------------------------------------------------------------- backward
 def backward_roles(U, fuse=True, ST=3):
     """k_bwd_dkdv: 64-query units of a key tile, a 3-stage Q/dO ring, S^T/dP^T
-    double-buffered in TMEM; issuer A (S^T, dP^T), issuer B (dV, dQ^T, dK),
-    softmax (P'^T into TMEM, dS^T into shared memory), dQ^T drain (fuse)."""
+    double-buffered in TMEM; issuer A (S^T, dP^T), issuer B (dV and dK with
+    P^T and dS^T read from TMEM, then dQ^T), softmax (P'^T over dP^T and dS^T
+    over S^T in TMEM, dS^T also into shared memory when fused), dQ^T drain
+    (fuse)."""
     def producer():
         yield ("arrive", "kv")
         for u in range(U):
@@ -201,7 +203,7 @@ def backward_roles(U, fuse=True, ST=3):
             b = u & 1
             yield ("wait", f"st_full{u % ST}", u // ST)
             if u >= 2:
-                yield ("wait", f"p_full{b}", (u - 2) >> 1)
+                yield ("wait", f"pd_done{b}", (u - 2) >> 1)          # S^T over dS^T(u - 2)
                 yield ("wait", f"dq_free{b}" if fuse else f"pd_done{b}", (u - 2) >> 1)
             yield ("arrive", f"s_full{b}")
 
@@ -209,10 +211,10 @@ def backward_roles(U, fuse=True, ST=3):
         for u in range(U):
             b = u & 1
             yield ("wait", f"p_full{b}", u >> 1)
-            if fuse:
-                yield ("arrive", f"dq_full{b}")
             yield ("arrive", f"pd_done{b}")
             yield ("arrive", f"st_empty{u % ST}")
+            if fuse:
+                yield ("arrive", f"dq_full{b}")
         yield ("arrive", "acc_done")
 
     def softmax():
@@ -220,8 +222,8 @@ def backward_roles(U, fuse=True, ST=3):
             b = u & 1
             yield ("wait", f"s_full{b}", u >> 1)
             yield ("wait", f"st_full{u % ST}", u // ST)
-            if u >= 2:
-                yield ("wait", f"pd_done{b}", (u - 2) >> 1)
+            if fuse and u >= 2:
+                yield ("wait", f"dq_full{b}", (u - 2) >> 1)          # dS^T(u - 2) in shared memory read
             yield ("arrive", f"p_full{b}")
         yield ("wait", "acc_done", 0)
 
