@@ -77,6 +77,8 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_plan_list_bytes": (i32, [vp, C.POINTER(sz), vp]),
         "prism_plan_attach_lists": (i32, [vp, vp, sz, vp]),
         "prism_plan": (i32, [pp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
+        "prism_plan_sharded": (i32, [pp, C.POINTER(vp), C.POINTER(vp), C.POINTER(vp), i32, i32, i32, vp,
+                                     vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import": (i32, [pp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import_cuts": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_attn_fwd": (i32, [vp, vp, vp, vp]),
@@ -294,6 +296,60 @@ def plan(Q, K, V, a_map, params: PrismParams, workspace=None, stream=None, compa
             lib.prism_plan_destroy(h)
             raise
     return Plan(params, h, workspace, (Q, K, V, a_map), lists)
+
+
+def plan_sharded(Qs, Ks, Vs, a_map, params: PrismParams, head0=0, heads_total=None, workspace=None,
+                 stream=None, compact=False) -> Plan:
+    """Stages 1-3 for heads head0 .. head0 + params.heads - 1 of inputs held as
+    token shards: Qs, Ks, Vs are equal-length lists (one entry per shard, shard s
+    holding frames [s T/n, (s + 1) T/n) of every head as [heads_total, N/n, D]),
+    each a contiguous CUDA tensor or a raw device address (an int: another GPU's
+    shard mapped for peer access).  The plan then runs like `plan` on those heads."""
+    import torch
+    lib = load()
+    n = len(Qs)
+    if n == 0 or len(Ks) != n or len(Vs) != n:
+        raise ValueError("Qs, Ks, Vs must be non-empty lists of the same length")
+    N = params.T * params.H * params.W
+    if params.T % n:
+        raise ValueError(f"{n} shards do not divide T = {params.T}")
+    want = torch.float32 if params.dtype == PRISM_F32 else torch.bfloat16
+    device, tensors = None, []
+    for t in (*Qs, *Ks, *Vs):
+        if isinstance(t, int):
+            continue
+        if t.dtype != want or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("shards must be contiguous CUDA tensors of the plan's dtype (or device addresses)")
+        if heads_total is None:
+            heads_total = t.shape[0]
+        if tuple(t.shape) != (heads_total, N // n, params.head_dim):
+            raise ValueError(f"expected shards of [heads_total, N/shards, D] = "
+                             f"{(heads_total, N // n, params.head_dim)}, got {tuple(t.shape)}")
+        device = device or t.device
+        tensors.append(t)
+    if heads_total is None:
+        raise ValueError("heads_total is needed when every shard is given as an address")
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    addr = lambda t: t if isinstance(t, int) else t.data_ptr()
+    arrs = [(C.c_void_p * n)(*[addr(t) for t in xs]) for xs in (Qs, Ks, Vs)]
+    need = core_bytes(params) if compact else workspace_bytes(params)
+    if need == 0:
+        raise PrismError(PRISM_ERR_INVALID_ARG, "prism_plan_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    h = C.c_void_p()
+    st = lib.prism_plan_sharded(C.byref(params), arrs[0], arrs[1], arrs[2], n, int(heads_total), int(head0),
+                                _ptr(a_map), _ptr(workspace), workspace.numel(), _stream(stream), C.byref(h))
+    if st:
+        raise PrismError(st, "prism_plan_sharded")
+    lists = None
+    if workspace.numel() < workspace_bytes(params):
+        try:
+            lists = _attach_lists(lib, h, device, stream)
+        except PrismError:
+            lib.prism_plan_destroy(h)
+            raise
+    return Plan(params, h, workspace, (tuple(tensors), a_map), lists)
 
 
 def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None, stream=None,

@@ -161,6 +161,41 @@ __constant__ int8_t c_log2shape[16][3] = {
     {1, 3, 3}, {2, 2, 3}, {2, 3, 2}, {3, 1, 3}, {3, 2, 2}, {3, 3, 1},
     {2, 3, 3}, {3, 2, 3}, {3, 3, 2}};
 
+// Where row (h, n) of a [heads][N][D] input lives.  A plain tensor is one
+// shard.  A sequence-parallel caller's input is `n` token shards, shard s
+// holding frames [s F, (s + 1) F) of every one of `stride_heads` heads as
+// [stride_heads][F H W][D] (a rank's part of the sequence); the plan covers
+// heads head0, head0 + 1, ... of them.  The shard pointers may be other GPUs'
+// memory mapped for peer access: the plan reads them with plain loads, so the
+// head-to-rank exchange and the reorder into block order are one pass.
+constexpr int kMaxShards = 16;
+struct TokenRows {
+    const void* p[kMaxShards];
+    int64_t S;             // tokens per shard (F H W)
+    int F;                 // frames per shard
+    int n;                 // shards
+    int stride_heads;      // heads held by each shard
+    int head0;             // the shard head of this plan's head 0
+    // row (h, token of frame t) as element offset into shard p[t / F]
+    template <typename T>
+    __device__ __forceinline__ const T* row(int h, int t, int64_t tok, int D) const {
+        const int sh = n == 1 ? 0 : t / F;
+        return static_cast<const T*>(p[sh]) +
+               ((int64_t)(head0 + h) * S + (tok - (int64_t)sh * S)) * D;
+    }
+};
+
+static TokenRows plain_rows(const void* x, int64_t N, int T, int heads) {
+    TokenRows r{};
+    r.p[0] = x;
+    r.S = N;
+    r.F = T;
+    r.n = 1;
+    r.stride_heads = heads;
+    r.head0 = 0;
+    return r;
+}
+
 struct DevPlan {
     int T, H, W, heads, D, Zh, Zw, Nz, NB, NT, WORDS;
     int64_t N;
@@ -437,7 +472,7 @@ struct Pair<float> {
 // MODE 2: statistics of the two parts of every split zone (grid z = part),
 // over the part's frames [t0, t1) only.
 template <typename T, int D, int MODE>
-__global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restrict__ V, float cut_ratio) {
+__global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const TokenRows V, float cut_ratio) {
     constexpr int CP = D / 2;            // channel pairs
     constexpr int G = 256 / CP;          // groups
     constexpr int RPG = 8 / G;           // h-rows per group
@@ -460,11 +495,10 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restri
     const int L = t1 - t0;
     const int zt = m / (d.Zh * d.Zw), zh = (m / d.Zw) % d.Zh, zw = m % d.Zw;
     const int cp = threadIdx.x % CP, grp = threadIdx.x / CP;
-    const T* Vh = V + (size_t)h * d.N * D;
     auto tok = [&](int lt, int lh, int lw) -> int64_t {
         return ((int64_t)(8 * zt + lt) * d.H + 8 * zh + lh) * d.W + 8 * zw + lw;
     };
-    const float2 ref = Pair<T>::load(Vh + tok(t0, 0, 0) * D + 2 * cp);
+    const float2 ref = Pair<T>::load(V.row<T>(h, 8 * zt + t0, tok(t0, 0, 0), D) + 2 * cp);
     float ST[2][8], SQ[2][8], SW[2][8], SH[2][RPG], Ds[2], Dq[2], Et[2][NE > 0 ? NE : 1];
     #pragma unroll
     for (int c = 0; c < 2; ++c) {
@@ -486,8 +520,9 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const T* __restri
         for (int lt = 0; lt < 8; ++lt) {
             if (MODE == 2 && (lt < t0 || lt >= t1)) continue;
             float2 x[8];
+            const T* vr = V.row<T>(h, 8 * zt + lt, tok(lt, lh, 0), D) + 2 * cp;   // 8 adjacent tokens
             #pragma unroll
-            for (int lw = 0; lw < 8; ++lw) x[lw] = Pair<T>::load(Vh + tok(lt, lh, lw) * D + 2 * cp);
+            for (int lw = 0; lw < 8; ++lw) x[lw] = Pair<T>::load(vr + lw * D);
             #pragma unroll
             for (int lw = 0; lw < 8; ++lw) {
                 const float v0 = x[lw].x - ref.x, v1 = x[lw].y - ref.y;
@@ -851,30 +886,31 @@ __global__ void __launch_bounds__(1024) k_zone_finalize_cut(DevPlan d, ShapeRule
 // One pass over 16-byte chunks (the inputs are 16-byte aligned and a head holds
 // N x D elements, a multiple of 16 bytes); see fold_abs.
 template <typename T>
-__global__ void __launch_bounds__(256) k_qkv_absmax(const T* __restrict__ Q, const T* __restrict__ K,
-                                                    const T* __restrict__ V, uint32_t* __restrict__ mx,
-                                                    int64_t n_per_head, int* err) {
-    static_assert(sizeof(T) == 2 || sizeof(T) == 4, "16- or 32-bit inputs");
+__global__ void __launch_bounds__(256) k_qkv_absmax(const TokenRows Q, const TokenRows K, const TokenRows V,
+                                                    uint32_t* __restrict__ mx, int D, int* err) {
     const int h = blockIdx.y;
-    const int64_t n16 = n_per_head * (int64_t)sizeof(T) / 16;
-    const uint4* q = reinterpret_cast<const uint4*>(Q + (size_t)h * n_per_head);
-    const uint4* k = reinterpret_cast<const uint4*>(K + (size_t)h * n_per_head);
-    const uint4* v = reinterpret_cast<const uint4*>(V + (size_t)h * n_per_head);
-    uint32_t m[3] = {0u, 0u, 0u};
+    const int64_t n16 = Q.S * D * (int64_t)sizeof(T) / 16;      // 16-byte chunks of one shard's head
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; i + stride < n16; i += 2 * stride) {     // two chunks of each tensor in flight
-        const uint4 q0 = __ldg(q + i), q1 = __ldg(q + i + stride);
-        const uint4 k0 = __ldg(k + i), k1 = __ldg(k + i + stride);
-        const uint4 v0 = __ldg(v + i), v1 = __ldg(v + i + stride);
-        m[0] = fold_abs<T>(fold_abs<T>(m[0], q0), q1);
-        m[1] = fold_abs<T>(fold_abs<T>(m[1], k0), k1);
-        m[2] = fold_abs<T>(fold_abs<T>(m[2], v0), v1);
-    }
-    if (i < n16) {
-        m[0] = fold_abs<T>(m[0], __ldg(q + i));
-        m[1] = fold_abs<T>(m[1], __ldg(k + i));
-        m[2] = fold_abs<T>(m[2], __ldg(v + i));
+    uint32_t m[3] = {0u, 0u, 0u};
+    for (int sh = 0; sh < Q.n; ++sh) {
+        const int64_t off = ((int64_t)(Q.head0 + h) * Q.S) * D;   // the same layout for Q, K, V
+        const uint4* q = reinterpret_cast<const uint4*>(static_cast<const T*>(Q.p[sh]) + off);
+        const uint4* k = reinterpret_cast<const uint4*>(static_cast<const T*>(K.p[sh]) + off);
+        const uint4* v = reinterpret_cast<const uint4*>(static_cast<const T*>(V.p[sh]) + off);
+        int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        for (; i + stride < n16; i += 2 * stride) {     // two chunks of each tensor in flight
+            const uint4 q0 = __ldg(q + i), q1 = __ldg(q + i + stride);
+            const uint4 k0 = __ldg(k + i), k1 = __ldg(k + i + stride);
+            const uint4 v0 = __ldg(v + i), v1 = __ldg(v + i + stride);
+            m[0] = fold_abs<T>(fold_abs<T>(m[0], q0), q1);
+            m[1] = fold_abs<T>(fold_abs<T>(m[1], k0), k1);
+            m[2] = fold_abs<T>(fold_abs<T>(m[2], v0), v1);
+        }
+        if (i < n16) {
+            m[0] = fold_abs<T>(m[0], __ldg(q + i));
+            m[1] = fold_abs<T>(m[1], __ldg(k + i));
+            m[2] = fold_abs<T>(m[2], __ldg(v + i));
+        }
     }
     #pragma unroll
     for (int t = 0; t < 3; ++t) {
@@ -895,9 +931,8 @@ __device__ __forceinline__ uint32_t ph2(float a, float b) {
 // Gather one block: rows in block order into the fp16 copies, raster index of
 // each slot into src, and fp32 block means of Q and K (from the input values).
 template <typename T, int D>
-__global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restrict__ Q,
-                                                     const T* __restrict__ K,
-                                                     const T* __restrict__ V) {
+__global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const TokenRows Q, const TokenRows K,
+                                                     const TokenRows V) {
     constexpr int EPC = 16 / sizeof(T);      // input elements per 16-byte chunk
     constexpr int CPR = D / EPC;             // chunks per row
     constexpr int RP = 256 / CPR;            // rows in flight
@@ -937,15 +972,14 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const T* __restr
     const size_t hoff = (size_t)h * d.N * D;
     for (int r = rl; r < vol; r += RP) {
         const int lw = r % bw, lh = (r / bw) % bh, lt = r / (bw * bh);
-        const int64_t n = ((int64_t)(8 * zt + toff + kt * bt + lt) * d.H + 8 * zh + kh * bh + lh) * d.W +
-                          8 * zw + kw * bw + lw;
+        const int ft = 8 * zt + toff + kt * bt + lt;
+        const int64_t n = ((int64_t)ft * d.H + 8 * zh + kh * bh + lh) * d.W + 8 * zw + kw * bw + lw;
         if (prism_bad_index(d.err, n >= 0 && n < d.N && start + r < d.N)) continue;
-        const size_t so = hoff + (size_t)n * D + (size_t)c * EPC;
         const size_t dst = hoff + (size_t)(start + r) * D + (size_t)c * EPC;
         if (c == 0) d.src[(size_t)h * d.N + start + r] = (int)n;
-        const uint4 q4 = *reinterpret_cast<const uint4*>(Q + so);
-        const uint4 k4 = *reinterpret_cast<const uint4*>(K + so);
-        const uint4 v4 = *reinterpret_cast<const uint4*>(V + so);
+        const uint4 q4 = *reinterpret_cast<const uint4*>(Q.row<T>(h, ft, n, D) + c * EPC);
+        const uint4 k4 = *reinterpret_cast<const uint4*>(K.row<T>(h, ft, n, D) + c * EPC);
+        const uint4 v4 = *reinterpret_cast<const uint4*>(V.row<T>(h, ft, n, D) + c * EPC);
         float fq[EPC], fk[EPC], fv[EPC];
         if constexpr (sizeof(T) == 2) {
             const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&q4);
@@ -1436,30 +1470,29 @@ static int plan_common(const prism_params* p, const void* Q, const void* K, cons
 }
 
 template <typename T, int D>
-static void launch_stats(prism_plan_s* P, const DevPlan& d, const void* V, cudaStream_t s) {
+static void launch_stats(prism_plan_s* P, const DevPlan& d, const TokenRows& V, cudaStream_t s) {
     const Geom& g = P->g;
     const int sm = (256 / (D / 2)) * D * 26 * (int)sizeof(float);
     if (!P->has_cuts) {
         cudaFuncSetAttribute(k_zone_stats<T, D, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V, 0.f);
+        k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, V, 0.f);
         return;
     }
     // whole zones with their energies and split decisions, then the parts of the split zones
     const int sm1 = (256 / (D / 2)) * D * 33 * (int)sizeof(float);
     cudaFuncSetAttribute(k_zone_stats<T, D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
-    k_zone_stats<T, D, 1><<<dim3(g.Nz, g.heads), 256, sm1, s>>>(d, (const T*)V, P->p.cut_ratio);
+    k_zone_stats<T, D, 1><<<dim3(g.Nz, g.heads), 256, sm1, s>>>(d, V, P->p.cut_ratio);
     cudaFuncSetAttribute(k_zone_stats<T, D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    k_zone_stats<T, D, 2><<<dim3(g.Nz, g.heads, 2), 256, sm, s>>>(d, (const T*)V, 0.f);
+    k_zone_stats<T, D, 2><<<dim3(g.Nz, g.heads, 2), 256, sm, s>>>(d, V, 0.f);
 }
 
 template <typename T, int D>
-static void launch_gather(prism_plan_s* P, const DevPlan& d, const void* Q, const void* K,
-                          const void* V, cudaStream_t s) {
+static void launch_gather(prism_plan_s* P, const DevPlan& d, const TokenRows& Q, const TokenRows& K,
+                          const TokenRows& V, cudaStream_t s) {
     const Geom& g = P->g;
     cudaMemsetAsync(d.qkv_max, 0, sizeof(uint32_t) * 3 * g.heads, s);
-    k_qkv_absmax<T><<<dim3(296, g.heads), 256, 0, s>>>((const T*)Q, (const T*)K, (const T*)V, d.qkv_max,
-                                                        g.N * D, d.err);
-    k_gather_pool<T, D><<<dim3(g.NB, g.heads), 256, 0, s>>>(d, (const T*)Q, (const T*)K, (const T*)V);
+    k_qkv_absmax<T><<<dim3(296, g.heads), 256, 0, s>>>(Q, K, V, d.qkv_max, D, d.err);
+    k_gather_pool<T, D><<<dim3(g.NB, g.heads), 256, 0, s>>>(d, Q, K, V);
 }
 
 // Counts and pointers of the index lists (CSR rows already counted by the
@@ -1494,7 +1527,7 @@ static void launch_list_fill(prism_plan_s* P, const DevPlan& d, cudaStream_t s) 
                                                             g.NB, g.NT, g.WORDS, 1, d.err);
 }
 
-static int run_plan(prism_plan_s* P, const void* Q, const void* K, const void* V, const float* amap,
+static int run_plan(prism_plan_s* P, const TokenRows& Q, const TokenRows& K, const TokenRows& V, const float* amap,
                     const uint8_t* given_shapes, const uint32_t* given_sel, cudaStream_t s,
                     const uint8_t* given_cut = nullptr, const uint8_t* given_sid2 = nullptr) {
     // kernels launched below: audio 1-3, stats 1-2, finalize 1, max + gather 2, select
@@ -1681,7 +1714,43 @@ extern "C" int prism_plan(const prism_params* p, const void* Q, const void* K, c
     if (st) return st;
     P->has_audio = a_map != nullptr;
     P->has_cuts = p->cut_ratio > 0.f;
-    st = run_plan(P, Q, K, V, a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+    const Geom& g = P->g;
+    st = run_plan(P, plain_rows(Q, g.N, g.T, g.heads), plain_rows(K, g.N, g.T, g.heads),
+                  plain_rows(V, g.N, g.T, g.heads), a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+    if (st) { delete P; return st; }
+    *out = P;
+    return PRISM_OK;
+}
+
+extern "C" int prism_plan_sharded(const prism_params* p, const void* const* Q, const void* const* K,
+                                  const void* const* V, int shards, int heads_total, int head0,
+                                  const float* a_map, void* workspace, size_t ws_bytes, void* stream,
+                                  prism_plan_t* out) {
+    if (!out) return PRISM_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!p || !Q || !K || !V || shards < 1 || shards > kMaxShards) return PRISM_ERR_INVALID_ARG;
+    if (a_map && !aligned16(a_map)) return PRISM_ERR_INVALID_ARG;
+    if (p->T % shards != 0 || head0 < 0 || heads_total < 1 || p->heads < 1 || head0 + p->heads > heads_total)
+        return PRISM_ERR_INVALID_ARG;
+    for (int i = 0; i < shards; ++i)
+        if (!Q[i] || !K[i] || !V[i] || !aligned16(Q[i]) || !aligned16(K[i]) || !aligned16(V[i]))
+            return PRISM_ERR_INVALID_ARG;
+    prism_plan_s* P = nullptr;
+    int st = plan_common(p, Q[0], K[0], V[0], workspace, ws_bytes, &P);
+    if (st) return st;
+    P->has_audio = a_map != nullptr;
+    P->has_cuts = p->cut_ratio > 0.f;
+    const Geom& g = P->g;
+    TokenRows rq{}, rk{}, rv{};
+    for (TokenRows* r : {&rq, &rk, &rv}) {
+        r->F = g.T / shards;
+        r->S = (int64_t)r->F * g.H * g.W;
+        r->n = shards;
+        r->stride_heads = heads_total;
+        r->head0 = head0;
+    }
+    for (int i = 0; i < shards; ++i) { rq.p[i] = Q[i]; rk.p[i] = K[i]; rv.p[i] = V[i]; }
+    st = run_plan(P, rq, rk, rv, a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
     if (st) { delete P; return st; }
     *out = P;
     return PRISM_OK;
@@ -1700,7 +1769,10 @@ extern "C" int prism_plan_import_cuts(const prism_params* p, const void* Q, cons
     if (st) return st;
     P->has_audio = 0;
     P->has_cuts = zone_cut != nullptr;
-    st = run_plan(P, Q, K, V, nullptr, shape_id, sel, static_cast<cudaStream_t>(stream), zone_cut, shape_id2);
+    const Geom& g = P->g;
+    st = run_plan(P, plain_rows(Q, g.N, g.T, g.heads), plain_rows(K, g.N, g.T, g.heads),
+                  plain_rows(V, g.N, g.T, g.heads), nullptr, shape_id, sel, static_cast<cudaStream_t>(stream),
+                  zone_cut, shape_id2);
     if (st) { delete P; return st; }
     *out = P;
     return PRISM_OK;
@@ -1933,7 +2005,7 @@ template <typename T, int D>
 static void noalloc_stats(const Geom& g, const DevPlan& d, const void* V, cudaStream_t s) {
     const int sm = (256 / (D / 2)) * D * 26 * (int)sizeof(float);
     cudaFuncSetAttribute(k_zone_stats<T, D, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, (const T*)V, 0.f);
+    k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, plain_rows(V, g.N, g.T, g.heads), 0.f);
 }
 
 // Device address of the scratch array, looked up once per device (with that

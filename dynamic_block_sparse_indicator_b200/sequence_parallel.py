@@ -18,6 +18,14 @@ layout and heads [r H/P, (r + 1) H/P) in the head layout.  Each direction is one
 all-to-all (NCCL over NVLink between GPUs; gloo on the host for the tests); the
 plan itself needs no collective.  The library computes nothing here: this
 module only moves tensors between ranks with torch.distributed.
+
+Where the ranks' sequence shards of Q, K and V are mapped into each other's
+address space (torch symmetric memory, CUDA IPC), the inbound exchange can be
+left out: `_lib.plan_sharded(qs, ks, vs, a, params, head0=h0, heads_total=H)`
+plans this rank's heads (`rank_heads`) straight from every rank's shard, the
+plan's reorder into block order reading the other GPUs' rows over NVLink, so
+the all-to-all and the reorder are one pass.  The plan then runs as above, and
+the results go back with `heads_to_seq`.
 """
 from __future__ import annotations
 
@@ -27,6 +35,13 @@ import torch.distributed as dist
 
 def _world(group):
     return dist.get_world_size(group), dist.get_rank(group)
+
+
+def rank_heads(rank: int, world: int, heads: int) -> tuple[int, int]:
+    """(first head, head count) of `rank` in the head layout: heads [r H/P, (r + 1) H/P)."""
+    if heads % world:
+        raise ValueError(f"heads ({heads}) must be a multiple of the group size ({world})")
+    return rank * (heads // world), heads // world
 
 
 def seq_to_heads(x: torch.Tensor, group=None) -> torch.Tensor:

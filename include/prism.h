@@ -203,6 +203,34 @@ PRISM_API int prism_plan(const prism_params* p, const void* Q, const void* K, co
                prism_plan_t* out);
 
 /*
+ * prism_plan_sharded -- prism_plan for inputs held as token shards, the layout
+ * a sequence-parallel rank holds (the pages train with sequence parallelism 8:
+ * page paper.rainbus.top, section "方法步骤详情").  The plan covers heads
+ * head0 .. head0 + p->heads - 1 of the shards' heads_total heads and reads
+ * their rows straight from the shards, so the sequence-to-head exchange that
+ * would precede a head-sharded plan and the plan's reorder into block order are
+ * one pass; everything after the plan (forward, backward, exports) is that of
+ * a prism_plan over those heads' [p->heads][N][head_dim] tensors.
+ * Arguments
+ *   Q, K, V      host arrays of `shards` device pointers.  Shard s holds frames
+ *                [s T/shards, (s + 1) T/shards) of every head as
+ *                [heads_total][(T/shards) H W][head_dim] of `dtype`, raster
+ *                order inside the shard; 16-byte aligned.  A pointer may be
+ *                another GPU's memory mapped for peer access (symmetric
+ *                memory, an IPC mapping): the kernels read it with plain
+ *                loads, never a TMA multicast.
+ *   shards       1 .. 16, dividing T.
+ *   heads_total  heads held by each shard; head0 + p->heads <= heads_total.
+ *   the rest     as prism_plan.
+ * Returns PRISM_ERR_INVALID_ARG for a shard count that does not divide T, a
+ * head range outside the shards, or a null or misaligned pointer.
+ */
+PRISM_API int prism_plan_sharded(const prism_params* p, const void* const* Q, const void* const* K,
+                                 const void* const* V, int shards, int heads_total, int head0,
+                                 const float* a_map, void* workspace, size_t ws_bytes, void* stream,
+                                 prism_plan_t* out);
+
+/*
  * prism_plan_import -- the same plan, but with stage 1's shapes and stage 3's
  * selection supplied by the caller instead of computed (a fixed-shape
  * comparator, a cached plan, or a plan computed elsewhere).  Runs stage 2

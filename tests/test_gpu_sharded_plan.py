@@ -1,0 +1,95 @@
+"""Plans read straight from sequence shards (prism_plan_sharded) on one GPU.
+
+A sequence-parallel rank holds frames [s T/P, (s + 1) T/P) of every head; the
+sharded plan of a head range reads every shard's rows itself (on several GPUs
+through peer mappings), so no all-to-all precedes it.  Here the P shards are
+separate buffers on one GPU standing in for the ranks' memory.  For every head
+range (the ranks of the head layout) the sharded plan must equal prism_plan on
+the gathered heads: shapes, block offsets, permutation, pooled means of every
+block, the per-head input maxima and the selection bit for bit, O and LSE bit for bit, the
+gradients to fp32 summation order.  Cases: bf16 with 4 shards of 4 frames
+(every 8-frame zone spans two shards) and adaptive temporal boundaries on, and
+the fp32 tiny workload with 2 shards.  Invalid shard counts and head ranges are
+rejected before any launch.
+"""
+import numpy as np
+import pytest
+import torch
+
+from dynamic_block_sparse_indicator_b200 import _lib
+from dynamic_block_sparse_indicator_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+ITEMS = ("shape_id", "nblocks", "blk_start", "src", "sel_bits", "qkv_max")
+
+
+def _shards(x, P):
+    n = x.shape[1] // P
+    return [x[:, s * n:(s + 1) * n].contiguous() for s in range(P)]
+
+
+def _run(pl, dO):
+    O, lse = pl.attn_fwd()
+    grads = pl.attn_bwd(dO, O, lse)
+    torch.cuda.synchronize()
+    assert pl.status() == _lib.PRISM_OK
+    return (O, lse) + tuple(grads)
+
+
+@pytest.mark.parametrize("case", ["bf16_4shards_cuts", "f32_2shards"])
+def test_sharded_plan_equals_gathered_plan(case, cuda_device):
+    if case == "bf16_4shards_cuts":
+        w = syn.workload(2, T=16, H=32, W=32, shot_cuts=[6])
+        P, heads, ranks, cut, dt = 4, 4, 2, 2.5, _lib.PRISM_BF16
+    else:
+        w = syn.workload(0)
+        P, heads, ranks, cut, dt = 2, 2, 2, 0.0, _lib.PRISM_F32
+    Q, K, V = syn.make_qkv(w, device="cuda", heads=heads)
+    dO = syn.make_dout(w, device="cuda", heads=heads, out_dtype=torch.bfloat16).float()
+    a = syn.make_amap(w, device="cuda")
+    qs, ks, vs = _shards(Q, P), _shards(K, P), _shards(V, P)
+    nh = heads // ranks
+    for r in range(ranks):
+        h0 = r * nh
+        sl = slice(h0, h0 + nh)
+        prm = _lib.make_params(w.T, w.H, w.W, nh, w.head_dim, dt, w.top_k, w.top_p, w.eps, cut_ratio=cut)
+        ref = _lib.plan(Q[sl].contiguous(), K[sl].contiguous(), V[sl].contiguous(), a, prm)
+        got = _lib.plan_sharded(qs, ks, vs, a, prm, head0=h0, heads_total=heads)
+        for item in ITEMS + (("zone_cut", "shape_id2") if cut else ()):
+            np.testing.assert_array_equal(got.export(item), ref.export(item), err_msg=f"{case} rank {r} {item}")
+        # pooled means of each head's blocks (rows past a head's block count are not written)
+        nb = ref.export("nblocks")
+        for item in ("qbar", "kbar"):
+            gm, rm = (x.export(item).reshape(nh, w.N // 64, w.head_dim) for x in (got, ref))
+            for h in range(nh):
+                np.testing.assert_array_equal(gm[h, :nb[h]], rm[h, :nb[h]], err_msg=f"{case} rank {r} {item} {h}")
+        g_out, r_out = _run(got, dO[sl].contiguous()), _run(ref, dO[sl].contiguous())
+        for g, e, nm in zip(g_out, r_out, ("O", "LSE", "dQ", "dK", "dV")):
+            g, e = g.cpu(), e.cpu()
+            if nm in ("O", "LSE"):
+                assert torch.equal(g, e), f"{case} rank {r} {nm}"
+            else:                      # partial sums reduced in the order the CTAs finish
+                diff, scale = (g - e).abs().max().item(), e.abs().max().item()
+                assert diff <= 1e-5 * scale, f"{case} rank {r} {nm}: {diff:.3e} at scale {scale:.3e}"
+
+
+def test_sharded_plan_rejects_bad_layouts(cuda_device):
+    w = syn.workload(0)
+    Q, K, V = syn.make_qkv(w, device="cuda", heads=2)
+    a = syn.make_amap(w, device="cuda")
+    prm = _lib.make_params(w.T, w.H, w.W, 2, w.head_dim, _lib.PRISM_F32, w.top_k, w.top_p, w.eps)
+    N = w.N
+    # 3 shards do not divide T = 8 (rejected by the binding before the call)
+    with pytest.raises(ValueError):
+        _lib.plan_sharded([Q] * 3, [K] * 3, [V] * 3, a, prm)
+    qs, ks, vs = _shards(Q, 2), _shards(K, 2), _shards(V, 2)
+    # the head range runs past the shards' heads: rejected by the library
+    with pytest.raises(_lib.PrismError) as e:
+        _lib.plan_sharded(qs, ks, vs, a, prm, head0=1, heads_total=2)
+    assert e.value.status == _lib.PRISM_ERR_INVALID_ARG
+    # a misaligned shard address
+    with pytest.raises(_lib.PrismError) as e:
+        _lib.plan_sharded([qs[0].data_ptr() + 4, qs[1].data_ptr()], ks, vs, a, prm, heads_total=2)
+    assert e.value.status == _lib.PRISM_ERR_INVALID_ARG
+    assert N % 2 == 0

@@ -3,7 +3,8 @@
 Every rank builds the same global [H, N, D] tensor from one seed and keeps its
 token slice; seq_to_heads must give exactly the global tensor's head slice of
 the rank (every token), heads_to_seq must undo it bit for bit, and gather_map
-must rebuild the whole per-token map on every rank.
+must rebuild the whole per-token map on every rank; rank_heads must name the
+rank's head slice (the head range a sharded plan on that rank covers).
 """
 import os
 import socket
@@ -42,7 +43,9 @@ def _worker(rank, world, port, out, H, N, D):
             sp.seq_to_heads(local[:H - 1] if H > 1 else local)   # heads not a multiple of the group
         except ValueError:
             bad = True
-        out[rank] = (ok_fwd, ok_back, ok_map, shape_ok, bad)
+        h0, nh = sp.rank_heads(rank, world, H)
+        ok_range = (h0, nh) == (rank * h, h) and torch.equal(heads, full[h0:h0 + nh])
+        out[rank] = (ok_fwd, ok_back, ok_map, shape_ok, bad, ok_range)
     finally:
         dist.destroy_process_group()
 
@@ -60,4 +63,4 @@ def test_seq_head_exchange(world, H, N, D):
         p.join(timeout=180)
         assert p.exitcode == 0
     for r in range(world):
-        assert out[r] == (True, True, True, True, True), (r, out[r])
+        assert out[r] == (True, True, True, True, True, True), (r, out[r])
