@@ -82,6 +82,9 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_plan_import": (i32, [pp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import_cuts": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_attn_fwd": (i32, [vp, vp, vp, vp]),
+        "prism_attn_fwd_sharded": (i32, [vp, C.POINTER(vp), i32, i32, i32, vp, vp]),
+        "prism_attn_bwd_sharded": (i32, [vp, C.POINTER(vp), C.POINTER(vp), vp, C.POINTER(vp), C.POINTER(vp),
+                                         C.POINTER(vp), i32, i32, i32, vp]),
         "prism_attn_bwd": (i32, [vp, vp, vp, vp, vp, vp, vp, vp]),
         "prism_plan_item_bytes": (sz, [vp, i32]),
         "prism_plan_export": (i32, [vp, i32, vp, sz, vp]),
@@ -137,6 +140,11 @@ def core_bytes(params: PrismParams) -> int:
 
 def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _addresses(xs):
+    """A ctypes array of device addresses from tensors or ints."""
+    return (C.c_void_p * len(xs))(*[x if isinstance(x, int) else x.data_ptr() for x in xs])
 
 
 def _stream(stream):
@@ -200,6 +208,34 @@ class Plan:
         if st:
             raise PrismError(st, "prism_attn_bwd")
         return dQ, dK, dV
+
+    def attn_fwd_sharded(self, O_shards, head0, heads_total, lse=None, stream=None):
+        """The forward writing O into token shards (lists of [heads_total, N/n, D] tensors or
+        device addresses, shard s = frames [s T/n, (s + 1) T/n)): rows of this plan's heads
+        head0 .. head0 + heads - 1.  The LSE stays [heads, N] on this device."""
+        import torch
+        p = self.params
+        if lse is None:
+            lse = torch.empty(p.heads, self.N, dtype=torch.float32, device=self._ws.device)
+        arr = _addresses(O_shards)
+        st = load().prism_attn_fwd_sharded(self._h, arr, len(O_shards), int(heads_total), int(head0), _ptr(lse),
+                                           _stream(stream))
+        if st:
+            raise PrismError(st, "prism_attn_fwd_sharded")
+        return lse
+
+    def attn_bwd_sharded(self, dO_shards, O_shards, lse, dQ_shards, dK_shards, dV_shards, head0, heads_total,
+                         stream=None):
+        """The backward reading dO and O from token shards and writing dQ, dK, dV into token
+        shards (the layout of attn_fwd_sharded)."""
+        n = len(dO_shards)
+        if not all(len(x) == n for x in (O_shards, dQ_shards, dK_shards, dV_shards)):
+            raise ValueError("every shard list must have the same length")
+        st = load().prism_attn_bwd_sharded(self._h, _addresses(dO_shards), _addresses(O_shards), _ptr(lse),
+                                           _addresses(dQ_shards), _addresses(dK_shards), _addresses(dV_shards),
+                                           n, int(heads_total), int(head0), _stream(stream))
+        if st:
+            raise PrismError(st, "prism_attn_bwd_sharded")
 
     def export(self, item: str, stream=None) -> np.ndarray:
         code, dt = ITEMS[item]

@@ -57,21 +57,25 @@ constexpr float kPScaleInv = 1.f / 32768.f;
 constexpr int kDsShift = 7;                 // dS' = dS 2^(kDsShift - E - ev): see k_bwd_pre
 
 // --------------------------------------------------------------- preprocess
-// max |dO| per head (fp32 bits, see fold_abs): one pass over 16-byte chunks (dO
-// is 16-byte aligned and a head holds N x head_dim values).
+// max |dO| per head (fp32 bits, see fold_abs): one pass over 16-byte chunks of
+// each shard's rows of the head (dO is 16-byte aligned and a shard holds
+// S x head_dim values of a head).
 template <typename OT>
-__global__ void __launch_bounds__(256) k_bwd_absmax(const OT* __restrict__ dO, uint32_t* dmax, int64_t n_per_head) {
+__global__ void __launch_bounds__(256) k_bwd_absmax(const TokenRows dO, uint32_t* dmax, int HD) {
     const int h = blockIdx.y;
-    const uint4* x = reinterpret_cast<const uint4*>(dO + (size_t)h * n_per_head);
-    const int64_t n16 = n_per_head * (int64_t)sizeof(OT) / 16;
+    const int64_t n16 = dO.S * HD * (int64_t)sizeof(OT) / 16;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0u;
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; i + stride < n16; i += 2 * stride) {         // two chunks in flight
-        const uint4 a = __ldg(x + i), b = __ldg(x + i + stride);
-        m = fold_abs<OT>(fold_abs<OT>(m, a), b);
+    for (int sh = 0; sh < dO.n; ++sh) {
+        const uint4* x = reinterpret_cast<const uint4*>(static_cast<const OT*>(dO.p[sh]) +
+                                                        (int64_t)(dO.head0 + h) * dO.S * HD);
+        int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        for (; i + stride < n16; i += 2 * stride) {         // two chunks in flight
+            const uint4 a = __ldg(x + i), b = __ldg(x + i + stride);
+            m = fold_abs<OT>(fold_abs<OT>(m, a), b);
+        }
+        if (i < n16) m = fold_abs<OT>(m, __ldg(x + i));
     }
-    if (i < n16) m = fold_abs<OT>(m, __ldg(x + i));
     uint32_t b = abs_bits<OT>(m);
     for (int o = 16; o > 0; o >>= 1) b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
     if ((threadIdx.x & 31) == 0) atomicMax(dmax + h, b);
@@ -88,7 +92,7 @@ __device__ __forceinline__ int dscale_exp(uint32_t bits, int* err) {
 }
 
 template <typename OT>
-__global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, const OT* __restrict__ O,
+__global__ void __launch_bounds__(256) k_bwd_pre(const TokenRows dO, const TokenRows O,
                                                  const float* __restrict__ lse,
                                                  const int* __restrict__ src, const uint32_t* dmax,
                                                  __half* __restrict__ dOp, float* __restrict__ lse_p,
@@ -101,8 +105,8 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const OT* __restrict__ dO, cons
     const float sc = ldexpf(1.f, -dscale_exp(dmax[h], err));
     const int64_t n = src[(size_t)h * N + p];
     if (prism_bad_index(err, n >= 0 && n < N)) return;
-    const OT* dr = dO + ((size_t)h * N + n) * HD;
-    const OT* orow = O + ((size_t)h * N + n) * HD;
+    const OT* dr = dO.row<const OT>(h, n, HD);
+    const OT* orow = O.row<const OT>(h, n, HD);
     __half* out = dOp + ((size_t)(h - h0) * N + p) * HD;
     float acc = 0.f;
     for (int c = lane; c < HD; c += 32) {
@@ -168,8 +172,7 @@ struct BwdArgs {
     const float* lse_p;    // [heads][N] 15 - LSE log2(e), block order
     const float* di_p;     // [heads][N] -D 2^-15 (D scaled like dO)
     const uint32_t* dmax;  // [heads] max |dO| bits: outputs are divided by the dO scale
-    void* out0;            // dK (dkdv) or dQ (dq), raster order
-    void* out1;            // dV (dkdv)
+    TokenRows out0;        // dQ (dq): rows of the output, a plain tensor or token shards
     float* dq_acc;         // (dkdv, head_dim 128) fp32 dQ accumulator, block order, head group
     int64_t N;
     int NT;
@@ -192,16 +195,15 @@ __device__ __forceinline__ int tiles_lower_bound(const int* e, int n, int key) {
     return lo;
 }
 
-__device__ __forceinline__ void store_row(void* base, size_t row, int HD, int c0, const uint32_t* v,
-                                          float mul, int out_f32) {
+__device__ __forceinline__ void store_row(void* rowp, int c0, const uint32_t* v, float mul, int out_f32) {
     if (out_f32) {
-        float4* op = reinterpret_cast<float4*>(static_cast<float*>(base) + row * HD + c0);
+        float4* op = reinterpret_cast<float4*>(static_cast<float*>(rowp) + c0);
         #pragma unroll
         for (int e = 0; e < 8; ++e)
             op[e] = make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
                                 __uint_as_float(v[4 * e + 2]) * mul, __uint_as_float(v[4 * e + 3]) * mul);
     } else {
-        uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + row * HD + c0);
+        uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(rowp) + c0);
         #pragma unroll
         for (int e = 0; e < 4; ++e)
             op[e] = make_uint4(pack_bf16(__uint_as_float(v[8 * e]) * mul, __uint_as_float(v[8 * e + 1]) * mul),
@@ -211,10 +213,10 @@ __device__ __forceinline__ void store_row(void* base, size_t row, int HD, int c0
     }
 }
 
-__device__ __forceinline__ void zero_row(void* base, size_t row, int HD, int out_f32) {
+__device__ __forceinline__ void zero_row(void* rowp, int HD, int out_f32) {
     for (int c = 0; c < HD; ++c) {
-        if (out_f32) static_cast<float*>(base)[row * HD + c] = 0.f;
-        else static_cast<__nv_bfloat16*>(base)[row * HD + c] = __float2bfloat16(0.f);
+        if (out_f32) static_cast<float*>(rowp)[c] = 0.f;
+        else static_cast<__nv_bfloat16*>(rowp)[c] = __float2bfloat16(0.f);
     }
 }
 
@@ -560,9 +562,9 @@ k_bwd_dkdv(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 // warp per row p, out[src[p]] = acc[p] * scale * 2^-e (the per-head dO scale).
 // Two accumulators (dK, dV) or one (dQ, acc1 == nullptr) per launch.
 template <typename OT>
-__global__ void __launch_bounds__(256) k_acc_finalize(const float* __restrict__ acc0, float scale0, OT* __restrict__ out0,
+__global__ void __launch_bounds__(256) k_acc_finalize(const float* __restrict__ acc0, float scale0, const TokenRows out0,
                                                       const float* __restrict__ acc1, float scale1,
-                                                      OT* __restrict__ out1, const int* __restrict__ src,
+                                                      const TokenRows out1, const int* __restrict__ src,
                                                       const uint32_t* dmax, int64_t N, int HD, int h0,
                                                       const uint32_t* __restrict__ qkv_max, int which0, int* err) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -576,10 +578,13 @@ __global__ void __launch_bounds__(256) k_acc_finalize(const float* __restrict__ 
         scale0 = ldexpf(scale0, 15 - qkv_shift(qkv_max[h * 3 + 2]) - kDsShift - qkv_shift(qkv_max[h * 3 + which0]));
     const int64_t n = src[(size_t)h * N + p];
     if (prism_bad_index(err, n >= 0 && n < N)) return;
-    const size_t ir = ((size_t)(h - h0) * N + p) * HD, orow = ((size_t)h * N + n) * HD;
-    for (int c = lane; c < HD; c += 32) out0[orow + c] = (OT)(acc0[ir + c] * (scale0 * unscale));
-    if (acc1)
-        for (int c = lane; c < HD; c += 32) out1[orow + c] = (OT)(acc1[ir + c] * (scale1 * unscale));
+    const size_t ir = ((size_t)(h - h0) * N + p) * HD;
+    OT* o0 = out0.row<OT>(h, n, HD);
+    for (int c = lane; c < HD; c += 32) o0[c] = (OT)(acc0[ir + c] * (scale0 * unscale));
+    if (acc1) {
+        OT* o1 = out1.row<OT>(h, n, HD);
+        for (int c = lane; c < HD; c += 32) o1[c] = (OT)(acc1[ir + c] * (scale1 * unscale));
+    }
 }
 
 // ------------------------------------------------------------------------ dQ
@@ -750,7 +755,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
         }
         int srow = a.src[prow];
         if (prism_bad_index(a.err, srow >= 0 && srow < a.N)) srow = 0;               // checking build
-        const size_t orow = (size_t)hrow + (size_t)srow;
+        void* orow = a.out_f32 ? static_cast<void*>(a.out0.row<float>(h, srow, HD))
+                               : static_cast<void*>(a.out0.row<__nv_bfloat16>(h, srow, HD));
         bool fin = false;
         if (ok && U > 0)
             fin = __all_sync(0xffffffffu, mbar_wait(&sm.dq_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, 2004));
@@ -762,11 +768,10 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
                 uint32_t o[32];
                 PRISM_TMEM_LD32(tmem + lane_off + TDQ + 32 * c, o);
                 tmem_wait_ld();
-                store_row(a.out0, orow, HD, 32 * c, o, ldexpf(a.inv_sqrt_d * unscale, ev - kDsShift - sk),
-                          a.out_f32);
+                store_row(orow, 32 * c, o, ldexpf(a.inv_sqrt_d * unscale, ev - kDsShift - sk), a.out_f32);
             }
         } else if (U == 0) {
-            zero_row(a.out0, orow, HD, a.out_f32);
+            zero_row(orow, HD, a.out_f32);
         }
     }
     tc_fence_before();
@@ -776,8 +781,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUten
 }
 
 template <int HD>
-static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse, void* dQ,
-                      void* dK, void* dV, cudaStream_t s) {
+static int launch_bwd(prism_plan_s* P, const TokenRows& dO, const TokenRows& O, const float* lse,
+                      const TokenRows& dQ, const TokenRows& dK, const TokenRows& dV, cudaStream_t s) {
     const Geom& g = P->g;
     char* b = P->ws;
     const int* src = (const int*)(b + P->L.src);
@@ -791,8 +796,8 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
     {
         PrismProf prof(P, PRISM_STAGE_BWD_PRE, s);
         const dim3 gmax(296, g.heads);
-        if (f32) k_bwd_absmax<float><<<gmax, 256, 0, s>>>((const float*)dO, dmax, g.N * HD);
-        else k_bwd_absmax<__nv_bfloat16><<<gmax, 256, 0, s>>>((const __nv_bfloat16*)dO, dmax, g.N * HD);
+        if (f32) k_bwd_absmax<float><<<gmax, 256, 0, s>>>(dO, dmax, HD);
+        else k_bwd_absmax<__nv_bfloat16><<<gmax, 256, 0, s>>>(dO, dmax, HD);
         P->launches += 1;
     }
     BwdArgs a{};
@@ -835,18 +840,15 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
         {
             PrismProf prof(P, PRISM_STAGE_BWD_PRE, s);
             if (f32)
-                k_bwd_pre<float><<<grows, 256, 0, s>>>((const float*)dO, (const float*)O, lse, src, dmax, dOp, lse_p,
-                                                       di_p, g.N, HD, h0, a.qkv_max, err);
+                k_bwd_pre<float><<<grows, 256, 0, s>>>(dO, O, lse, src, dmax, dOp, lse_p, di_p, g.N, HD, h0,
+                                                       a.qkv_max, err);
             else
-                k_bwd_pre<__nv_bfloat16><<<grows, 256, 0, s>>>((const __nv_bfloat16*)dO, (const __nv_bfloat16*)O,
-                                                               lse, src, dmax, dOp, lse_p, di_p, g.N, HD, h0,
-                                                               a.qkv_max, err);
+                k_bwd_pre<__nv_bfloat16><<<grows, 256, 0, s>>>(dO, O, lse, src, dmax, dOp, lse_p, di_p, g.N, HD,
+                                                               h0, a.qkv_max, err);
         }
         // dK, dV (and for head_dim 128 dQ) per key tile over the transposed lists
         a.ptr = (const int*)(b + P->L.kt_ptr);
         a.ent_off = loff + LIST_BWD * (size_t)g.heads;
-        a.out0 = dK;
-        a.out1 = dV;
         {
             PrismProf prof(P, PRISM_STAGE_BWD_DKDV, s);
             if (FUSE) cudaMemsetAsync(dq_acc, 0, acc_bytes, s);
@@ -855,29 +857,27 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
             k_bwd_dkdv<HD, FUSE><<<dim3(g.NT, chunks, nh), FUSE ? 480 : 352, sm1, s>>>(
                 P->tm_k, P->tm_v, P->tm_q64, P->tm_do64, P->tm_dk, P->tm_dv, a);
             if (f32)
-                k_acc_finalize<float><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (float*)dK, dv_acc, 1.f / kPScale,
-                                                            (float*)dV, src, dmax, g.N, HD, h0, a.qkv_max, 0, err);
+                k_acc_finalize<float><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, dK, dv_acc, 1.f / kPScale, dV, src,
+                                                            dmax, g.N, HD, h0, a.qkv_max, 0, err);
             else
-                k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, (__nv_bfloat16*)dK, dv_acc,
-                                                                    1.f / kPScale, (__nv_bfloat16*)dV, src, dmax,
-                                                                    g.N, HD, h0, a.qkv_max, 0, err);
+                k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dk_acc, a.inv_sqrt_d, dK, dv_acc, 1.f / kPScale,
+                                                                    dV, src, dmax, g.N, HD, h0, a.qkv_max, 0, err);
         }
         {
             PrismProf prof(P, PRISM_STAGE_BWD_DQ, s);
             if (FUSE) {
                 if (f32)
-                    k_acc_finalize<float><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (float*)dQ, nullptr, 0.f,
-                                                                nullptr, src, dmax, g.N, HD, h0, a.qkv_max, 1, err);
+                    k_acc_finalize<float><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, dQ, nullptr, 0.f, TokenRows{},
+                                                                src, dmax, g.N, HD, h0, a.qkv_max, 1, err);
                 else
-                    k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, (__nv_bfloat16*)dQ,
-                                                                        nullptr, 0.f, nullptr, src, dmax, g.N, HD,
-                                                                        h0, a.qkv_max, 1, err);
+                    k_acc_finalize<__nv_bfloat16><<<grows, 256, 0, s>>>(dq_acc, a.inv_sqrt_d, dQ, nullptr, 0.f,
+                                                                        TokenRows{}, src, dmax, g.N, HD, h0,
+                                                                        a.qkv_max, 1, err);
             } else {
                 // dQ per query tile over the forward lists (head_dim 64)
                 a.ptr = (const int*)(b + P->L.qt_ptr);
                 a.ent_off = loff + LIST_FWD * (size_t)g.heads;
                 a.out0 = dQ;
-                a.out1 = nullptr;
                 k_bwd_dq<HD><<<dim3(g.NT, nh), 192, sm2, s>>>(P->tm_q, P->tm_do, P->tm_k64, P->tm_v64, a);
             }
         }
@@ -888,8 +888,9 @@ static int launch_bwd(prism_plan_s* P, const void* dO, const void* O, const floa
 
 }  // namespace prism
 
-int prism_launch_attn_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse, void* dQ,
-                          void* dK, void* dV, void* stream) {
+int prism_launch_attn_bwd(prism_plan_s* P, const prism::TokenRows& dO, const prism::TokenRows& O, const float* lse,
+                          const prism::TokenRows& dQ, const prism::TokenRows& dK, const prism::TokenRows& dV,
+                          void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return P->g.D == 128 ? prism::launch_bwd<128>(P, dO, O, lse, dQ, dK, dV, s)
                          : prism::launch_bwd<64>(P, dO, O, lse, dQ, dK, dV, s);

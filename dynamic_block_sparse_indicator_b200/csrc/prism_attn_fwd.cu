@@ -81,7 +81,7 @@ struct FwdArgs {
     const int64_t* qt_off; // [heads]
     int h0;                // first head of this launch (grid y = heads h0, h0 + 1, ...)
     const int* src;        // [heads][N]
-    void* O;               // [heads][N][HD] raster order
+    TokenRows O;           // row (h, raster token) of the output, a plain tensor or token shards
     float* lse;            // [heads][N]
     int64_t N;
     int NT;
@@ -440,11 +440,11 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     #pragma unroll
                     for (int e = 0; e < 8; ++e) sp[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
                 } else if (a.out_f32) {
-                    float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow * HD + c0);
+                    float4* op = reinterpret_cast<float4*>(a.O.row<float>(h, srow, HD) + c0);
                     #pragma unroll
                     for (int e = 0; e < 8; ++e) op[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
                 } else {
-                    uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + orow * HD + c0);
+                    uint4* op = reinterpret_cast<uint4*>(a.O.row<__nv_bfloat16>(h, srow, HD) + c0);
                     #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         op[e] = make_uint4(pack_bf16(x[8 * e], x[8 * e + 1]), pack_bf16(x[8 * e + 2], x[8 * e + 3]),
@@ -484,7 +484,7 @@ __global__ void k_selftest_wait(int* err) {
 }
 
 template <int HD>
-static int launch_fwd(prism_plan_s* P, void* O, float* lse, cudaStream_t s) {
+static int launch_fwd(prism_plan_s* P, const TokenRows& O, float* lse, cudaStream_t s) {
     const Geom& g = P->g;
     FwdArgs a;
     char* b = P->ws;
@@ -538,7 +538,7 @@ int prism_launch_selftest_wait(prism_plan_s* P, void* stream) {
     return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
 }
 
-int prism_launch_attn_fwd(prism_plan_s* P, void* O, float* lse, void* stream) {
+int prism_launch_attn_fwd(prism_plan_s* P, const prism::TokenRows& O, float* lse, void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return P->g.D == 128 ? prism::launch_fwd<128>(P, O, lse, s) : prism::launch_fwd<64>(P, O, lse, s);
 }

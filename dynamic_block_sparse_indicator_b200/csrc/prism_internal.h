@@ -47,6 +47,63 @@ __device__ __forceinline__ int qkv_shift(uint32_t max_bits) {
 }
 #endif
 
+// Where row (h, token n) of a [heads][N][D] tensor lives.  A plain tensor is
+// one shard.  A sequence-parallel caller's tensor is `n` token shards, shard s
+// holding frames [s F, (s + 1) F) of every one of `stride_heads` heads as
+// [stride_heads][F HW][D] (a rank's part of the sequence); a plan covers heads
+// head0, head0 + 1, ... of them.  The shard pointers may be other GPUs' memory
+// mapped for peer access: the kernels read and write them with plain loads and
+// stores, so the exchange between sequence and head layouts happens inside the
+// passes the plan and the attention make anyway.
+constexpr int kMaxShards = 16;
+struct TokenRows {
+    void* p[kMaxShards];
+    int64_t S;             // tokens per shard (F HW)
+    int64_t HW;            // tokens per frame
+    int F;                 // frames per shard
+    int n;                 // shards
+    int stride_heads;      // heads held by each shard
+    int head0;             // the shard head of plan head 0
+#if defined(__CUDACC__)
+    // row (h, token tok of frame t)
+    template <typename T>
+    __device__ __forceinline__ T* row_t(int h, int t, int64_t tok, int D) const {
+        const int sh = n == 1 ? 0 : t / F;
+        return static_cast<T*>(p[sh]) + ((int64_t)(head0 + h) * S + (tok - (int64_t)sh * S)) * D;
+    }
+    template <typename T>
+    __device__ __forceinline__ T* row(int h, int64_t tok, int D) const {
+        return row_t<T>(h, n == 1 ? 0 : (int)(tok / HW), tok, D);
+    }
+#endif
+};
+
+// One plain [heads][N][D] tensor.
+inline TokenRows plain_rows(const void* x, int T, int64_t HW, int heads) {
+    TokenRows r{};
+    r.p[0] = const_cast<void*>(x);
+    r.HW = HW;
+    r.F = T;
+    r.S = (int64_t)T * HW;
+    r.n = 1;
+    r.stride_heads = heads;
+    r.head0 = 0;
+    return r;
+}
+
+// `shards` token shards of `heads_total` heads; the plan's head 0 is shard head head0.
+inline TokenRows shard_rows(const void* const* xs, int shards, int T, int64_t HW, int heads_total, int head0) {
+    TokenRows r{};
+    for (int i = 0; i < shards; ++i) r.p[i] = const_cast<void*>(xs[i]);
+    r.HW = HW;
+    r.F = T / shards;
+    r.S = (int64_t)r.F * HW;
+    r.n = shards;
+    r.stride_heads = heads_total;
+    r.head0 = head0;
+    return r;
+}
+
 // Geometry derived from prism_params.
 struct Geom {
     int T, H, W, heads, D, dtype;
@@ -165,8 +222,10 @@ struct PrismProf {
     ~PrismProf() { close(); }
 };
 
-// Internal entry points of the attention translation units.
-int prism_launch_attn_fwd(prism_plan_s* P, void* O, float* lse, void* stream);
+// Internal entry points of the attention translation units (O, dO, dQ, dK, dV
+// addressed through TokenRows; the LSE is the plan's [heads][N]).
+int prism_launch_attn_fwd(prism_plan_s* P, const prism::TokenRows& O, float* lse, void* stream);
 int prism_launch_selftest_wait(prism_plan_s* P, void* stream);
-int prism_launch_attn_bwd(prism_plan_s* P, const void* dO, const void* O, const float* lse,
-                          void* dQ, void* dK, void* dV, void* stream);
+int prism_launch_attn_bwd(prism_plan_s* P, const prism::TokenRows& dO, const prism::TokenRows& O, const float* lse,
+                          const prism::TokenRows& dQ, const prism::TokenRows& dK, const prism::TokenRows& dV,
+                          void* stream);

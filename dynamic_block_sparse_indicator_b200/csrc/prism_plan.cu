@@ -32,6 +32,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <new>
 
@@ -160,41 +161,6 @@ __constant__ int8_t c_log2shape[16][3] = {
     {1, 2, 3}, {1, 3, 2}, {2, 1, 3}, {2, 2, 2}, {2, 3, 1}, {3, 1, 2}, {3, 2, 1},
     {1, 3, 3}, {2, 2, 3}, {2, 3, 2}, {3, 1, 3}, {3, 2, 2}, {3, 3, 1},
     {2, 3, 3}, {3, 2, 3}, {3, 3, 2}};
-
-// Where row (h, n) of a [heads][N][D] input lives.  A plain tensor is one
-// shard.  A sequence-parallel caller's input is `n` token shards, shard s
-// holding frames [s F, (s + 1) F) of every one of `stride_heads` heads as
-// [stride_heads][F H W][D] (a rank's part of the sequence); the plan covers
-// heads head0, head0 + 1, ... of them.  The shard pointers may be other GPUs'
-// memory mapped for peer access: the plan reads them with plain loads, so the
-// head-to-rank exchange and the reorder into block order are one pass.
-constexpr int kMaxShards = 16;
-struct TokenRows {
-    const void* p[kMaxShards];
-    int64_t S;             // tokens per shard (F H W)
-    int F;                 // frames per shard
-    int n;                 // shards
-    int stride_heads;      // heads held by each shard
-    int head0;             // the shard head of this plan's head 0
-    // row (h, token of frame t) as element offset into shard p[t / F]
-    template <typename T>
-    __device__ __forceinline__ const T* row(int h, int t, int64_t tok, int D) const {
-        const int sh = n == 1 ? 0 : t / F;
-        return static_cast<const T*>(p[sh]) +
-               ((int64_t)(head0 + h) * S + (tok - (int64_t)sh * S)) * D;
-    }
-};
-
-static TokenRows plain_rows(const void* x, int64_t N, int T, int heads) {
-    TokenRows r{};
-    r.p[0] = x;
-    r.S = N;
-    r.F = T;
-    r.n = 1;
-    r.stride_heads = heads;
-    r.head0 = 0;
-    return r;
-}
 
 struct DevPlan {
     int T, H, W, heads, D, Zh, Zw, Nz, NB, NT, WORDS;
@@ -498,7 +464,7 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const TokenRows V
     auto tok = [&](int lt, int lh, int lw) -> int64_t {
         return ((int64_t)(8 * zt + lt) * d.H + 8 * zh + lh) * d.W + 8 * zw + lw;
     };
-    const float2 ref = Pair<T>::load(V.row<T>(h, 8 * zt + t0, tok(t0, 0, 0), D) + 2 * cp);
+    const float2 ref = Pair<T>::load(V.row_t<const T>(h, 8 * zt + t0, tok(t0, 0, 0), D) + 2 * cp);
     float ST[2][8], SQ[2][8], SW[2][8], SH[2][RPG], Ds[2], Dq[2], Et[2][NE > 0 ? NE : 1];
     #pragma unroll
     for (int c = 0; c < 2; ++c) {
@@ -520,7 +486,7 @@ __global__ void __launch_bounds__(256) k_zone_stats(DevPlan d, const TokenRows V
         for (int lt = 0; lt < 8; ++lt) {
             if (MODE == 2 && (lt < t0 || lt >= t1)) continue;
             float2 x[8];
-            const T* vr = V.row<T>(h, 8 * zt + lt, tok(lt, lh, 0), D) + 2 * cp;   // 8 adjacent tokens
+            const T* vr = V.row_t<const T>(h, 8 * zt + lt, tok(lt, lh, 0), D) + 2 * cp;   // 8 adjacent tokens
             #pragma unroll
             for (int lw = 0; lw < 8; ++lw) x[lw] = Pair<T>::load(vr + lw * D);
             #pragma unroll
@@ -977,9 +943,9 @@ __global__ void __launch_bounds__(256) k_gather_pool(DevPlan d, const TokenRows 
         if (prism_bad_index(d.err, n >= 0 && n < d.N && start + r < d.N)) continue;
         const size_t dst = hoff + (size_t)(start + r) * D + (size_t)c * EPC;
         if (c == 0) d.src[(size_t)h * d.N + start + r] = (int)n;
-        const uint4 q4 = *reinterpret_cast<const uint4*>(Q.row<T>(h, ft, n, D) + c * EPC);
-        const uint4 k4 = *reinterpret_cast<const uint4*>(K.row<T>(h, ft, n, D) + c * EPC);
-        const uint4 v4 = *reinterpret_cast<const uint4*>(V.row<T>(h, ft, n, D) + c * EPC);
+        const uint4 q4 = *reinterpret_cast<const uint4*>(Q.row_t<const T>(h, ft, n, D) + c * EPC);
+        const uint4 k4 = *reinterpret_cast<const uint4*>(K.row_t<const T>(h, ft, n, D) + c * EPC);
+        const uint4 v4 = *reinterpret_cast<const uint4*>(V.row_t<const T>(h, ft, n, D) + c * EPC);
         float fq[EPC], fk[EPC], fv[EPC];
         if constexpr (sizeof(T) == 2) {
             const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&q4);
@@ -1715,8 +1681,8 @@ extern "C" int prism_plan(const prism_params* p, const void* Q, const void* K, c
     P->has_audio = a_map != nullptr;
     P->has_cuts = p->cut_ratio > 0.f;
     const Geom& g = P->g;
-    st = run_plan(P, plain_rows(Q, g.N, g.T, g.heads), plain_rows(K, g.N, g.T, g.heads),
-                  plain_rows(V, g.N, g.T, g.heads), a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+    st = run_plan(P, plain_rows(Q, g.T, (int64_t)g.H * g.W, g.heads), plain_rows(K, g.T, (int64_t)g.H * g.W, g.heads),
+                  plain_rows(V, g.T, (int64_t)g.H * g.W, g.heads), a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
     if (st) { delete P; return st; }
     *out = P;
     return PRISM_OK;
@@ -1741,16 +1707,10 @@ extern "C" int prism_plan_sharded(const prism_params* p, const void* const* Q, c
     P->has_audio = a_map != nullptr;
     P->has_cuts = p->cut_ratio > 0.f;
     const Geom& g = P->g;
-    TokenRows rq{}, rk{}, rv{};
-    for (TokenRows* r : {&rq, &rk, &rv}) {
-        r->F = g.T / shards;
-        r->S = (int64_t)r->F * g.H * g.W;
-        r->n = shards;
-        r->stride_heads = heads_total;
-        r->head0 = head0;
-    }
-    for (int i = 0; i < shards; ++i) { rq.p[i] = Q[i]; rk.p[i] = K[i]; rv.p[i] = V[i]; }
-    st = run_plan(P, rq, rk, rv, a_map, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+    const int64_t HW = (int64_t)g.H * g.W;
+    st = run_plan(P, shard_rows(Q, shards, g.T, HW, heads_total, head0), shard_rows(K, shards, g.T, HW, heads_total, head0),
+                  shard_rows(V, shards, g.T, HW, heads_total, head0), a_map, nullptr, nullptr,
+                  static_cast<cudaStream_t>(stream));
     if (st) { delete P; return st; }
     *out = P;
     return PRISM_OK;
@@ -1770,8 +1730,8 @@ extern "C" int prism_plan_import_cuts(const prism_params* p, const void* Q, cons
     P->has_audio = 0;
     P->has_cuts = zone_cut != nullptr;
     const Geom& g = P->g;
-    st = run_plan(P, plain_rows(Q, g.N, g.T, g.heads), plain_rows(K, g.N, g.T, g.heads),
-                  plain_rows(V, g.N, g.T, g.heads), nullptr, shape_id, sel, static_cast<cudaStream_t>(stream),
+    st = run_plan(P, plain_rows(Q, g.T, (int64_t)g.H * g.W, g.heads), plain_rows(K, g.T, (int64_t)g.H * g.W, g.heads),
+                  plain_rows(V, g.T, (int64_t)g.H * g.W, g.heads), nullptr, shape_id, sel, static_cast<cudaStream_t>(stream),
                   zone_cut, shape_id2);
     if (st) { delete P; return st; }
     *out = P;
@@ -1940,7 +1900,8 @@ extern "C" const char* prism_version(void) { return "prism-b200 0.1 sm_100a"; }
 extern "C" int prism_attn_fwd(prism_plan_t P, void* O, float* lse, void* stream) {
     if (!P || !O || !lse || !P->lists_ready) return PRISM_ERR_INVALID_ARG;
     if (!aligned16(O) || !aligned16(lse)) return PRISM_ERR_INVALID_ARG;
-    return prism_launch_attn_fwd(P, O, lse, stream);
+    const Geom& g = P->g;
+    return prism_launch_attn_fwd(P, plain_rows(O, g.T, (int64_t)g.H * g.W, g.heads), lse, stream);
 }
 
 extern "C" int prism_attn_bwd(prism_plan_t P, const void* dO, const void* O, const float* lse,
@@ -1949,7 +1910,45 @@ extern "C" int prism_attn_bwd(prism_plan_t P, const void* dO, const void* O, con
     if (!aligned16(dO) || !aligned16(O) || !aligned16(lse) || !aligned16(dQ) || !aligned16(dK) ||
         !aligned16(dV))
         return PRISM_ERR_INVALID_ARG;
-    return prism_launch_attn_bwd(P, dO, O, lse, dQ, dK, dV, stream);
+    const Geom& g = P->g;
+    const int64_t HW = (int64_t)g.H * g.W;
+    return prism_launch_attn_bwd(P, plain_rows(dO, g.T, HW, g.heads), plain_rows(O, g.T, HW, g.heads), lse,
+                                 plain_rows(dQ, g.T, HW, g.heads), plain_rows(dK, g.T, HW, g.heads),
+                                 plain_rows(dV, g.T, HW, g.heads), stream);
+}
+
+// The shard layout arguments of the *_sharded entry points: shards dividing T,
+// a head range inside the shards' heads, non-null 16-byte aligned pointers.
+static bool shards_ok(const prism_plan_s* P, int shards, int heads_total, int head0,
+                      std::initializer_list<const void* const*> arrays) {
+    if (!P || shards < 1 || shards > kMaxShards || P->g.T % shards != 0) return false;
+    if (head0 < 0 || heads_total < 1 || head0 + P->g.heads > heads_total) return false;
+    for (const void* const* xs : arrays) {
+        if (!xs) return false;
+        for (int i = 0; i < shards; ++i)
+            if (!xs[i] || !aligned16(xs[i])) return false;
+    }
+    return true;
+}
+
+extern "C" int prism_attn_fwd_sharded(prism_plan_t P, void* const* O, int shards, int heads_total, int head0,
+                                      float* lse, void* stream) {
+    if (!P || !lse || !aligned16(lse) || !P->lists_ready) return PRISM_ERR_INVALID_ARG;
+    if (!shards_ok(P, shards, heads_total, head0, {O})) return PRISM_ERR_INVALID_ARG;
+    const Geom& g = P->g;
+    return prism_launch_attn_fwd(P, shard_rows(O, shards, g.T, (int64_t)g.H * g.W, heads_total, head0), lse,
+                                 stream);
+}
+
+extern "C" int prism_attn_bwd_sharded(prism_plan_t P, const void* const* dO, const void* const* O,
+                                      const float* lse, void* const* dQ, void* const* dK, void* const* dV,
+                                      int shards, int heads_total, int head0, void* stream) {
+    if (!P || !lse || !aligned16(lse) || !P->lists_ready) return PRISM_ERR_INVALID_ARG;
+    if (!shards_ok(P, shards, heads_total, head0, {dO, O, dQ, dK, dV})) return PRISM_ERR_INVALID_ARG;
+    const Geom& g = P->g;
+    const int64_t HW = (int64_t)g.H * g.W;
+    auto rows = [&](const void* const* xs) { return shard_rows(xs, shards, g.T, HW, heads_total, head0); };
+    return prism_launch_attn_bwd(P, rows(dO), rows(O), lse, rows(dQ), rows(dK), rows(dV), stream);
 }
 
 // ====================================================== no-allocation stage 1
@@ -2005,7 +2004,7 @@ template <typename T, int D>
 static void noalloc_stats(const Geom& g, const DevPlan& d, const void* V, cudaStream_t s) {
     const int sm = (256 / (D / 2)) * D * 26 * (int)sizeof(float);
     cudaFuncSetAttribute(k_zone_stats<T, D, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, plain_rows(V, g.N, g.T, g.heads), 0.f);
+    k_zone_stats<T, D, 0><<<dim3(g.Nz, g.heads), 256, sm, s>>>(d, plain_rows(V, g.T, (int64_t)g.H * g.W, g.heads), 0.f);
 }
 
 // Device address of the scratch array, looked up once per device (with that

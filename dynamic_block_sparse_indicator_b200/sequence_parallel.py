@@ -19,13 +19,13 @@ all-to-all (NCCL over NVLink between GPUs; gloo on the host for the tests); the
 plan itself needs no collective.  The library computes nothing here: this
 module only moves tensors between ranks with torch.distributed.
 
-Where the ranks' sequence shards of Q, K and V are mapped into each other's
-address space (torch symmetric memory, CUDA IPC), the inbound exchange can be
-left out: `_lib.plan_sharded(qs, ks, vs, a, params, head0=h0, heads_total=H)`
-plans this rank's heads (`rank_heads`) straight from every rank's shard, the
-plan's reorder into block order reading the other GPUs' rows over NVLink, so
-the all-to-all and the reorder are one pass.  The plan then runs as above, and
-the results go back with `heads_to_seq`.
+Where the ranks' sequence shards are mapped into each other's address space
+(torch symmetric memory, CUDA IPC), both exchanges can be left out:
+`_lib.plan_sharded(qs, ks, vs, a, params, head0=h0, heads_total=H)` plans this
+rank's heads (`rank_heads`) straight from every rank's Q, K, V shard (the
+plan's reorder reads the other GPUs' rows over NVLink), and the plan's
+`attn_fwd_sharded` / `attn_bwd_sharded` write O, dQ, dK, dV into (and read dO,
+O from) the shards in place, so no all-to-all runs around the layer.
 """
 from __future__ import annotations
 

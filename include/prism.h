@@ -292,6 +292,26 @@ PRISM_API int prism_attn_bwd(prism_plan_t plan, const void* dO, const void* O, c
                    void* dQ, void* dK, void* dV, void* stream);
 
 /*
+ * prism_attn_fwd_sharded / prism_attn_bwd_sharded -- prism_attn_fwd and
+ * prism_attn_bwd with O, dO, dQ, dK, dV held as token shards in the layout of
+ * prism_plan_sharded (host arrays of `shards` device pointers, shard s holding
+ * frames [s T/shards, (s + 1) T/shards) of `heads_total` heads as
+ * [heads_total][(T/shards) H W][head_dim] of `out_dtype`; the plan's heads are
+ * head0 .. head0 + heads - 1 there).  The rows of the plan's heads are written
+ * (and O, dO read) in place, so a sequence-parallel rank needs no all-to-all
+ * after the forward or around the backward: with peer-mapped shards the
+ * kernels store and load other GPUs' rows with plain stores and loads.  The
+ * LSE stays [heads][N] fp32 on this device.  Returns PRISM_ERR_INVALID_ARG for
+ * a shard count that does not divide T, a head range outside the shards, or a
+ * null or misaligned pointer.
+ */
+PRISM_API int prism_attn_fwd_sharded(prism_plan_t plan, void* const* O, int shards, int heads_total, int head0,
+                                     float* lse, void* stream);
+PRISM_API int prism_attn_bwd_sharded(prism_plan_t plan, const void* const* dO, const void* const* O,
+                                     const float* lse, void* const* dQ, void* const* dK, void* const* dV,
+                                     int shards, int heads_total, int head0, void* stream);
+
+/*
  * prism_zone_shapes_noalloc -- stage 1 alone (zone statistics, block volume,
  *   snapped shape) for callers that cannot allocate device memory: a plugin
  *   that may only use the buffers another engine's memory plan hands it, a

@@ -9,8 +9,10 @@ the gathered heads: shapes, block offsets, permutation, pooled means of every
 block, the per-head input maxima and the selection bit for bit, O and LSE bit for bit, the
 gradients to fp32 summation order.  Cases: bf16 with 4 shards of 4 frames
 (every 8-frame zone spans two shards) and adaptive temporal boundaries on, and
-the fp32 tiny workload with 2 shards.  Invalid shard counts and head ranges are
-rejected before any launch.
+the fp32 tiny workload with 2 shards.  The forward and the backward in the
+shard layout (prism_attn_fwd_sharded, prism_attn_bwd_sharded): every rank's
+rows of O, dQ, dK, dV land in the shards equal to the gathered run's.  Invalid
+shard counts and head ranges are rejected before any launch.
 """
 import numpy as np
 import pytest
@@ -70,6 +72,52 @@ def test_sharded_plan_equals_gathered_plan(case, cuda_device):
             if nm in ("O", "LSE"):
                 assert torch.equal(g, e), f"{case} rank {r} {nm}"
             else:                      # partial sums reduced in the order the CTAs finish
+                diff, scale = (g - e).abs().max().item(), e.abs().max().item()
+                assert diff <= 1e-5 * scale, f"{case} rank {r} {nm}: {diff:.3e} at scale {scale:.3e}"
+
+
+@pytest.mark.parametrize("case", ["bf16_4shards", "f32_2shards"])
+def test_sequence_parallel_round_trip_in_place(case, cuda_device):
+    """Every rank plans its heads from the shards and runs the forward and the
+    backward with O, dO, dQ, dK, dV in the shard layout: the shards then hold
+    exactly the gathered run's outputs (O bit for bit, the gradients to fp32
+    summation order), with no exchange outside the kernels."""
+    if case == "bf16_4shards":
+        w = syn.workload(2, T=16, H=32, W=32)
+        P, heads, ranks, dt = 4, 4, 2, _lib.PRISM_BF16
+    else:
+        w = syn.workload(0)
+        P, heads, ranks, dt = 2, 2, 2, _lib.PRISM_F32
+    Q, K, V = syn.make_qkv(w, device="cuda", heads=heads)
+    dO = syn.make_dout(w, device="cuda", heads=heads, out_dtype=torch.float32)
+    a = syn.make_amap(w, device="cuda")
+    qs, ks, vs, dos = _shards(Q, P), _shards(K, P), _shards(V, P), _shards(dO, P)
+    n = w.N // P
+    mk = lambda: [torch.full((heads, n, w.head_dim), float("nan"), device="cuda") for _ in range(P)]
+    o_s, dq_s, dk_s, dv_s = mk(), mk(), mk(), mk()
+    nh = heads // ranks
+    want = {}
+    for r in range(ranks):
+        h0 = r * nh
+        sl = slice(h0, h0 + nh)
+        prm = _lib.make_params(w.T, w.H, w.W, nh, w.head_dim, dt, w.top_k, w.top_p, w.eps)
+        pl = _lib.plan_sharded(qs, ks, vs, a, prm, head0=h0, heads_total=heads)
+        lse = pl.attn_fwd_sharded(o_s, h0, heads)
+        torch.cuda.synchronize()
+        pl.attn_bwd_sharded(dos, o_s, lse, dq_s, dk_s, dv_s, h0, heads)
+        torch.cuda.synchronize()
+        assert pl.status() == _lib.PRISM_OK
+        ref = _lib.plan(Q[sl].contiguous(), K[sl].contiguous(), V[sl].contiguous(), a, prm)
+        want[r] = _run(ref, dO[sl].contiguous())
+    gather = lambda xs: torch.cat([x.cpu() for x in xs], dim=1)
+    got = {nm: gather(xs) for nm, xs in (("O", o_s), ("dQ", dq_s), ("dK", dk_s), ("dV", dv_s))}
+    for r in range(ranks):
+        sl = slice(r * nh, (r + 1) * nh)
+        for nm, e in zip(("O", "dQ", "dK", "dV"), (want[r][0], want[r][2], want[r][3], want[r][4])):
+            g, e = got[nm][sl], e.cpu()
+            if nm == "O":
+                assert torch.equal(g, e), f"{case} rank {r} O"
+            else:
                 diff, scale = (g - e).abs().max().item(), e.abs().max().item()
                 assert diff <= 1e-5 * scale, f"{case} rank {r} {nm}: {diff:.3e} at scale {scale:.3e}"
 
