@@ -23,6 +23,21 @@ def test_plan_rejects_host_tensors_and_bad_shapes():
         _lib.plan_import(x, x, x, None, None, p)
 
 
+def test_plan_sharded_rejects_bad_shard_lists():
+    p = _params()
+    x = torch.zeros(2, 1024, 64, dtype=torch.bfloat16)          # one of 2 shards of 2,048 tokens
+    with pytest.raises(ValueError):
+        _lib.plan_sharded([], [], [], None, p)                   # no shards
+    with pytest.raises(ValueError):
+        _lib.plan_sharded([x, x], [x], [x, x], None, p)          # lists of different lengths
+    with pytest.raises(ValueError):
+        _lib.plan_sharded([x] * 3, [x] * 3, [x] * 3, None, p)    # 3 shards do not divide T = 8
+    with pytest.raises(ValueError):
+        _lib.plan_sharded([x, x], [x, x], [x, x], None, p)       # host memory
+    with pytest.raises(ValueError):
+        _lib.plan_sharded([0, 0], [0, 0], [0, 0], None, p)       # addresses only: heads_total needed
+
+
 def test_av_norm_rejects_bad_inputs():
     q = torch.zeros(2, 256, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
