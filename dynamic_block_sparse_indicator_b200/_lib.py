@@ -79,6 +79,8 @@ def load(path: str | None = None) -> C.CDLL:
         "prism_plan": (i32, [pp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_sharded": (i32, [pp, C.POINTER(vp), C.POINTER(vp), C.POINTER(vp), i32, i32, i32, vp,
                                      vp, sz, vp, C.POINTER(vp)]),
+        "prism_plan_import_sharded": (i32, [pp, C.POINTER(vp), C.POINTER(vp), C.POINTER(vp), i32, i32, i32, vp,
+                                            vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import": (i32, [pp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_plan_import_cuts": (i32, [pp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, C.POINTER(vp)]),
         "prism_attn_fwd": (i32, [vp, vp, vp, vp]),
@@ -334,15 +336,9 @@ def plan(Q, K, V, a_map, params: PrismParams, workspace=None, stream=None, compa
     return Plan(params, h, workspace, (Q, K, V, a_map), lists)
 
 
-def plan_sharded(Qs, Ks, Vs, a_map, params: PrismParams, head0=0, heads_total=None, workspace=None,
-                 stream=None, compact=False) -> Plan:
-    """Stages 1-3 for heads head0 .. head0 + params.heads - 1 of inputs held as
-    token shards: Qs, Ks, Vs are equal-length lists (one entry per shard, shard s
-    holding frames [s T/n, (s + 1) T/n) of every head as [heads_total, N/n, D]),
-    each a contiguous CUDA tensor or a raw device address (an int: another GPU's
-    shard mapped for peer access).  The plan then runs like `plan` on those heads."""
+def _shard_args(Qs, Ks, Vs, params, heads_total):
+    """Checks a shard layout; returns (address arrays, heads_total, device, tensors)."""
     import torch
-    lib = load()
     n = len(Qs)
     if n == 0 or len(Ks) != n or len(Vs) != n:
         raise ValueError("Qs, Ks, Vs must be non-empty lists of the same length")
@@ -366,8 +362,46 @@ def plan_sharded(Qs, Ks, Vs, a_map, params: PrismParams, head0=0, heads_total=No
     if heads_total is None:
         raise ValueError("heads_total is needed when every shard is given as an address")
     device = device or torch.device("cuda", torch.cuda.current_device())
-    addr = lambda t: t if isinstance(t, int) else t.data_ptr()
-    arrs = [(C.c_void_p * n)(*[addr(t) for t in xs]) for xs in (Qs, Ks, Vs)]
+    return [_addresses(xs) for xs in (Qs, Ks, Vs)], int(heads_total), device, tuple(tensors)
+
+
+def plan_import_sharded(Qs, Ks, Vs, shape_id, sel_bits, params: PrismParams, head0=0, heads_total=None,
+                        zone_cut=None, shape_id2=None, workspace=None, stream=None, compact=False) -> Plan:
+    """plan_import for inputs held as token shards (the layout of plan_sharded)."""
+    import torch
+    lib = load()
+    arrs, heads_total, device, tensors = _shard_args(Qs, Ks, Vs, params, heads_total)
+    need = core_bytes(params) if compact else workspace_bytes(params)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    h = C.c_void_p()
+    st = lib.prism_plan_import_sharded(C.byref(params), arrs[0], arrs[1], arrs[2], len(Qs), heads_total,
+                                       int(head0), _ptr(shape_id), _ptr(zone_cut), _ptr(shape_id2),
+                                       _ptr(sel_bits), _ptr(workspace), workspace.numel(), _stream(stream),
+                                       C.byref(h))
+    if st:
+        raise PrismError(st, "prism_plan_import_sharded")
+    lists = None
+    if workspace.numel() < workspace_bytes(params):
+        try:
+            lists = _attach_lists(lib, h, device, stream)
+        except PrismError:
+            lib.prism_plan_destroy(h)
+            raise
+    return Plan(params, h, workspace, (tensors, shape_id, sel_bits, zone_cut, shape_id2), lists)
+
+
+def plan_sharded(Qs, Ks, Vs, a_map, params: PrismParams, head0=0, heads_total=None, workspace=None,
+                 stream=None, compact=False) -> Plan:
+    """Stages 1-3 for heads head0 .. head0 + params.heads - 1 of inputs held as
+    token shards: Qs, Ks, Vs are equal-length lists (one entry per shard, shard s
+    holding frames [s T/n, (s + 1) T/n) of every head as [heads_total, N/n, D]),
+    each a contiguous CUDA tensor or a raw device address (an int: another GPU's
+    shard mapped for peer access).  The plan then runs like `plan` on those heads."""
+    import torch
+    lib = load()
+    arrs, heads_total, device, tensors = _shard_args(Qs, Ks, Vs, params, heads_total)
+    n = len(Qs)
     need = core_bytes(params) if compact else workspace_bytes(params)
     if need == 0:
         raise PrismError(PRISM_ERR_INVALID_ARG, "prism_plan_workspace_bytes")
@@ -385,7 +419,7 @@ def plan_sharded(Qs, Ks, Vs, a_map, params: PrismParams, head0=0, heads_total=No
         except PrismError:
             lib.prism_plan_destroy(h)
             raise
-    return Plan(params, h, workspace, (tuple(tensors), a_map), lists)
+    return Plan(params, h, workspace, (tensors, a_map), lists)
 
 
 def plan_import(Q, K, V, shape_id, sel_bits, params: PrismParams, workspace=None, stream=None,

@@ -1738,6 +1738,36 @@ extern "C" int prism_plan_import_cuts(const prism_params* p, const void* Q, cons
     return PRISM_OK;
 }
 
+extern "C" int prism_plan_import_sharded(const prism_params* p, const void* const* Q, const void* const* K,
+                                         const void* const* V, int shards, int heads_total, int head0,
+                                         const uint8_t* shape_id, const uint8_t* zone_cut,
+                                         const uint8_t* shape_id2, const uint32_t* sel, void* workspace,
+                                         size_t ws_bytes, void* stream, prism_plan_t* out) {
+    if (!out) return PRISM_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!p || !Q || !K || !V || shards < 1 || shards > kMaxShards) return PRISM_ERR_INVALID_ARG;
+    if (!shape_id || !sel || !aligned16(sel)) return PRISM_ERR_INVALID_ARG;
+    if ((zone_cut == nullptr) != (shape_id2 == nullptr)) return PRISM_ERR_INVALID_ARG;
+    if (p->T % shards != 0 || head0 < 0 || heads_total < 1 || p->heads < 1 || head0 + p->heads > heads_total)
+        return PRISM_ERR_INVALID_ARG;
+    for (int i = 0; i < shards; ++i)
+        if (!Q[i] || !K[i] || !V[i] || !aligned16(Q[i]) || !aligned16(K[i]) || !aligned16(V[i]))
+            return PRISM_ERR_INVALID_ARG;
+    prism_plan_s* P = nullptr;
+    int st = plan_common(p, Q[0], K[0], V[0], workspace, ws_bytes, &P);
+    if (st) return st;
+    P->has_audio = 0;
+    P->has_cuts = zone_cut != nullptr;
+    const Geom& g = P->g;
+    const int64_t HW = (int64_t)g.H * g.W;
+    st = run_plan(P, shard_rows(Q, shards, g.T, HW, heads_total, head0), shard_rows(K, shards, g.T, HW, heads_total, head0),
+                  shard_rows(V, shards, g.T, HW, heads_total, head0), nullptr, shape_id, sel,
+                  static_cast<cudaStream_t>(stream), zone_cut, shape_id2);
+    if (st) { delete P; return st; }
+    *out = P;
+    return PRISM_OK;
+}
+
 extern "C" int prism_plan_import(const prism_params* p, const void* Q, const void* K, const void* V,
                                  const uint8_t* shape_id, const uint32_t* sel, void* workspace,
                                  size_t ws_bytes, void* stream, prism_plan_t* out) {

@@ -260,6 +260,18 @@ PRISM_API int prism_plan_import_cuts(const prism_params* p, const void* Q, const
                                      size_t ws_bytes, void* stream, prism_plan_t* out);
 
 /*
+ * prism_plan_import_sharded -- prism_plan_import_cuts for inputs held as token
+ * shards (the layout and the head range of prism_plan_sharded): the given
+ * shapes, splits (zone_cut and shape_id2 both NULL without adaptive temporal
+ * boundaries) and selection, with the reorder reading every shard's rows.
+ */
+PRISM_API int prism_plan_import_sharded(const prism_params* p, const void* const* Q, const void* const* K,
+                                        const void* const* V, int shards, int heads_total, int head0,
+                                        const uint8_t* shape_id, const uint8_t* zone_cut,
+                                        const uint8_t* shape_id2, const uint32_t* sel, void* workspace,
+                                        size_t ws_bytes, void* stream, prism_plan_t* out);
+
+/*
  * prism_plan_list_bytes -- for a plan made with a core-only workspace: the
  *   bytes its index lists need (0 once they are built).  Synchronises `stream`
  *   (reads each head's list lengths).

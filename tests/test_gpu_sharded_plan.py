@@ -11,8 +11,10 @@ gradients to fp32 summation order.  Cases: bf16 with 4 shards of 4 frames
 (every 8-frame zone spans two shards) and adaptive temporal boundaries on, and
 the fp32 tiny workload with 2 shards.  The forward and the backward in the
 shard layout (prism_attn_fwd_sharded, prism_attn_bwd_sharded): every rank's
-rows of O, dQ, dK, dV land in the shards equal to the gathered run's.  Invalid
-shard counts and head ranges are rejected before any launch.
+rows of O, dQ, dK, dV land in the shards equal to the gathered run's.  The
+sharded import (prism_plan_import_sharded) rebuilds a sharded plan from its own
+shapes, splits and selection.  Invalid shard counts and head ranges are
+rejected before any launch.
 """
 import numpy as np
 import pytest
@@ -120,6 +122,31 @@ def test_sequence_parallel_round_trip_in_place(case, cuda_device):
             else:
                 diff, scale = (g - e).abs().max().item(), e.abs().max().item()
                 assert diff <= 1e-5 * scale, f"{case} rank {r} {nm}: {diff:.3e} at scale {scale:.3e}"
+
+
+def test_sharded_import_equals_sharded_plan(cuda_device):
+    """prism_plan_import_sharded given a sharded plan's own shapes, splits and
+    selection rebuilds that plan: the reorder and pooling from the shards, and
+    the forward, bit for bit."""
+    w = syn.workload(2, T=16, H=32, W=32, shot_cuts=[6])
+    P, heads, nh, h0 = 4, 4, 2, 2
+    Q, K, V = syn.make_qkv(w, device="cuda", heads=heads)
+    a = syn.make_amap(w, device="cuda")
+    qs, ks, vs = _shards(Q, P), _shards(K, P), _shards(V, P)
+    prm = _lib.make_params(w.T, w.H, w.W, nh, w.head_dim, _lib.PRISM_BF16, w.top_k, w.top_p, w.eps, cut_ratio=2.5)
+    pl = _lib.plan_sharded(qs, ks, vs, a, prm, head0=h0, heads_total=heads)
+    dev = lambda item, dt: torch.from_numpy(pl.export(item).view(dt)).cuda()
+    sid, cut, sid2 = dev("shape_id", np.uint8), dev("zone_cut", np.uint8), dev("shape_id2", np.uint8)
+    bits = dev("sel_bits", np.int32)
+    im = _lib.plan_import_sharded(qs, ks, vs, sid, bits, prm, head0=h0, heads_total=heads, zone_cut=cut,
+                                  shape_id2=sid2)
+    for item in ("blk_start", "src", "sel_bits", "qkv_max"):
+        np.testing.assert_array_equal(im.export(item), pl.export(item), err_msg=item)
+    O1, l1 = pl.attn_fwd()
+    O2, l2 = im.attn_fwd()
+    torch.cuda.synchronize()
+    assert im.status() == _lib.PRISM_OK
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
 
 
 def test_sharded_plan_rejects_bad_layouts(cuda_device):
