@@ -20,7 +20,7 @@ plan itself needs no collective.  The library computes nothing here: this
 module only moves tensors between ranks with torch.distributed.
 
 Where the ranks' sequence shards are mapped into each other's address space
-(torch symmetric memory, CUDA IPC), both exchanges can be left out:
+(`symmetric_shard`: torch symmetric memory), both exchanges can be left out:
 `_lib.plan_sharded(qs, ks, vs, a, params, head0=h0, heads_total=H)` plans this
 rank's heads (`rank_heads`) straight from every rank's Q, K, V shard (the
 plan's reorder reads the other GPUs' rows over NVLink), and the plan's
@@ -35,6 +35,23 @@ import torch.distributed as dist
 
 def _world(group):
     return dist.get_world_size(group), dist.get_rank(group)
+
+
+def symmetric_shard(shape, dtype, group=None):
+    """A sequence shard in symmetric memory, for the `_sharded` entry points.
+
+    Returns (t, addresses, handle): the local shard tensor `t` (write this rank's
+    rows into it), every rank's shard mapped into this process as device addresses
+    in rank order (pass them as the shard list), and the rendezvous handle, which
+    must outlive every plan and launch that uses the addresses.  The ranks must have
+    written their shards (a barrier on `group`, with the writes synchronised) before
+    a kernel reads them, and must not reuse a shard while another rank's kernels may
+    still read or write it.  Needs one GPU per rank with peer access (NVLink)."""
+    import torch.distributed._symmetric_memory as symm_mem
+    t = symm_mem.empty(*shape, dtype=dtype, device=torch.device("cuda", torch.cuda.current_device()))
+    handle = symm_mem.rendezvous(t, group if group is not None else dist.group.WORLD)
+    delta = t.data_ptr() - handle.buffer_ptrs[handle.rank]
+    return t, [p + delta for p in handle.buffer_ptrs], handle
 
 
 def rank_heads(rank: int, world: int, heads: int) -> tuple[int, int]:
