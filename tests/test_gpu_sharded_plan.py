@@ -13,8 +13,9 @@ the fp32 tiny workload with 2 shards.  The forward and the backward in the
 shard layout (prism_attn_fwd_sharded, prism_attn_bwd_sharded): every rank's
 rows of O, dQ, dK, dV land in the shards equal to the gathered run's.  The
 sharded import (prism_plan_import_sharded) rebuilds a sharded plan from its own
-shapes, splits and selection.  Invalid shard counts and head ranges are
-rejected before any launch.
+shapes, splits and selection.  sequence_parallel.symmetric_shard, in an NCCL
+group of one rank, gives shard addresses the sharded plan reads.  Invalid shard
+counts and head ranges are rejected before any launch.
 """
 import numpy as np
 import pytest
@@ -168,3 +169,60 @@ def test_sharded_plan_rejects_bad_layouts(cuda_device):
         _lib.plan_sharded([qs[0].data_ptr() + 4, qs[1].data_ptr()], ks, vs, a, prm, heads_total=2)
     assert e.value.status == _lib.PRISM_ERR_INVALID_ARG
     assert N % 2 == 0
+
+
+SYMM_CHILD = r"""
+import os, sys, json
+import torch, torch.distributed as dist
+sys.path.insert(0, sys.argv[1])
+from dynamic_block_sparse_indicator_b200 import _lib
+from dynamic_block_sparse_indicator_b200 import sequence_parallel as sp
+from dynamic_block_sparse_indicator_b200 import synthetic as syn
+os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=sys.argv[2], RANK="0", WORLD_SIZE="1")
+torch.cuda.set_device(0)
+dist.init_process_group("nccl", rank=0, world_size=1)
+try:
+    w = syn.workload(0)
+    Q, K, V = syn.make_qkv(w, device="cuda", heads=2)
+    a = syn.make_amap(w, device="cuda")
+    shards, keep = [], []
+    for x in (Q, K, V):
+        t, addrs, h = sp.symmetric_shard(tuple(x.shape), x.dtype)
+        t.copy_(x)
+        keep.append((t, h))
+        shards.append(addrs)
+    torch.cuda.synchronize()
+    dist.barrier()
+    prm = _lib.make_params(w.T, w.H, w.W, 2, w.head_dim, _lib.PRISM_F32, w.top_k, w.top_p, w.eps)
+    got = _lib.plan_sharded(shards[0], shards[1], shards[2], a, prm, heads_total=2)
+    ref = _lib.plan(Q, K, V, a, prm)
+    O1, _ = got.attn_fwd()
+    O2, _ = ref.attn_fwd()
+    torch.cuda.synchronize()
+    same = bool(torch.equal(O1, O2)) and got.status() == 0
+    print(json.dumps({"same": same, "n": len(shards[0])}))
+    del got, ref
+finally:
+    dist.destroy_process_group()
+"""
+
+
+def test_symmetric_shard_single_rank(cuda_device, tmp_path):
+    """symmetric_shard on one rank (NCCL group of one): its address list feeds
+    plan_sharded, whose forward equals prism_plan's."""
+    import json
+    import os
+    import socket
+    import subprocess
+    import sys
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    script = tmp_path / "child.py"
+    script.write_text(SYMM_CHILD)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, str(script), root, str(port)], capture_output=True, text=True,
+                         timeout=300, env=dict(os.environ, NCCL_NVLS_ENABLE="0"))
+    assert res.returncode == 0, res.stderr[-3000:]
+    out = json.loads(res.stdout.strip().splitlines()[-1])
+    assert out == {"same": True, "n": 1}
